@@ -1,0 +1,168 @@
+"""Seeded synthetic inputs for the FP8 scaled GEMM workloads.
+
+Only random numbers and shapes live here: no quantization, no scaling, no
+GEMM arithmetic.  Both the CUDA path (through the bindings) and the CPU oracle
+(in tests and the CPU-baseline leg of bench.py) are fed the same tensors from
+this module.
+
+Every tensor is drawn on the CPU from a ``torch.Generator`` in fp32 and then
+rounded to bf16 (round-to-nearest-even), in the order listed for each
+workload; the seed of workload ``i`` (0-based, in the order below) is
+``1000 + i`` (``+100`` for the second (N, K) shape of the blockwise pair).
+
+Workloads (shapes and distributions from the pages' benchmark and test
+descriptions; no public dataset is involved):
+  0 tensorwise  M=N=K=256, A,B ~ N(0,1)
+  1 rowwise     M=N=K=4096, A ~ N(0,1) with 0.1% of entries x50 (outliers),
+                W ~ N(0, 0.02^2), bias ~ N(0, 0.01^2)
+  2 blockwise 1x128_128x128  M=16640, (N,K) in {(5120,8192), (8192,5120)},
+                A ~ N(0,1), W ~ N(0, 0.02^2)
+  3 blockwise 1x128_128x1    M=16640, same (N,K) pair,
+                L ~ N(0, 1e-3^2) (M,K), R ~ N(0,1) stored (N,K)
+  4 grouped     E=16, W ~ N(0, 0.02^2) (16,4096,4096), A ~ N(0,1) (32768,4096),
+                group sizes: 2048 chunks of 16 rows, each chunk given to an
+                expert drawn from p(r) ~ r^-1.2 over ranks r=1..16, ranks mapped
+                to experts by a seeded permutation; offs = cumulative ends
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import Dict, List, Optional
+
+import numpy as np
+import torch
+
+WORKLOAD_NAMES = [
+    "tensorwise_256",
+    "rowwise_4096",
+    "blockwise_1x128_128x128",
+    "blockwise_1x128_128x1",
+    "grouped_e16",
+]
+
+
+def generator(seed: int) -> torch.Generator:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    return g
+
+
+def randn_bf16(shape, std: float, g: torch.Generator,
+               outlier_frac: float = 0.0, outlier_mult: float = 1.0) -> torch.Tensor:
+    """N(0, std^2) in fp32, optional outliers (a seeded random subset of exactly
+    round(frac * numel) entries multiplied by ``outlier_mult``), then bf16."""
+    x = torch.randn(*shape, generator=g, dtype=torch.float32)
+    if std != 1.0:
+        x.mul_(std)
+    if outlier_frac > 0.0:
+        n = int(round(outlier_frac * x.numel()))
+        idx = torch.randperm(x.numel(), generator=g)[:n]
+        x.view(-1)[idx] *= outlier_mult
+    return x.to(torch.bfloat16)
+
+
+def bf16_bits(t: torch.Tensor) -> np.ndarray:
+    """uint16 bit patterns of a CPU bf16 tensor (no copy of the values' meaning)."""
+    assert t.dtype == torch.bfloat16
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def zipf_group_sizes(total_rows: int, E: int, chunk: int, s: float,
+                     g: torch.Generator) -> torch.Tensor:
+    """Group sizes (multiples of ``chunk``) summing to ``total_rows``."""
+    assert total_rows % chunk == 0
+    ranks = torch.arange(1, E + 1, dtype=torch.float64)
+    p = ranks.pow(-s)
+    p = p / p.sum()
+    n_chunks = total_rows // chunk
+    chunk_rank = torch.multinomial(p, n_chunks, replacement=True, generator=g)
+    perm = torch.randperm(E, generator=g)
+    expert = perm[chunk_rank]
+    return torch.bincount(expert, minlength=E).to(torch.int64) * chunk
+
+
+def offsets_from_sizes(sizes) -> torch.Tensor:
+    """Cumulative end offsets, int32."""
+    sizes = torch.as_tensor(sizes, dtype=torch.int64)
+    return torch.cumsum(sizes, 0).to(torch.int32)
+
+
+@dataclass
+class Workload:
+    name: str
+    recipe: str                      # tensor | row | 1x128_128x128 | 1x128_128x1 | grouped
+    M: int
+    N: int
+    K: int
+    a: torch.Tensor                  # bf16 (M, K) CPU
+    b: torch.Tensor                  # bf16 (N, K) or (E, N, K) CPU
+    bias: Optional[torch.Tensor] = None   # bf16 (N,) CPU
+    offs: Optional[torch.Tensor] = None   # int32 (E,) CPU
+    E: int = 0
+    seed: int = 0
+    extra: Dict = field(default_factory=dict)
+
+    @property
+    def flops(self) -> int:
+        return 2 * self.M * self.N * self.K
+
+
+def make_workload(index: int, shape_index: int = 0, scale_down: int = 1) -> Workload:
+    """Build workload ``index`` (see module doc).  ``scale_down`` > 1 divides M
+    (and, for the grouped case, the token count) to make a smaller case with
+    the same distributions; sizes stay multiples of 16."""
+    seed = 1000 + index + 100 * shape_index
+    g = generator(seed)
+    name = WORKLOAD_NAMES[index]
+    if index == 0:
+        M = N = K = 256
+        a = randn_bf16((M, K), 1.0, g)
+        b = randn_bf16((N, K), 1.0, g)
+        return Workload(name, "tensor", M, N, K, a, b, seed=seed)
+    if index == 1:
+        M = N = K = 4096
+        M //= scale_down
+        a = randn_bf16((M, K), 1.0, g, outlier_frac=0.001, outlier_mult=50.0)
+        b = randn_bf16((N, K), 0.02, g)
+        bias = randn_bf16((N,), 0.01, g)
+        return Workload(name, "row", M, N, K, a, b, bias=bias, seed=seed)
+    if index in (2, 3):
+        NK = [(5120, 8192), (8192, 5120)][shape_index]
+        M = 16640 // scale_down
+        M -= M % 16
+        N, K = NK
+        if index == 2:
+            a = randn_bf16((M, K), 1.0, g)
+            b = randn_bf16((N, K), 0.02, g)
+            return Workload(name, "1x128_128x128", M, N, K, a, b, seed=seed)
+        a = randn_bf16((M, K), 1e-3, g)
+        b = randn_bf16((N, K), 1.0, g)
+        return Workload(name, "1x128_128x1", M, N, K, a, b, seed=seed)
+    if index == 4:
+        E, N, K = 16, 4096, 4096
+        T = 32768 // scale_down
+        b = randn_bf16((E, N, K), 0.02, g)
+        a = randn_bf16((T, K), 1.0, g)
+        sizes = zipf_group_sizes(T, E, 16, 1.2, g)
+        offs = offsets_from_sizes(sizes)
+        return Workload(name, "grouped", T, N, K, a, b, offs=offs, E=E, seed=seed)
+    raise ValueError(f"unknown workload {index}")
+
+
+def small_case(recipe: str, M: int, N: int, K: int, seed: int,
+               a_std: float = 1.0, b_std: float = 0.02, bias: bool = False,
+               E: int = 0, group_sizes: Optional[List[int]] = None) -> Workload:
+    """A parity-test case of arbitrary (ragged) size with the workloads'
+    distributions."""
+    g = generator(seed)
+    if recipe == "grouped":
+        assert group_sizes is not None and len(group_sizes) == E
+        b = randn_bf16((E, N, K), b_std, g)
+        a = randn_bf16((M, K), a_std, g)
+        offs = offsets_from_sizes(group_sizes)
+        assert int(offs[-1]) == M
+        return Workload("small_grouped", recipe, M, N, K, a, b, offs=offs, E=E, seed=seed)
+    a = randn_bf16((M, K), a_std, g)
+    b = randn_bf16((N, K), b_std, g)
+    bb = randn_bf16((N,), 0.01, g) if bias else None
+    return Workload(f"small_{recipe}", recipe, M, N, K, a, b, bias=bb, seed=seed)
