@@ -1,0 +1,498 @@
+#!/usr/bin/env python
+"""Benchmark of the FP8 scaled-GEMM hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+dynamic quantization of both operands (amax -> scale -> e4m3 cast) and the
+scaled GEMM with its epilogue (scales, bias, bf16 cast) -- or, for the MoE
+workload, the grouped GEMM over the offs array.  Inputs are resident in HBM
+when the timed region starts; L2 is flushed (a 256 MB write) between steps,
+outside the per-step CUDA events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference]
+
+Prints ONE JSON line (rank 0).  `value` is GEMM TFLOP/s over the whole step
+(quantize + GEMM) summed over ranks; `roofline` describes the GEMM kernel
+alone against the measured peak; `e2e` is the same metric through the public
+API with host buffers and the copies inside the timed region;
+`cpu_baseline` is the CPU oracle on a bounded sample of the same workload.
+
+With --impl reference the oracle itself is timed on the host cores (rank 0
+only), as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from fp8_scaled_matrix_b200 import workloads as W  # noqa: E402
+
+WORKLOADS = {
+    # name: (workload index, shape index)
+    "tensorwise_256": (0, 0),
+    "rowwise_4096": (1, 0),
+    "blockwise_1x128_128x128": (2, 0),
+    "blockwise_1x128_128x128_b": (2, 1),
+    "blockwise_1x128_128x1": (3, 0),
+    "blockwise_1x128_128x1_b": (3, 1),
+    "grouped_e16": (4, 0),
+}
+DEFAULT_WORKLOAD = "rowwise_4096"
+# Page 5's context numbers (TFLOP/s of torch._scaled_mm, hardware not stated)
+PAGE_NUMBERS = {
+    "blockwise_1x128_128x128": 1008.91, "blockwise_1x128_128x128_b": 1002.23,
+    "blockwise_1x128_128x1": 808.271, "blockwise_1x128_128x1_b": 807.015,
+}
+OPERAND_GROUPS = {"tensor": ("tensor", "tensor"), "row": ("row", "row"),
+                  "1x128_128x128": ("1x128", "128x128"),
+                  "1x128_128x1": ("1x128", "1x128"), "grouped": ("row", "row")}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_OVER_BF16 = 2.0   # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+L2_FLUSH_BYTES = 256 << 20
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ------------------------------------------------------------------ peaks
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_sources_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "fp8_scaled_matrix_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per GEMM launch from the committed ncu summary, if it was
+    taken on the current kernel sources; otherwise None."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        e = d.get(workload)
+        if e and e.get("sources") == kernel_sources_hash():
+            return float(e["bytes_per_launch"])
+    except Exception:
+        return None
+    return None
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.t:
+            self.t.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- our path
+
+class Step:
+    """Device buffers and the launches of one step of a workload."""
+
+    def __init__(self, wl: W.Workload, dev: torch.device):
+        from fp8_scaled_matrix_b200 import fp8sm
+        self.f = fp8sm
+        self.wl = wl
+        self.dev = dev
+        ga, gb = OPERAND_GROUPS[wl.recipe]
+        self.qa_recipe = fp8sm.QUANT_RECIPES[ga]
+        self.qb_recipe = fp8sm.QUANT_RECIPES[gb]
+        self.a = wl.a.to(dev)
+        if wl.recipe == "grouped":
+            E, N, K = wl.b.shape
+            self.b = wl.b.to(dev).reshape(E * N, K)
+            self.offs = wl.offs.to(dev)
+        else:
+            self.b = wl.b.to(dev)
+            self.offs = None
+        self.bias = None if wl.bias is None else wl.bias.to(dev)
+        rows_a, cols = self.a.shape
+        rows_b = self.b.shape[0]
+        self.qa = torch.empty(rows_a, cols, dtype=torch.uint8, device=dev)
+        self.qb = torch.empty(rows_b, cols, dtype=torch.uint8, device=dev)
+        self.sa = torch.empty(max(fp8sm.scale_count(rows_a, cols, self.qa_recipe), 1),
+                              dtype=torch.float32, device=dev)
+        self.sb = torch.empty(max(fp8sm.scale_count(rows_b, cols, self.qb_recipe), 1),
+                              dtype=torch.float32, device=dev)
+        self.ws = torch.zeros(64, dtype=torch.uint8, device=dev)
+        self.out = torch.empty(wl.M, wl.N, dtype=torch.bfloat16, device=dev)
+        self.launches_per_step = 3
+
+    def quantize(self):
+        f = self.f
+        f.fp8_quantize(self.a, self.qa_recipe, out=self.qa, scales=self.sa, workspace=self.ws)
+        f.fp8_quantize(self.b, self.qb_recipe, out=self.qb, scales=self.sb, workspace=self.ws)
+
+    def gemm(self):
+        f = self.f
+        wl = self.wl
+        if wl.recipe == "grouped":
+            E, N, K = wl.b.shape
+            f.fp8_grouped_scaled_mm(self.qa, self.qb.view(E, N, K), self.sa,
+                                    self.sb.view(E, N), self.offs, out=self.out)
+        else:
+            f.fp8_scaled_mm(self.qa, self.qb, self.sa, self.sb,
+                            f.MM_RECIPES[wl.recipe], bias=self.bias, out=self.out)
+
+    def quant_bytes(self) -> int:
+        """Algorithmic HBM bytes of the two quantize launches: 2 B read +
+        1 B written per element, 4 B per scale."""
+        n = self.a.numel() + self.b.numel()
+        return 3 * n + 4 * (self.sa.numel() + self.sb.numel())
+
+
+def run_ours(args, wl, dev, rank, world):
+    torch.cuda.set_device(dev)
+    st = Step(wl, dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        st.quantize()
+        st.gemm()
+    torch.cuda.synchronize()
+    st.f.check_device_status()
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.25)  # let the sampler start before the timed work
+    for i in range(K):
+        flush.zero_()  # evict L2 (outside the step's events)
+        ev[i][0].record(stream)
+        st.quantize()
+        ev[i][1].record(stream)
+        st.gemm()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    st.f.check_device_status()
+    q_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    g_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    step_ms = [q + g for q, g in zip(q_ms, g_ms)]
+    total_ms = float(np.sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    res = {
+        "total_ms": total_ms,
+        "q_ms": float(np.mean(q_ms)), "g_ms": float(np.mean(g_ms)),
+        "g_ms_median": float(np.median(g_ms)), "q_ms_median": float(np.median(q_ms)),
+        "quant_bytes": st.quant_bytes(), "launches": st.launches_per_step * K,
+        "clocks": clocks,
+    }
+    if not args.no_e2e:
+        res["e2e"] = run_e2e(args, wl, dev, world)
+    return res
+
+
+def run_e2e(args, wl, dev, world):
+    """Same step through the public API from pinned HOST buffers: H2D copies
+    of the bf16 inputs, quantize, GEMM, D2H copy of the bf16 result, all in
+    the timed region."""
+    from fp8_scaled_matrix_b200 import fp8sm
+    ha = wl.a.pin_memory()
+    hb = (wl.b.reshape(-1, wl.K) if wl.recipe == "grouped" else wl.b).contiguous().pin_memory()
+    hbias = None if wl.bias is None else wl.bias.pin_memory()
+    hout = torch.empty(wl.M, wl.N, dtype=torch.bfloat16).pin_memory()
+    st = Step(wl, dev)
+    da, db = st.a, st.b
+    dbias = st.bias
+    stream = torch.cuda.current_stream()
+    steps = max(3, min(args.steps, args.e2e_steps))
+
+    def one():
+        da.copy_(ha, non_blocking=True)
+        db.copy_(hb, non_blocking=True)
+        if hbias is not None:
+            dbias.copy_(hbias, non_blocking=True)
+        st.quantize()
+        st.gemm()
+        hout.copy_(st.out, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    h2d = ha.numel() * 2 + hb.numel() * 2 + (0 if hbias is None else hbias.numel() * 2)
+    d2h = hout.numel() * 2
+    return {"ms": ms, "h2d": h2d, "d2h": d2h, "steps": steps}
+
+
+# ---------------------------------------------------------------- oracle
+
+def oracle_sample(wl, max_rows: int):
+    """Time the CPU oracle on a bounded sample of the workload: quantize of
+    both operands in full, the GEMM on the first `max_rows` output rows.
+    Returns (seconds for the sample, fraction of the GEMM it covers,
+    seconds for quantize, threads)."""
+    import oracle
+    ga, gb = OPERAND_GROUPS[wl.recipe]
+    G = {"tensor": oracle.GROUP_TENSOR, "row": oracle.GROUP_ROW,
+         "1x128": oracle.GROUP_1x128, "128x128": oracle.GROUP_128x128}
+    MMR = {"tensor": oracle.MM_TENSOR_TENSOR, "row": oracle.MM_ROW_ROW,
+           "1x128_128x128": oracle.MM_1x128_128x128, "1x128_128x1": oracle.MM_1x128_128x1}
+    t0 = time.perf_counter()
+    qa, sa = oracle.quantize(W.bf16_bits(wl.a), G[ga])
+    if wl.recipe == "grouped":
+        E, N, K = wl.b.shape
+        qb, sb = oracle.quantize(W.bf16_bits(wl.b.reshape(E * N, K)), G[gb])
+    else:
+        qb, sb = oracle.quantize(W.bf16_bits(wl.b), G[gb])
+    tq = time.perf_counter() - t0
+    rows = np.arange(min(max_rows, wl.M), dtype=np.int64)
+    t0 = time.perf_counter()
+    if wl.recipe == "grouped":
+        E, N, K = wl.b.shape
+        oracle.grouped_scaled_mm(qa, qb.reshape(E, N, K), sa, sb.reshape(E, N),
+                                 wl.offs.numpy(), rows=rows)
+    else:
+        bias = None if wl.bias is None else W.bf16_bits(wl.bias)
+        oracle.scaled_mm(qa, qb, sa, sb, MMR[wl.recipe], bias_bits=bias, rows=rows)
+    tg = time.perf_counter() - t0
+    return tg, rows.size / wl.M, tq, oracle.num_threads()
+
+
+def cpu_baseline(wl, rows: int):
+    tg, frac, tq, threads = oracle_sample(wl, rows)
+    est_s = tq + tg / frac
+    value = wl.flops / est_s / 1e12
+    return {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": (f"quantize of both operands in full ({tq:.2f} s) + GEMM on "
+                       f"{int(round(frac * wl.M))} of {wl.M} output rows ({tg:.2f} s), "
+                       f"scaled to all rows"),
+            "seconds_est_per_step": est_s}
+
+
+def baseline_rows(wl, target_s: float = 12.0) -> int:
+    """Rows of the GEMM that take about target_s on the oracle (probe with 8)."""
+    tg, frac, _, _ = oracle_sample(wl, 8)
+    per_row = tg / max(1, int(round(frac * wl.M)))
+    return int(max(8, min(wl.M, target_s / max(per_row, 1e-9))))
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=0,
+                    help="output rows for the CPU oracle sample (0: about 12 s of work)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    idx, shape_index = WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        wl = W.make_workload(idx, shape_index)
+        steps = args.steps or 1
+        rows = args.cpu_rows or baseline_rows(wl, 20.0 / max(1, steps + args.warmup))
+        for _ in range(min(args.warmup, 1)):
+            oracle_sample(wl, max(8, rows // 4))
+        times = []
+        for _ in range(steps):
+            b = cpu_baseline(wl, rows)
+            times.append(b["seconds_est_per_step"])
+        ms = float(np.mean(times)) * 1e3
+        value = wl.flops / (ms * 1e-3) / 1e12
+        line = {
+            "impl": "reference", "metric": "fp8_scaled_gemm_tflops", "value": value,
+            "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp8e4m3/int64-exact/f64", "data": "synthetic",
+            "config": {"workload": args.workload, "M": wl.M, "N": wl.N, "K": wl.K},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": b["cores"],
+                             "kind": "oracle", "sample": b["sample"]},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+        return 0
+
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local_rank)
+    from fp8_scaled_matrix_b200 import build
+    build.build()
+
+    wl = W.make_workload(idx, shape_index)
+    if args.steps is None:
+        # about a second of timed work per workload
+        args.steps = {"tensorwise_256": 4000, "rowwise_4096": 3000,
+                      "grouped_e16": 1000}.get(args.workload, 600)
+    res = run_ours(args, wl, dev, rank, world)
+
+    peaks, peak_src = load_peaks()
+    fp8_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])) * FP8_OVER_BF16
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    K = args.steps
+    ms_per_step = res["total_ms"] / K
+    value = wl.flops * world / (ms_per_step * 1e-3) / 1e12
+    gemm_tflops = wl.flops / (res["g_ms"] * 1e-3) / 1e12
+    quant_gbs = res["quant_bytes"] / (res["q_ms"] * 1e-3) / 1e9
+    line = {
+        "metric": "fp8_scaled_gemm_tflops",
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": (value / world / PAGE_NUMBERS[args.workload]
+                        if args.workload in PAGE_NUMBERS else None),
+        "dtype": "fp8e4m3 (fp32 accumulate)",
+        "data": "synthetic",
+        "config": {
+            "workload": args.workload, "M": wl.M, "N": wl.N, "K": wl.K,
+            "recipe": wl.recipe, "E": wl.E or None, "bias": wl.bias is not None,
+            "out_dtype": "bf16", "l2": "flushed between steps (256 MB write, outside the step events)",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "step": "quantize A + quantize B + scaled GEMM",
+        },
+        "roofline": {
+            "bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak,
+            "unit": "TFLOP/s", "frac": gemm_tflops / fp8_peak,
+            "traffic": recorded_traffic(args.workload),
+            "kernel": "fp8_gemm_kernel", "peak_source":
+                f"{peak_src} bf16 burst x {FP8_OVER_BF16:g} (nominal fp8/bf16 dense ratio)",
+            "ms_per_launch": res["g_ms"],
+        },
+        "roofline_quantize": {
+            "bound": "hbm", "achieved": quant_gbs, "peak": hbm_peak, "unit": "GB/s",
+            "frac": quant_gbs / hbm_peak, "ms_per_step": res["q_ms"],
+            "bytes_per_step": res["quant_bytes"], "peak_source": peak_src,
+        },
+        "gpu_launches": res["launches"],
+        "clocks": res["clocks"],
+    }
+    if "e2e" in res:
+        e = res["e2e"]
+        line["e2e"] = {"value": wl.flops * world / (e["ms"] * 1e-3) / 1e12, "unit": "TFLOP/s",
+                       "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
+                       "ms_per_step": e["ms"], "steps": e["steps"]}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows = args.cpu_rows or baseline_rows(wl)
+        line["cpu_baseline"] = {k: v for k, v in cpu_baseline(wl, rows).items()
+                                if k != "seconds_est_per_step"}
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

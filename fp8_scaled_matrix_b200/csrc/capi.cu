@@ -1,0 +1,266 @@
+// C ABI of the library (declared in include/fp8sm.h): argument validation,
+// recipe -> kernel selection (one kernel per recipe, no fallback), the
+// per-device status word and per-thread error messages.
+//
+// Error classes follow "Add _scaled_mm_v2 API" (Blas.cpp review): invalid
+// arguments are a user error (FP8_ERR_VALUE), combinations that could exist
+// but are not implemented are FP8_ERR_UNSUPPORTED, everything else
+// (CUDA failures) FP8_ERR_CUDA.  "Add _grouped_mm dispatch handler to
+// Float8Tensor" requires that an unsupported granularity raises instead of
+// silently running something else; nothing here ever falls back.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+#include <string>
+
+#include "../../include/fp8sm.h"
+#include "internal.h"
+
+namespace fp8sm {
+// Device status words (one per device, since __device__ variables are
+// instantiated per device): [0] first error code, [1] site.
+__device__ uint32_t g_status_word[2];
+}  // namespace fp8sm
+
+namespace {
+
+thread_local std::string t_last_error;
+
+constexpr int kMaxDevices = 64;
+struct DeviceInfo {
+  bool ready = false;
+  uint32_t* status = nullptr;
+  int num_sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+fp8_status fail(fp8_status s, const std::string& msg) {
+  t_last_error = msg;
+  return s;
+}
+
+fp8_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(FP8_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+// Per-device set-up on first use: the status word's device address (taken
+// with the device current) and the SM count.
+fp8_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(FP8_ERR_CUDA, "device index out of range");
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, fp8sm::g_status_word);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status)");
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (major != 10 || minor != 0)
+      return fail(FP8_ERR_UNSUPPORTED,
+                  "this library is built for sm_100a (B200); device has compute capability " +
+                      std::to_string(major) + "." + std::to_string(minor));
+    d.status = static_cast<uint32_t*>(p);
+    d.num_sms = sms;
+    d.ready = true;
+  }
+  *out = &d;
+  return FP8_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) {
+  return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+fp8_status finish_launch(cudaError_t e, const std::string& err, const char* what) {
+  if (e == cudaSuccess) {
+    t_last_error.clear();
+    return FP8_OK;
+  }
+  if (!err.empty()) return fail(FP8_ERR_VALUE, std::string(what) + ": " + err);
+  return cuda_fail(e, what);
+}
+
+}  // namespace
+
+extern "C" {
+
+int fp8_version(void) { return 100; }
+
+const char* fp8_last_error(void) { return t_last_error.c_str(); }
+
+size_t fp8_quantize_workspace_bytes(fp8_quant_recipe recipe, int64_t rows,
+                                    int64_t cols) {
+  (void)rows;
+  (void)cols;
+  return recipe == FP8_SCALE_TENSOR ? 16 : 0;
+}
+
+fp8_status fp8_quantize(const void* x_bf16, int64_t rows, int64_t cols,
+                        int64_t ld_x, fp8_quant_recipe recipe, void* out_fp8,
+                        float* out_scales, void* workspace, size_t ws_bytes,
+                        fp8_stream_t stream) {
+  if (recipe < FP8_SCALE_TENSOR || recipe > FP8_SCALE_BLOCK_128x128)
+    return fail(FP8_ERR_VALUE, "fp8_quantize: unknown recipe");
+  if (rows < 0 || cols < 0) return fail(FP8_ERR_VALUE, "fp8_quantize: negative size");
+  if (rows > (int64_t(1) << 31) || cols > (int64_t(1) << 31))
+    return fail(FP8_ERR_VALUE, "fp8_quantize: size too large");
+  if (ld_x < cols) return fail(FP8_ERR_VALUE, "fp8_quantize: ld_x < cols");
+  if (cols % 8 != 0 || ld_x % 8 != 0)
+    return fail(FP8_ERR_VALUE, "fp8_quantize: cols and ld_x must be multiples of 8");
+  if ((recipe == FP8_SCALE_BLOCK_1x128 || recipe == FP8_SCALE_BLOCK_128x128) &&
+      cols % 128 != 0)
+    return fail(FP8_ERR_VALUE, "fp8_quantize: blockwise recipes need cols % 128 == 0");
+  const bool empty = rows == 0 || cols == 0;
+  const bool writes_scales = !(rows == 0 && recipe != FP8_SCALE_TENSOR) &&
+                             !(cols == 0 && (recipe == FP8_SCALE_BLOCK_1x128 ||
+                                             recipe == FP8_SCALE_BLOCK_128x128));
+  if (!empty && (x_bf16 == nullptr || out_fp8 == nullptr))
+    return fail(FP8_ERR_VALUE, "fp8_quantize: null tensor pointer");
+  if (writes_scales && out_scales == nullptr)
+    return fail(FP8_ERR_VALUE, "fp8_quantize: null scale pointer");
+  if (!empty && (!aligned(x_bf16, 16) || !aligned(out_fp8, 16)))
+    return fail(FP8_ERR_VALUE, "fp8_quantize: x and out_fp8 must be 16-byte aligned");
+  if (out_scales && !aligned(out_scales, 4))
+    return fail(FP8_ERR_VALUE, "fp8_quantize: out_scales must be 4-byte aligned");
+  const size_t need = fp8_quantize_workspace_bytes(recipe, rows, cols);
+  if (need > 0 && (workspace == nullptr || ws_bytes < need || !aligned(workspace, 16)))
+    return fail(FP8_ERR_VALUE, "fp8_quantize: tensorwise recipe needs a 16-byte aligned "
+                               "workspace of fp8_quantize_workspace_bytes() bytes");
+  if (!writes_scales) {
+    t_last_error.clear();
+    return FP8_OK;
+  }
+  DeviceInfo* d = nullptr;
+  fp8_status s = device_info(&d);
+  if (s != FP8_OK) return s;
+  std::string err;
+  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status,
+                       d->num_sms, &err};
+  cudaError_t e = fp8sm::launch_quantize(x_bf16, rows, cols, ld_x, (int)recipe,
+                                         out_fp8, out_scales, workspace, ctx);
+  return finish_launch(e, err, "fp8_quantize");
+}
+
+fp8_status fp8_scaled_mm(const void* a, const void* b, int64_t M, int64_t N,
+                         int64_t K, const float* scale_a, const float* scale_b,
+                         fp8_mm_recipe recipe, const void* bias_bf16,
+                         fp8_out_dtype out_dtype, void* out,
+                         fp8_stream_t stream) {
+  if (recipe < FP8_MM_TENSOR_TENSOR || recipe > FP8_MM_1x128_128x1)
+    return fail(FP8_ERR_VALUE, "fp8_scaled_mm: unknown recipe");
+  if (out_dtype != FP8_OUT_BF16 && out_dtype != FP8_OUT_F32)
+    return fail(FP8_ERR_VALUE, "fp8_scaled_mm: unknown out_dtype");
+  if (M < 0 || N < 0 || K < 0) return fail(FP8_ERR_VALUE, "fp8_scaled_mm: negative size");
+  if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+    return fail(FP8_ERR_VALUE, "fp8_scaled_mm: size too large");
+  if (K % 16 != 0) return fail(FP8_ERR_VALUE, "fp8_scaled_mm: K must be a multiple of 16");
+  if (N % 16 != 0) return fail(FP8_ERR_VALUE, "fp8_scaled_mm: N must be a multiple of 16");
+  const bool blockwise = recipe == FP8_MM_1x128_128x128 || recipe == FP8_MM_1x128_128x1;
+  if (blockwise && K % 128 != 0)
+    return fail(FP8_ERR_VALUE, "fp8_scaled_mm: blockwise recipes need K % 128 == 0");
+  if (M == 0 || N == 0) {
+    t_last_error.clear();
+    return FP8_OK;
+  }
+  if (out == nullptr) return fail(FP8_ERR_VALUE, "fp8_scaled_mm: null out");
+  if (K > 0 && (a == nullptr || b == nullptr || scale_a == nullptr || scale_b == nullptr))
+    return fail(FP8_ERR_VALUE, "fp8_scaled_mm: null operand or scale pointer");
+  if (!aligned(out, 16) || (a && !aligned(a, 16)) || (b && !aligned(b, 16)) ||
+      (bias_bf16 && !aligned(bias_bf16, 16)) || (scale_a && !aligned(scale_a, 16)) ||
+      (scale_b && !aligned(scale_b, 16)))
+    return fail(FP8_ERR_VALUE, "fp8_scaled_mm: pointers must be 16-byte aligned");
+  DeviceInfo* d = nullptr;
+  fp8_status s = device_info(&d);
+  if (s != FP8_OK) return s;
+  std::string err;
+  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status,
+                       d->num_sms, &err};
+  cudaError_t e = fp8sm::launch_scaled_mm(a, b, M, N, K, scale_a, scale_b,
+                                          (int)recipe, bias_bf16,
+                                          out_dtype == FP8_OUT_F32, out, ctx);
+  return finish_launch(e, err, "fp8_scaled_mm");
+}
+
+fp8_status fp8_grouped_scaled_mm(const void* a, const void* b_experts,
+                                 int64_t M_total, int64_t N, int64_t K,
+                                 int32_t E, const float* scale_a,
+                                 const float* scale_b, const int32_t* offs,
+                                 fp8_out_dtype out_dtype, void* out,
+                                 fp8_stream_t stream) {
+  if (out_dtype != FP8_OUT_BF16 && out_dtype != FP8_OUT_F32)
+    return fail(FP8_ERR_VALUE, "fp8_grouped_scaled_mm: unknown out_dtype");
+  if (offs == nullptr)
+    return fail(FP8_ERR_VALUE, "fp8_grouped_scaled_mm: offs is required");
+  if (M_total < 0 || N < 0 || K < 0 || E < 1 || E > 65535)
+    return fail(FP8_ERR_VALUE, "fp8_grouped_scaled_mm: bad size or expert count");
+  if (M_total >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+    return fail(FP8_ERR_VALUE, "fp8_grouped_scaled_mm: size too large");
+  if (K % 16 != 0 || N % 16 != 0)
+    return fail(FP8_ERR_VALUE, "fp8_grouped_scaled_mm: K and N must be multiples of 16");
+  if (M_total == 0 || N == 0) {
+    t_last_error.clear();
+    return FP8_OK;
+  }
+  if (out == nullptr || (K > 0 && (a == nullptr || b_experts == nullptr ||
+                                   scale_a == nullptr || scale_b == nullptr)))
+    return fail(FP8_ERR_VALUE, "fp8_grouped_scaled_mm: null pointer");
+  if (!aligned(out, 16) || (a && !aligned(a, 16)) || (b_experts && !aligned(b_experts, 16)) ||
+      (scale_a && !aligned(scale_a, 16)) || (scale_b && !aligned(scale_b, 16)) ||
+      !aligned(offs, 4))
+    return fail(FP8_ERR_VALUE, "fp8_grouped_scaled_mm: pointers must be 16-byte aligned");
+  DeviceInfo* d = nullptr;
+  fp8_status s = device_info(&d);
+  if (s != FP8_OK) return s;
+  std::string err;
+  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status,
+                       d->num_sms, &err};
+  cudaError_t e = fp8sm::launch_grouped_scaled_mm(a, b_experts, M_total, N, K, E,
+                                                  scale_a, scale_b, offs,
+                                                  out_dtype == FP8_OUT_F32, out, ctx);
+  return finish_launch(e, err, "fp8_grouped_scaled_mm");
+}
+
+fp8_status fp8_get_device_status(fp8_stream_t stream) {
+  DeviceInfo* d = nullptr;
+  fp8_status s = device_info(&d);
+  if (s != FP8_OK) return s;
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "fp8_get_device_status: sync");
+  uint32_t w[2] = {0, 0};
+  e = cudaMemcpy(w, d->status, sizeof(w), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "fp8_get_device_status: read");
+  const uint32_t zero[2] = {0, 0};
+  e = cudaMemcpy(d->status, zero, sizeof(zero), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "fp8_get_device_status: clear");
+  if (w[0] == 0) {
+    t_last_error.clear();
+    return FP8_OK;
+  }
+  return fail(static_cast<fp8_status>(w[0]),
+              "device status " + std::to_string(w[0]) + " recorded at site " +
+                  std::to_string(w[1]));
+}
+
+fp8_status fp8_debug_timeout_probe(uint32_t limit_us, fp8_stream_t stream) {
+  if (limit_us < 1 || limit_us > 2000000)
+    return fail(FP8_ERR_VALUE, "fp8_debug_timeout_probe: limit_us out of range");
+  DeviceInfo* d = nullptr;
+  fp8_status s = device_info(&d);
+  if (s != FP8_OK) return s;
+  std::string err;
+  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status,
+                       d->num_sms, &err};
+  return finish_launch(fp8sm::launch_timeout_probe(limit_us, ctx), err,
+                       "fp8_debug_timeout_probe");
+}
+
+}  // extern "C"

@@ -1,0 +1,43 @@
+// Internal launcher interface between the C-ABI layer (capi.cu) and the
+// kernel translation units.  Launchers assume arguments were validated.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+namespace fp8sm {
+
+struct LaunchCtx {
+  cudaStream_t stream;
+  uint32_t* status;   // device status word of the current device
+  int num_sms;
+  std::string* err;   // filled on failure
+};
+
+// Quantizers (quantize.cu).  recipe: 0 tensor, 1 row, 2 1x128, 3 128x128.
+cudaError_t launch_quantize(const void* x, int64_t rows, int64_t cols,
+                            int64_t ld, int recipe, void* q, float* scales,
+                            void* workspace, const LaunchCtx& ctx);
+
+// Dense scaled GEMM (gemm.cu).  recipe: 0 tensor, 1 row, 2 1x128_128x128,
+// 3 1x128_128x1.  out_f32: 0 -> bf16 output, 1 -> fp32 output.
+cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
+                             int64_t N, int64_t K, const float* sa,
+                             const float* sb, int recipe, const void* bias,
+                             int out_f32, void* out, const LaunchCtx& ctx);
+
+// Grouped rowwise scaled GEMM (gemm.cu).
+cudaError_t launch_grouped_scaled_mm(const void* a, const void* b,
+                                     int64_t M_total, int64_t N, int64_t K,
+                                     int32_t E, const float* sa,
+                                     const float* sb, const int32_t* offs,
+                                     int out_f32, void* out,
+                                     const LaunchCtx& ctx);
+
+// Failure-detection probe (gemm.cu): one CTA waits on a barrier nothing
+// completes, with the given limit.
+cudaError_t launch_timeout_probe(uint32_t limit_us, const LaunchCtx& ctx);
+
+}  // namespace fp8sm

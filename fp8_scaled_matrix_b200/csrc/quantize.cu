@@ -1,0 +1,368 @@
+// Dynamic e4m3 quantizers ("per-token scaling for fp8 linear", Highlights:
+// per-row amax -> scale, input pre-scaled, fp8 cast; the 1x128 / 128x128
+// groups of "Add _scaled_mm_v2 API" and "improve fp8 blockwise gemm perf").
+//
+// Per group G:  a = max(max|x|, 1e-12);  scale = a / 448;  inv = 448 / a;
+//               q = cvt.rn.satfinite.e4m3(x * inv)
+// Every step is one IEEE fp32 operation (no FMA contraction, no fast math),
+// so the codes and scales are bit-identical to any other implementation of
+// the same steps.
+//
+// HBM-bound: 2 bytes read + 1 byte written per element.  All kernels move
+// 16-byte vectors (8 bf16 in, 8 e4m3 out or 16 in / 16 out), reduce the
+// amax with warp shuffles, and keep the group in registers between the amax
+// and the cast so x is read from HBM once (the tensorwise recipe re-reads x
+// when it does not fit on chip).
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace fp8sm {
+namespace {
+
+constexpr float kE4M3Max = 448.0f;
+constexpr float kEps = 1e-12f;
+
+struct ScalePair {
+  float s;    // dequantization multiplier, stored
+  float inv;  // quantization multiplier
+};
+
+__device__ __forceinline__ ScalePair scales_from_amax(float amax) {
+  const float a = fmaxf(amax, kEps);
+  return {__fdiv_rn(a, kE4M3Max), __fdiv_rn(kE4M3Max, a)};
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) {
+  return __uint_as_float(w << 16);
+}
+__device__ __forceinline__ float bf16_hi(uint32_t w) {
+  return __uint_as_float(w & 0xFFFF0000u);
+}
+
+__device__ __forceinline__ float amax8(const uint4& v, float m) {
+  m = fmaxf(m, fabsf(bf16_lo(v.x)));
+  m = fmaxf(m, fabsf(bf16_hi(v.x)));
+  m = fmaxf(m, fabsf(bf16_lo(v.y)));
+  m = fmaxf(m, fabsf(bf16_hi(v.y)));
+  m = fmaxf(m, fabsf(bf16_lo(v.z)));
+  m = fmaxf(m, fabsf(bf16_hi(v.z)));
+  m = fmaxf(m, fabsf(bf16_lo(v.w)));
+  m = fmaxf(m, fabsf(bf16_hi(v.w)));
+  return m;
+}
+
+__device__ __forceinline__ uint32_t cast2(uint32_t w, float inv) {
+  const float2 y = make_float2(__fmul_rn(bf16_lo(w), inv),
+                               __fmul_rn(bf16_hi(w), inv));
+  return static_cast<uint32_t>(
+      __nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3));
+}
+
+// 8 bf16 -> 8 e4m3 bytes (little-endian order preserved).
+__device__ __forceinline__ uint2 cast8(const uint4& v, float inv) {
+  return make_uint2(cast2(v.x, inv) | (cast2(v.y, inv) << 16),
+                    cast2(v.z, inv) | (cast2(v.w, inv) << 16));
+}
+
+__device__ __forceinline__ float warp_max(float m) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  return m;
+}
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+  return __ldcs(p);
+}
+
+// ------------------------------------------------------------ rowwise
+// One warp per row; lane l holds vectors l, l+32, ... (VPT of them) in
+// registers, so each row is read once.  cols <= 256 * VPT.
+template <int VPT>
+__global__ void __launch_bounds__(256) quant_row_kernel(
+    const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+    uint8_t* __restrict__ q, float* __restrict__ scales) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int nvec = static_cast<int>(cols >> 3);
+  const uint4* xr = reinterpret_cast<const uint4*>(x + row * ld);
+  uint4 v[VPT];
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int idx = i * 32 + lane;
+    if (idx < nvec) {
+      v[i] = ld_stream(xr + idx);
+      m = amax8(v[i], m);
+    }
+  }
+  m = warp_max(m);
+  const ScalePair sp = scales_from_amax(m);
+  if (lane == 0) scales[row] = sp.s;
+  uint2* qr = reinterpret_cast<uint2*>(q + row * cols);
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int idx = i * 32 + lane;
+    if (idx < nvec) qr[idx] = cast8(v[i], sp.inv);
+  }
+}
+
+// Rows longer than 256*16 elements: amax pass, then a second read (served
+// from L2 for the row just read) for the cast.
+__global__ void __launch_bounds__(256) quant_row_long_kernel(
+    const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+    uint8_t* __restrict__ q, float* __restrict__ scales) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int64_t nvec = cols >> 3;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + row * ld);
+  float m = 0.0f;
+  for (int64_t base = 0; base < nvec; base += 128) {
+    uint4 v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t idx = base + i * 32 + lane;
+      if (idx < nvec) v[i] = __ldg(xr + idx);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t idx = base + i * 32 + lane;
+      if (idx < nvec) m = amax8(v[i], m);
+    }
+  }
+  m = warp_max(m);
+  const ScalePair sp = scales_from_amax(m);
+  if (lane == 0) scales[row] = sp.s;
+  uint2* qr = reinterpret_cast<uint2*>(q + row * cols);
+  for (int64_t idx = lane; idx < nvec; idx += 32)
+    qr[idx] = cast8(ld_stream(xr + idx), sp.inv);
+}
+
+// -------------------------------------------------------------- 1x128
+// A warp handles 4 rows x one 128-column block per task: lane = 8*g + j
+// covers row r0+g, columns kb*128 + 16j .. +16 (two 16-byte loads, one
+// 16-byte store).  Scales K-block-major: scales[kb*rows + r], so one warp
+// writes 4 consecutive floats.  Each warp runs kTasks tasks (the next K
+// blocks of the same rows) with all loads issued first.
+constexpr int k1x128Tasks = 4;
+
+__global__ void __launch_bounds__(256) quant_1x128_kernel(
+    const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+    uint8_t* __restrict__ q, float* __restrict__ scales) {
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 3;
+  const int j = lane & 7;
+  const int64_t KB = cols >> 7;
+  const int64_t kb_groups = (KB + k1x128Tasks - 1) / k1x128Tasks;
+  const int64_t warp = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int64_t quad = warp / kb_groups;
+  const int64_t kb0 = (warp % kb_groups) * k1x128Tasks;
+  const int64_t row = quad * 4 + g;
+  const bool row_ok = row < rows;
+  if (quad * 4 >= rows) return;
+  uint4 v[k1x128Tasks][2];
+#pragma unroll
+  for (int t = 0; t < k1x128Tasks; ++t) {
+    const int64_t kb = kb0 + t;
+    if (row_ok && kb < KB) {
+      const uint4* p = reinterpret_cast<const uint4*>(x + row * ld + kb * 128 + j * 16);
+      v[t][0] = ld_stream(p);
+      v[t][1] = ld_stream(p + 1);
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < k1x128Tasks; ++t) {
+    const int64_t kb = kb0 + t;
+    if (kb >= KB) break;  // uniform across the warp
+    float m = 0.0f;
+    if (row_ok) m = amax8(v[t][1], amax8(v[t][0], 0.0f));
+    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+    if (!row_ok) continue;
+    const ScalePair sp = scales_from_amax(m);
+    if (j == 0) scales[kb * rows + row] = sp.s;
+    const uint2 lo = cast8(v[t][0], sp.inv);
+    const uint2 hi = cast8(v[t][1], sp.inv);
+    *reinterpret_cast<uint4*>(q + row * cols + kb * 128 + j * 16) =
+        make_uint4(lo.x, lo.y, hi.x, hi.y);
+  }
+}
+
+// ------------------------------------------------------------ 128x128
+// One CTA (256 threads) per 128x128 tile: thread t covers row t/2 and
+// 64 columns (8 x 16-byte loads held in registers).  Ragged last row block:
+// rows past the end take no part in the amax and are not written.
+__global__ void __launch_bounds__(256) quant_128x128_kernel(
+    const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+    uint8_t* __restrict__ q, float* __restrict__ scales) {
+  __shared__ float warp_amax[8];
+  const int64_t RB = (rows + 127) >> 7;
+  const int64_t rb = blockIdx.x % RB;
+  const int64_t kb = blockIdx.x / RB;
+  const int t = threadIdx.x;
+  const int64_t row = rb * 128 + (t >> 1);
+  const int64_t col = kb * 128 + (t & 1) * 64;
+  const bool ok = row < rows;
+  uint4 v[8];
+  float m = 0.0f;
+  if (ok) {
+    const uint4* p = reinterpret_cast<const uint4*>(x + row * ld + col);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = ld_stream(p + i);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = amax8(v[i], m);
+  }
+  m = warp_max(m);
+  if ((t & 31) == 0) warp_amax[t >> 5] = m;
+  __syncthreads();
+  float tm = warp_amax[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) tm = fmaxf(tm, warp_amax[i]);
+  const ScalePair sp = scales_from_amax(tm);
+  if (t == 0) scales[kb * RB + rb] = sp.s;
+  if (!ok) return;
+  uint4* qp = reinterpret_cast<uint4*>(q + row * cols + col);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint2 lo = cast8(v[2 * i], sp.inv);
+    const uint2 hi = cast8(v[2 * i + 1], sp.inv);
+    qp[i] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+  }
+}
+
+// ------------------------------------------------------------- tensor
+// One amax for the whole matrix.  Cooperative launch (all CTAs resident):
+// phase 1 reduces each CTA's amax and folds it into ws[0] with an atomic
+// max on the fp32 bit pattern (non-negative floats order like unsigned
+// integers); a bounded grid barrier on ws[1]; phase 2 casts.  When every
+// thread holds at most one vector (small tensors) phase 2 reuses the
+// registers, otherwise it re-reads x (from L2 when it fits there).
+// ws[0..1] must be zero on entry (the launcher clears them).
+__global__ void __launch_bounds__(256) quant_tensor_kernel(
+    const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+    uint8_t* __restrict__ q, float* __restrict__ scale, uint32_t* ws,
+    uint32_t* status) {
+  __shared__ float warp_amax[8];
+  __shared__ uint32_t ok_flag;
+  const int64_t nvec = cols >> 3;
+  const bool single = (rows <= gridDim.x) && (nvec <= blockDim.x);
+  uint4 keep = make_uint4(0, 0, 0, 0);
+  float m = 0.0f;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + r * ld);
+    for (int64_t c = threadIdx.x; c < nvec; c += blockDim.x) {
+      const uint4 v = __ldg(xr + c);
+      keep = v;
+      m = amax8(v, m);
+    }
+  }
+  m = warp_max(m);
+  if ((threadIdx.x & 31) == 0) warp_amax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float bm = warp_amax[0];
+    for (int i = 1; i < (int)(blockDim.x >> 5); ++i) bm = fmaxf(bm, warp_amax[i]);
+    atomicMax(ws, __float_as_uint(bm));
+    __threadfence();
+    atomicAdd(ws + 1, 1u);
+    // bounded grid barrier
+    uint32_t ok = 1;
+    const uint64_t t0 = globaltimer_ns();
+    while (*reinterpret_cast<volatile uint32_t*>(ws + 1) < gridDim.x) {
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        record_status(status, FP8_DEV_TIMEOUT, SITE_GRID_BARRIER);
+        ok = 0;
+        break;
+      }
+    }
+    __threadfence();
+    ok_flag = ok;
+  }
+  __syncthreads();
+  if (!ok_flag) return;
+  const float amax = __uint_as_float(*reinterpret_cast<volatile uint32_t*>(ws));
+  const ScalePair sp = scales_from_amax(amax);
+  if (blockIdx.x == 0 && threadIdx.x == 0) scale[0] = sp.s;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + r * ld);
+    uint2* qr = reinterpret_cast<uint2*>(q + r * cols);
+    for (int64_t c = threadIdx.x; c < nvec; c += blockDim.x)
+      qr[c] = cast8(single ? keep : __ldg(xr + c), sp.inv);
+  }
+}
+
+int g_tensor_blocks_per_sm = -1;
+
+}  // namespace
+
+cudaError_t launch_quantize(const void* xv, int64_t rows, int64_t cols,
+                            int64_t ld, int recipe, void* qv, float* scales,
+                            void* workspace, const LaunchCtx& ctx) {
+  const uint16_t* x = static_cast<const uint16_t*>(xv);
+  uint8_t* q = static_cast<uint8_t*>(qv);
+  cudaStream_t st = ctx.stream;
+  if (recipe == 1) {  // rowwise
+    if (rows == 0) return cudaSuccess;
+    const unsigned grid = static_cast<unsigned>((rows + 7) / 8);
+    const int64_t nvec = cols / 8;
+    if (nvec <= 32)
+      quant_row_kernel<1><<<grid, 256, 0, st>>>(x, rows, cols, ld, q, scales);
+    else if (nvec <= 64)
+      quant_row_kernel<2><<<grid, 256, 0, st>>>(x, rows, cols, ld, q, scales);
+    else if (nvec <= 128)
+      quant_row_kernel<4><<<grid, 256, 0, st>>>(x, rows, cols, ld, q, scales);
+    else if (nvec <= 256)
+      quant_row_kernel<8><<<grid, 256, 0, st>>>(x, rows, cols, ld, q, scales);
+    else if (nvec <= 512)
+      quant_row_kernel<16><<<grid, 256, 0, st>>>(x, rows, cols, ld, q, scales);
+    else
+      quant_row_long_kernel<<<grid, 256, 0, st>>>(x, rows, cols, ld, q, scales);
+    return cudaGetLastError();
+  }
+  if (recipe == 2) {  // 1x128
+    if (rows == 0 || cols == 0) return cudaSuccess;
+    const int64_t KB = cols / 128;
+    const int64_t kb_groups = (KB + k1x128Tasks - 1) / k1x128Tasks;
+    const int64_t warps = ((rows + 3) / 4) * kb_groups;
+    const unsigned grid = static_cast<unsigned>((warps + 7) / 8);
+    quant_1x128_kernel<<<grid, 256, 0, st>>>(x, rows, cols, ld, q, scales);
+    return cudaGetLastError();
+  }
+  if (recipe == 3) {  // 128x128
+    if (rows == 0 || cols == 0) return cudaSuccess;
+    const int64_t tiles = ((rows + 127) / 128) * (cols / 128);
+    quant_128x128_kernel<<<static_cast<unsigned>(tiles), 256, 0, st>>>(
+        x, rows, cols, ld, q, scales);
+    return cudaGetLastError();
+  }
+  // tensorwise
+  uint32_t* ws = static_cast<uint32_t*>(workspace);
+  cudaError_t e = cudaMemsetAsync(ws, 0, 2 * sizeof(uint32_t), st);
+  if (e != cudaSuccess) return e;
+  if (g_tensor_blocks_per_sm < 0) {
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quant_tensor_kernel,
+                                                      256, 0);
+    if (e != cudaSuccess) return e;
+    g_tensor_blocks_per_sm = n;
+  }
+  int64_t max_grid = static_cast<int64_t>(ctx.num_sms) *
+                     (g_tensor_blocks_per_sm > 0 ? g_tensor_blocks_per_sm : 1);
+  int64_t grid = rows < max_grid ? rows : max_grid;
+  if (grid < 1) grid = 1;
+  unsigned g = static_cast<unsigned>(grid);
+  uint32_t* status = ctx.status;
+  void* args[] = {(void*)&x, (void*)&rows, (void*)&cols, (void*)&ld,
+                  (void*)&q, (void*)&scales, (void*)&ws, (void*)&status};
+  return cudaLaunchCooperativeKernel((const void*)quant_tensor_kernel, dim3(g),
+                                     dim3(256), args, 0, st);
+}
+
+}  // namespace fp8sm

@@ -1,0 +1,225 @@
+"""Thin Python binding over the C ABI in include/fp8sm.h (libfp8sm.so).
+
+Argument marshalling only: torch tensors supply device memory and the
+current CUDA stream; every step of the computation runs in the library's
+kernels.  There is no fallback: if the library cannot be loaded, or a call
+returns an error, an exception is raised.
+
+Names match the C entry points (fp8_quantize, fp8_scaled_mm,
+fp8_grouped_scaled_mm, fp8_get_device_status, fp8_last_error, ...).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfp8sm.so")
+
+# enums (include/fp8sm.h)
+FP8_OK, FP8_ERR_VALUE, FP8_ERR_UNSUPPORTED, FP8_ERR_CUDA, FP8_ERR_TIMEOUT = 0, 1, 2, 3, 4
+FP8_SCALE_TENSOR, FP8_SCALE_ROW, FP8_SCALE_BLOCK_1x128, FP8_SCALE_BLOCK_128x128 = 0, 1, 2, 3
+FP8_MM_TENSOR_TENSOR, FP8_MM_ROW_ROW, FP8_MM_1x128_128x128, FP8_MM_1x128_128x1 = 0, 1, 2, 3
+FP8_OUT_BF16, FP8_OUT_F32 = 0, 1
+
+QUANT_RECIPES = {"tensor": FP8_SCALE_TENSOR, "row": FP8_SCALE_ROW,
+                 "1x128": FP8_SCALE_BLOCK_1x128, "128x128": FP8_SCALE_BLOCK_128x128}
+MM_RECIPES = {"tensor": FP8_MM_TENSOR_TENSOR, "row": FP8_MM_ROW_ROW,
+              "1x128_128x128": FP8_MM_1x128_128x128, "1x128_128x1": FP8_MM_1x128_128x1}
+
+EXPORTED = ["fp8_version", "fp8_last_error", "fp8_quantize_workspace_bytes",
+            "fp8_quantize", "fp8_scaled_mm", "fp8_grouped_scaled_mm",
+            "fp8_get_device_status", "fp8_debug_timeout_probe"]
+
+
+class Fp8Error(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"[status {status}] {msg}")
+        self.status = status
+
+
+class Fp8ValueError(Fp8Error, ValueError):
+    pass
+
+
+class Fp8Unsupported(Fp8Error, NotImplementedError):
+    pass
+
+
+class Fp8Timeout(Fp8Error):
+    pass
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libfp8sm.so (raises if it is missing; there is no other path)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with `python -m fp8_scaled_matrix_b200.build` "
+            "(there is no fallback implementation)")
+    L = ctypes.CDLL(path)
+    P, I64, I32, U32, SZ = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32,
+                           ctypes.c_uint32, ctypes.c_size_t)
+    E = ctypes.c_int
+    L.fp8_version.restype = ctypes.c_int
+    L.fp8_version.argtypes = []
+    L.fp8_last_error.restype = ctypes.c_char_p
+    L.fp8_last_error.argtypes = []
+    L.fp8_quantize_workspace_bytes.restype = SZ
+    L.fp8_quantize_workspace_bytes.argtypes = [E, I64, I64]
+    L.fp8_quantize.restype = E
+    L.fp8_quantize.argtypes = [P, I64, I64, I64, E, P, P, P, SZ, P]
+    L.fp8_scaled_mm.restype = E
+    L.fp8_scaled_mm.argtypes = [P, P, I64, I64, I64, P, P, E, P, E, P, P]
+    L.fp8_grouped_scaled_mm.restype = E
+    L.fp8_grouped_scaled_mm.argtypes = [P, P, I64, I64, I64, I32, P, P, P, E, P, P]
+    L.fp8_get_device_status.restype = E
+    L.fp8_get_device_status.argtypes = [P]
+    L.fp8_debug_timeout_probe.restype = E
+    L.fp8_debug_timeout_probe.argtypes = [U32, P]
+    _lib = L
+    return L
+
+
+def _check(status: int):
+    if status == FP8_OK:
+        return
+    msg = load_library().fp8_last_error().decode(errors="replace")
+    cls = {FP8_ERR_VALUE: Fp8ValueError, FP8_ERR_UNSUPPORTED: Fp8Unsupported,
+           FP8_ERR_TIMEOUT: Fp8Timeout}.get(status, Fp8Error)
+    raise cls(status, msg)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("tensors must live in CUDA device memory")
+
+
+def fp8_version() -> int:
+    return load_library().fp8_version()
+
+
+def fp8_last_error() -> str:
+    return load_library().fp8_last_error().decode(errors="replace")
+
+
+def scale_count(rows: int, cols: int, recipe: int) -> int:
+    if recipe == FP8_SCALE_TENSOR:
+        return 1
+    if recipe == FP8_SCALE_ROW:
+        return rows
+    if recipe == FP8_SCALE_BLOCK_1x128:
+        return (cols // 128) * rows
+    return (cols // 128) * ((rows + 127) // 128)
+
+
+def fp8_quantize_workspace_bytes(recipe: int, rows: int, cols: int) -> int:
+    return load_library().fp8_quantize_workspace_bytes(recipe, rows, cols)
+
+
+def fp8_quantize(x: torch.Tensor, recipe: int, out: Optional[torch.Tensor] = None,
+                 scales: Optional[torch.Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None,
+                 stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Quantize a 2-D bf16 CUDA tensor (row stride x.stride(0)).
+
+    Returns (codes uint8 (rows, cols), scales float32).  `out`, `scales` and
+    `workspace` may be passed to avoid allocations."""
+    L = load_library()
+    _need_cuda(x)
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D bf16 tensor with unit column stride")
+    rows, cols = x.shape
+    if out is None:
+        out = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(max(scale_count(rows, cols, recipe), 1),
+                             dtype=torch.float32, device=x.device)
+    ws_bytes = L.fp8_quantize_workspace_bytes(recipe, rows, cols)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=x.device)
+    _check(L.fp8_quantize(_ptr(x), rows, cols, x.stride(0), recipe, _ptr(out),
+                          _ptr(scales), _ptr(workspace),
+                          0 if workspace is None else workspace.numel() * workspace.element_size(),
+                          _stream(stream)))
+    return out, scales
+
+
+def fp8_scaled_mm(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor,
+                  scale_b: torch.Tensor, recipe: int,
+                  bias: Optional[torch.Tensor] = None, out_dtype=torch.bfloat16,
+                  out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """out = (a * scale_a) @ (b * scale_b)^T (+ bias); a (M,K), b (N,K) uint8 e4m3 codes."""
+    L = load_library()
+    _need_cuda(a, b, scale_a, scale_b, bias)
+    M, K = a.shape
+    N = b.shape[0]
+    if b.shape[1] != K:
+        raise ValueError("a and b must share K")
+    for t in (a, b):
+        if t.dtype not in (torch.uint8, torch.float8_e4m3fn) or not t.is_contiguous():
+            raise ValueError("a and b must be contiguous e4m3 (uint8 codes)")
+    if bias is not None and (bias.dtype != torch.bfloat16 or not bias.is_contiguous()):
+        raise ValueError("bias must be a contiguous bf16 tensor")
+    od = FP8_OUT_F32 if out_dtype == torch.float32 else FP8_OUT_BF16
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=a.device)
+    _check(L.fp8_scaled_mm(_ptr(a), _ptr(b), M, N, K, _ptr(scale_a), _ptr(scale_b),
+                           recipe, _ptr(bias), od, _ptr(out), _stream(stream)))
+    return out
+
+
+def fp8_grouped_scaled_mm(a: torch.Tensor, b_experts: torch.Tensor,
+                          scale_a: torch.Tensor, scale_b: torch.Tensor,
+                          offs: torch.Tensor, out_dtype=torch.bfloat16,
+                          out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Grouped rowwise GEMM: rows [offs[g-1], offs[g]) of a times expert g."""
+    L = load_library()
+    _need_cuda(a, b_experts, scale_a, scale_b, offs)
+    if offs is None:
+        raise ValueError("offs is required")
+    if offs.dtype != torch.int32:
+        raise ValueError("offs must be int32")
+    M, K = a.shape
+    E, N, K2 = b_experts.shape
+    if K2 != K or offs.numel() != E:
+        raise ValueError("shape mismatch")
+    od = FP8_OUT_F32 if out_dtype == torch.float32 else FP8_OUT_BF16
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=a.device)
+    _check(L.fp8_grouped_scaled_mm(_ptr(a), _ptr(b_experts), M, N, K, E, _ptr(scale_a),
+                                   _ptr(scale_b), _ptr(offs), od, _ptr(out),
+                                   _stream(stream)))
+    return out
+
+
+def fp8_get_device_status(stream=None) -> int:
+    """Synchronize and return (and clear) the device status word."""
+    return load_library().fp8_get_device_status(_stream(stream))
+
+
+def check_device_status(stream=None):
+    _check(fp8_get_device_status(stream))
+
+
+def fp8_debug_timeout_probe(limit_us: int, stream=None):
+    _check(load_library().fp8_debug_timeout_probe(limit_us, _stream(stream)))

@@ -1,0 +1,209 @@
+/*
+ * fp8sm — FP8 (e4m3) scaled matrix multiply and dynamic quantizer for
+ * NVIDIA B200 (sm_100a).  C ABI.
+ *
+ *   out = (A_fp8 * s_A) @ (B_fp8 * s_B)^T (+ bias)
+ *
+ * Sources for the operations (public pull-request pages):
+ *   [P1] "Fix: Handle LowLevelZeroPlugin with use_fp8=True" (ColossalAI PR
+ *        #6419), Solution: the FP8 linear forward calls a scaled matmul
+ *        whose result equals dequantize-then-matmul plus bias; scales are
+ *        dequantization multipliers; tensorwise scales presented as (1, 1).
+ *   [P2] "Add _grouped_mm dispatch handler to Float8Tensor" (torchao PR
+ *        #4390): MoE expert weights (E, N, K) used as weight.transpose(-2,-1);
+ *        rowwise activation scales and (E, N) weight scales; offs required;
+ *        an unsupported granularity must raise, never fall back silently.
+ *   [P3] "per-token scaling for fp8 linear" (DiffSynth-Engine PR #160),
+ *        Highlights: per-row amax -> scale, input pre-scaled (epsilon guard)
+ *        and cast to fp8 before one scaled matmul.
+ *   [P4] "Add _scaled_mm_v2 API" (PyTorch PR #164141): explicit (declared,
+ *        not inferred) scaling recipes per operand; A and B fp8 with fp32
+ *        scales; Blockwise_1x128 (A) x Blockwise_128x128 (B); argument errors
+ *        are ValueError-class, unimplemented combinations NotImplementedError-
+ *        class, everything else RuntimeError-class.
+ *   [P5] "improve fp8 blockwise gemm perf" (torchao PR #2784): the
+ *        1x128_128x128 GEMM (output = input @ weight.t()) and the
+ *        1x128_128x1 GEMM (grad_weight = grad_output_t @ input).
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE memory owned by the caller; the library
+ *     never allocates, frees or keeps them.  Calls are asynchronous on the
+ *     given stream and return once the work is enqueued.
+ *   - Matrices are row-major.  A is (M, K) with K contiguous; B is stored
+ *     (N, K) with K contiguous (i.e. the GEMM computes input @ weight.t()).
+ *     FP8 tensors are e4m3 bytes; bf16 tensors are raw 16-bit patterns.
+ *   - Argument errors (null pointers, bad sizes, misaligned pointers, a scale
+ *     layout that does not fit the recipe) return FP8_ERR_VALUE before
+ *     anything is launched.  A recipe / dtype combination that is not
+ *     implemented returns FP8_ERR_UNSUPPORTED; there is no fallback path of
+ *     any kind.  A failed CUDA launch returns FP8_ERR_CUDA.  fp8_last_error()
+ *     then describes the problem (per host thread).
+ *   - Errors found on the device (a malformed offs array, a pipeline wait
+ *     that ran past its time limit) are recorded in a per-device status word
+ *     and read back with fp8_get_device_status().
+ */
+#ifndef FP8SM_H
+#define FP8SM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FP8SM_API __attribute__((visibility("default")))
+#else
+#define FP8SM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* fp8_stream_t;
+
+/* Status codes: [P4] error classes (ValueError / NotImplementedError /
+ * RuntimeError) mapped to codes; TIMEOUT is a device wait that gave up. */
+typedef enum {
+  FP8_OK = 0,
+  FP8_ERR_VALUE = 1,        /* invalid argument (user error)                */
+  FP8_ERR_UNSUPPORTED = 2,  /* valid request, not implemented: no fallback  */
+  FP8_ERR_CUDA = 3,         /* CUDA runtime / launch failure                */
+  FP8_ERR_TIMEOUT = 4       /* a device-side wait ran past its limit        */
+} fp8_status;
+
+/* Quantization group shapes ([P3] per-row, [P4]/[P5] 1x128 and 128x128,
+ * [P1] per-tensor). */
+typedef enum {
+  FP8_SCALE_TENSOR = 0,         /* one scale for the whole matrix           */
+  FP8_SCALE_ROW = 1,            /* one scale per row                        */
+  FP8_SCALE_BLOCK_1x128 = 2,    /* one scale per row per 128 columns        */
+  FP8_SCALE_BLOCK_128x128 = 3   /* one scale per 128x128 tile               */
+} fp8_quant_recipe;
+
+/* GEMM scaling recipes, named A-recipe_B-recipe as in [P4]; B orientation as
+ * in [P5] (the B operand is stored (N, K), so "128x1" means one scale per
+ * output column n per 128-wide K block). */
+typedef enum {
+  FP8_MM_TENSOR_TENSOR = 0,     /* s_A[0] * s_B[0]                           */
+  FP8_MM_ROW_ROW = 1,           /* s_A[m] * s_B[n]                           */
+  FP8_MM_1x128_128x128 = 2,     /* s_A[kb*M + m] * s_B[kb*ceil(N/128) + n/128] */
+  FP8_MM_1x128_128x1 = 3        /* s_A[kb*M + m] * s_B[kb*N + n]             */
+} fp8_mm_recipe;
+
+typedef enum {
+  FP8_OUT_BF16 = 0,   /* round to nearest even from the fp32 result        */
+  FP8_OUT_F32 = 1     /* the fp32 result before any bf16 cast              */
+} fp8_out_dtype;
+
+/*
+ * Dynamic quantization ([P3] Highlights; scale = max(amax, 1e-12)/448).
+ *
+ * For every group G of x (shape set by `recipe`):
+ *   amax = max |x| over G;  a = max(amax, 1e-12f)
+ *   scale[G] = a / 448 (fp32, IEEE division)   -- the dequantization multiplier
+ *   q = e4m3_rn_satfinite(x * (448 / a))        -- one fp32 multiply, then the
+ *                                                  RNE cast saturating at +-448
+ *
+ *   x_bf16     (rows, cols) bf16, row stride ld_x elements; 16-byte aligned,
+ *              ld_x % 8 == 0, cols % 8 == 0.
+ *   out_fp8    (rows, cols) e4m3, row stride cols; 16-byte aligned.
+ *   out_scales fp32, 4-byte aligned:
+ *                TENSOR:   1 value
+ *                ROW:      rows values, scale[r]
+ *                1x128:    (cols/128) * rows values, scale[kb*rows + r]
+ *                          (K-block-major: one block's scales for consecutive
+ *                          rows are contiguous)
+ *                128x128:  (cols/128) * ceil(rows/128) values,
+ *                          scale[kb*ceil(rows/128) + r/128]
+ *              Blockwise recipes need cols % 128 == 0 (rows may be ragged).
+ *   workspace  device scratch of fp8_quantize_workspace_bytes() bytes (may be
+ *              NULL when that is 0).  TENSOR needs 16 bytes; the library
+ *              clears it on the stream before use.  Calls that share one
+ *              workspace must not overlap on the GPU.
+ * Empty inputs are valid: rows == 0 writes nothing; cols == 0 writes the
+ * epsilon scale for each (row) group.
+ */
+FP8SM_API size_t fp8_quantize_workspace_bytes(fp8_quant_recipe recipe, int64_t rows,
+                                    int64_t cols);
+
+FP8SM_API fp8_status fp8_quantize(const void* x_bf16, int64_t rows, int64_t cols,
+                        int64_t ld_x, fp8_quant_recipe recipe, void* out_fp8,
+                        float* out_scales, void* workspace, size_t ws_bytes,
+                        fp8_stream_t stream);
+
+/*
+ * Scaled GEMM ([P1] forward; [P4] recipes; [P5] blockwise recipes):
+ *   out[m, n] = sum_k (a[m,k] * sA) * (b[n,k] * sB)  (+ bias[n])
+ * with the scales picked per recipe (see fp8_mm_recipe).  Products are
+ * accumulated in fp32 on the tensor cores; the blockwise recipes accumulate
+ * each 128-wide K block separately and apply its scales on the CUDA cores
+ * before summing in fp32.
+ *
+ *   a        (M, K) e4m3, K contiguous, 16-byte aligned.
+ *   b        (N, K) e4m3, K contiguous, 16-byte aligned.
+ *   scale_a, scale_b  fp32 scale arrays in the recipe's layout; 16-byte aligned.
+ *   bias_bf16 (N) bf16 or NULL; 16-byte aligned.
+ *   out      (M, N) row-major, bf16 or fp32 per `out_dtype`; 16-byte aligned.
+ * Requirements: K % 16 == 0 (K % 128 == 0 for the blockwise recipes),
+ * N % 16 == 0.  M is arbitrary.  M == 0 or N == 0 is a no-op; K == 0 writes
+ * bias (or zeros).
+ */
+FP8SM_API fp8_status fp8_scaled_mm(const void* a, const void* b, int64_t M, int64_t N,
+                         int64_t K, const float* scale_a, const float* scale_b,
+                         fp8_mm_recipe recipe, const void* bias_bf16,
+                         fp8_out_dtype out_dtype, void* out,
+                         fp8_stream_t stream);
+
+/*
+ * Grouped (MoE) scaled GEMM, rowwise recipe only ([P2] Design, RowWise path;
+ * other weight granularities return FP8_ERR_UNSUPPORTED as [P2]'s review
+ * requires):
+ *   for g in 0..E-1, rows m in [offs[g-1], offs[g])  (offs[-1] = 0):
+ *     out[m, n] = sum_k (a[m,k] * scale_a[m]) * (b_experts[g,n,k] * scale_b[g*N + n])
+ *
+ *   a          (M_total, K) e4m3, 16-byte aligned.
+ *   b_experts  (E, N, K) e4m3, 16-byte aligned (the experts' weights as
+ *              stored, used as weight.transpose(-2, -1)).
+ *   scale_a    (M_total) fp32 per-token scales.
+ *   scale_b    (E, N) fp32 per-expert per-output-channel scales.
+ *   offs       DEVICE (E) int32 cumulative END offsets: non-decreasing,
+ *              offs[E-1] == M_total; empty groups allowed.  It is read on the
+ *              device; if it is malformed nothing is written and the device
+ *              status becomes FP8_ERR_VALUE.
+ *   out        (M_total, N) row-major, bf16 or fp32.
+ * Requirements: K % 16 == 0, N % 16 == 0, 1 <= E <= 65535.
+ */
+FP8SM_API fp8_status fp8_grouped_scaled_mm(const void* a, const void* b_experts,
+                                 int64_t M_total, int64_t N, int64_t K,
+                                 int32_t E, const float* scale_a,
+                                 const float* scale_b, const int32_t* offs,
+                                 fp8_out_dtype out_dtype, void* out,
+                                 fp8_stream_t stream);
+
+/*
+ * Synchronizes `stream`, then returns and clears the current device's status
+ * word: FP8_OK, FP8_ERR_VALUE (malformed offs), FP8_ERR_TIMEOUT (a pipeline
+ * wait gave up; the kernel released its resources and returned), or
+ * FP8_ERR_CUDA if the synchronization itself failed.
+ */
+FP8SM_API fp8_status fp8_get_device_status(fp8_stream_t stream);
+
+/* Message for the last error returned on this host thread ("" if none). */
+FP8SM_API const char* fp8_last_error(void);
+
+/*
+ * Test hook for the failure-detection path: launches one CTA that waits on a
+ * pipeline barrier nothing will ever complete, with a wait limit of
+ * `limit_us` microseconds (1..2000000).  The wait gives up, the kernel
+ * records FP8_ERR_TIMEOUT in the status word and returns normally, so the
+ * CUDA context stays usable.  No counterpart on the pages.
+ */
+FP8SM_API fp8_status fp8_debug_timeout_probe(uint32_t limit_us, fp8_stream_t stream);
+
+/* Library version (major*10000 + minor*100 + patch). */
+FP8SM_API int fp8_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FP8SM_H */

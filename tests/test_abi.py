@@ -1,0 +1,127 @@
+"""The C-ABI library loads on a machine without a GPU, exports every symbol
+include/fp8sm.h declares, and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from fp8_scaled_matrix_b200 import fp8sm
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_symbols():
+    src = open(os.path.join(ROOT, "include", "fp8sm.h")).read()
+    return re.findall(r"FP8SM_API\s+[\w\s\*]+?\b(fp8_\w+)\s*\(", src)
+
+
+def test_header_declares_expected_entry_points():
+    syms = set(header_symbols())
+    assert {"fp8_quantize", "fp8_scaled_mm", "fp8_grouped_scaled_mm",
+            "fp8_get_device_status", "fp8_last_error"} <= syms
+
+
+def test_library_exports_every_header_symbol(lib):
+    for name in header_symbols():
+        assert hasattr(lib, name), name
+    assert set(fp8sm.EXPORTED) == set(header_symbols())
+    assert lib.fp8_version() == 100
+
+
+def test_workspace_sizes(lib):
+    assert lib.fp8_quantize_workspace_bytes(fp8sm.FP8_SCALE_TENSOR, 256, 256) == 16
+    for r in (fp8sm.FP8_SCALE_ROW, fp8sm.FP8_SCALE_BLOCK_1x128, fp8sm.FP8_SCALE_BLOCK_128x128):
+        assert lib.fp8_quantize_workspace_bytes(r, 256, 256) == 0
+
+
+P = ctypes.c_void_p
+FAKE = P(1 << 20)  # never dereferenced: every call below fails validation first
+
+
+@pytest.mark.parametrize("args,frag", [
+    ((FAKE, 4, 100, 100, fp8sm.FP8_SCALE_ROW), "multiples of 8"),
+    ((FAKE, 4, 200, 200, fp8sm.FP8_SCALE_BLOCK_1x128), "cols % 128"),
+    ((FAKE, 4, 128, 64, fp8sm.FP8_SCALE_ROW), "ld_x < cols"),
+    ((FAKE, -1, 128, 128, fp8sm.FP8_SCALE_ROW), "negative"),
+    ((FAKE, 4, 128, 128, 7), "unknown recipe"),
+    ((None, 4, 128, 128, fp8sm.FP8_SCALE_ROW), "null"),
+])
+def test_quantize_rejects_bad_arguments(lib, args, frag):
+    x, rows, cols, ld, recipe = args
+    st = lib.fp8_quantize(x, rows, cols, ld, recipe, FAKE, FAKE, None, 0, None)
+    assert st == fp8sm.FP8_ERR_VALUE
+    assert frag in lib.fp8_last_error().decode()
+
+
+def test_quantize_tensorwise_needs_workspace(lib):
+    st = lib.fp8_quantize(FAKE, 4, 128, 128, fp8sm.FP8_SCALE_TENSOR, FAKE, FAKE, None, 0, None)
+    assert st == fp8sm.FP8_ERR_VALUE
+    assert "workspace" in lib.fp8_last_error().decode()
+
+
+def test_quantize_misaligned_pointer(lib):
+    st = lib.fp8_quantize(P((1 << 20) + 2), 4, 128, 128, fp8sm.FP8_SCALE_ROW, FAKE, FAKE,
+                          None, 0, None)
+    assert st == fp8sm.FP8_ERR_VALUE and "aligned" in lib.fp8_last_error().decode()
+
+
+@pytest.mark.parametrize("M,N,K,recipe,frag", [
+    (128, 100, 128, fp8sm.FP8_MM_ROW_ROW, "N must be a multiple of 16"),
+    (128, 128, 100, fp8sm.FP8_MM_ROW_ROW, "K must be a multiple of 16"),
+    (128, 128, 144, fp8sm.FP8_MM_1x128_128x128, "K % 128"),
+    (128, 128, 144, fp8sm.FP8_MM_1x128_128x1, "K % 128"),
+    (-1, 128, 128, fp8sm.FP8_MM_ROW_ROW, "negative"),
+    (128, 128, 128, 9, "unknown recipe"),
+])
+def test_scaled_mm_rejects_bad_arguments(lib, M, N, K, recipe, frag):
+    st = lib.fp8_scaled_mm(FAKE, FAKE, M, N, K, FAKE, FAKE, recipe, None,
+                           fp8sm.FP8_OUT_BF16, FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE
+    assert frag in lib.fp8_last_error().decode()
+
+
+def test_scaled_mm_null_and_alignment(lib):
+    st = lib.fp8_scaled_mm(None, FAKE, 128, 128, 128, FAKE, FAKE, fp8sm.FP8_MM_ROW_ROW,
+                           None, fp8sm.FP8_OUT_BF16, FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE
+    st = lib.fp8_scaled_mm(FAKE, P((1 << 20) + 8), 128, 128, 128, FAKE, FAKE,
+                           fp8sm.FP8_MM_ROW_ROW, None, fp8sm.FP8_OUT_BF16, FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE and "aligned" in lib.fp8_last_error().decode()
+    st = lib.fp8_scaled_mm(FAKE, FAKE, 128, 128, 128, FAKE, FAKE, fp8sm.FP8_MM_ROW_ROW,
+                           None, 5, FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE and "out_dtype" in lib.fp8_last_error().decode()
+
+
+def test_empty_gemm_is_a_noop_without_cuda(lib):
+    # M == 0 or N == 0 returns before any CUDA call
+    assert lib.fp8_scaled_mm(None, None, 0, 128, 128, None, None, fp8sm.FP8_MM_ROW_ROW,
+                             None, fp8sm.FP8_OUT_BF16, None, None) == fp8sm.FP8_OK
+    assert lib.fp8_scaled_mm(None, None, 64, 0, 128, None, None, fp8sm.FP8_MM_ROW_ROW,
+                             None, fp8sm.FP8_OUT_BF16, None, None) == fp8sm.FP8_OK
+
+
+def test_grouped_requires_offs(lib):
+    st = lib.fp8_grouped_scaled_mm(FAKE, FAKE, 64, 128, 128, 4, FAKE, FAKE, None,
+                                   fp8sm.FP8_OUT_BF16, FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE and "offs is required" in lib.fp8_last_error().decode()
+    st = lib.fp8_grouped_scaled_mm(FAKE, FAKE, 64, 128, 128, 0, FAKE, FAKE, FAKE,
+                                   fp8sm.FP8_OUT_BF16, FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE
+
+
+def test_python_binding_rejects_host_tensors():
+    x = torch.zeros(4, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fp8sm.fp8_quantize(x, fp8sm.FP8_SCALE_ROW)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError, match="no fallback"):
+        saved = fp8sm._lib
+        fp8sm._lib = None
+        try:
+            fp8sm.load_library(str(tmp_path / "nope.so"))
+        finally:
+            fp8sm._lib = saved
