@@ -157,7 +157,9 @@ def fp8_quantize(x: torch.Tensor, recipe: int, out: Optional[torch.Tensor] = Non
     ws_bytes = L.fp8_quantize_workspace_bytes(recipe, rows, cols)
     if ws_bytes and workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=x.device)
-    _check(L.fp8_quantize(_ptr(x), rows, cols, x.stride(0), recipe, _ptr(out),
+    # the row stride only matters when there is more than one non-empty row
+    ld = x.stride(0) if (rows > 1 and cols > 0) else cols
+    _check(L.fp8_quantize(_ptr(x), rows, cols, ld, recipe, _ptr(out),
                           _ptr(scales), _ptr(workspace),
                           0 if workspace is None else workspace.numel() * workspace.element_size(),
                           _stream(stream)))
