@@ -150,6 +150,34 @@ fp8_status fp8_quantize(const void* x_bf16, int64_t rows, int64_t cols,
   return finish_launch(e, err, "fp8_quantize");
 }
 
+fp8_status fp8_quantize_noalloc(const void* x_bf16, int64_t rows, int64_t cols,
+                                int64_t ld_x, fp8_quant_recipe recipe,
+                                void* out_fp8, float* out_scales,
+                                fp8_stream_t stream) {
+  if (recipe < FP8_SCALE_TENSOR || recipe > FP8_SCALE_BLOCK_128x128)
+    return fail(FP8_ERR_VALUE, "fp8_quantize_noalloc: unknown recipe");
+  const size_t need = fp8_quantize_workspace_bytes(recipe, rows, cols);
+  const size_t have = fp8sm::noalloc_scratch_bytes();
+  if (need > have)
+    return fail(FP8_ERR_VALUE,
+                "fp8_quantize_noalloc: this call needs " + std::to_string(need) +
+                    " bytes of scratch, more than the library's fixed " +
+                    std::to_string(have) + "-byte scratch");
+  void* scratch = nullptr;
+  if (need > 0) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "fp8_quantize_noalloc: cudaGetDevice");
+    e = fp8sm::noalloc_scratch_ptr(dev, &scratch);
+    if (e != cudaSuccess)
+      return cuda_fail(e, "fp8_quantize_noalloc: cudaGetSymbolAddress(scratch)");
+  }
+  // Same validation and kernels as fp8_quantize, with the library's own
+  // scratch standing in for the caller's workspace.
+  return fp8_quantize(x_bf16, rows, cols, ld_x, recipe, out_fp8, out_scales,
+                      scratch, need > 0 ? have : 0, stream);
+}
+
 fp8_status fp8_scaled_mm(const void* a, const void* b, int64_t M, int64_t N,
                          int64_t K, const float* scale_a, const float* scale_b,
                          fp8_mm_recipe recipe, const void* bias_bf16,

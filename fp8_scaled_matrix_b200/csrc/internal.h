@@ -21,6 +21,12 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t cols,
                             int64_t ld, int recipe, void* q, float* scales,
                             void* workspace, const LaunchCtx& ctx);
 
+// Library-owned scratch for the no-allocation quantize entry point
+// (quantize.cu): its size, and its device address on `device` (looked up
+// once per device; the device must be current).
+size_t noalloc_scratch_bytes();
+cudaError_t noalloc_scratch_ptr(int device, void** out);
+
 // Dense scaled GEMM (gemm.cu).  recipe: 0 tensor, 1 row, 2 1x128_128x128,
 // 3 1x128_128x1.  out_f32: 0 -> bf16 output, 1 -> fp32 output.
 cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,

@@ -17,6 +17,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -300,7 +302,35 @@ __global__ void __launch_bounds__(256) quant_tensor_kernel(
 
 int g_tensor_blocks_per_sm = -1;
 
+// Scratch for fp8_quantize_noalloc: a fixed array in device memory that the
+// library owns.  Every GPU that loads the library holds one copy until the
+// process exits.  All calls share it; a call leaves its contents behind, so
+// the launcher clears what must start at zero before each use, and two
+// calls that run at the same time on the GPU (different streams) race on it.
+constexpr size_t kNoAllocScratchBytes = 256;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch for each device, taken once with that
+// device current (in host code the array's name is only a stand-in).
+void* g_noalloc_ptr[64] = {nullptr};
+std::mutex g_noalloc_mu;
+
 }  // namespace
+
+size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+cudaError_t noalloc_scratch_ptr(int device, void** out) {
+  if (device < 0 || device >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[device] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[device] = p;
+  }
+  *out = g_noalloc_ptr[device];
+  return cudaSuccess;
+}
 
 cudaError_t launch_quantize(const void* xv, int64_t rows, int64_t cols,
                             int64_t ld, int recipe, void* qv, float* scales,

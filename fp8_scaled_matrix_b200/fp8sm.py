@@ -32,7 +32,8 @@ MM_RECIPES = {"tensor": FP8_MM_TENSOR_TENSOR, "row": FP8_MM_ROW_ROW,
 
 EXPORTED = ["fp8_version", "fp8_last_error", "fp8_quantize_workspace_bytes",
             "fp8_quantize", "fp8_scaled_mm", "fp8_grouped_scaled_mm",
-            "fp8_get_device_status", "fp8_debug_timeout_probe"]
+            "fp8_get_device_status", "fp8_debug_timeout_probe",
+            "fp8_quantize_noalloc"]
 
 
 class Fp8Error(RuntimeError):
@@ -85,6 +86,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fp8_get_device_status.argtypes = [P]
     L.fp8_debug_timeout_probe.restype = E
     L.fp8_debug_timeout_probe.argtypes = [U32, P]
+    L.fp8_quantize_noalloc.restype = E
+    L.fp8_quantize_noalloc.argtypes = [P, I64, I64, I64, E, P, P, P]
     _lib = L
     return L
 
@@ -163,6 +166,25 @@ def fp8_quantize(x: torch.Tensor, recipe: int, out: Optional[torch.Tensor] = Non
                           _ptr(scales), _ptr(workspace),
                           0 if workspace is None else workspace.numel() * workspace.element_size(),
                           _stream(stream)))
+    return out, scales
+
+
+def fp8_quantize_noalloc(x: torch.Tensor, recipe: int, out: torch.Tensor,
+                         scales: torch.Tensor, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Quantize like fp8_quantize without any allocation, for callers that
+    may not allocate device memory (for example a plugin inside a host
+    application that owns every allocation, or a service whose memory plan
+    is fixed at start-up).  The caller passes the output buffers; the library
+    uses its own fixed scratch, shared by all calls (order calls on one
+    stream: concurrent calls race on it)."""
+    L = load_library()
+    _need_cuda(x, out, scales)
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D bf16 tensor with unit column stride")
+    rows, cols = x.shape
+    ld = x.stride(0) if (rows > 1 and cols > 0) else cols
+    _check(L.fp8_quantize_noalloc(_ptr(x), rows, cols, ld, recipe, _ptr(out),
+                                  _ptr(scales), _stream(stream)))
     return out, scales
 
 

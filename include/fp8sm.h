@@ -132,6 +132,35 @@ FP8SM_API fp8_status fp8_quantize(const void* x_bf16, int64_t rows, int64_t cols
                         fp8_stream_t stream);
 
 /*
+ * Dynamic quantization exactly as fp8_quantize (same recipes, layouts,
+ * results and errors), but without a workspace argument, for callers that
+ * cannot allocate device memory: for example a plugin running inside a host
+ * application that owns every device allocation and hands its plugins no
+ * scratch, or a service that fixes its memory plan at start-up and may not
+ * call cudaMalloc afterwards (it synchronizes the device and can fail under
+ * memory pressure).  The caller still passes x, out_fp8 and out_scales.
+ *
+ * This entry point allocates nothing and calls no allocating routine.  The
+ * scratch it needs (the tensorwise recipe's amax word and grid-barrier
+ * counter) lives in a fixed FP8_NOALLOC_SCRATCH_BYTES-byte array inside the
+ * library's device code; every GPU that loads the library holds one copy
+ * until the process exits.  The first call on each device looks up that
+ * array's device address (cudaGetSymbolAddress) with the device current;
+ * make that first call before any stream capture.  All calls share the
+ * array and each call clears the part that must start at zero, so calls that
+ * run at the same time on the GPU (for example on two streams) race with
+ * each other: order them on one stream.  A call that would need more scratch
+ * than the array holds returns FP8_ERR_VALUE.  No counterpart on the pages.
+ */
+#define FP8_NOALLOC_SCRATCH_BYTES 256
+
+FP8SM_API fp8_status fp8_quantize_noalloc(const void* x_bf16, int64_t rows,
+                                          int64_t cols, int64_t ld_x,
+                                          fp8_quant_recipe recipe,
+                                          void* out_fp8, float* out_scales,
+                                          fp8_stream_t stream);
+
+/*
  * Scaled GEMM ([P1] forward; [P4] recipes; [P5] blockwise recipes):
  *   out[m, n] = sum_k (a[m,k] * sA) * (b[n,k] * sB)  (+ bias[n])
  * with the scales picked per recipe (see fp8_mm_recipe).  Products are
