@@ -111,7 +111,7 @@ fp8_status fp8_quantize(const void* x_bf16, int64_t rows, int64_t cols,
   if (recipe < FP8_SCALE_TENSOR || recipe > FP8_SCALE_BLOCK_128x128)
     return fail(FP8_ERR_VALUE, "fp8_quantize: unknown recipe");
   if (rows < 0 || cols < 0) return fail(FP8_ERR_VALUE, "fp8_quantize: negative size");
-  if (rows > (int64_t(1) << 31) || cols > (int64_t(1) << 31))
+  if (rows >= (int64_t(1) << 31) || cols >= (int64_t(1) << 31))
     return fail(FP8_ERR_VALUE, "fp8_quantize: size too large");
   if (ld_x < cols) return fail(FP8_ERR_VALUE, "fp8_quantize: ld_x < cols");
   if (cols % 8 != 0 || ld_x % 8 != 0)

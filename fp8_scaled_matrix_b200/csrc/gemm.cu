@@ -9,14 +9,18 @@
 // perf"), and the grouped rowwise MoE form over (E, N, K) experts with
 // cumulative offs ("Add _grouped_mm dispatch handler to Float8Tensor").
 //
-// One persistent kernel, one CTA per SM, 10 warps with fixed roles:
+// One persistent kernel, one CTA per SM, 12 warps with fixed roles:
 //   warp 0      TMA producer: A (128 x 128 B) and B (256 x 128 B) tiles into
 //               a 4-stage shared-memory ring (128-byte swizzle)
 //   warp 1      TMEM owner + MMA issuer: one thread issues
 //               tcgen05.mma.kind::f8f6f4 (M=128, N=256, K=32) x 4 per stage
 //               into fp32 TMEM accumulators; tcgen05.commit frees stages
-//   warps 2-9   epilogue: warp w reads TMEM lanes 32*(w%4).. (the hardware's
-//               lane quarter) and columns 128*((w-2)/4).. of each tile
+//   warps 2-3   idle after the prologue (warp 2 validates offs)
+//   warps 4-11  epilogue: warp w reads TMEM lanes 32*(w%4).. (the hardware's
+//               lane quarter) and columns 128*((w-4)/4).. of each tile
+// The blockwise kernels move registers from warpgroup 0 to the epilogue
+// warpgroups (setmaxnreg) so each epilogue thread can hold its 128 fp32
+// accumulators plus 64 freshly loaded TMEM values.
 // TMEM holds two 256-column fp32 buffers.  Tensorwise / rowwise: each buffer
 // is one whole tile's accumulator, so the epilogue of tile i overlaps the
 // MMAs of tile i+1.  Blockwise: each 128-wide K block is accumulated into a
@@ -34,6 +38,8 @@
 #include <cudaTypedefs.h>
 #include <stdint.h>
 
+#include <cstdlib>
+
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -44,26 +50,49 @@ constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 128;  // bytes == e4m3 elements per stage along K
 constexpr int UMMA_K = 32;
-constexpr int STAGES = 4;
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kFirstEpiWarp = 4;  // warps 0-3 = warpgroup 0 (producer, MMA, 2 idle)
+constexpr int kThreads = 32 * kFirstEpiWarp + 32 * kEpiWarps;
+// Register split (blockwise kernels): warpgroup 0 gives registers up, the two
+// epilogue warpgroups take them.  Launch: 384 threads x 168 registers =
+// 64512 = 128 x kRegsLow + 256 x kRegsHigh.  The host refuses to launch a
+// kernel that was compiled with fewer than kRegsAtLaunch registers.
+constexpr uint32_t kRegsLow = 56;
+constexpr uint32_t kRegsHigh = 224;
+constexpr uint32_t kRegsAtLaunch = 168;
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsAtLaunch,
+              "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;  // two 256-column fp32 buffers
-constexpr uint32_t kAStage = BM * BK;
-constexpr uint32_t kBStage = BN * BK;
 constexpr uint32_t kEpiBuf = 32 * 64;  // 32 rows x 64 bytes, 64-byte swizzle
-constexpr uint32_t kSbBuf = 128 * 4;   // 128 fp32 column scales per warp
+constexpr int kScaleAhead = 4;         // K blocks of scales fetched ahead
+constexpr int kRingAhead = 3;          // 128x1: K blocks of scales in the smem ring
+constexpr int kSbSlot = 128 + 32;      // 128x1 ring slot: column + row scales
+constexpr uint32_t kSbBuf = kRingAhead * kSbSlot * 4;  // per-warp 128x1 scale ring
 
-constexpr uint32_t kOffA = 0;
-constexpr uint32_t kOffB = kOffA + STAGES * kAStage;
-constexpr uint32_t kOffEpi = kOffB + STAGES * kBStage;
-constexpr uint32_t kOffSb = kOffEpi + kEpiWarps * kEpiBuf;
-constexpr uint32_t kOffBar = kOffSb + kEpiWarps * kSbBuf;
-// barriers: full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain
-constexpr uint32_t kNumBars = 2 * STAGES + 5;
-constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
-constexpr uint32_t kSmemUsed = kOffMisc + 16;
-constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // + alignment slack
-static_assert(kSmemBytes <= 232448, "shared memory budget");
+// Shared-memory layout.  Single-CTA tiles are 128 x 256: each stage holds
+// A (128 rows) and B (256 rows) of a 128-byte K slice.  CTA-pair tiles are
+// 256 x 256 (cta_group::2): each CTA holds its own 128 rows of A and its own
+// 128 rows (half of N) of B, so a stage is a third smaller and two more
+// stages fit.
+template <bool kPair>
+struct Cfg {
+  static constexpr int kStages = kPair ? 6 : 4;
+  static constexpr int kTileM = kPair ? 2 * BM : BM;   // output rows per work item
+  static constexpr uint32_t kBRows = kPair ? BN / 2 : BN;  // B rows held per CTA
+  static constexpr uint32_t kAStage = BM * BK;
+  static constexpr uint32_t kBStage = kBRows * BK;
+  static constexpr uint32_t kOffA = 0;
+  static constexpr uint32_t kOffB = kOffA + kStages * kAStage;
+  static constexpr uint32_t kOffEpi = kOffB + kStages * kBStage;
+  static constexpr uint32_t kOffSb = kOffEpi + kEpiWarps * kEpiBuf;
+  static constexpr uint32_t kOffBar = kOffSb + kEpiWarps * kSbBuf;
+  // barriers: full[kStages], empty[kStages], acc_full[2], acc_empty[2], drain
+  static constexpr uint32_t kNumBars = 2 * kStages + 5;
+  static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr uint32_t kSmemUsed = kOffMisc + 16;
+  static constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // + alignment slack
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
 
 enum Recipe : int { kTensor = 0, kRow = 1, kBlock128 = 2, kBlock1 = 3 };
 
@@ -79,6 +108,12 @@ struct GemmParams {
   int32_t m_tiles;   // tiles along M (dense)
   int32_t k_blocks;
   uint32_t* status;
+  // Dense kernels: work items [0, split_start) are whole 128 x 256 tiles in
+  // M-major order; when the last wave would leave more than half of the SMs
+  // idle, each of its tiles becomes two 128 x 128 items (split_start ..
+  // total_items), so twice as many SMs finish it in half the time.
+  int64_t split_start;
+  int64_t total_items;
 };
 
 // Walks the concatenated per-group M tiles in increasing order.
@@ -88,20 +123,20 @@ struct GroupCursor {
   int64_t row_start;
   int64_t row_end;
   int64_t m_tiles;  // M tiles of group g
-  __device__ void init(const int32_t* offs) {
+  __device__ void init(const int32_t* offs, int64_t tm) {
     g = 0;
     tiles_before = 0;
     row_start = 0;
     row_end = offs[0];
-    m_tiles = (row_end + BM - 1) / BM;
+    m_tiles = (row_end + tm - 1) / tm;
   }
-  __device__ void seek(int64_t mt, const int32_t* offs, int32_t E) {
+  __device__ void seek(int64_t mt, const int32_t* offs, int32_t E, int64_t tm) {
     while (mt >= tiles_before + m_tiles && g + 1 < E) {
       tiles_before += m_tiles;
       ++g;
       row_start = row_end;
       row_end = offs[g];
-      m_tiles = (row_end - row_start + BM - 1) / BM;
+      m_tiles = (row_end - row_start + tm - 1) / tm;
     }
   }
 };
@@ -109,22 +144,34 @@ struct GroupCursor {
 struct TileCoord {
   int32_t m0, n0, g;
   int64_t row_end;
+  bool half_n;  // 128-wide item (columns n0 .. n0+127 only)
 };
 
-template <bool kGrouped>
+// Work item t -> output tile (rows m0 .. m0 + kTM - 1).
+template <bool kGrouped, int kTM>
 __device__ __forceinline__ TileCoord tile_coord(int64_t t, const GemmParams& p,
                                                 GroupCursor& cur) {
   TileCoord c;
+  c.half_n = false;
+  int32_t sub = 0;
+  if constexpr (!kGrouped) {
+    if (t >= p.split_start) {
+      const int64_t h = t - p.split_start;
+      t = p.split_start + (h >> 1);
+      sub = static_cast<int32_t>(h & 1);
+      c.half_n = true;
+    }
+  }
   const int64_t mt = t / p.n_tiles;
-  c.n0 = static_cast<int32_t>((t % p.n_tiles) * BN);
+  c.n0 = static_cast<int32_t>((t % p.n_tiles) * BN) + sub * (BN / 2);
   if constexpr (kGrouped) {
-    cur.seek(mt, p.offs, p.E);
+    cur.seek(mt, p.offs, p.E, kTM);
     c.g = cur.g;
-    c.m0 = static_cast<int32_t>(cur.row_start + (mt - cur.tiles_before) * BM);
+    c.m0 = static_cast<int32_t>(cur.row_start + (mt - cur.tiles_before) * kTM);
     c.row_end = cur.row_end;
   } else {
     c.g = 0;
-    c.m0 = static_cast<int32_t>(mt * BM);
+    c.m0 = static_cast<int32_t>(mt * kTM);
     c.row_end = p.M;
   }
   return c;
@@ -186,6 +233,11 @@ __device__ __forceinline__ void store_box64(
     uint8_t* buf, const uint4 (&chunk)[4], const CUtensorMap* tm_out,
     int32_t col0 /*elements*/, int32_t row0, int64_t row_end, uint8_t* out,
     int64_t N, uint32_t elem_bytes, uint32_t lane) {
+  if constexpr (!kGrouped) {
+    // the previous box's TMA store must have read the buffer
+    if (lane == 0) bulk_wait_group_read0();
+    __syncwarp();
+  }
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const uint32_t slot = static_cast<uint32_t>(j) ^ ((lane >> 1) & 3u);
@@ -199,9 +251,7 @@ __device__ __forceinline__ void store_box64(
     if (lane == 0 && row0 < row_end && col0 < N) {
       tma_store_2d(tm_out, buf, col0, row0);
       bulk_commit_group();
-      bulk_wait_group_read0();
     }
-    __syncwarp();
   } else {
     __syncwarp();
     const uint32_t elems_per_chunk = 16u / elem_bytes;
@@ -252,23 +302,25 @@ __device__ __forceinline__ void store_cols32(
   }
 }
 
-template <int kRecipe, bool kOutF32, bool kGrouped>
+template <int kRecipe, bool kOutF32, bool kGrouped, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
                     const __grid_constant__ CUtensorMap tm_b,
+                    const __grid_constant__ CUtensorMap tm_b_half,
                     const __grid_constant__ CUtensorMap tm_out,
                     const GemmParams p) {
   constexpr bool kBlockwise = (kRecipe == kBlock128 || kRecipe == kBlock1);
+  using C = Cfg<kPair>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* full = bars;
-  uint64_t* empty = bars + STAGES;
-  uint64_t* acc_full = bars + 2 * STAGES;
-  uint64_t* acc_empty = bars + 2 * STAGES + 2;
-  uint64_t* drain = bars + 2 * STAGES + 4;
-  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+  uint64_t* empty = bars + C::kStages;
+  uint64_t* acc_full = bars + 2 * C::kStages;
+  uint64_t* acc_empty = bars + 2 * C::kStages + 2;
+  uint64_t* drain = bars + 2 * C::kStages + 4;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   uint32_t* tmem_slot = misc + 0;
   volatile uint32_t* abort_flag = misc + 1;
   int64_t* total_tiles_slot = reinterpret_cast<int64_t*>(misc + 2);
@@ -277,24 +329,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t lane = lane_id();
 
   if (warp == 0 && lane == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], kEpiWarps);
+      // pair: the leader's barrier collects both CTAs' epilogue warps
+      mbar_init(&acc_empty[i], kPair ? 2 * kEpiWarps : kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0u;
     fence_barrier_init();
     prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_b);
-    if constexpr (!kGrouped) prefetch_tmap(&tm_out);
+    if constexpr (!kGrouped) {
+      prefetch_tmap(&tm_b_half);
+      prefetch_tmap(&tm_out);
+    }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    if constexpr (kPair) {
+      tmem_alloc_pair(tmem_slot, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, kTmemCols);
+      tmem_relinquish();
+    }
   }
   if (warp == 2) {
     int64_t total;
@@ -306,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int32_t e = p.offs[i];
         const int32_t prev = i ? p.offs[i - 1] : 0;
         if (e < prev || prev < 0) bad = true;
-        else mt += (static_cast<int64_t>(e) - prev + BM - 1) / BM;
+        else mt += (static_cast<int64_t>(e) - prev + C::kTileM - 1) / C::kTileM;
       }
       if (lane == 0 && static_cast<int64_t>(p.offs[p.E - 1]) != p.M) bad = true;
       bad = __any_sync(0xFFFFFFFFu, bad);
@@ -317,66 +378,94 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (bad && lane == 0 && blockIdx.x == 0)
         record_status(p.status, FP8_DEV_VALUE, SITE_OFFS);
     } else {
-      total = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
+      total = p.total_items;
     }
     if (lane == 0) *total_tiles_slot = total;
   }
   __syncthreads();
+  // pair: both CTAs' barriers are initialised before any cross-CTA traffic
+  if constexpr (kPair) cluster_sync();
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
   const int64_t total_tiles = *total_tiles_slot;
   const int32_t KB = p.k_blocks;
+  // work items: one per CTA, or one per CTA pair (cluster of two)
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+  const int64_t item0 = kPair ? (blockIdx.x >> 1) : blockIdx.x;
+  const int64_t item_stride = kPair ? (gridDim.x >> 1) : gridDim.x;
+  constexpr int kTM = C::kTileM;
 
-  if (warp == 0) {
+  if (warp < kFirstEpiWarp) {
+   // warpgroup 0: all four warps execute the same setmaxnreg
+   if constexpr (kBlockwise) warpgroup_reg_dealloc<kRegsLow>();
+   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
       GroupCursor cur;
-      if constexpr (kGrouped) cur.init(p.offs);
+      if constexpr (kGrouped) cur.init(p.offs, kTM);
       uint32_t stage = 0, phase = 0;
       uint64_t issued = 0;
       bool ok = true;
-      for (int64_t t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-        const TileCoord c = tile_coord<kGrouped>(t, p, cur);
+      for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
+        const TileCoord c = tile_coord<kGrouped, kTM>(t, p, cur);
         for (int32_t kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status,
                          SITE_PRODUCER_EMPTY, kWaitLimitNs)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], kAStage + kBStage);
-          tma_load_2d(smem + kOffA + stage * kAStage, &tm_a, &full[stage],
-                      kb * BK, c.m0);
-          if constexpr (kGrouped)
-            tma_load_3d(smem + kOffB + stage * kBStage, &tm_b, &full[stage],
-                        kb * BK, c.n0, c.g);
-          else
-            tma_load_2d(smem + kOffB + stage * kBStage, &tm_b, &full[stage],
-                        kb * BK, c.n0);
+          const uint32_t b_bytes = c.half_n ? C::kBStage / 2 : C::kBStage;
+          uint8_t* a_dst = smem + C::kOffA + stage * C::kAStage;
+          uint8_t* b_dst = smem + C::kOffB + stage * C::kBStage;
+          if constexpr (kPair) {
+            // This CTA's 128 rows of A and its half of the item's B rows;
+            // both CTAs' bytes complete on the leader's barrier, which the
+            // leader arms for the pair.
+            const uint32_t lead_full = mapa_shared(smem_u32(&full[stage]), 0);
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * (C::kAStage + b_bytes));
+            const int32_t b_row = c.n0 + static_cast<int32_t>(rank) * (c.half_n ? BN / 4 : BN / 2);
+            tma_load_2d_pair(a_dst, &tm_a, lead_full, kb * BK,
+                             c.m0 + static_cast<int32_t>(rank) * BM);
+            if constexpr (kGrouped)
+              tma_load_3d_pair(b_dst, &tm_b, lead_full, kb * BK, b_row, c.g);
+            else
+              tma_load_2d_pair(b_dst, c.half_n ? &tm_b_half : &tm_b, lead_full, kb * BK, b_row);
+          } else {
+            mbar_arrive_expect_tx(&full[stage], C::kAStage + b_bytes);
+            tma_load_2d(a_dst, &tm_a, &full[stage], kb * BK, c.m0);
+            if constexpr (kGrouped)
+              tma_load_3d(b_dst, &tm_b, &full[stage], kb * BK, c.n0, c.g);
+            else
+              tma_load_2d(b_dst, c.half_n ? &tm_b_half : &tm_b, &full[stage], kb * BK, c.n0);
+          }
           ++issued;
-          if (++stage == STAGES) {
+          if (++stage == C::kStages) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
-      if (!ok) {
+      if (!ok && rank == 0) {
         // Let the copies already in flight land before the CTA exits.
-        const uint64_t first = issued > STAGES ? issued - STAGES : 0;
+        const uint64_t first = issued > C::kStages ? issued - C::kStages : 0;
         for (uint64_t i = first; i < issued; ++i) {
           uint32_t dummy_abort = 0;
-          mbar_wait(&full[i % STAGES], static_cast<uint32_t>((i / STAGES) & 1u),
+          mbar_wait(&full[i % C::kStages], static_cast<uint32_t>((i / C::kStages) & 1u),
                     &dummy_abort, nullptr, SITE_TEARDOWN, 10000000ull);
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = idesc_e4m3_f32(BM, BN);
+    // (pair: the leader CTA issues for both; the peer only drains)
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc_full = idesc_e4m3_f32(kTM, BN);
+      const uint32_t idesc_half = idesc_e4m3_f32(kTM, BN / 2);
       uint32_t stage = 0, phase = 0;
       uint32_t acc = 0, acc_phase = 0;
       bool ok = true;
-      for (int64_t t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+      for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
+        const uint32_t idesc = (!kGrouped && t >= p.split_start) ? idesc_half : idesc_full;
         if constexpr (!kBlockwise) {
           if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag, p.status,
                          SITE_MMA_ACC_EMPTY, kWaitLimitNs)) {
@@ -402,58 +491,77 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after_sync();
           const uint32_t d = tmem_base + acc * BN;
           const uint64_t da =
-              smem_desc_k_sw128(smem_u32(smem + kOffA + stage * kAStage));
+              smem_desc_k_sw128(smem_u32(smem + C::kOffA + stage * C::kAStage));
           const uint64_t db =
-              smem_desc_k_sw128(smem_u32(smem + kOffB + stage * kBStage));
+              smem_desc_k_sw128(smem_u32(smem + C::kOffB + stage * C::kBStage));
 #pragma unroll
           for (int k = 0; k < BK / UMMA_K; ++k) {
             const uint32_t accumulate =
                 kBlockwise ? (k > 0) : ((kb > 0) || (k > 0));
-            mma_e4m3(d, da + (k * UMMA_K) / 16, db + (k * UMMA_K) / 16, idesc,
-                     accumulate);
+            if constexpr (kPair)
+              mma_e4m3_pair(d, da + (k * UMMA_K) / 16, db + (k * UMMA_K) / 16, idesc,
+                            accumulate);
+            else
+              mma_e4m3(d, da + (k * UMMA_K) / 16, db + (k * UMMA_K) / 16, idesc,
+                       accumulate);
           }
-          mma_commit(&empty[stage]);
-          if (++stage == STAGES) {
+          if constexpr (kPair) mma_commit_pair(&empty[stage], 0x3);
+          else mma_commit(&empty[stage]);
+          if (++stage == C::kStages) {
             stage = 0;
             phase ^= 1u;
           }
           if constexpr (kBlockwise) {
-            mma_commit(&acc_full[acc]);
+            if constexpr (kPair) mma_commit_pair(&acc_full[acc], 0x3);
+            else mma_commit(&acc_full[acc]);
             acc ^= 1u;
             if (acc == 0) acc_phase ^= 1u;
           }
         }
         if constexpr (!kBlockwise) {
           if (ok) {
-            mma_commit(&acc_full[acc]);
+            if constexpr (kPair) mma_commit_pair(&acc_full[acc], 0x3);
+            else mma_commit(&acc_full[acc]);
             acc ^= 1u;
             if (acc == 0) acc_phase ^= 1u;
           }
         }
       }
-      // All MMAs issued by this thread complete before TMEM is released.
-      mma_commit(drain);
+      // All MMAs issued by this thread complete before TMEM is released
+      // (pair: in both CTAs).
+      if constexpr (kPair) mma_commit_pair(drain, 0x3);
+      else mma_commit(drain);
+    }
+    if (lane == 0) {
       uint32_t dummy_abort = 0;
       mbar_wait(drain, 0, &dummy_abort, p.status, SITE_TEARDOWN, kWaitLimitNs);
     }
+   }
   } else {
     // --------------------------------------------------------- epilogue
-    const uint32_t ew = warp - 2;          // 0..7
+    if constexpr (kBlockwise) warpgroup_reg_alloc<kRegsHigh>();
+    const uint32_t ew = warp - kFirstEpiWarp;  // 0..7
     const uint32_t q = warp & 3u;          // TMEM lane quarter of this warp
     const uint32_t half = ew >> 2;         // which 128 columns of the tile
-    uint8_t* ebuf = smem + kOffEpi + ew * kEpiBuf;
-    float* sbbuf = reinterpret_cast<float*>(smem + kOffSb + ew * kSbBuf);
+    uint8_t* ebuf = smem + C::kOffEpi + ew * kEpiBuf;
+    float* sbbuf = reinterpret_cast<float*>(smem + C::kOffSb + ew * kSbBuf);
     const uint32_t lane_base = (q * 32u) << 16;
     GroupCursor cur;
-    if constexpr (kGrouped) cur.init(p.offs);
+    if constexpr (kGrouped) cur.init(p.offs, kTM);
     uint32_t acc = 0, acc_phase = 0;
     bool ok = true;
-    for (int64_t t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-      const TileCoord c = tile_coord<kGrouped>(t, p, cur);
-      const int64_t row = static_cast<int64_t>(c.m0) + q * 32 + lane;
+    // TMEM buffers are handed back on the leader's barrier (pair: from both CTAs)
+    const uint32_t acc_empty_addr0 =
+        kPair ? mapa_shared(smem_u32(&acc_empty[0]), 0) : smem_u32(&acc_empty[0]);
+    const uint32_t acc_empty_addr1 =
+        kPair ? mapa_shared(smem_u32(&acc_empty[1]), 0) : smem_u32(&acc_empty[1]);
+    for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
+      const TileCoord c = tile_coord<kGrouped, kTM>(t, p, cur);
+      const int32_t cta_m0 = c.m0 + static_cast<int32_t>(rank) * BM;  // this CTA's rows
+      const int64_t row = static_cast<int64_t>(cta_m0) + q * 32 + lane;
       const bool row_ok = row < c.row_end;
       const int64_t ncol0 = static_cast<int64_t>(c.n0) + half * 128;
-      const int32_t row0 = c.m0 + static_cast<int32_t>(q * 32);
+      const int32_t row0 = cta_m0 + static_cast<int32_t>(q * 32);
 
       if constexpr (!kBlockwise) {
         if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status,
@@ -462,6 +570,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after_sync();
+        if (c.half_n && half == 1) {
+          // 128-wide item: this warp's columns are not part of it
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(acc ? acc_empty_addr1 : acc_empty_addr0);
+          acc ^= 1u;
+          if (acc == 0) acc_phase ^= 1u;
+          continue;
+        }
         float sa;
         if constexpr (kRecipe == kTensor) sa = __ldg(p.sa) * __ldg(p.sb);
         else sa = row_ok ? __ldg(p.sa + row) : 0.0f;
@@ -475,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (cc == 3) {
             tc_fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+            if (lane == 0) mbar_arrive_cluster(acc ? acc_empty_addr1 : acc_empty_addr0);
           }
           const int64_t n = ncol0 + cc * 32;
           float bias[32];
@@ -498,44 +614,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         acc ^= 1u;
         if (acc == 0) acc_phase ^= 1u;
-      } else {
-        // Blockwise: promote each K block's partial product into registers.
+      } else if constexpr (kRecipe == kBlock128) {
+        // 1x128_128x128: promote each K block's partial product into
+        // registers; the scale product sA[m,kb] * sB[n/128,kb] is one value
+        // per thread per K block.
         float2 accr[64];
 #pragma unroll
         for (int i = 0; i < 64; ++i) accr[i] = make_float2(0.0f, 0.0f);
         const int64_t NB = (p.N + 127) / 128;
         const int64_t nb = ncol0 / 128;  // 128-column block of this warp
         const bool nb_ok = ncol0 < p.N;
-        // first K block's scales
-        float sa_next = row_ok ? __ldg(p.sa + row) : 0.0f;
-        float sb_next = 0.0f;
-        float4 sb4_next = make_float4(0.f, 0.f, 0.f, 0.f);
-        if constexpr (kRecipe == kBlock128) {
-          sb_next = nb_ok ? __ldg(p.sb + nb) : 0.0f;
-        } else {
-          const int64_t n = ncol0 + 4 * lane;
-          if (n < p.N) sb4_next = __ldg(reinterpret_cast<const float4*>(p.sb + n));
+        // scales fetched kScaleAhead K blocks ahead through a shift register
+        auto load_sa = [&](int32_t k) -> float {
+          return (row_ok && k < KB) ? __ldg(p.sa + static_cast<int64_t>(k) * p.M + row) : 0.0f;
+        };
+        auto load_sb = [&](int32_t k) -> float {
+          return (nb_ok && k < KB) ? __ldg(p.sb + static_cast<int64_t>(k) * NB + nb) : 0.0f;
+        };
+        float sa_r[kScaleAhead], sb_r[kScaleAhead];
+#pragma unroll
+        for (int i = 0; i < kScaleAhead; ++i) {
+          sa_r[i] = load_sa(i);
+          sb_r[i] = load_sb(i);
         }
         for (int32_t kb = 0; kb < KB; ++kb) {
-          const float sa_kb = sa_next;
-          const float sb_kb = sb_next;
-          if constexpr (kRecipe == kBlock1) {
-            __syncwarp();
-            reinterpret_cast<float4*>(sbbuf)[lane] = sb4_next;
-            __syncwarp();
+          const float f = sa_r[0] * sb_r[0];
+#pragma unroll
+          for (int i = 0; i + 1 < kScaleAhead; ++i) {
+            sa_r[i] = sa_r[i + 1];
+            sb_r[i] = sb_r[i + 1];
           }
-          // prefetch the next K block's scales
-          if (kb + 1 < KB) {
-            sa_next = row_ok ? __ldg(p.sa + static_cast<int64_t>(kb + 1) * p.M + row) : 0.0f;
-            if constexpr (kRecipe == kBlock128) {
-              sb_next = nb_ok ? __ldg(p.sb + static_cast<int64_t>(kb + 1) * NB + nb) : 0.0f;
-            } else {
-              const int64_t n = ncol0 + 4 * lane;
-              if (n < p.N)
-                sb4_next = __ldg(reinterpret_cast<const float4*>(
-                    p.sb + static_cast<int64_t>(kb + 1) * p.N + n));
-            }
-          }
+          sa_r[kScaleAhead - 1] = load_sa(kb + kScaleAhead);
+          sb_r[kScaleAhead - 1] = load_sb(kb + kScaleAhead);
           if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status,
                          SITE_EPI_ACC_FULL, kWaitLimitNs)) {
             ok = false;
@@ -543,40 +653,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after_sync();
           const uint32_t tcol = tmem_base + lane_base + acc * BN + half * 128;
-          const float f = sa_kb * sb_kb;
+          const float2 f2 = make_float2(f, f);
 #pragma unroll
-          for (int cc = 0; cc < 8; ++cc) {
-            uint32_t r[16];
-            tmem_ld_32x32b_x16(tcol + cc * 16, r);
+          for (int hc = 0; hc < 2; ++hc) {
+            uint32_t r[2][32];
+            tmem_ld_32x32b_x32(tcol + hc * 64, r[0]);
+            tmem_ld_32x32b_x32(tcol + hc * 64 + 32, r[1]);
             tmem_ld_wait();
-            if constexpr (kRecipe == kBlock128) {
-              const float2 f2 = make_float2(f, f);
+            if (hc == 1) {
+              // every TMEM read of this buffer is done: hand it back
+              tc_fence_before_sync();
+              __syncwarp();
+              if (lane == 0) mbar_arrive_cluster(acc ? acc_empty_addr1 : acc_empty_addr0);
+            }
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const float2 pv = make_float2(__uint_as_float(r[2 * i]),
-                                              __uint_as_float(r[2 * i + 1]));
-                accr[cc * 8 + i] = fma2(pv, f2, accr[cc * 8 + i]);
-              }
-            } else {
-              const float2 sa2 = make_float2(sa_kb, sa_kb);
-              const float4* sbv = reinterpret_cast<const float4*>(sbbuf) + cc * 4;
+            for (int c2 = 0; c2 < 2; ++c2) {
+              const int base = hc * 32 + c2 * 16;  // float2 index of column hc*64 + c2*32
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const float4 s4 = sbv[i];
-                const float2 p0 = make_float2(__uint_as_float(r[4 * i]),
-                                              __uint_as_float(r[4 * i + 1]));
-                const float2 p1 = make_float2(__uint_as_float(r[4 * i + 2]),
-                                              __uint_as_float(r[4 * i + 3]));
-                const float2 t0 = mul2(p0, make_float2(s4.x, s4.y));
-                const float2 t1 = mul2(p1, make_float2(s4.z, s4.w));
-                accr[cc * 8 + 2 * i] = fma2(t0, sa2, accr[cc * 8 + 2 * i]);
-                accr[cc * 8 + 2 * i + 1] = fma2(t1, sa2, accr[cc * 8 + 2 * i + 1]);
+              for (int i = 0; i < 16; ++i) {
+                const float2 pv = make_float2(__uint_as_float(r[c2][2 * i]),
+                                              __uint_as_float(r[c2][2 * i + 1]));
+                accr[base + i] = fma2(pv, f2, accr[base + i]);
               }
             }
           }
-          tc_fence_before_sync();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[acc]);
           acc ^= 1u;
           if (acc == 0) acc_phase ^= 1u;
         }
@@ -595,6 +695,142 @@ __global__ void __launch_bounds__(kThreads, 1)
                                           static_cast<int32_t>(n), row0,
                                           c.row_end, p.out, p.N, lane);
         }
+      } else {
+        // 1x128_128x1: a different scale for every output column.  TMEM is
+        // read in the 16x256b shape: thread t holds rows g, g+8, g+16, g+24
+        // (g = t/4) of the warp's lane quarter and, in every 8-column group j,
+        // the two columns 8j + 2c, 8j + 2c + 1 (c = t%4): 4 rows x 32 columns.
+        // So it needs 4 row scales and 32 column scales per K block (8-byte
+        // shared loads that 8 lanes share) instead of 128 column scales.
+        // Scales come through a per-warp cp.async ring, kRingAhead K blocks
+        // ahead: slot = [128 column scales | 32 row scales].
+        const uint32_t g = lane >> 2, cq = lane & 3;
+        float2 accr[64];  // accr[ri * 16 + j]: row g + 8 ri, columns 8j + 2cq + {0,1}
+#pragma unroll
+        for (int i = 0; i < 64; ++i) accr[i] = make_float2(0.0f, 0.0f);
+        const int64_t ncol_lane = ncol0 + 4 * lane;
+        auto fetch = [&](int32_t k) {
+          float* dst = sbbuf + (k % kRingAhead) * kSbSlot;
+          const bool vc = k < KB && ncol_lane < p.N;
+          cp_async_16(dst + 4 * lane,
+                      vc ? p.sb + static_cast<int64_t>(k) * p.N + ncol_lane : p.sb,
+                      vc ? 16u : 0u);
+          const bool vr = k < KB && row_ok;
+          cp_async_4(dst + 128 + lane, vr ? p.sa + static_cast<int64_t>(k) * p.M + row : p.sa,
+                     vr ? 4u : 0u);
+          cp_async_commit();
+        };
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < kRingAhead - 1; ++i) fetch(i);
+        for (int32_t kb = 0; kb < KB; ++kb) {
+          __syncwarp();  // every lane is done reading the slot refilled next
+          fetch(kb + kRingAhead - 1);
+          cp_async_wait<kRingAhead - 1>();  // this K block's slot has landed
+          __syncwarp();
+          if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status,
+                         SITE_EPI_ACC_FULL, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const float* sl = sbbuf + (kb % kRingAhead) * kSbSlot;
+          const float sa_i[4] = {sl[128 + g], sl[128 + g + 8], sl[128 + g + 16],
+                                 sl[128 + g + 24]};
+          const uint32_t tcol = tmem_base + lane_base + acc * BN + half * 128;
+#pragma unroll
+          for (int lh = 0; lh < 2; ++lh) {  // TMEM lanes 0-15 / 16-31 of the quarter
+            uint32_t r[2][32];
+            tmem_ld_16x256b_x8(tcol + ((16u * lh) << 16), r[0]);
+            tmem_ld_16x256b_x8(tcol + ((16u * lh) << 16) + 64, r[1]);
+            tmem_ld_wait();
+            if (lh == 1) {
+              tc_fence_before_sync();
+              __syncwarp();
+              if (lane == 0) mbar_arrive_cluster(acc ? acc_empty_addr1 : acc_empty_addr0);
+            }
+            const float2 sat = make_float2(sa_i[2 * lh], sa_i[2 * lh]);
+            const float2 sab = make_float2(sa_i[2 * lh + 1], sa_i[2 * lh + 1]);
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const int j = ch * 8 + k;
+                const float2 s2 = *reinterpret_cast<const float2*>(sl + 8 * j + 2 * cq);
+                const float2 pt = make_float2(__uint_as_float(r[ch][4 * k]),
+                                              __uint_as_float(r[ch][4 * k + 1]));
+                const float2 pb = make_float2(__uint_as_float(r[ch][4 * k + 2]),
+                                              __uint_as_float(r[ch][4 * k + 3]));
+                accr[(2 * lh) * 16 + j] = fma2(mul2(pt, s2), sat, accr[(2 * lh) * 16 + j]);
+                accr[(2 * lh + 1) * 16 + j] =
+                    fma2(mul2(pb, s2), sab, accr[(2 * lh + 1) * 16 + j]);
+              }
+            }
+          }
+          acc ^= 1u;
+          if (acc == 0) acc_phase ^= 1u;
+        }
+        if (!ok) break;
+        // Final store: per 32-column chunk cc (column groups j = 4cc..4cc+3),
+        // each thread writes its 4 rows x 4 column pairs into the warp's
+        // staging box (32 rows x 64 bytes, 64-byte swizzle), then the box is
+        // stored like the other recipes' (bf16: one box per chunk; fp32: two).
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const int64_t n = ncol0 + cc * 32;
+          float bias2[4][2];
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            const int64_t col = n + 8 * jj + 2 * cq;
+            if (p.bias != nullptr && col < p.N) {
+              const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(p.bias + col));
+              bias2[jj][0] = __uint_as_float(w << 16);
+              bias2[jj][1] = __uint_as_float(w & 0xFFFF0000u);
+            } else {
+              bias2[jj][0] = bias2[jj][1] = 0.0f;
+            }
+          }
+          constexpr int kBoxes = kOutF32 ? 2 : 1;   // 64-byte boxes per 32 columns
+#pragma unroll
+          for (int bx = 0; bx < kBoxes; ++bx) {
+            if constexpr (!kGrouped) {
+              if (lane == 0) bulk_wait_group_read0();
+              __syncwarp();
+            }
+#pragma unroll
+            for (int ri = 0; ri < 4; ++ri) {
+              const uint32_t rr = g + 8 * ri;  // row within the warp's 32
+#pragma unroll
+              for (int jj = 0; jj < 4; ++jj) {
+                const float2 a = accr[ri * 16 + cc * 4 + jj];
+                const float o0 = a.x + bias2[jj][0], o1 = a.y + bias2[jj][1];
+                if constexpr (!kOutF32) {
+                  // bf16: column 8jj + 2cq -> byte 16jj + 4cq of the 64-byte row
+                  const uint32_t slot = static_cast<uint32_t>(jj) ^ ((rr >> 1) & 3u);
+                  *reinterpret_cast<uint32_t*>(ebuf + rr * 64 + slot * 16 + 4 * cq) =
+                      pack_bf16x2(o0, o1);
+                } else {
+                  // fp32: box bx holds columns 16bx .. 16bx+15 -> jj in {2bx, 2bx+1}
+                  if ((jj >> 1) == bx) {
+                    const uint32_t cb = (8 * (jj & 1) + 2 * cq) * 4;  // byte within the row
+                    const uint32_t slot = (cb >> 4) ^ ((rr >> 1) & 3u);
+                    *reinterpret_cast<float2*>(ebuf + rr * 64 + slot * 16 + (cb & 15)) =
+                        make_float2(o0, o1);
+                  }
+                }
+              }
+            }
+            const int32_t col0 = static_cast<int32_t>(n) + (kOutF32 ? 16 * bx : 0);
+            if constexpr (!kGrouped) {
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0 && row0 < c.row_end && col0 < p.N) {
+                tma_store_2d(&tm_out, ebuf, col0, row0);
+                bulk_commit_group();
+              }
+            }
+          }
+        }
       }
     }
     if (lane == 0) bulk_wait_group0();
@@ -603,9 +839,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before_sync();
   __syncthreads();
+  // pair: no CTA leaves (or frees TMEM) while the other may still touch its
+  // barriers or shared memory
+  if constexpr (kPair) cluster_sync();
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if constexpr (kPair) tmem_dealloc_pair(tmem_base, kTmemCols);
+    else tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
@@ -672,30 +912,55 @@ bool make_tmap(CUtensorMap* m, CUtensorMapDataType dt, uint32_t rank,
   return true;
 }
 
-template <int kRecipe, bool kOutF32, bool kGrouped>
+template <int kRecipe, bool kOutF32, bool kGrouped, bool kPair>
 cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb,
-                          const CUtensorMap& to, const GemmParams& p,
-                          unsigned grid, cudaStream_t st) {
+                          const CUtensorMap& tbh, const CUtensorMap& to,
+                          const GemmParams& p, unsigned grid, cudaStream_t st) {
+  using C = Cfg<kPair>;
   static bool configured = false;
-  auto kern = fp8_gemm_kernel<kRecipe, kOutF32, kGrouped>;
+  auto kern = fp8_gemm_kernel<kRecipe, kOutF32, kGrouped, kPair>;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(
-        kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
+    if (kRecipe == kBlock128 || kRecipe == kBlock1) {
+      // setmaxnreg.inc would wait forever if the launch allocation were
+      // smaller than the split assumes: check before the first launch.
+      cudaFuncAttributes attr;
+      e = cudaFuncGetAttributes(&attr, kern);
+      if (e != cudaSuccess) return e;
+      if (attr.numRegs < static_cast<int>(kRegsAtLaunch)) return cudaErrorInvalidConfiguration;
+    }
     configured = true;
   }
-  kern<<<grid, kThreads, kSmemBytes, st>>>(ta, tb, to, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kPair ? 2 : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, tbh, to, p);
 }
 
 template <bool kGrouped>
-cudaError_t dispatch(int recipe, int out_f32, const CUtensorMap& ta,
-                     const CUtensorMap& tb, const CUtensorMap& to,
-                     const GemmParams& p, unsigned grid, cudaStream_t st) {
-#define FP8SM_CASE(R)                                                        \
-  if (recipe == R)                                                           \
-    return out_f32 ? launch_kernel<R, true, kGrouped>(ta, tb, to, p, grid, st) \
-                   : launch_kernel<R, false, kGrouped>(ta, tb, to, p, grid, st);
+cudaError_t dispatch(int recipe, int out_f32, bool pair, const CUtensorMap& ta,
+                     const CUtensorMap& tb, const CUtensorMap& tbh,
+                     const CUtensorMap& to, const GemmParams& p, unsigned grid,
+                     cudaStream_t st) {
+#define FP8SM_CASE(R)                                                                   \
+  if (recipe == R) {                                                                    \
+    if (pair)                                                                           \
+      return out_f32 ? launch_kernel<R, true, kGrouped, true>(ta, tb, tbh, to, p, grid, st)   \
+                     : launch_kernel<R, false, kGrouped, true>(ta, tb, tbh, to, p, grid, st); \
+    return out_f32 ? launch_kernel<R, true, kGrouped, false>(ta, tb, tbh, to, p, grid, st)    \
+                   : launch_kernel<R, false, kGrouped, false>(ta, tb, tbh, to, p, grid, st);  \
+  }
   if constexpr (kGrouped) {
     FP8SM_CASE(kRow)
   } else {
@@ -719,6 +984,27 @@ bool out_map(CUtensorMap* m, void* out, int64_t rows, int64_t N, int out_f32,
                    2, out, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B, err);
 }
 
+// A operand map: 128-row boxes (one CTA's rows) in both modes.
+bool a_map(CUtensorMap* m, const void* a, int64_t rows, int64_t K, std::string* err) {
+  uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(rows)};
+  uint64_t strides[1] = {static_cast<uint64_t>(K)};
+  uint32_t box[2] = {BK, BM};
+  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a, dims, strides, box,
+                   CU_TENSOR_MAP_SWIZZLE_128B, err);
+}
+
+// Whether to run a problem on CTA pairs (256-row items, cta_group::2).
+// Measured on B200: the pair kernel halves B traffic per CTA but adds a
+// cross-SM handshake per accumulator hand-off; it is not faster for any
+// recipe here (2x slower for the blockwise recipes, whose hand-off is per
+// K block), so single CTAs are used.  Kept selectable for tuning.
+// FP8SM_CTA_PAIRS=1 selects the pair kernel (read per call; for tuning and
+// for the tests that keep it covered).
+bool use_pair(int64_t M) {
+  const char* e = std::getenv("FP8SM_CTA_PAIRS");
+  return e != nullptr && e[0] == '1' && M > BM;
+}
+
 }  // namespace
 
 cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
@@ -738,20 +1024,19 @@ cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
           static_cast<const uint16_t*>(bias), M, N, out);
     return cudaGetLastError();
   }
-  CUtensorMap ta, tb, to;
-  {
-    uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
-    uint64_t strides[1] = {static_cast<uint64_t>(K)};
-    uint32_t box[2] = {BK, BM};
-    if (!make_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a, dims, strides, box,
-                   CU_TENSOR_MAP_SWIZZLE_128B, ctx.err))
-      return cudaErrorInvalidValue;
-  }
+  const bool pair = use_pair(M);
+  const uint32_t b_rows = pair ? Cfg<true>::kBRows : Cfg<false>::kBRows;
+  CUtensorMap ta, tb, tbh, to;
+  if (!a_map(&ta, a, M, K, ctx.err)) return cudaErrorInvalidValue;
   {
     uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N)};
     uint64_t strides[1] = {static_cast<uint64_t>(K)};
-    uint32_t box[2] = {BK, BN};
+    uint32_t box[2] = {BK, b_rows};
     if (!make_tmap(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, b, dims, strides, box,
+                   CU_TENSOR_MAP_SWIZZLE_128B, ctx.err))
+      return cudaErrorInvalidValue;
+    uint32_t box_half[2] = {BK, b_rows / 2};
+    if (!make_tmap(&tbh, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, b, dims, strides, box_half,
                    CU_TENSOR_MAP_SWIZZLE_128B, ctx.err))
       return cudaErrorInvalidValue;
   }
@@ -766,13 +1051,27 @@ cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
   p.out = out;
   p.offs = nullptr;
   p.E = 0;
+  const int64_t tile_m = pair ? 2 * BM : BM;
   p.n_tiles = static_cast<int32_t>((N + BN - 1) / BN);
-  p.m_tiles = static_cast<int32_t>((M + BM - 1) / BM);
+  p.m_tiles = static_cast<int32_t>((M + tile_m - 1) / tile_m);
   p.k_blocks = static_cast<int32_t>((K + BK - 1) / BK);
   p.status = ctx.status;
   const int64_t tiles = static_cast<int64_t>(p.n_tiles) * p.m_tiles;
-  const unsigned grid = static_cast<unsigned>(tiles < ctx.num_sms ? tiles : ctx.num_sms);
-  return dispatch<false>(recipe, out_f32, ta, tb, to, p, grid, ctx.stream);
+  const int64_t G = pair ? ctx.num_sms / 2 : ctx.num_sms;  // CTAs or CTA pairs
+  p.split_start = tiles;
+  p.total_items = tiles;
+  const bool blockwise = recipe == kBlock128 || recipe == kBlock1;
+  if (!blockwise) {
+    const int64_t waves = (tiles + G - 1) / G;
+    const int64_t last = tiles - (waves - 1) * G;  // tiles in the last wave
+    if (2 * last <= G) {
+      p.split_start = (waves - 1) * G;
+      p.total_items = p.split_start + 2 * last;
+    }
+  }
+  const int64_t units = p.total_items < G ? p.total_items : G;
+  const unsigned grid = static_cast<unsigned>(pair ? 2 * units : units);
+  return dispatch<false>(recipe, out_f32, pair, ta, tb, tbh, to, p, grid, ctx.stream);
 }
 
 cudaError_t launch_grouped_scaled_mm(const void* a, const void* b,
@@ -781,31 +1080,20 @@ cudaError_t launch_grouped_scaled_mm(const void* a, const void* b,
                                      const float* sb, const int32_t* offs,
                                      int out_f32, void* out,
                                      const LaunchCtx& ctx) {
-  if (M_total == 0 || N == 0) {
-    // Nothing to write; offs still has to end at 0, which the caller's
-    // host-side checks cannot see.  A one-CTA launch would only validate.
-    if (M_total == 0 && N == 0) return cudaSuccess;
-  }
-  if (K == 0 || M_total == 0 || N == 0) {
-    if (M_total == 0 || N == 0) return cudaSuccess;
+  if (M_total == 0 || N == 0) return cudaSuccess;
+  if (K == 0)
     return launch_scaled_mm(nullptr, nullptr, M_total, N, 0, nullptr, nullptr,
                             1, nullptr, out_f32, out, ctx);
-  }
+  const bool pair = use_pair(M_total);
+  const uint32_t b_rows = pair ? Cfg<true>::kBRows : Cfg<false>::kBRows;
   CUtensorMap ta, tb, to;
-  {
-    uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M_total)};
-    uint64_t strides[1] = {static_cast<uint64_t>(K)};
-    uint32_t box[2] = {BK, BM};
-    if (!make_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a, dims, strides, box,
-                   CU_TENSOR_MAP_SWIZZLE_128B, ctx.err))
-      return cudaErrorInvalidValue;
-  }
+  if (!a_map(&ta, a, M_total, K, ctx.err)) return cudaErrorInvalidValue;
   {
     uint64_t dims[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N),
                         static_cast<uint64_t>(E)};
     uint64_t strides[2] = {static_cast<uint64_t>(K),
                            static_cast<uint64_t>(N) * static_cast<uint64_t>(K)};
-    uint32_t box[3] = {BK, BN, 1};
+    uint32_t box[3] = {BK, b_rows, 1};
     if (!make_tmap(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, b, dims, strides, box,
                    CU_TENSOR_MAP_SWIZZLE_128B, ctx.err))
       return cudaErrorInvalidValue;
@@ -827,8 +1115,10 @@ cudaError_t launch_grouped_scaled_mm(const void* a, const void* b,
   p.m_tiles = 0;
   p.k_blocks = static_cast<int32_t>((K + BK - 1) / BK);
   p.status = ctx.status;
-  return dispatch<true>(1, out_f32, ta, tb, to, p,
-                        static_cast<unsigned>(ctx.num_sms), ctx.stream);
+  p.split_start = INT64_MAX;
+  p.total_items = 0;
+  const unsigned grid = static_cast<unsigned>(pair ? (ctx.num_sms / 2) * 2 : ctx.num_sms);
+  return dispatch<true>(1, out_f32, pair, ta, tb, tb, to, p, grid, ctx.stream);
 }
 
 cudaError_t launch_timeout_probe(uint32_t limit_us, const LaunchCtx& ctx) {

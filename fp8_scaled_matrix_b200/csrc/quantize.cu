@@ -114,6 +114,44 @@ __global__ void __launch_bounds__(256) quant_row_kernel(
   }
 }
 
+// One CTA per row (rows up to 16384 columns): thread t holds 16 consecutive
+// elements (two 16-byte loads, one 16-byte store); warp amax -> shared
+// memory -> block amax.  Many small CTAs keep enough loads in flight and let
+// the stores of finishing CTAs overlap the loads of new ones.
+__global__ void __launch_bounds__(1024) quant_row_cta_kernel(
+    const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+    uint8_t* __restrict__ q, float* __restrict__ scales) {
+  __shared__ float warp_amax[32];
+  const int64_t row = blockIdx.x;
+  const int t = threadIdx.x;
+  const int nvec = static_cast<int>(cols >> 3);
+  const uint4* xr = reinterpret_cast<const uint4*>(x + row * ld);
+  const int i0 = 2 * t;
+  const bool v0 = i0 < nvec, v1 = i0 + 1 < nvec;
+  uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+  if (v0) a = ld_stream(xr + i0);
+  if (v1) b = ld_stream(xr + i0 + 1);
+  float m = amax8(b, amax8(a, 0.0f));  // zero padding does not change the max
+  m = warp_max(m);
+  if ((t & 31) == 0) warp_amax[t >> 5] = m;
+  __syncthreads();
+  const int nw = static_cast<int>(blockDim.x >> 5);
+  float bm = warp_amax[0];
+  for (int i = 1; i < nw; ++i) bm = fmaxf(bm, warp_amax[i]);
+  const ScalePair sp = scales_from_amax(bm);
+  if (t == 0) scales[row] = sp.s;
+  uint8_t* qr = q + row * cols + static_cast<int64_t>(i0) * 8;
+  // 16-byte stores need cols % 16 == 0 (row starts 16-byte aligned);
+  // otherwise two 8-byte stores.
+  if (v1 && (cols & 15) == 0) {
+    const uint2 lo = cast8(a, sp.inv), hi = cast8(b, sp.inv);
+    *reinterpret_cast<uint4*>(qr) = make_uint4(lo.x, lo.y, hi.x, hi.y);
+  } else {
+    if (v0) *reinterpret_cast<uint2*>(qr) = cast8(a, sp.inv);
+    if (v1) *reinterpret_cast<uint2*>(qr + 8) = cast8(b, sp.inv);
+  }
+}
+
 // Rows longer than 256*16 elements: amax pass, then a second read (served
 // from L2 for the row just read) for the cast.
 __global__ void __launch_bounds__(256) quant_row_long_kernel(
@@ -342,7 +380,12 @@ cudaError_t launch_quantize(const void* xv, int64_t rows, int64_t cols,
     if (rows == 0) return cudaSuccess;
     const unsigned grid = static_cast<unsigned>((rows + 7) / 8);
     const int64_t nvec = cols / 8;
-    if (nvec <= 32)
+    if (nvec >= 64 && nvec <= 2048) {
+      // one CTA per row, 16 elements per thread
+      const int64_t threads = ((nvec + 1) / 2 + 31) / 32 * 32;
+      quant_row_cta_kernel<<<static_cast<unsigned>(rows), static_cast<unsigned>(threads), 0,
+                             st>>>(x, rows, cols, ld, q, scales);
+    } else if (nvec <= 32)
       quant_row_kernel<1><<<grid, 256, 0, st>>>(x, rows, cols, ld, q, scales);
     else if (nvec <= 64)
       quant_row_kernel<2><<<grid, 256, 0, st>>>(x, rows, cols, ld, q, scales);

@@ -46,6 +46,7 @@ CASES = [
     ("row", 300, 272, 528, True),
     ("row", 129, 512, 4096, True),
     ("row", 2048, 4096, 256, False),         # 256 tiles > SM count: persistent loop
+    ("row", 4096, 4096, 256, True),          # 512 tiles: last wave split into 128-wide items
     ("row", 7, 48, 32, True),
     ("1x128_128x128", 260, 400, 384, False),
     ("1x128_128x128", 128, 256, 128, True),
@@ -130,3 +131,17 @@ def test_end_to_end_full_size_sampled(idx, shape_index):
     err = got - exact
     sqnr = 10 * np.log10((exact ** 2).sum() / (err ** 2).sum())
     assert sqnr >= 20.0, sqnr
+
+
+@pytest.mark.parametrize("recipe,M,N,K,bias", [
+    ("row", 300, 272, 528, True),
+    ("row", 4096, 4096, 256, False),
+    ("1x128_128x128", 1100, 2304, 1024, False),
+    ("1x128_128x1", 130, 528, 256, False),
+    ("tensor", 256, 256, 256, False),
+])
+def test_gemm_parity_cta_pairs(recipe, M, N, K, bias, monkeypatch):
+    """The CTA-pair kernel (cta_group::2, 256-row items), selected with
+    FP8SM_CTA_PAIRS=1, against the oracle."""
+    monkeypatch.setenv("FP8SM_CTA_PAIRS", "1")
+    test_gemm_parity(recipe, M, N, K, bias, torch.float32)
