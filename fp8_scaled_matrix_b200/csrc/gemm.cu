@@ -13,22 +13,27 @@
 //   warp 0      TMA producer: A (128 x 128 B) and B (256 x 128 B) tiles into
 //               a 4-stage shared-memory ring (128-byte swizzle)
 //   warp 1      TMEM owner + MMA issuer: one thread issues
-//               tcgen05.mma.kind::f8f6f4 (M=128, N=256, K=32) x 4 per stage
-//               into fp32 TMEM accumulators; tcgen05.commit frees stages
-//   warps 2-3   idle after the prologue (warp 2 validates offs)
+//               tcgen05.mma.kind::f8f6f4 into fp32 TMEM accumulators;
+//               tcgen05.commit frees stages and hands accumulators over
+//   warp 2      blockwise: scale producer (cp.async ring of per-K-block row
+//               and column scales, kSclSlots K blocks ahead); grouped:
+//               validates offs in the prologue
+//   warp 3      idle after the prologue
 //   warps 4-11  epilogue: warp w reads TMEM lanes 32*(w%4).. (the hardware's
 //               lane quarter) and columns 128*((w-4)/4).. of each tile
 // The blockwise kernels move registers from warpgroup 0 to the epilogue
 // warpgroups (setmaxnreg) so each epilogue thread can hold its 128 fp32
 // accumulators plus 64 freshly loaded TMEM values.
 // TMEM holds two 256-column fp32 buffers.  Tensorwise / rowwise: each buffer
-// is one whole tile's accumulator, so the epilogue of tile i overlaps the
-// MMAs of tile i+1.  Blockwise: each 128-wide K block is accumulated into a
-// buffer on its own (no carry-in), and the epilogue warps promote it --
-// acc += partial * sA[m,kb] * sB[.,kb] -- into fp32 registers while the tensor
-// core fills the other buffer.  Results are scaled, biased, rounded to bf16
-// (or kept fp32), staged in shared memory and written by TMA stores (the
-// grouped kernel masks rows past its group with plain 16-byte stores).
+// is one whole tile's accumulator (M=128, N=256, K=32 MMAs), so the epilogue
+// of tile i overlaps the MMAs of tile i+1.  Blockwise: each 128-wide K block
+// is accumulated into a buffer on its own (no carry-in), as two N=128 halves
+// with separate hand-back barriers; the four epilogue warps of a half promote
+// it -- acc += partial * sA[m,kb] * sB[.,kb] -- into fp32 registers while the
+// tensor core fills the other half and the other buffer.  Results are scaled,
+// biased, rounded to bf16 (or kept fp32), staged in shared memory and written
+// by TMA stores (the grouped kernel masks rows past its group with plain
+// 16-byte stores).
 //
 // Every wait is bounded (one second); a wait that gives up records
 // FP8_ERR_TIMEOUT in the device status word, the CTA drains its in-flight
@@ -64,10 +69,12 @@ static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsAtLaunch,
               "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;  // two 256-column fp32 buffers
 constexpr uint32_t kEpiBuf = 32 * 64;  // 32 rows x 64 bytes, 64-byte swizzle
-constexpr int kScaleAhead = 4;         // K blocks of scales fetched ahead
-constexpr int kRingAhead = 3;          // 128x1: K blocks of scales in the smem ring
-constexpr int kSbSlot = 128 + 32;      // 128x1 ring slot: column + row scales
-constexpr uint32_t kSbBuf = kRingAhead * kSbSlot * 4;  // per-warp 128x1 scale ring
+// Blockwise scale ring: one slot per K block, filled ahead by warp 2 with
+// cp.async: [128 row scales sA[kb, m0..] | column scales: sB[kb, nb0],
+// sB[kb, nb0 + 1] (1x128_128x128) or sB[kb, n0 .. n0 + 255] (1x128_128x1)].
+constexpr int kSclSlots = 8;
+constexpr int kSclSlotFloats = 128 + 256;
+constexpr uint32_t kSclBytes = kSclSlots * kSclSlotFloats * 4;
 
 // Shared-memory layout.  Single-CTA tiles are 128 x 256: each stage holds
 // A (128 rows) and B (256 rows) of a 128-byte K slice.  CTA-pair tiles are
@@ -84,10 +91,11 @@ struct Cfg {
   static constexpr uint32_t kOffA = 0;
   static constexpr uint32_t kOffB = kOffA + kStages * kAStage;
   static constexpr uint32_t kOffEpi = kOffB + kStages * kBStage;
-  static constexpr uint32_t kOffSb = kOffEpi + kEpiWarps * kEpiBuf;
-  static constexpr uint32_t kOffBar = kOffSb + kEpiWarps * kSbBuf;
-  // barriers: full[kStages], empty[kStages], acc_full[2], acc_empty[2], drain
-  static constexpr uint32_t kNumBars = 2 * kStages + 5;
+  static constexpr uint32_t kOffScl = kOffEpi + kEpiWarps * kEpiBuf;
+  static constexpr uint32_t kOffBar = kOffScl + kSclBytes;
+  // barriers: full[kStages], empty[kStages], acc_full[2], acc_empty[4], drain,
+  // scale ring sfull[kSclSlots], sempty[kSclSlots]
+  static constexpr uint32_t kNumBars = 2 * kStages + 7 + 2 * kSclSlots;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
   static constexpr uint32_t kSmemUsed = kOffMisc + 16;
   static constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // + alignment slack
@@ -318,8 +326,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* full = bars;
   uint64_t* empty = bars + C::kStages;
   uint64_t* acc_full = bars + 2 * C::kStages;
-  uint64_t* acc_empty = bars + 2 * C::kStages + 2;
-  uint64_t* drain = bars + 2 * C::kStages + 4;
+  uint64_t* acc_empty = bars + 2 * C::kStages + 2;  // [2] dense; [2 * buf + half] blockwise
+  uint64_t* drain = bars + 2 * C::kStages + 6;
+  uint64_t* sfull = bars + 2 * C::kStages + 7;
+  uint64_t* sempty = sfull + kSclSlots;
+  float* scl = reinterpret_cast<float*>(smem + C::kOffScl);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   uint32_t* tmem_slot = misc + 0;
   volatile uint32_t* abort_flag = misc + 1;
@@ -333,12 +344,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&acc_full[i], 1);
-      // pair: the leader's barrier collects both CTAs' epilogue warps
-      mbar_init(&acc_empty[i], kPair ? 2 * kEpiWarps : kEpiWarps);
-    }
+    for (int i = 0; i < 2; ++i) mbar_init(&acc_full[i], 1);
+    // pair: the leader's barrier collects both CTAs' epilogue warps
+    // dense: every epilogue warp hands a buffer back (pair: from both CTAs);
+    // blockwise: the four warps that read a half hand that half back
+    for (int i = 0; i < 4; ++i)
+      mbar_init(&acc_empty[i], kBlockwise ? kEpiWarps / 2 : (kPair ? 2 * kEpiWarps : kEpiWarps));
     mbar_init(drain, 1);
+    for (int i = 0; i < kSclSlots; ++i) {
+      mbar_init(&sfull[i], 32);            // one cp.async arrival per lane of warp 2
+      mbar_init(&sempty[i], kEpiWarps);
+    }
     *abort_flag = 0u;
     fence_barrier_init();
     prefetch_tmap(&tm_a);
@@ -409,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
         const TileCoord c = tile_coord<kGrouped, kTM>(t, p, cur);
         for (int32_t kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status,
+          if (!mbar_wait<kPair>(&empty[stage], phase ^ 1u, abort_flag, p.status,
                          SITE_PRODUCER_EMPTY, kWaitLimitNs)) {
             ok = false;
             break;
@@ -450,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t first = issued > C::kStages ? issued - C::kStages : 0;
         for (uint64_t i = first; i < issued; ++i) {
           uint32_t dummy_abort = 0;
-          mbar_wait(&full[i % C::kStages], static_cast<uint32_t>((i / C::kStages) & 1u),
+          mbar_wait<kPair>(&full[i % C::kStages], static_cast<uint32_t>((i / C::kStages) & 1u),
                     &dummy_abort, nullptr, SITE_TEARDOWN, 10000000ull);
         }
       }
@@ -464,64 +480,100 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t stage = 0, phase = 0;
       uint32_t acc = 0, acc_phase = 0;
       bool ok = true;
-      for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
-        const uint32_t idesc = (!kGrouped && t >= p.split_start) ? idesc_half : idesc_full;
-        if constexpr (!kBlockwise) {
-          if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag, p.status,
-                         SITE_MMA_ACC_EMPTY, kWaitLimitNs)) {
+      // The issue loop is kept lean (the single issuing thread, not the
+      // tensor core, is the limit at 4 MMAs per stage): no fence after a
+      // stage wait (TMA writes and MMA reads are both async-proxy, ordered by
+      // the barrier), and the next stage's barrier is peeked while this
+      // stage's MMAs go out.
+      bool ready = mbar_test_wait<kPair>(&full[stage], phase);
+      if constexpr (!kBlockwise) {
+        for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
+          const uint32_t idesc = (!kGrouped && t >= p.split_start) ? idesc_half : idesc_full;
+          if (!mbar_wait<kPair>(&acc_empty[acc], acc_phase ^ 1u, abort_flag, p.status,
+                                SITE_MMA_ACC_EMPTY, kWaitLimitNs)) {
             ok = false;
             break;
           }
           tc_fence_after_sync();
-        }
-        for (int32_t kb = 0; kb < KB; ++kb) {
-          if constexpr (kBlockwise) {
-            if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag,
-                           p.status, SITE_MMA_ACC_EMPTY, kWaitLimitNs)) {
+          for (int32_t kb = 0; kb < KB; ++kb) {
+            if (!ready && !mbar_wait<kPair>(&full[stage], phase, abort_flag, p.status,
+                                            SITE_MMA_FULL, kWaitLimitNs)) {
               ok = false;
               break;
             }
-            tc_fence_after_sync();
-          }
-          if (!mbar_wait(&full[stage], phase, abort_flag, p.status,
-                         SITE_MMA_FULL, kWaitLimitNs)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after_sync();
-          const uint32_t d = tmem_base + acc * BN;
-          const uint64_t da =
-              smem_desc_k_sw128(smem_u32(smem + C::kOffA + stage * C::kAStage));
-          const uint64_t db =
-              smem_desc_k_sw128(smem_u32(smem + C::kOffB + stage * C::kBStage));
+            const uint32_t cur = stage;
+            if (++stage == C::kStages) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            ready = mbar_test_wait<kPair>(&full[stage], phase);  // peek at the next stage
+            const uint32_t d = tmem_base + acc * BN;
+            const uint64_t da = smem_desc_k_sw128(smem_u32(smem + C::kOffA + cur * C::kAStage));
+            const uint64_t db = smem_desc_k_sw128(smem_u32(smem + C::kOffB + cur * C::kBStage));
 #pragma unroll
-          for (int k = 0; k < BK / UMMA_K; ++k) {
-            const uint32_t accumulate =
-                kBlockwise ? (k > 0) : ((kb > 0) || (k > 0));
-            if constexpr (kPair)
-              mma_e4m3_pair(d, da + (k * UMMA_K) / 16, db + (k * UMMA_K) / 16, idesc,
-                            accumulate);
-            else
-              mma_e4m3(d, da + (k * UMMA_K) / 16, db + (k * UMMA_K) / 16, idesc,
-                       accumulate);
+            for (int k = 0; k < BK / UMMA_K; ++k) {
+              const uint32_t accumulate = (kb > 0) || (k > 0);
+              if constexpr (kPair)
+                mma_e4m3_pair(d, da + (k * UMMA_K) / 16, db + (k * UMMA_K) / 16, idesc,
+                              accumulate);
+              else
+                mma_e4m3(d, da + (k * UMMA_K) / 16, db + (k * UMMA_K) / 16, idesc,
+                         accumulate);
+            }
+            if constexpr (kPair) mma_commit_pair(&empty[cur], 0x3);
+            else mma_commit(&empty[cur]);
           }
-          if constexpr (kPair) mma_commit_pair(&empty[stage], 0x3);
-          else mma_commit(&empty[stage]);
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
-          if constexpr (kBlockwise) {
+          if (ok) {
             if constexpr (kPair) mma_commit_pair(&acc_full[acc], 0x3);
             else mma_commit(&acc_full[acc]);
             acc ^= 1u;
             if (acc == 0) acc_phase ^= 1u;
           }
         }
-        if constexpr (!kBlockwise) {
-          if (ok) {
-            if constexpr (kPair) mma_commit_pair(&acc_full[acc], 0x3);
-            else mma_commit(&acc_full[acc]);
+      } else {
+        // Blockwise: each K block goes into a buffer on its own, as two
+        // N = 128 halves (TMEM columns [0,128) and [128,256) of the buffer,
+        // B rows 0-127 and 128-255 of the stage).  Each half has its own
+        // hand-back barrier, so the half-0 MMAs of K block kb+2 start as soon
+        // as the epilogue has read half 0 of K block kb, while it still reads
+        // half 1.  Signals: acc_full[buf] = half 0 done; empty[stage] = half 1
+        // done (and the stage free).
+        const uint32_t idesc = idesc_e4m3_f32(BM, BN / 2);
+        constexpr uint64_t kBHalfDesc = (BN / 2) * BK / 16;  // descriptor units (16 B)
+        for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
+          for (int32_t kb = 0; kb < KB && ok; ++kb) {
+            uint32_t cur = 0;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              if (!mbar_wait<kPair>(&acc_empty[2 * acc + h], acc_phase ^ 1u, abort_flag,
+                                    p.status, SITE_MMA_ACC_EMPTY, kWaitLimitNs)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after_sync();
+              if (h == 0) {
+                if (!ready && !mbar_wait<kPair>(&full[stage], phase, abort_flag, p.status,
+                                                SITE_MMA_FULL, kWaitLimitNs)) {
+                  ok = false;
+                  break;
+                }
+                cur = stage;
+                if (++stage == C::kStages) {
+                  stage = 0;
+                  phase ^= 1u;
+                }
+                ready = mbar_test_wait<kPair>(&full[stage], phase);
+              }
+              const uint32_t d = tmem_base + acc * BN + h * (BN / 2);
+              const uint64_t da = smem_desc_k_sw128(smem_u32(smem + C::kOffA + cur * C::kAStage));
+              const uint64_t db = smem_desc_k_sw128(smem_u32(smem + C::kOffB + cur * C::kBStage)) +
+                                  h * kBHalfDesc;
+#pragma unroll
+              for (int k = 0; k < BK / UMMA_K; ++k)
+                mma_e4m3(d, da + (k * UMMA_K) / 16, db + (k * UMMA_K) / 16, idesc, k > 0);
+              if (h == 0) mma_commit(&acc_full[acc]);
+              else mma_commit(&empty[cur]);
+            }
             acc ^= 1u;
             if (acc == 0) acc_phase ^= 1u;
           }
@@ -534,7 +586,59 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (lane == 0) {
       uint32_t dummy_abort = 0;
-      mbar_wait(drain, 0, &dummy_abort, p.status, SITE_TEARDOWN, kWaitLimitNs);
+      mbar_wait<kPair>(drain, 0, &dummy_abort, p.status, SITE_TEARDOWN, kWaitLimitNs);
+    }
+   } else if (warp == 2) {
+    // ----------------------------------------------- blockwise scale producer
+    // Fills the scale ring kSclSlots K blocks ahead of the epilogue, so the
+    // epilogue never waits on a global load: row scales of the tile's 128
+    // rows (lane l: rows 4l .. 4l+3) and its column scales, by cp.async with
+    // zero fill past the matrix; each lane's copies then arrive on the slot's
+    // sfull barrier.
+    if constexpr (kBlockwise) {
+      const int64_t NB = (p.N + 127) / 128;
+      uint32_t slot = 0, sphase = 0;
+      bool ok = true;
+      GroupCursor cur;
+      for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
+        const TileCoord c = tile_coord<kGrouped, kTM>(t, p, cur);
+        for (int32_t kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&sempty[slot], sphase ^ 1u, abort_flag, p.status, SITE_SCALE_EMPTY,
+                         kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          float* dst = scl + slot * kSclSlotFloats;
+          const float* sa_k = p.sa + static_cast<int64_t>(kb) * p.M;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int64_t r = static_cast<int64_t>(c.m0) + 4 * lane + i;
+            cp_async_4(dst + 4 * lane + i, r < p.M ? sa_k + r : p.sa, r < p.M ? 4u : 0u);
+          }
+          if constexpr (kRecipe == kBlock128) {
+            if (lane < 2) {
+              const bool v = static_cast<int64_t>(c.n0) + 128 * lane < p.N;
+              cp_async_4(dst + 128 + lane,
+                         v ? p.sb + static_cast<int64_t>(kb) * NB + c.n0 / 128 + lane : p.sb,
+                         v ? 4u : 0u);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const int64_t n = static_cast<int64_t>(c.n0) + 8 * lane + 4 * i;
+              cp_async_16(dst + 128 + 8 * lane + 4 * i,
+                          n < p.N ? p.sb + static_cast<int64_t>(kb) * p.N + n : p.sb,
+                          n < p.N ? 16u : 0u);
+            }
+          }
+          cp_async_mbar_arrive_noinc(&sfull[slot]);
+          if (++slot == kSclSlots) {
+            slot = 0;
+            sphase ^= 1u;
+          }
+        }
+      }
+      cp_async_wait_all();  // nothing lands in shared memory after the CTA exits
     }
    }
   } else {
@@ -544,17 +648,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t q = warp & 3u;          // TMEM lane quarter of this warp
     const uint32_t half = ew >> 2;         // which 128 columns of the tile
     uint8_t* ebuf = smem + C::kOffEpi + ew * kEpiBuf;
-    float* sbbuf = reinterpret_cast<float*>(smem + C::kOffSb + ew * kSbBuf);
     const uint32_t lane_base = (q * 32u) << 16;
     GroupCursor cur;
     if constexpr (kGrouped) cur.init(p.offs, kTM);
     uint32_t acc = 0, acc_phase = 0;
+    uint32_t ep_stage = 0, ep_phase = 0;  // blockwise: mirrors the MMA's stage sequence
+    uint32_t sslot = 0, sphase = 0;       // blockwise: scale ring position
+    // blockwise: wait until the scale ring holds this K block's scales
+    auto wait_scales = [&]() -> const float* {
+      if (!mbar_wait(&sfull[sslot], sphase, abort_flag, p.status, SITE_EPI_SCALE_FULL,
+                     kWaitLimitNs))
+        return nullptr;
+      return scl + sslot * kSclSlotFloats;
+    };
+    // ... and hand the slot back once every lane has read it
+    auto release_scales = [&]() {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sempty[sslot]);
+      if (++sslot == kSclSlots) {
+        sslot = 0;
+        sphase ^= 1u;
+      }
+    };
     bool ok = true;
     // TMEM buffers are handed back on the leader's barrier (pair: from both CTAs)
     const uint32_t acc_empty_addr0 =
         kPair ? mapa_shared(smem_u32(&acc_empty[0]), 0) : smem_u32(&acc_empty[0]);
     const uint32_t acc_empty_addr1 =
         kPair ? mapa_shared(smem_u32(&acc_empty[1]), 0) : smem_u32(&acc_empty[1]);
+    // Single CTA: a CTA-scope arrive.  Pair: the leader's barrier, at cluster
+    // scope (a cluster-scope release costs a fence, so it is used only there).
+    auto release_acc = [&](uint32_t a) {
+      if constexpr (kPair) mbar_arrive_cluster(a ? acc_empty_addr1 : acc_empty_addr0);
+      else mbar_arrive(&acc_empty[a]);
+    };
     for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
       const TileCoord c = tile_coord<kGrouped, kTM>(t, p, cur);
       const int32_t cta_m0 = c.m0 + static_cast<int32_t>(rank) * BM;  // this CTA's rows
@@ -564,7 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t row0 = cta_m0 + static_cast<int32_t>(q * 32);
 
       if constexpr (!kBlockwise) {
-        if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status,
+        if (!mbar_wait<kPair>(&acc_full[acc], acc_phase, abort_flag, p.status,
                        SITE_EPI_ACC_FULL, kWaitLimitNs)) {
           ok = false;
           break;
@@ -573,7 +700,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (c.half_n && half == 1) {
           // 128-wide item: this warp's columns are not part of it
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(acc ? acc_empty_addr1 : acc_empty_addr0);
+          if (lane == 0) release_acc(acc);
           acc ^= 1u;
           if (acc == 0) acc_phase ^= 1u;
           continue;
@@ -591,7 +718,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (cc == 3) {
             tc_fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(acc ? acc_empty_addr1 : acc_empty_addr0);
+            if (lane == 0) release_acc(acc);
           }
           const int64_t n = ncol0 + cc * 32;
           float bias[32];
@@ -616,65 +743,58 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (acc == 0) acc_phase ^= 1u;
       } else if constexpr (kRecipe == kBlock128) {
         // 1x128_128x128: promote each K block's partial product into
-        // registers; the scale product sA[m,kb] * sB[n/128,kb] is one value
-        // per thread per K block.
-        float2 accr[64];
+        // registers.  Warp (q, half) reads TMEM lanes 32q.. and the 128
+        // columns of its half of the tile, so the four warps of half 0 work on
+        // K block kb while the tensor core still writes half 1 of it, and the
+        // two warps that share a scheduler are a half apart.  Its scale
+        // product sA[m,kb] * sB[nb,kb] is one value per thread per K block.
+        // The four 32-column TMEM loads are pipelined against the FMAs.
+        float2 accr[64];  // accr[16 c + i]: columns 32c + 2i, 32c + 2i + 1
 #pragma unroll
         for (int i = 0; i < 64; ++i) accr[i] = make_float2(0.0f, 0.0f);
-        const int64_t NB = (p.N + 127) / 128;
-        const int64_t nb = ncol0 / 128;  // 128-column block of this warp
-        const bool nb_ok = ncol0 < p.N;
-        // scales fetched kScaleAhead K blocks ahead through a shift register
-        auto load_sa = [&](int32_t k) -> float {
-          return (row_ok && k < KB) ? __ldg(p.sa + static_cast<int64_t>(k) * p.M + row) : 0.0f;
-        };
-        auto load_sb = [&](int32_t k) -> float {
-          return (nb_ok && k < KB) ? __ldg(p.sb + static_cast<int64_t>(k) * NB + nb) : 0.0f;
-        };
-        float sa_r[kScaleAhead], sb_r[kScaleAhead];
-#pragma unroll
-        for (int i = 0; i < kScaleAhead; ++i) {
-          sa_r[i] = load_sa(i);
-          sb_r[i] = load_sb(i);
-        }
-        for (int32_t kb = 0; kb < KB; ++kb) {
-          const float f = sa_r[0] * sb_r[0];
-#pragma unroll
-          for (int i = 0; i + 1 < kScaleAhead; ++i) {
-            sa_r[i] = sa_r[i + 1];
-            sb_r[i] = sb_r[i + 1];
-          }
-          sa_r[kScaleAhead - 1] = load_sa(kb + kScaleAhead);
-          sb_r[kScaleAhead - 1] = load_sb(kb + kScaleAhead);
-          if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status,
-                         SITE_EPI_ACC_FULL, kWaitLimitNs)) {
+        for (int32_t kb = 0; kb < KB && ok; ++kb) {
+          const float* sl = wait_scales();
+          if (sl == nullptr) {
             ok = false;
             break;
+          }
+          const float f = sl[q * 32 + lane] * sl[128 + half];
+          release_scales();
+          // half 0: its own commit; half 1: the stage's release
+          const bool got =
+              half == 0 ? mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status,
+                                    SITE_EPI_ACC_FULL, kWaitLimitNs)
+                        : mbar_wait(&empty[ep_stage], ep_phase, abort_flag, p.status,
+                                    SITE_EPI_ACC_FULL, kWaitLimitNs);
+          if (!got) {
+            ok = false;
+            break;
+          }
+          if (++ep_stage == C::kStages) {
+            ep_stage = 0;
+            ep_phase ^= 1u;
           }
           tc_fence_after_sync();
           const uint32_t tcol = tmem_base + lane_base + acc * BN + half * 128;
           const float2 f2 = make_float2(f, f);
+          uint32_t r[2][32];
+          tmem_ld_32x32b_x32(tcol, r[0]);
+          tmem_ld_wait();
 #pragma unroll
-          for (int hc = 0; hc < 2; ++hc) {
-            uint32_t r[2][32];
-            tmem_ld_32x32b_x32(tcol + hc * 64, r[0]);
-            tmem_ld_32x32b_x32(tcol + hc * 64 + 32, r[1]);
-            tmem_ld_wait();
-            if (hc == 1) {
-              // every TMEM read of this buffer is done: hand it back
+          for (int c = 0; c < 4; ++c) {
+            if (c < 3) tmem_ld_32x32b_x32(tcol + 32 * (c + 1), r[(c + 1) & 1]);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float2 pv = make_float2(__uint_as_float(r[c & 1][2 * i]),
+                                            __uint_as_float(r[c & 1][2 * i + 1]));
+              accr[16 * c + i] = fma2(pv, f2, accr[16 * c + i]);
+            }
+            if (c < 3) tmem_ld_wait();
+            if (c == 2) {
+              // every TMEM read of this half is done: hand it back
               tc_fence_before_sync();
               __syncwarp();
-              if (lane == 0) mbar_arrive_cluster(acc ? acc_empty_addr1 : acc_empty_addr0);
-            }
-#pragma unroll
-            for (int c2 = 0; c2 < 2; ++c2) {
-              const int base = hc * 32 + c2 * 16;  // float2 index of column hc*64 + c2*32
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const float2 pv = make_float2(__uint_as_float(r[c2][2 * i]),
-                                              __uint_as_float(r[c2][2 * i + 1]));
-                accr[base + i] = fma2(pv, f2, accr[base + i]);
-              }
+              if (lane == 0) mbar_arrive(&acc_empty[2 * acc + half]);
             }
           }
           acc ^= 1u;
@@ -696,77 +816,76 @@ __global__ void __launch_bounds__(kThreads, 1)
                                           c.row_end, p.out, p.N, lane);
         }
       } else {
-        // 1x128_128x1: a different scale for every output column.  TMEM is
-        // read in the 16x256b shape: thread t holds rows g, g+8, g+16, g+24
-        // (g = t/4) of the warp's lane quarter and, in every 8-column group j,
-        // the two columns 8j + 2c, 8j + 2c + 1 (c = t%4): 4 rows x 32 columns.
-        // So it needs 4 row scales and 32 column scales per K block (8-byte
-        // shared loads that 8 lanes share) instead of 128 column scales.
-        // Scales come through a per-warp cp.async ring, kRingAhead K blocks
-        // ahead: slot = [128 column scales | 32 row scales].
+        // 1x128_128x1: a different scale for every output column.  Same
+        // warp/half split as 1x128_128x128.  TMEM is read in the 16x256b
+        // shape: thread t holds rows g, g+8, g+16, g+24 (g = t/4) of the
+        // warp's lane quarter and, in every 8-column group j, the two columns
+        // 8j + 2c, 8j + 2c + 1 (c = t%4).  So it needs 4 row scales and 32
+        // column scales per K block (8-byte shared loads that 8 lanes share)
+        // instead of 128 column scales; both come from the scale ring.  The
+        // four loads (64 columns x 16 lanes each) are pipelined against the
+        // FMAs.
         const uint32_t g = lane >> 2, cq = lane & 3;
         float2 accr[64];  // accr[ri * 16 + j]: row g + 8 ri, columns 8j + 2cq + {0,1}
 #pragma unroll
         for (int i = 0; i < 64; ++i) accr[i] = make_float2(0.0f, 0.0f);
-        const int64_t ncol_lane = ncol0 + 4 * lane;
-        auto fetch = [&](int32_t k) {
-          float* dst = sbbuf + (k % kRingAhead) * kSbSlot;
-          const bool vc = k < KB && ncol_lane < p.N;
-          cp_async_16(dst + 4 * lane,
-                      vc ? p.sb + static_cast<int64_t>(k) * p.N + ncol_lane : p.sb,
-                      vc ? 16u : 0u);
-          const bool vr = k < KB && row_ok;
-          cp_async_4(dst + 128 + lane, vr ? p.sa + static_cast<int64_t>(k) * p.M + row : p.sa,
-                     vr ? 4u : 0u);
-          cp_async_commit();
-        };
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < kRingAhead - 1; ++i) fetch(i);
-        for (int32_t kb = 0; kb < KB; ++kb) {
-          __syncwarp();  // every lane is done reading the slot refilled next
-          fetch(kb + kRingAhead - 1);
-          cp_async_wait<kRingAhead - 1>();  // this K block's slot has landed
-          __syncwarp();
-          if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status,
-                         SITE_EPI_ACC_FULL, kWaitLimitNs)) {
+        for (int32_t kb = 0; kb < KB && ok; ++kb) {
+          const float* sl = wait_scales();
+          if (sl == nullptr) {
             ok = false;
             break;
           }
+          const float sa_i[4] = {sl[q * 32 + g], sl[q * 32 + g + 8], sl[q * 32 + g + 16],
+                                 sl[q * 32 + g + 24]};
+          const float* sbl = sl + 128 + half * 128;  // this warp's 128 column scales
+          const bool got =
+              half == 0 ? mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status,
+                                    SITE_EPI_ACC_FULL, kWaitLimitNs)
+                        : mbar_wait(&empty[ep_stage], ep_phase, abort_flag, p.status,
+                                    SITE_EPI_ACC_FULL, kWaitLimitNs);
+          if (!got) {
+            ok = false;
+            break;
+          }
+          if (++ep_stage == C::kStages) {
+            ep_stage = 0;
+            ep_phase ^= 1u;
+          }
           tc_fence_after_sync();
-          const float* sl = sbbuf + (kb % kRingAhead) * kSbSlot;
-          const float sa_i[4] = {sl[128 + g], sl[128 + g + 8], sl[128 + g + 16],
-                                 sl[128 + g + 24]};
           const uint32_t tcol = tmem_base + lane_base + acc * BN + half * 128;
+          // chunk c: 64-column block cb = c / 2, TMEM lanes 16 lh .. (lh = c % 2)
+          uint32_t r[2][32];
+          tmem_ld_16x256b_x8(tcol, r[0]);
+          tmem_ld_wait();
 #pragma unroll
-          for (int lh = 0; lh < 2; ++lh) {  // TMEM lanes 0-15 / 16-31 of the quarter
-            uint32_t r[2][32];
-            tmem_ld_16x256b_x8(tcol + ((16u * lh) << 16), r[0]);
-            tmem_ld_16x256b_x8(tcol + ((16u * lh) << 16) + 64, r[1]);
-            tmem_ld_wait();
-            if (lh == 1) {
-              tc_fence_before_sync();
-              __syncwarp();
-              if (lane == 0) mbar_arrive_cluster(acc ? acc_empty_addr1 : acc_empty_addr0);
+          for (int c = 0; c < 4; ++c) {
+            if (c < 3) {
+              const int cn = c + 1;
+              tmem_ld_16x256b_x8(tcol + (((cn & 1) * 16u) << 16) + (cn >> 1) * 64,
+                                 r[cn & 1]);
             }
+            const int cb = c >> 1, lh = c & 1;
             const float2 sat = make_float2(sa_i[2 * lh], sa_i[2 * lh]);
             const float2 sab = make_float2(sa_i[2 * lh + 1], sa_i[2 * lh + 1]);
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-#pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                const int j = ch * 8 + k;
-                const float2 s2 = *reinterpret_cast<const float2*>(sl + 8 * j + 2 * cq);
-                const float2 pt = make_float2(__uint_as_float(r[ch][4 * k]),
-                                              __uint_as_float(r[ch][4 * k + 1]));
-                const float2 pb = make_float2(__uint_as_float(r[ch][4 * k + 2]),
-                                              __uint_as_float(r[ch][4 * k + 3]));
-                accr[(2 * lh) * 16 + j] = fma2(mul2(pt, s2), sat, accr[(2 * lh) * 16 + j]);
-                accr[(2 * lh + 1) * 16 + j] =
-                    fma2(mul2(pb, s2), sab, accr[(2 * lh + 1) * 16 + j]);
-              }
+            for (int k = 0; k < 8; ++k) {
+              const int j = cb * 8 + k;
+              const float2 s2 = *reinterpret_cast<const float2*>(sbl + 8 * j + 2 * cq);
+              const float2 pt = make_float2(__uint_as_float(r[c & 1][4 * k]),
+                                            __uint_as_float(r[c & 1][4 * k + 1]));
+              const float2 pb = make_float2(__uint_as_float(r[c & 1][4 * k + 2]),
+                                            __uint_as_float(r[c & 1][4 * k + 3]));
+              accr[(2 * lh) * 16 + j] = fma2(mul2(pt, s2), sat, accr[(2 * lh) * 16 + j]);
+              accr[(2 * lh + 1) * 16 + j] = fma2(mul2(pb, s2), sab, accr[(2 * lh + 1) * 16 + j]);
+            }
+            if (c < 3) tmem_ld_wait();
+            if (c == 2) {
+              tc_fence_before_sync();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&acc_empty[2 * acc + half]);
             }
           }
+          release_scales();
           acc ^= 1u;
           if (acc == 0) acc_phase ^= 1u;
         }
@@ -916,36 +1035,42 @@ template <int kRecipe, bool kOutF32, bool kGrouped, bool kPair>
 cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb,
                           const CUtensorMap& tbh, const CUtensorMap& to,
                           const GemmParams& p, unsigned grid, cudaStream_t st) {
-  using C = Cfg<kPair>;
-  static bool configured = false;
-  auto kern = fp8_gemm_kernel<kRecipe, kOutF32, kGrouped, kPair>;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(
-        kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    if (kRecipe == kBlock128 || kRecipe == kBlock1) {
-      // setmaxnreg.inc would wait forever if the launch allocation were
-      // smaller than the split assumes: check before the first launch.
-      cudaFuncAttributes attr;
-      e = cudaFuncGetAttributes(&attr, kern);
+  constexpr bool kBlockwise = kRecipe == kBlock128 || kRecipe == kBlock1;
+  if constexpr (kPair && kBlockwise) {
+    return cudaErrorInvalidValue;  // CTA pairs serve the dense recipes only
+  } else {
+    using C = Cfg<kPair>;
+    static bool configured = false;
+    auto kern = fp8_gemm_kernel<kRecipe, kOutF32, kGrouped, kPair>;
+    if (!configured) {
+      cudaError_t e = cudaFuncSetAttribute(
+          kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
       if (e != cudaSuccess) return e;
-      if (attr.numRegs < static_cast<int>(kRegsAtLaunch)) return cudaErrorInvalidConfiguration;
+      if (kBlockwise) {
+        // setmaxnreg.inc would wait forever if the launch allocation were
+        // smaller than the split assumes: check before the first launch.
+        cudaFuncAttributes attr;
+        e = cudaFuncGetAttributes(&attr, kern);
+        if (e != cudaSuccess) return e;
+        if (attr.numRegs < static_cast<int>(kRegsAtLaunch)) return cudaErrorInvalidConfiguration;
+      }
+      configured = true;
     }
-    configured = true;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    // single-CTA kernels are launched without a cluster attribute
+    cfg.attrs = attr;
+    cfg.numAttrs = kPair ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, ta, tb, tbh, to, p);
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = C::kSmemBytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kPair ? 2 : 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, ta, tb, tbh, to, p);
 }
 
 template <bool kGrouped>
@@ -998,11 +1123,12 @@ bool a_map(CUtensorMap* m, const void* a, int64_t rows, int64_t K, std::string* 
 // cross-SM handshake per accumulator hand-off; it is not faster for any
 // recipe here (2x slower for the blockwise recipes, whose hand-off is per
 // K block), so single CTAs are used.  Kept selectable for tuning.
-// FP8SM_CTA_PAIRS=1 selects the pair kernel (read per call; for tuning and
-// for the tests that keep it covered).
-bool use_pair(int64_t M) {
+// FP8SM_CTA_PAIRS=1 selects the pair kernel for the dense recipes (read per
+// call; for tuning and for the tests that keep it covered).  The blockwise
+// kernels always run on single CTAs.
+bool use_pair(int64_t M, int recipe) {
   const char* e = std::getenv("FP8SM_CTA_PAIRS");
-  return e != nullptr && e[0] == '1' && M > BM;
+  return e != nullptr && e[0] == '1' && M > BM && recipe != kBlock128 && recipe != kBlock1;
 }
 
 }  // namespace
@@ -1024,7 +1150,7 @@ cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
           static_cast<const uint16_t*>(bias), M, N, out);
     return cudaGetLastError();
   }
-  const bool pair = use_pair(M);
+  const bool pair = use_pair(M, recipe);
   const uint32_t b_rows = pair ? Cfg<true>::kBRows : Cfg<false>::kBRows;
   CUtensorMap ta, tb, tbh, to;
   if (!a_map(&ta, a, M, K, ctx.err)) return cudaErrorInvalidValue;
@@ -1084,7 +1210,7 @@ cudaError_t launch_grouped_scaled_mm(const void* a, const void* b,
   if (K == 0)
     return launch_scaled_mm(nullptr, nullptr, M_total, N, 0, nullptr, nullptr,
                             1, nullptr, out_f32, out, ctx);
-  const bool pair = use_pair(M_total);
+  const bool pair = use_pair(M_total, kRow);
   const uint32_t b_rows = pair ? Cfg<true>::kBRows : Cfg<false>::kBRows;
   CUtensorMap ta, tb, to;
   if (!a_map(&ta, a, M_total, K, ctx.err)) return cudaErrorInvalidValue;

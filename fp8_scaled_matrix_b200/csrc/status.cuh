@@ -25,6 +25,8 @@ enum : uint32_t {
   SITE_GRID_BARRIER = 6,
   SITE_OFFS = 7,
   SITE_PROBE = 8,
+  SITE_SCALE_EMPTY = 9,
+  SITE_EPI_SCALE_FULL = 10,
 };
 
 // Wait limit for every pipeline wait inside the GEMM / quantize kernels.
