@@ -27,10 +27,9 @@
 // TMEM holds two 256-column fp32 buffers.  Tensorwise / rowwise: each buffer
 // is one whole tile's accumulator (M=128, N=256, K=32 MMAs), so the epilogue
 // of tile i overlaps the MMAs of tile i+1.  Blockwise: each 128-wide K block
-// is accumulated into a buffer on its own (no carry-in), as two N=128 halves
-// with separate hand-back barriers; the four epilogue warps of a half promote
-// it -- acc += partial * sA[m,kb] * sB[.,kb] -- into fp32 registers while the
-// tensor core fills the other half and the other buffer.  Results are scaled,
+// is accumulated into a buffer on its own (no carry-in), and the epilogue
+// warps promote it -- acc += partial * sA[m,kb] * sB[.,kb] -- into fp32
+// registers while the tensor core fills the other buffer.  Results are scaled,
 // biased, rounded to bf16 (or kept fp32), staged in shared memory and written
 // by TMA stores (the grouped kernel masks rows past its group with plain
 // 16-byte stores).
@@ -93,9 +92,9 @@ struct Cfg {
   static constexpr uint32_t kOffEpi = kOffB + kStages * kBStage;
   static constexpr uint32_t kOffScl = kOffEpi + kEpiWarps * kEpiBuf;
   static constexpr uint32_t kOffBar = kOffScl + kSclBytes;
-  // barriers: full[kStages], empty[kStages], acc_full[2], acc_empty[4], drain,
+  // barriers: full[kStages], empty[kStages], acc_full[2], acc_empty[2], drain,
   // scale ring sfull[kSclSlots], sempty[kSclSlots]
-  static constexpr uint32_t kNumBars = 2 * kStages + 7 + 2 * kSclSlots;
+  static constexpr uint32_t kNumBars = 2 * kStages + 5 + 2 * kSclSlots;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
   static constexpr uint32_t kSmemUsed = kOffMisc + 16;
   static constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // + alignment slack
@@ -326,9 +325,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* full = bars;
   uint64_t* empty = bars + C::kStages;
   uint64_t* acc_full = bars + 2 * C::kStages;
-  uint64_t* acc_empty = bars + 2 * C::kStages + 2;  // [2] dense; [2 * buf + half] blockwise
-  uint64_t* drain = bars + 2 * C::kStages + 6;
-  uint64_t* sfull = bars + 2 * C::kStages + 7;
+  uint64_t* acc_empty = bars + 2 * C::kStages + 2;
+  uint64_t* drain = bars + 2 * C::kStages + 4;
+  uint64_t* sfull = bars + 2 * C::kStages + 5;
   uint64_t* sempty = sfull + kSclSlots;
   float* scl = reinterpret_cast<float*>(smem + C::kOffScl);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
@@ -346,10 +345,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) mbar_init(&acc_full[i], 1);
     // pair: the leader's barrier collects both CTAs' epilogue warps
-    // dense: every epilogue warp hands a buffer back (pair: from both CTAs);
-    // blockwise: the four warps that read a half hand that half back
-    for (int i = 0; i < 4; ++i)
-      mbar_init(&acc_empty[i], kBlockwise ? kEpiWarps / 2 : (kPair ? 2 * kEpiWarps : kEpiWarps));
+    // every epilogue warp hands a buffer back (pair: from both CTAs)
+    for (int i = 0; i < 2; ++i) mbar_init(&acc_empty[i], kPair ? 2 * kEpiWarps : kEpiWarps);
     mbar_init(drain, 1);
     for (int i = 0; i < kSclSlots; ++i) {
       mbar_init(&sfull[i], 32);            // one cp.async arrival per lane of warp 2
@@ -531,49 +528,38 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else {
-        // Blockwise: each K block goes into a buffer on its own, as two
-        // N = 128 halves (TMEM columns [0,128) and [128,256) of the buffer,
-        // B rows 0-127 and 128-255 of the stage).  Each half has its own
-        // hand-back barrier, so the half-0 MMAs of K block kb+2 start as soon
-        // as the epilogue has read half 0 of K block kb, while it still reads
-        // half 1.  Signals: acc_full[buf] = half 0 done; empty[stage] = half 1
-        // done (and the stage free).
-        const uint32_t idesc = idesc_e4m3_f32(BM, BN / 2);
-        constexpr uint64_t kBHalfDesc = (BN / 2) * BK / 16;  // descriptor units (16 B)
+        // Blockwise: each K block goes into a TMEM buffer on its own (no
+        // carry-in).  The stage's release commit also tells the epilogue that
+        // the K block's partial product is complete.  (Splitting a K block
+        // into two N = 128 halves with their own hand-back costs twice the
+        // MMA instructions and commits, and the single issuing thread, not
+        // the tensor core, then sets the pace.)
         for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
-          for (int32_t kb = 0; kb < KB && ok; ++kb) {
-            uint32_t cur = 0;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              if (!mbar_wait<kPair>(&acc_empty[2 * acc + h], acc_phase ^ 1u, abort_flag,
-                                    p.status, SITE_MMA_ACC_EMPTY, kWaitLimitNs)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after_sync();
-              if (h == 0) {
-                if (!ready && !mbar_wait<kPair>(&full[stage], phase, abort_flag, p.status,
-                                                SITE_MMA_FULL, kWaitLimitNs)) {
-                  ok = false;
-                  break;
-                }
-                cur = stage;
-                if (++stage == C::kStages) {
-                  stage = 0;
-                  phase ^= 1u;
-                }
-                ready = mbar_test_wait<kPair>(&full[stage], phase);
-              }
-              const uint32_t d = tmem_base + acc * BN + h * (BN / 2);
-              const uint64_t da = smem_desc_k_sw128(smem_u32(smem + C::kOffA + cur * C::kAStage));
-              const uint64_t db = smem_desc_k_sw128(smem_u32(smem + C::kOffB + cur * C::kBStage)) +
-                                  h * kBHalfDesc;
-#pragma unroll
-              for (int k = 0; k < BK / UMMA_K; ++k)
-                mma_e4m3(d, da + (k * UMMA_K) / 16, db + (k * UMMA_K) / 16, idesc, k > 0);
-              if (h == 0) mma_commit(&acc_full[acc]);
-              else mma_commit(&empty[cur]);
+          for (int32_t kb = 0; kb < KB; ++kb) {
+            if (!mbar_wait<kPair>(&acc_empty[acc], acc_phase ^ 1u, abort_flag, p.status,
+                                  SITE_MMA_ACC_EMPTY, kWaitLimitNs)) {
+              ok = false;
+              break;
             }
+            tc_fence_after_sync();
+            if (!ready && !mbar_wait<kPair>(&full[stage], phase, abort_flag, p.status,
+                                            SITE_MMA_FULL, kWaitLimitNs)) {
+              ok = false;
+              break;
+            }
+            const uint32_t cur = stage;
+            if (++stage == C::kStages) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            ready = mbar_test_wait<kPair>(&full[stage], phase);
+            const uint32_t d = tmem_base + acc * BN;
+            const uint64_t da = smem_desc_k_sw128(smem_u32(smem + C::kOffA + cur * C::kAStage));
+            const uint64_t db = smem_desc_k_sw128(smem_u32(smem + C::kOffB + cur * C::kBStage));
+#pragma unroll
+            for (int k = 0; k < BK / UMMA_K; ++k)
+              mma_e4m3(d, da + (k * UMMA_K) / 16, db + (k * UMMA_K) / 16, idesc_full, k > 0);
+            mma_commit(&empty[cur]);
             acc ^= 1u;
             if (acc == 0) acc_phase ^= 1u;
           }
@@ -744,11 +730,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if constexpr (kRecipe == kBlock128) {
         // 1x128_128x128: promote each K block's partial product into
         // registers.  Warp (q, half) reads TMEM lanes 32q.. and the 128
-        // columns of its half of the tile, so the four warps of half 0 work on
-        // K block kb while the tensor core still writes half 1 of it, and the
-        // two warps that share a scheduler are a half apart.  Its scale
-        // product sA[m,kb] * sB[nb,kb] is one value per thread per K block.
-        // The four 32-column TMEM loads are pipelined against the FMAs.
+        // columns of its half of the tile (one 128-column block of B), so its
+        // scale product sA[m,kb] * sB[nb,kb] is one value per thread per K
+        // block.  The four 32-column TMEM loads are pipelined against the
+        // FMAs: the next chunk is in flight while this one is promoted.
         float2 accr[64];  // accr[16 c + i]: columns 32c + 2i, 32c + 2i + 1
 #pragma unroll
         for (int i = 0; i < 64; ++i) accr[i] = make_float2(0.0f, 0.0f);
@@ -760,13 +745,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const float f = sl[q * 32 + lane] * sl[128 + half];
           release_scales();
-          // half 0: its own commit; half 1: the stage's release
-          const bool got =
-              half == 0 ? mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status,
-                                    SITE_EPI_ACC_FULL, kWaitLimitNs)
-                        : mbar_wait(&empty[ep_stage], ep_phase, abort_flag, p.status,
-                                    SITE_EPI_ACC_FULL, kWaitLimitNs);
-          if (!got) {
+          // the K block's MMAs are done when its stage is released
+          if (!mbar_wait(&empty[ep_stage], ep_phase, abort_flag, p.status, SITE_EPI_ACC_FULL,
+                         kWaitLimitNs)) {
             ok = false;
             break;
           }
@@ -794,7 +775,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               // every TMEM read of this half is done: hand it back
               tc_fence_before_sync();
               __syncwarp();
-              if (lane == 0) mbar_arrive(&acc_empty[2 * acc + half]);
+              if (lane == 0) mbar_arrive(&acc_empty[acc]);
             }
           }
           acc ^= 1u;
@@ -817,7 +798,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         // 1x128_128x1: a different scale for every output column.  Same
-        // warp/half split as 1x128_128x128.  TMEM is read in the 16x256b
+        // warp/column split as 1x128_128x128.  TMEM is read in the 16x256b
         // shape: thread t holds rows g, g+8, g+16, g+24 (g = t/4) of the
         // warp's lane quarter and, in every 8-column group j, the two columns
         // 8j + 2c, 8j + 2c + 1 (c = t%4).  So it needs 4 row scales and 32
@@ -838,12 +819,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float sa_i[4] = {sl[q * 32 + g], sl[q * 32 + g + 8], sl[q * 32 + g + 16],
                                  sl[q * 32 + g + 24]};
           const float* sbl = sl + 128 + half * 128;  // this warp's 128 column scales
-          const bool got =
-              half == 0 ? mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status,
-                                    SITE_EPI_ACC_FULL, kWaitLimitNs)
-                        : mbar_wait(&empty[ep_stage], ep_phase, abort_flag, p.status,
-                                    SITE_EPI_ACC_FULL, kWaitLimitNs);
-          if (!got) {
+          // the K block's MMAs are done when its stage is released
+          if (!mbar_wait(&empty[ep_stage], ep_phase, abort_flag, p.status, SITE_EPI_ACC_FULL,
+                         kWaitLimitNs)) {
             ok = false;
             break;
           }
@@ -882,7 +860,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (c == 2) {
               tc_fence_before_sync();
               __syncwarp();
-              if (lane == 0) mbar_arrive(&acc_empty[2 * acc + half]);
+              if (lane == 0) mbar_arrive(&acc_empty[acc]);
             }
           }
           release_scales();
