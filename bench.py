@@ -101,6 +101,24 @@ def recorded_traffic(workload: str):
     return None
 
 
+# ------------------------------------------------------- multi-rank plumbing
+
+def max_over_ranks(x: float, dev) -> float:
+    """The largest of every rank's `x` (a device time): one all-reduce(MAX)
+    over the default process group, or `x` itself on a single rank."""
+    dist = torch.distributed
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job throughput: every rank's work over the slowest rank's time."""
+    return flops_per_rank * world / (ms * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -232,16 +250,36 @@ class Step:
         return 3 * n + 4 * (self.sa.numel() + self.sb.numel())
 
 
+def capture(fn, pool=None):
+    """Record the launches `fn` makes (through the C ABI) into a CUDA graph."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, pool=pool):
+        fn()
+    return g
+
+
 def run_ours(args, wl, dev, rank, world):
     torch.cuda.set_device(dev)
     st = Step(wl, dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
         st.quantize()
         st.gemm()
     torch.cuda.synchronize()
     st.f.check_device_status()
+    quantize, gemm = st.quantize, st.gemm
+    if args.graphs:
+        # The step's launches replayed from CUDA graphs: the same kernels on
+        # the same buffers, without the host's per-call cost between them.
+        gq = capture(st.quantize)
+        gg = capture(st.gemm, pool=gq.pool())
+        quantize, gemm = gq.replay, gg.replay
+        for _ in range(3):
+            quantize()
+            gemm()
+        torch.cuda.synchronize()
+        st.f.check_device_status()
+    stream = torch.cuda.current_stream()
 
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
@@ -254,9 +292,9 @@ def run_ours(args, wl, dev, rank, world):
     for i in range(K):
         flush.zero_()  # evict L2 (outside the step's events)
         ev[i][0].record(stream)
-        st.quantize()
+        quantize()
         ev[i][1].record(stream)
-        st.gemm()
+        gemm()
         ev[i][2].record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -266,11 +304,7 @@ def run_ours(args, wl, dev, rank, world):
     q_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
     g_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
     step_ms = [q + g for q, g in zip(q_ms, g_ms)]
-    total_ms = float(np.sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(float(np.sum(step_ms)), dev)
     res = {
         "total_ms": total_ms,
         "q_ms": float(np.mean(q_ms)), "g_ms": float(np.mean(g_ms)),
@@ -319,11 +353,7 @@ def run_e2e(args, wl, dev, world):
         one()
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / steps
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, dev)
     h2d = ha.numel() * 2 + hb.numel() * 2 + (0 if hbias is None else hbias.numel() * 2)
     d2h = hout.numel() * 2
     return {"ms": ms, "h2d": h2d, "d2h": d2h, "steps": steps}
@@ -383,7 +413,7 @@ def baseline_rows(wl, target_s: float = 12.0) -> int:
 
 # ------------------------------------------------------------------ main
 
-def main():
+def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
@@ -391,11 +421,14 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--graphs", type=int, default=1, choices=[0, 1],
+                    help="replay the step's launches from CUDA graphs (1, default) or "
+                         "call the API per launch (0)")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=0,
                     help="output rows for the CPU oracle sample (0: about 12 s of work)")
-    args = ap.parse_args()
+    args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
@@ -452,7 +485,7 @@ def main():
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     K = args.steps
     ms_per_step = res["total_ms"] / K
-    value = wl.flops * world / (ms_per_step * 1e-3) / 1e12
+    value = job_tflops(wl.flops, world, ms_per_step)
     gemm_tflops = wl.flops / (res["g_ms"] * 1e-3) / 1e12
     quant_gbs = res["quant_bytes"] / (res["q_ms"] * 1e-3) / 1e9
     line = {
@@ -475,6 +508,8 @@ def main():
             "out_dtype": "bf16", "l2": "flushed between steps (256 MB write, outside the step events)",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "step": "quantize A || quantize B (two streams), then scaled GEMM",
+            "launch": ("CUDA graphs of the step's C-ABI launches" if args.graphs
+                       else "one C-ABI call per launch"),
         },
         "roofline": {
             "bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak,
@@ -494,7 +529,7 @@ def main():
     }
     if "e2e" in res:
         e = res["e2e"]
-        line["e2e"] = {"value": wl.flops * world / (e["ms"] * 1e-3) / 1e12, "unit": "TFLOP/s",
+        line["e2e"] = {"value": job_tflops(wl.flops, world, e["ms"]), "unit": "TFLOP/s",
                        "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
                        "ms_per_step": e["ms"], "steps": e["steps"]}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
