@@ -578,7 +578,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ----------------------------------------------- blockwise scale producer
     // Fills the scale ring kSclSlots K blocks ahead of the epilogue, so the
     // epilogue never waits on a global load: row scales of the tile's 128
-    // rows (lane l: rows 4l .. 4l+3) and its column scales, by cp.async with
+    // rows (lane l: rows l, l+32, l+64, l+96 -- coalesced reads,
+    // conflict-free writes) and its column scales, by cp.async with
     // zero fill past the matrix; each lane's copies then arrive on the slot's
     // sfull barrier.
     if constexpr (kBlockwise) {
@@ -598,8 +599,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float* sa_k = p.sa + static_cast<int64_t>(kb) * p.M;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const int64_t r = static_cast<int64_t>(c.m0) + 4 * lane + i;
-            cp_async_4(dst + 4 * lane + i, r < p.M ? sa_k + r : p.sa, r < p.M ? 4u : 0u);
+            const int64_t r = static_cast<int64_t>(c.m0) + lane + 32 * i;
+            cp_async_4(dst + lane + 32 * i, r < p.M ? sa_k + r : p.sa, r < p.M ? 4u : 0u);
           }
           if constexpr (kRecipe == kBlock128) {
             if (lane < 2) {
@@ -727,14 +728,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         acc ^= 1u;
         if (acc == 0) acc_phase ^= 1u;
-      } else if constexpr (kRecipe == kBlock128) {
-        // 1x128_128x128: promote each K block's partial product into
-        // registers.  Warp (q, half) reads TMEM lanes 32q.. and the 128
-        // columns of its half of the tile (one 128-column block of B), so its
-        // scale product sA[m,kb] * sB[nb,kb] is one value per thread per K
-        // block.  The four 32-column TMEM loads are pipelined against the
-        // FMAs: the next chunk is in flight while this one is promoted.
-        float2 accr[64];  // accr[16 c + i]: columns 32c + 2i, 32c + 2i + 1
+      } else {
+        // Blockwise: promote each K block's partial product into registers.
+        // Warp (q, half) reads TMEM lanes 32q.. and the 128 columns of its
+        // half of the tile, in the 32x32b shape (thread = one row, 32
+        // consecutive columns per load; the 16x256b shape reads TMEM at about
+        // a third of the rate).  The four 32-column loads are pipelined
+        // against the FMAs: the next chunk is in flight while this one is
+        // promoted.
+        //   1x128_128x128: the half is one 128-column block of B, so the
+        //     scale product sA[m,kb] * sB[nb,kb] is one value per thread.
+        //   1x128_128x1: acc += (P * sB[n,kb]) * sA[m,kb] per column, the
+        //     column scales read from the scale ring (the same address in
+        //     every lane: a broadcast).
+        float2 accr[64];  // accr[16 c + i]: columns 32c + 2i, 32c + 2i + 1 of the warp's 128
 #pragma unroll
         for (int i = 0; i < 64; ++i) accr[i] = make_float2(0.0f, 0.0f);
         for (int32_t kb = 0; kb < KB && ok; ++kb) {
@@ -743,8 +750,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          const float f = sl[q * 32 + lane] * sl[128 + half];
-          release_scales();
+          const float sa = sl[q * 32 + lane];
+          float f = sa;
+          if constexpr (kRecipe == kBlock128) {
+            f = sa * sl[128 + half];
+            release_scales();
+          }
+          const float2 f2 = make_float2(f, f);
+          const float* sbl = sl + 128 + half * 128;  // 1x128_128x1: this warp's column scales
           // the K block's MMAs are done when its stage is released
           if (!mbar_wait(&empty[ep_stage], ep_phase, abort_flag, p.status, SITE_EPI_ACC_FULL,
                          kWaitLimitNs)) {
@@ -757,7 +770,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after_sync();
           const uint32_t tcol = tmem_base + lane_base + acc * BN + half * 128;
-          const float2 f2 = make_float2(f, f);
           uint32_t r[2][32];
           tmem_ld_32x32b_x32(tcol, r[0]);
           tmem_ld_wait();
@@ -766,18 +778,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (c < 3) tmem_ld_32x32b_x32(tcol + 32 * (c + 1), r[(c + 1) & 1]);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const float2 pv = make_float2(__uint_as_float(r[c & 1][2 * i]),
-                                            __uint_as_float(r[c & 1][2 * i + 1]));
+              float2 pv = make_float2(__uint_as_float(r[c & 1][2 * i]),
+                                      __uint_as_float(r[c & 1][2 * i + 1]));
+              if constexpr (kRecipe == kBlock1)
+                pv = mul2(pv, *reinterpret_cast<const float2*>(sbl + 32 * c + 2 * i));
               accr[16 * c + i] = fma2(pv, f2, accr[16 * c + i]);
             }
             if (c < 3) tmem_ld_wait();
             if (c == 2) {
-              // every TMEM read of this half is done: hand it back
+              // every TMEM read of this buffer is done: hand it back
               tc_fence_before_sync();
               __syncwarp();
               if (lane == 0) mbar_arrive(&acc_empty[acc]);
             }
           }
+          if constexpr (kRecipe == kBlock1) release_scales();
           acc ^= 1u;
           if (acc == 0) acc_phase ^= 1u;
         }
@@ -795,138 +810,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           store_cols32<kOutF32, kGrouped>(ebuf, v, &tm_out,
                                           static_cast<int32_t>(n), row0,
                                           c.row_end, p.out, p.N, lane);
-        }
-      } else {
-        // 1x128_128x1: a different scale for every output column.  Same
-        // warp/column split as 1x128_128x128.  TMEM is read in the 16x256b
-        // shape: thread t holds rows g, g+8, g+16, g+24 (g = t/4) of the
-        // warp's lane quarter and, in every 8-column group j, the two columns
-        // 8j + 2c, 8j + 2c + 1 (c = t%4).  So it needs 4 row scales and 32
-        // column scales per K block (8-byte shared loads that 8 lanes share)
-        // instead of 128 column scales; both come from the scale ring.  The
-        // four loads (64 columns x 16 lanes each) are pipelined against the
-        // FMAs.
-        const uint32_t g = lane >> 2, cq = lane & 3;
-        float2 accr[64];  // accr[ri * 16 + j]: row g + 8 ri, columns 8j + 2cq + {0,1}
-#pragma unroll
-        for (int i = 0; i < 64; ++i) accr[i] = make_float2(0.0f, 0.0f);
-        for (int32_t kb = 0; kb < KB && ok; ++kb) {
-          const float* sl = wait_scales();
-          if (sl == nullptr) {
-            ok = false;
-            break;
-          }
-          const float sa_i[4] = {sl[q * 32 + g], sl[q * 32 + g + 8], sl[q * 32 + g + 16],
-                                 sl[q * 32 + g + 24]};
-          const float* sbl = sl + 128 + half * 128;  // this warp's 128 column scales
-          // the K block's MMAs are done when its stage is released
-          if (!mbar_wait(&empty[ep_stage], ep_phase, abort_flag, p.status, SITE_EPI_ACC_FULL,
-                         kWaitLimitNs)) {
-            ok = false;
-            break;
-          }
-          if (++ep_stage == C::kStages) {
-            ep_stage = 0;
-            ep_phase ^= 1u;
-          }
-          tc_fence_after_sync();
-          const uint32_t tcol = tmem_base + lane_base + acc * BN + half * 128;
-          // chunk c: 64-column block cb = c / 2, TMEM lanes 16 lh .. (lh = c % 2)
-          uint32_t r[2][32];
-          tmem_ld_16x256b_x8(tcol, r[0]);
-          tmem_ld_wait();
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            if (c < 3) {
-              const int cn = c + 1;
-              tmem_ld_16x256b_x8(tcol + (((cn & 1) * 16u) << 16) + (cn >> 1) * 64,
-                                 r[cn & 1]);
-            }
-            const int cb = c >> 1, lh = c & 1;
-            const float2 sat = make_float2(sa_i[2 * lh], sa_i[2 * lh]);
-            const float2 sab = make_float2(sa_i[2 * lh + 1], sa_i[2 * lh + 1]);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const int j = cb * 8 + k;
-              const float2 s2 = *reinterpret_cast<const float2*>(sbl + 8 * j + 2 * cq);
-              const float2 pt = make_float2(__uint_as_float(r[c & 1][4 * k]),
-                                            __uint_as_float(r[c & 1][4 * k + 1]));
-              const float2 pb = make_float2(__uint_as_float(r[c & 1][4 * k + 2]),
-                                            __uint_as_float(r[c & 1][4 * k + 3]));
-              accr[(2 * lh) * 16 + j] = fma2(mul2(pt, s2), sat, accr[(2 * lh) * 16 + j]);
-              accr[(2 * lh + 1) * 16 + j] = fma2(mul2(pb, s2), sab, accr[(2 * lh + 1) * 16 + j]);
-            }
-            if (c < 3) tmem_ld_wait();
-            if (c == 2) {
-              tc_fence_before_sync();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&acc_empty[acc]);
-            }
-          }
-          release_scales();
-          acc ^= 1u;
-          if (acc == 0) acc_phase ^= 1u;
-        }
-        if (!ok) break;
-        // Final store: per 32-column chunk cc (column groups j = 4cc..4cc+3),
-        // each thread writes its 4 rows x 4 column pairs into the warp's
-        // staging box (32 rows x 64 bytes, 64-byte swizzle), then the box is
-        // stored like the other recipes' (bf16: one box per chunk; fp32: two).
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int64_t n = ncol0 + cc * 32;
-          float bias2[4][2];
-#pragma unroll
-          for (int jj = 0; jj < 4; ++jj) {
-            const int64_t col = n + 8 * jj + 2 * cq;
-            if (p.bias != nullptr && col < p.N) {
-              const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(p.bias + col));
-              bias2[jj][0] = __uint_as_float(w << 16);
-              bias2[jj][1] = __uint_as_float(w & 0xFFFF0000u);
-            } else {
-              bias2[jj][0] = bias2[jj][1] = 0.0f;
-            }
-          }
-          constexpr int kBoxes = kOutF32 ? 2 : 1;   // 64-byte boxes per 32 columns
-#pragma unroll
-          for (int bx = 0; bx < kBoxes; ++bx) {
-            if constexpr (!kGrouped) {
-              if (lane == 0) bulk_wait_group_read0();
-              __syncwarp();
-            }
-#pragma unroll
-            for (int ri = 0; ri < 4; ++ri) {
-              const uint32_t rr = g + 8 * ri;  // row within the warp's 32
-#pragma unroll
-              for (int jj = 0; jj < 4; ++jj) {
-                const float2 a = accr[ri * 16 + cc * 4 + jj];
-                const float o0 = a.x + bias2[jj][0], o1 = a.y + bias2[jj][1];
-                if constexpr (!kOutF32) {
-                  // bf16: column 8jj + 2cq -> byte 16jj + 4cq of the 64-byte row
-                  const uint32_t slot = static_cast<uint32_t>(jj) ^ ((rr >> 1) & 3u);
-                  *reinterpret_cast<uint32_t*>(ebuf + rr * 64 + slot * 16 + 4 * cq) =
-                      pack_bf16x2(o0, o1);
-                } else {
-                  // fp32: box bx holds columns 16bx .. 16bx+15 -> jj in {2bx, 2bx+1}
-                  if ((jj >> 1) == bx) {
-                    const uint32_t cb = (8 * (jj & 1) + 2 * cq) * 4;  // byte within the row
-                    const uint32_t slot = (cb >> 4) ^ ((rr >> 1) & 3u);
-                    *reinterpret_cast<float2*>(ebuf + rr * 64 + slot * 16 + (cb & 15)) =
-                        make_float2(o0, o1);
-                  }
-                }
-              }
-            }
-            const int32_t col0 = static_cast<int32_t>(n) + (kOutF32 ? 16 * bx : 0);
-            if constexpr (!kGrouped) {
-              fence_proxy_async_smem();
-              __syncwarp();
-              if (lane == 0 && row0 < c.row_end && col0 < p.N) {
-                tma_store_2d(&tm_out, ebuf, col0, row0);
-                bulk_commit_group();
-              }
-            }
-          }
         }
       }
     }
