@@ -236,45 +236,48 @@ __global__ void __launch_bounds__(256) quant_1x128_kernel(
 }
 
 // ------------------------------------------------------------ 128x128
-// One CTA (256 threads) per 128x128 tile: thread t covers row t/2 and
-// 64 columns (8 x 16-byte loads held in registers).  Ragged last row block:
-// rows past the end take no part in the amax and are not written.
-__global__ void __launch_bounds__(256) quant_128x128_kernel(
+// One CTA (512 threads) per 128x128 tile: thread t covers the 16-byte chunk
+// t%16 of rows t/16 + 32 i (i < 4), so each warp-wide load reads two whole
+// 256-byte row segments (coalesced); the 4 chunks stay in registers.
+// Ragged last row block: rows past the end take no part in the amax and are
+// not written.
+constexpr int k128Threads = 512;
+__global__ void __launch_bounds__(k128Threads) quant_128x128_kernel(
     const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
     uint8_t* __restrict__ q, float* __restrict__ scales) {
-  __shared__ float warp_amax[8];
+  constexpr int kWarps = k128Threads / 32;
+  constexpr int kRowStep = k128Threads / 16;       // rows covered per load round
+  constexpr int kRounds = 128 / kRowStep;
+  __shared__ float warp_amax[kWarps];
   const int64_t RB = (rows + 127) >> 7;
   const int64_t rb = blockIdx.x % RB;
   const int64_t kb = blockIdx.x / RB;
   const int t = threadIdx.x;
-  const int64_t row = rb * 128 + (t >> 1);
-  const int64_t col = kb * 128 + (t & 1) * 64;
-  const bool ok = row < rows;
-  uint4 v[8];
+  const int64_t row0 = rb * 128 + (t >> 4);
+  const int64_t col = kb * 128 + (t & 15) * 8;
+  const uint16_t* xp = x + row0 * ld + col;
+  uint4 v[kRounds];
   float m = 0.0f;
-  if (ok) {
-    const uint4* p = reinterpret_cast<const uint4*>(x + row * ld + col);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = ld_stream(p + i);
+  for (int i = 0; i < kRounds; ++i)
+    v[i] = row0 + kRowStep * i < rows
+               ? ld_stream(reinterpret_cast<const uint4*>(xp + kRowStep * i * ld))
+               : make_uint4(0, 0, 0, 0);  // zero padding does not change the max
 #pragma unroll
-    for (int i = 0; i < 8; ++i) m = amax8(v[i], m);
-  }
+  for (int i = 0; i < kRounds; ++i) m = amax8(v[i], m);
   m = warp_max(m);
   if ((t & 31) == 0) warp_amax[t >> 5] = m;
   __syncthreads();
   float tm = warp_amax[0];
 #pragma unroll
-  for (int i = 1; i < 8; ++i) tm = fmaxf(tm, warp_amax[i]);
+  for (int i = 1; i < kWarps; ++i) tm = fmaxf(tm, warp_amax[i]);
   const ScalePair sp = scales_from_amax(tm);
   if (t == 0) scales[kb * RB + rb] = sp.s;
-  if (!ok) return;
-  uint4* qp = reinterpret_cast<uint4*>(q + row * cols + col);
+  uint8_t* qp = q + row0 * cols + col;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint2 lo = cast8(v[2 * i], sp.inv);
-    const uint2 hi = cast8(v[2 * i + 1], sp.inv);
-    qp[i] = make_uint4(lo.x, lo.y, hi.x, hi.y);
-  }
+  for (int i = 0; i < kRounds; ++i)
+    if (row0 + kRowStep * i < rows)
+      *reinterpret_cast<uint2*>(qp + kRowStep * i * cols) = cast8(v[i], sp.inv);
 }
 
 // ------------------------------------------------------------- tensor
@@ -411,7 +414,7 @@ cudaError_t launch_quantize(const void* xv, int64_t rows, int64_t cols,
   if (recipe == 3) {  // 128x128
     if (rows == 0 || cols == 0) return cudaSuccess;
     const int64_t tiles = ((rows + 127) / 128) * (cols / 128);
-    quant_128x128_kernel<<<static_cast<unsigned>(tiles), 256, 0, st>>>(
+    quant_128x128_kernel<<<static_cast<unsigned>(tiles), k128Threads, 0, st>>>(
         x, rows, cols, ld, q, scales);
     return cudaGetLastError();
   }
