@@ -6,6 +6,7 @@ statically so the .so needs nothing but the driver at load time.  No fast
 math: the quantizer's fp32 divisions and multiplies must stay IEEE.
 """
 import concurrent.futures as cf
+import fcntl
 import os
 import shutil
 import subprocess
@@ -40,12 +41,31 @@ def _deps():
     return files
 
 
+def _up_to_date() -> bool:
+    if not os.path.exists(LIB):
+        return False
+    newest = max(os.path.getmtime(f) for f in _deps())
+    return os.path.getmtime(LIB) >= newest
+
+
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    if not force and os.path.exists(LIB):
-        newest = max(os.path.getmtime(f) for f in _deps())
-        if os.path.getmtime(LIB) >= newest:
-            return LIB
+    """Compile the library if it is missing or older than its sources.
+    Several processes (one per GPU) may call this at once: an exclusive file
+    lock serialises them, and the ones that wait find the library built."""
+    if not force and _up_to_date():
+        return LIB
     os.makedirs(BUILD_DIR, exist_ok=True)
+    with open(os.path.join(BUILD_DIR, ".lock"), "w") as lock:
+        fcntl.flock(lock, fcntl.LOCK_EX)
+        try:
+            if not force and _up_to_date():
+                return LIB
+            return _build_locked(verbose_ptxas)
+        finally:
+            fcntl.flock(lock, fcntl.LOCK_UN)
+
+
+def _build_locked(verbose_ptxas: bool) -> str:
     objs = []
     cmds = []
     for src in SOURCES:
@@ -59,13 +79,14 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
             sys.stderr.write(r.stdout + r.stderr)
         if r.returncode != 0:
             raise RuntimeError("nvcc failed: " + " ".join(c))
-    link = [nvcc(), "-shared", "-o", LIB + ".tmp"] + objs + ARCH + [
+    tmp = f"{LIB}.tmp{os.getpid()}"
+    link = [nvcc(), "-shared", "-o", tmp] + objs + ARCH + [
         "-cudart", "static", "-Xcompiler", "-fPIC"]
     r = subprocess.run(link, capture_output=True, text=True)
     if r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)
         raise RuntimeError("link failed")
-    os.replace(LIB + ".tmp", LIB)
+    os.replace(tmp, LIB)
     return LIB
 
 
