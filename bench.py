@@ -48,6 +48,8 @@ WORKLOADS = {
     "blockwise_1x128_128x1": (3, 0),
     "blockwise_1x128_128x1_b": (3, 1),
     "grouped_e16": (4, 0),
+    "grad_input_1x128_128x128": (5, 0),
+    "grad_weight_1x128_128x1": (6, 0),
 }
 DEFAULT_WORKLOAD = "rowwise_4096"
 # Page 5's context numbers (TFLOP/s of torch._scaled_mm, hardware not stated)
@@ -57,7 +59,12 @@ PAGE_NUMBERS = {
 }
 OPERAND_GROUPS = {"tensor": ("tensor", "tensor"), "row": ("row", "row"),
                   "1x128_128x128": ("1x128", "128x128"),
-                  "1x128_128x1": ("1x128", "1x128"), "grouped": ("row", "row")}
+                  "1x128_128x1": ("1x128", "1x128"), "grouped": ("row", "row"),
+                  "grad_input": ("1x128", "128x128"), "grad_weight": ("1x128", "1x128")}
+# GEMM recipe of each workload recipe, and which operands are quantized
+# transposed (the training GEMMs contract along the stored rows)
+GEMM_RECIPE = {"grad_input": "1x128_128x128", "grad_weight": "1x128_128x1"}
+TRANSPOSED = {"grad_input": (False, True), "grad_weight": (True, True)}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_OVER_BF16 = 2.0   # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 L2_FLUSH_BYTES = 256 << 20
@@ -200,8 +207,10 @@ class Step:
             self.b = wl.b.to(dev)
             self.offs = None
         self.bias = None if wl.bias is None else wl.bias.to(dev)
-        rows_a, cols = self.a.shape
-        rows_b = self.b.shape[0]
+        self.t_a, self.t_b = TRANSPOSED.get(wl.recipe, (False, False))
+        # quantized operands: A (M, K), B (N, K) (grouped: (E N, K))
+        rows_a, rows_b = wl.M, self.b.shape[1] if self.t_b else self.b.shape[0]
+        cols = wl.K
         self.qa = torch.empty(rows_a, cols, dtype=torch.uint8, device=dev)
         self.qb = torch.empty(rows_b, cols, dtype=torch.uint8, device=dev)
         self.sa = torch.empty(max(fp8sm.scale_count(rows_a, cols, self.qa_recipe), 1),
@@ -225,10 +234,18 @@ class Step:
         self.ev_fork.record(main)
         self.side.wait_event(self.ev_fork)
         with torch.cuda.stream(self.side):
-            f.fp8_quantize(self.b, self.qb_recipe, out=self.qb, scales=self.sb,
-                           workspace=self.ws_b, stream=self.side)
-        f.fp8_quantize(self.a, self.qa_recipe, out=self.qa, scales=self.sa, workspace=self.ws,
-                       stream=main)
+            if self.t_b:
+                f.fp8_quantize_transposed(self.b, self.qb_recipe, out=self.qb, scales=self.sb,
+                                          stream=self.side)
+            else:
+                f.fp8_quantize(self.b, self.qb_recipe, out=self.qb, scales=self.sb,
+                               workspace=self.ws_b, stream=self.side)
+        if self.t_a:
+            f.fp8_quantize_transposed(self.a, self.qa_recipe, out=self.qa, scales=self.sa,
+                                      stream=main)
+        else:
+            f.fp8_quantize(self.a, self.qa_recipe, out=self.qa, scales=self.sa,
+                           workspace=self.ws, stream=main)
         self.ev_join.record(self.side)
         main.wait_event(self.ev_join)
 
@@ -241,7 +258,8 @@ class Step:
                                     self.sb.view(E, N), self.offs, out=self.out)
         else:
             f.fp8_scaled_mm(self.qa, self.qb, self.sa, self.sb,
-                            f.MM_RECIPES[wl.recipe], bias=self.bias, out=self.out)
+                            f.MM_RECIPES[GEMM_RECIPE.get(wl.recipe, wl.recipe)],
+                            bias=self.bias, out=self.out)
 
     def quant_bytes(self) -> int:
         """Algorithmic HBM bytes of the two quantize launches: 2 B read +
@@ -380,13 +398,18 @@ def oracle_sample(wl, max_rows: int):
          "1x128": oracle.GROUP_1x128, "128x128": oracle.GROUP_128x128}
     MMR = {"tensor": oracle.MM_TENSOR_TENSOR, "row": oracle.MM_ROW_ROW,
            "1x128_128x128": oracle.MM_1x128_128x128, "1x128_128x1": oracle.MM_1x128_128x1}
+    t_a, t_b = TRANSPOSED.get(wl.recipe, (False, False))
+
+    def bits(x, transposed):
+        b = W.bf16_bits(x)
+        return np.ascontiguousarray(b.T) if transposed else b
     t0 = time.perf_counter()
-    qa, sa = oracle.quantize(W.bf16_bits(wl.a), G[ga])
+    qa, sa = oracle.quantize(bits(wl.a, t_a), G[ga])
     if wl.recipe == "grouped":
         E, N, K = wl.b.shape
         qb, sb = oracle.quantize(W.bf16_bits(wl.b.reshape(E * N, K)), G[gb])
     else:
-        qb, sb = oracle.quantize(W.bf16_bits(wl.b), G[gb])
+        qb, sb = oracle.quantize(bits(wl.b, t_b), G[gb])
     tq = time.perf_counter() - t0
     rows = np.arange(min(max_rows, wl.M), dtype=np.int64)
     t0 = time.perf_counter()
@@ -396,7 +419,8 @@ def oracle_sample(wl, max_rows: int):
                                  wl.offs.numpy(), rows=rows)
     else:
         bias = None if wl.bias is None else W.bf16_bits(wl.bias)
-        oracle.scaled_mm(qa, qb, sa, sb, MMR[wl.recipe], bias_bits=bias, rows=rows)
+        oracle.scaled_mm(qa, qb, sa, sb, MMR[GEMM_RECIPE.get(wl.recipe, wl.recipe)],
+                         bias_bits=bias, rows=rows)
     tg = time.perf_counter() - t0
     return tg, rows.size / wl.M, tq, oracle.num_threads()
 

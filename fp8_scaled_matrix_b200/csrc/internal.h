@@ -21,6 +21,12 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t cols,
                             int64_t ld, int recipe, void* q, float* scales,
                             void* workspace, const LaunchCtx& ctx);
 
+// Quantization of x^T (quantize.cu), recipe 2 (1x128) or 3 (128x128);
+// rows % 128 == 0.  q is (cols, rows) with row stride rows.
+cudaError_t launch_quantize_transposed(const void* x, int64_t rows, int64_t cols,
+                                       int64_t ld, int recipe, void* q, float* scales,
+                                       const LaunchCtx& ctx);
+
 // Library-owned scratch for the no-allocation quantize entry point
 // (quantize.cu): its size, and its device address on `device` (looked up
 // once per device; the device must be current).

@@ -280,6 +280,89 @@ __global__ void __launch_bounds__(k128Threads) quant_128x128_kernel(
       *reinterpret_cast<uint2*>(qp + kRowStep * i * cols) = cast8(v[i], sp.inv);
 }
 
+// ------------------------------------------------------- transposed
+// Quantizes x^T ((cols, rows)) for the training GEMMs ("improve fp8
+// blockwise gemm perf": grad_input = grad_output @ weight and grad_weight =
+// grad_output_t @ input both need an operand whose contraction runs along
+// x's rows).  The result equals the 1x128 / 128x128 quantization of the
+// transposed matrix: a group is 128 consecutive rows of x within one column
+// (1x128) or a 128 x 128 tile (128x128).
+// One CTA (512 threads) per 128-row x 128-column tile of x: coalesced
+// 16-byte loads (4 per thread) into shared memory, then thread t takes
+// column t % 128 and rows 32 (t / 128) .. +31 of the tile: it reads them from
+// shared memory (a warp reads 32 consecutive columns of one row), the four
+// quarter-columns' amax meet in shared memory, and the thread writes its 32
+// codes as 32 consecutive bytes of the output row (x's column).
+constexpr int kTrRows = 128;
+constexpr int kTrCols = 128;
+constexpr int kTrThreads = 512;
+constexpr int kTrPitch = kTrCols + 8;  // bf16 elements per shared row (16-byte pad)
+
+template <bool k128x128>
+__global__ void __launch_bounds__(kTrThreads) quant_transposed_kernel(
+    const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+    uint8_t* __restrict__ q, float* __restrict__ scales) {
+  __shared__ __align__(16) uint16_t tile[kTrRows * kTrPitch];
+  __shared__ float part[4][kTrCols];
+  __shared__ float warp_amax[kTrThreads / 32];
+  const int64_t kb = blockIdx.x;                          // 128-row block of x
+  const int64_t c0 = static_cast<int64_t>(blockIdx.y) * kTrCols;
+  const int t = threadIdx.x;
+  // load: chunk t % 16 (8 columns) of rows t / 16 + 32 i
+  {
+    const int ch = t & 15;
+    const int64_t col = c0 + ch * 8;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = (t >> 4) + 32 * i;
+      uint4 v = make_uint4(0, 0, 0, 0);  // columns past the end: zero (no effect on the max)
+      if (col < cols)
+        v = ld_stream(reinterpret_cast<const uint4*>(x + (kb * kTrRows + r) * ld + col));
+      *reinterpret_cast<uint4*>(&tile[r * kTrPitch + ch * 8]) = v;
+    }
+  }
+  __syncthreads();
+  const int c = t & (kTrCols - 1);   // column within the tile = output row
+  const int qr = t >> 7;             // rows 32 qr .. 32 qr + 31
+  uint32_t w[16];                    // the 32 values, packed bf16 pairs
+  float m = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t lo = tile[(32 * qr + 2 * j) * kTrPitch + c];
+    const uint32_t hi = tile[(32 * qr + 2 * j + 1) * kTrPitch + c];
+    w[j] = lo | (hi << 16);
+    m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[j])), fabsf(bf16_hi(w[j]))));
+  }
+  part[qr][c] = m;
+  float gm;
+  if constexpr (k128x128) {
+    m = warp_max(m);
+    if ((t & 31) == 0) warp_amax[t >> 5] = m;
+    __syncthreads();
+    gm = warp_amax[0];
+#pragma unroll
+    for (int i = 1; i < kTrThreads / 32; ++i) gm = fmaxf(gm, warp_amax[i]);
+  } else {
+    __syncthreads();
+    gm = fmaxf(fmaxf(part[0][c], part[1][c]), fmaxf(part[2][c], part[3][c]));
+  }
+  const ScalePair sp = scales_from_amax(gm);
+  const int64_t col = c0 + c;
+  if constexpr (k128x128) {
+    if (t == 0) scales[kb * ((cols + kTrCols - 1) / kTrCols) + blockIdx.y] = sp.s;
+  } else {
+    if (qr == 0 && col < cols) scales[kb * cols + col] = sp.s;
+  }
+  if (col >= cols) return;
+  uint4 out[2];
+  uint32_t* o = reinterpret_cast<uint32_t*>(out);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) o[j] = cast2(w[2 * j], sp.inv) | (cast2(w[2 * j + 1], sp.inv) << 16);
+  uint4* dst = reinterpret_cast<uint4*>(q + col * rows + kb * kTrRows + 32 * qr);
+  dst[0] = out[0];
+  dst[1] = out[1];
+}
+
 // ------------------------------------------------------------- tensor
 // One amax for the whole matrix.  Cooperative launch (all CTAs resident):
 // phase 1 reduces each CTA's amax and folds it into ws[0] with an atomic
@@ -371,6 +454,23 @@ cudaError_t noalloc_scratch_ptr(int device, void** out) {
   }
   *out = g_noalloc_ptr[device];
   return cudaSuccess;
+}
+
+cudaError_t launch_quantize_transposed(const void* xv, int64_t rows, int64_t cols,
+                                       int64_t ld, int recipe, void* qv, float* scales,
+                                       const LaunchCtx& ctx) {
+  if (rows == 0 || cols == 0) return cudaSuccess;
+  const uint16_t* x = static_cast<const uint16_t*>(xv);
+  uint8_t* q = static_cast<uint8_t*>(qv);
+  const dim3 grid(static_cast<unsigned>(rows / kTrRows),
+                  static_cast<unsigned>((cols + kTrCols - 1) / kTrCols));
+  if (recipe == 3)
+    quant_transposed_kernel<true><<<grid, kTrThreads, 0, ctx.stream>>>(x, rows, cols, ld, q,
+                                                                       scales);
+  else
+    quant_transposed_kernel<false><<<grid, kTrThreads, 0, ctx.stream>>>(x, rows, cols, ld, q,
+                                                                        scales);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_quantize(const void* xv, int64_t rows, int64_t cols,

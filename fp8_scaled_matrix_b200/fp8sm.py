@@ -33,7 +33,7 @@ MM_RECIPES = {"tensor": FP8_MM_TENSOR_TENSOR, "row": FP8_MM_ROW_ROW,
 EXPORTED = ["fp8_version", "fp8_last_error", "fp8_quantize_workspace_bytes",
             "fp8_quantize", "fp8_scaled_mm", "fp8_grouped_scaled_mm",
             "fp8_get_device_status", "fp8_debug_timeout_probe",
-            "fp8_quantize_noalloc"]
+            "fp8_quantize_noalloc", "fp8_quantize_transposed"]
 
 
 class Fp8Error(RuntimeError):
@@ -88,6 +88,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fp8_debug_timeout_probe.argtypes = [U32, P]
     L.fp8_quantize_noalloc.restype = E
     L.fp8_quantize_noalloc.argtypes = [P, I64, I64, I64, E, P, P, P]
+    L.fp8_quantize_transposed.restype = E
+    L.fp8_quantize_transposed.argtypes = [P, I64, I64, I64, E, P, P, P]
     _lib = L
     return L
 
@@ -185,6 +187,30 @@ def fp8_quantize_noalloc(x: torch.Tensor, recipe: int, out: torch.Tensor,
     ld = x.stride(0) if (rows > 1 and cols > 0) else cols
     _check(L.fp8_quantize_noalloc(_ptr(x), rows, cols, ld, recipe, _ptr(out),
                                   _ptr(scales), _stream(stream)))
+    return out, scales
+
+
+def fp8_quantize_transposed(x: torch.Tensor, recipe: int, out: Optional[torch.Tensor] = None,
+                            scales: Optional[torch.Tensor] = None,
+                            stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Quantize x^T (x: 2-D bf16 CUDA tensor (rows, cols), rows % 128 == 0)
+    with the 1x128 or 128x128 recipe, as fp8_quantize(x.t()) would.
+
+    Returns (codes uint8 (cols, rows), scales float32 in the recipe's layout
+    for a (cols, rows) matrix)."""
+    L = load_library()
+    _need_cuda(x)
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D bf16 tensor with unit column stride")
+    rows, cols = x.shape
+    if out is None:
+        out = torch.empty((cols, rows), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(max(scale_count(cols, rows, recipe), 1),
+                             dtype=torch.float32, device=x.device)
+    ld = x.stride(0) if (rows > 1 and cols > 0) else cols
+    _check(L.fp8_quantize_transposed(_ptr(x), rows, cols, ld, recipe, _ptr(out),
+                                     _ptr(scales), _stream(stream)))
     return out, scales
 
 

@@ -23,6 +23,13 @@ descriptions; no public dataset is involved):
                 group sizes: 2048 chunks of 16 rows, each chunk given to an
                 expert drawn from p(r) ~ r^-1.2 over ranks r=1..16, ranks mapped
                 to experts by a seeded permutation; offs = cumulative ends
+  5 grad_input  the training GEMM grad_input = grad_output @ weight of the
+                blockwise benchmark's linear layer (16640 tokens, 8192 in,
+                5120 out): dY ~ N(0,1) (16640, 5120), W ~ N(0, 0.02^2)
+                (5120, 8192) as stored; GEMM M=16640, N=8192, K=5120
+  6 grad_weight grad_weight = grad_output_t @ input of the same layer:
+                dY ~ N(0, 1e-3^2) (16640, 5120), X ~ N(0,1) (16640, 8192);
+                GEMM M=5120, N=8192, K=16640
 """
 from __future__ import annotations
 
@@ -38,6 +45,8 @@ WORKLOAD_NAMES = [
     "blockwise_1x128_128x128",
     "blockwise_1x128_128x1",
     "grouped_e16",
+    "grad_input_1x128_128x128",
+    "grad_weight_1x128_128x1",
 ]
 
 
@@ -90,12 +99,17 @@ def offsets_from_sizes(sizes) -> torch.Tensor:
 @dataclass
 class Workload:
     name: str
-    recipe: str                      # tensor | row | 1x128_128x128 | 1x128_128x1 | grouped
+    # tensor | row | 1x128_128x128 | 1x128_128x1 | grouped | grad_input | grad_weight
+    recipe: str
     M: int
     N: int
     K: int
-    a: torch.Tensor                  # bf16 (M, K) CPU
-    b: torch.Tensor                  # bf16 (N, K) or (E, N, K) CPU
+    # GEMM sizes M, N, K; the bf16 operands as a caller holds them (CPU):
+    #   a  (M, K); grad_weight: (K, M) (grad_output, tokens x out)
+    #   b  (N, K) or (E, N, K); grad_input: (K, N) (the weight as stored);
+    #      grad_weight: (K, N) (the layer input, tokens x in)
+    a: torch.Tensor
+    b: torch.Tensor
     bias: Optional[torch.Tensor] = None   # bf16 (N,) CPU
     offs: Optional[torch.Tensor] = None   # int32 (E,) CPU
     E: int = 0
@@ -146,6 +160,16 @@ def make_workload(index: int, shape_index: int = 0, scale_down: int = 1) -> Work
         sizes = zipf_group_sizes(T, E, 16, 1.2, g)
         offs = offsets_from_sizes(sizes)
         return Workload(name, "grouped", T, N, K, a, b, offs=offs, E=E, seed=seed)
+    if index in (5, 6):
+        T, K_in, N_out = 16640 // scale_down, 8192, 5120
+        T -= T % 128
+        if index == 5:
+            dy = randn_bf16((T, N_out), 1.0, g)
+            w = randn_bf16((N_out, K_in), 0.02, g)
+            return Workload(name, "grad_input", T, K_in, N_out, dy, w, seed=seed)
+        dy = randn_bf16((T, N_out), 1e-3, g)
+        x = randn_bf16((T, K_in), 1.0, g)
+        return Workload(name, "grad_weight", N_out, K_in, T, dy, x, seed=seed)
     raise ValueError(f"unknown workload {index}")
 
 

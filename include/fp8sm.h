@@ -161,6 +161,32 @@ FP8SM_API fp8_status fp8_quantize_noalloc(const void* x_bf16, int64_t rows,
                                           fp8_stream_t stream);
 
 /*
+ * Transposed dynamic quantization, for the training GEMMs of [P5] (the
+ * 1x128_128x128 GEMM also serves grad_input = grad_output @ weight, the
+ * 1x128_128x1 GEMM serves grad_weight = grad_output_t @ input) and [P1]'s
+ * backward pass: both need an operand whose contraction runs along x's
+ * rows.  The result is exactly what fp8_quantize() gives for the transpose
+ * of x, without materializing the bf16 transpose:
+ *
+ *   x_bf16     (rows, cols) bf16, row stride ld_x elements; 16-byte aligned,
+ *              ld_x % 8 == 0, cols % 8 == 0, rows % 128 == 0.
+ *   out_fp8    (cols, rows) e4m3 = quantized x^T, row stride rows;
+ *              16-byte aligned.
+ *   out_scales the recipe's layout for a (cols, rows) matrix, 4-byte aligned:
+ *                1x128:    (rows/128) * cols values, scale[kb*cols + c]
+ *                          (group: rows 128 kb .. 128 kb + 127 of column c)
+ *                128x128:  (rows/128) * ceil(cols/128) values,
+ *                          scale[kb*ceil(cols/128) + c/128]
+ *   recipe     FP8_SCALE_BLOCK_1x128 or FP8_SCALE_BLOCK_128x128; the
+ *              tensorwise and rowwise recipes return FP8_ERR_UNSUPPORTED.
+ * rows == 0 or cols == 0 writes nothing.  No workspace is needed.
+ */
+FP8SM_API fp8_status fp8_quantize_transposed(const void* x_bf16, int64_t rows,
+                                             int64_t cols, int64_t ld_x,
+                                             fp8_quant_recipe recipe, void* out_fp8,
+                                             float* out_scales, fp8_stream_t stream);
+
+/*
  * Scaled GEMM ([P1] forward; [P4] recipes; [P5] blockwise recipes):
  *   out[m, n] = sum_k (a[m,k] * sA) * (b[n,k] * sB)  (+ bias[n])
  * with the scales picked per recipe (see fp8_mm_recipe).  Products are

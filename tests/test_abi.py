@@ -67,6 +67,30 @@ def test_quantize_misaligned_pointer(lib):
     assert st == fp8sm.FP8_ERR_VALUE and "aligned" in lib.fp8_last_error().decode()
 
 
+@pytest.mark.parametrize("args,status,frag", [
+    ((FAKE, 256, 128, 128, fp8sm.FP8_SCALE_ROW), fp8sm.FP8_ERR_UNSUPPORTED, "1x128 and 128x128"),
+    ((FAKE, 256, 128, 128, fp8sm.FP8_SCALE_TENSOR), fp8sm.FP8_ERR_UNSUPPORTED, "1x128 and 128x128"),
+    ((FAKE, 200, 128, 128, fp8sm.FP8_SCALE_BLOCK_1x128), fp8sm.FP8_ERR_VALUE, "rows must be a multiple of 128"),
+    ((FAKE, 256, 100, 100, fp8sm.FP8_SCALE_BLOCK_1x128), fp8sm.FP8_ERR_VALUE, "multiples of 8"),
+    ((FAKE, 256, 128, 64, fp8sm.FP8_SCALE_BLOCK_128x128), fp8sm.FP8_ERR_VALUE, "ld_x < cols"),
+    ((None, 256, 128, 128, fp8sm.FP8_SCALE_BLOCK_1x128), fp8sm.FP8_ERR_VALUE, "null"),
+    ((P((1 << 20) + 2), 256, 128, 128, fp8sm.FP8_SCALE_BLOCK_1x128), fp8sm.FP8_ERR_VALUE, "aligned"),
+    ((FAKE, 256, 128, 128, 9), fp8sm.FP8_ERR_VALUE, "unknown recipe"),
+])
+def test_quantize_transposed_rejects_bad_arguments(lib, args, status, frag):
+    x, rows, cols, ld, recipe = args
+    st = lib.fp8_quantize_transposed(x, rows, cols, ld, recipe, FAKE, FAKE, None)
+    assert st == status
+    assert frag in lib.fp8_last_error().decode()
+
+
+def test_quantize_transposed_empty_is_a_noop_without_cuda(lib):
+    assert lib.fp8_quantize_transposed(None, 0, 128, 128, fp8sm.FP8_SCALE_BLOCK_1x128,
+                                       None, None, None) == fp8sm.FP8_OK
+    assert lib.fp8_quantize_transposed(None, 256, 0, 0, fp8sm.FP8_SCALE_BLOCK_128x128,
+                                       None, None, None) == fp8sm.FP8_OK
+
+
 @pytest.mark.parametrize("M,N,K,recipe,frag", [
     (128, 100, 128, fp8sm.FP8_MM_ROW_ROW, "N must be a multiple of 16"),
     (128, 128, 100, fp8sm.FP8_MM_ROW_ROW, "K must be a multiple of 16"),
