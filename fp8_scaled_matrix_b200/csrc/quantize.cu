@@ -287,80 +287,105 @@ __global__ void __launch_bounds__(k128Threads) quant_128x128_kernel(
 // x's rows).  The result equals the 1x128 / 128x128 quantization of the
 // transposed matrix: a group is 128 consecutive rows of x within one column
 // (1x128) or a 128 x 128 tile (128x128).
-// One CTA (512 threads) per 128-row x 128-column tile of x: coalesced
-// 16-byte loads (4 per thread) into shared memory, then thread t takes
-// column t % 128 and rows 32 (t / 128) .. +31 of the tile: it reads them from
-// shared memory (a warp reads 32 consecutive columns of one row), the four
-// quarter-columns' amax meet in shared memory, and the thread writes its 32
-// codes as 32 consecutive bytes of the output row (x's column).
+// Persistent CTAs (512 threads) walk the 128-row x 128-column tiles of x
+// with a two-buffer cp.async pipeline: the next tile's 16-byte chunks
+// (coalesced rows of x) stream into shared memory while this tile is
+// processed.  Thread t takes column t % 128 and rows 32 (t / 128) .. +31 of
+// the tile: it reads them from shared memory (a warp reads 32 consecutive
+// columns of one row), the four quarter-columns' amax meet in shared memory,
+// and the thread writes its 32 codes as 32 consecutive bytes of the output
+// row (x's column).
 constexpr int kTrRows = 128;
 constexpr int kTrCols = 128;
 constexpr int kTrThreads = 512;
 constexpr int kTrPitch = kTrCols + 8;  // bf16 elements per shared row (16-byte pad)
+constexpr int kTrTileElems = kTrRows * kTrPitch;
+constexpr size_t kTrSmemBytes = 2 * kTrTileElems * sizeof(uint16_t);
+constexpr int kTrCtasPerSm = 2;
 
 template <bool k128x128>
 __global__ void __launch_bounds__(kTrThreads) quant_transposed_kernel(
     const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
     uint8_t* __restrict__ q, float* __restrict__ scales) {
-  __shared__ __align__(16) uint16_t tile[kTrRows * kTrPitch];
+  extern __shared__ __align__(16) uint16_t tiles_smem[];
   __shared__ float part[4][kTrCols];
   __shared__ float warp_amax[kTrThreads / 32];
-  const int64_t kb = blockIdx.x;                          // 128-row block of x
-  const int64_t c0 = static_cast<int64_t>(blockIdx.y) * kTrCols;
+  const int64_t n_kb = rows / kTrRows;
+  const int64_t n_cb = (cols + kTrCols - 1) / kTrCols;
+  const int64_t n_tiles = n_kb * n_cb;
   const int t = threadIdx.x;
-  // load: chunk t % 16 (8 columns) of rows t / 16 + 32 i
-  {
+  // copy tile `tile` into buffer `buf`: chunk t % 16 (8 columns) of rows
+  // t / 16 + 32 i; columns past the end are zero-filled (no effect on the max)
+  auto issue = [&](int64_t tile, int buf) {
+    const int64_t kb = tile % n_kb, cb = tile / n_kb;
     const int ch = t & 15;
-    const int64_t col = c0 + ch * 8;
+    const int64_t col = cb * kTrCols + ch * 8;
+    uint16_t* dst = tiles_smem + buf * kTrTileElems;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int r = (t >> 4) + 32 * i;
-      uint4 v = make_uint4(0, 0, 0, 0);  // columns past the end: zero (no effect on the max)
-      if (col < cols)
-        v = ld_stream(reinterpret_cast<const uint4*>(x + (kb * kTrRows + r) * ld + col));
-      *reinterpret_cast<uint4*>(&tile[r * kTrPitch + ch * 8]) = v;
+      const bool in = col < cols;
+      cp_async_16(dst + r * kTrPitch + ch * 8, in ? x + (kb * kTrRows + r) * ld + col : x,
+                  in ? 16u : 0u);
     }
-  }
-  __syncthreads();
+    cp_async_commit();
+  };
+  int64_t tile = blockIdx.x;
+  if (tile < n_tiles) issue(tile, 0);
   const int c = t & (kTrCols - 1);   // column within the tile = output row
   const int qr = t >> 7;             // rows 32 qr .. 32 qr + 31
-  uint32_t w[16];                    // the 32 values, packed bf16 pairs
-  float m = 0.0f;
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const uint32_t lo = tile[(32 * qr + 2 * j) * kTrPitch + c];
-    const uint32_t hi = tile[(32 * qr + 2 * j + 1) * kTrPitch + c];
-    w[j] = lo | (hi << 16);
-    m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[j])), fabsf(bf16_hi(w[j]))));
-  }
-  part[qr][c] = m;
-  float gm;
-  if constexpr (k128x128) {
-    m = warp_max(m);
-    if ((t & 31) == 0) warp_amax[t >> 5] = m;
+  for (int it = 0; tile < n_tiles; tile += gridDim.x, ++it) {
+    const int buf = it & 1;
+    if (tile + gridDim.x < n_tiles) issue(tile + gridDim.x, buf ^ 1);
+    else cp_async_commit();          // empty group: the wait below counts groups
+    cp_async_wait<1>();              // this tile's copies have landed
     __syncthreads();
-    gm = warp_amax[0];
+    const uint16_t* tl = tiles_smem + buf * kTrTileElems;
+    const int64_t kb = tile % n_kb, cb = tile / n_kb;
+    uint32_t w[16];                  // the 32 values, packed bf16 pairs
+    float m = 0.0f;
 #pragma unroll
-    for (int i = 1; i < kTrThreads / 32; ++i) gm = fmaxf(gm, warp_amax[i]);
-  } else {
+    for (int j = 0; j < 16; ++j) {
+      const uint32_t lo = tl[(32 * qr + 2 * j) * kTrPitch + c];
+      const uint32_t hi = tl[(32 * qr + 2 * j + 1) * kTrPitch + c];
+      w[j] = lo | (hi << 16);
+      m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[j])), fabsf(bf16_hi(w[j]))));
+    }
+    float gm;
+    if constexpr (k128x128) {
+      m = warp_max(m);
+      if ((t & 31) == 0) warp_amax[t >> 5] = m;
+      __syncthreads();
+      gm = warp_amax[0];
+#pragma unroll
+      for (int i = 1; i < kTrThreads / 32; ++i) gm = fmaxf(gm, warp_amax[i]);
+    } else {
+      part[qr][c] = m;
+      __syncthreads();
+      gm = fmaxf(fmaxf(part[0][c], part[1][c]), fmaxf(part[2][c], part[3][c]));
+    }
+    const ScalePair sp = scales_from_amax(gm);
+    const int64_t col = cb * kTrCols + c;
+    if constexpr (k128x128) {
+      if (t == 0) scales[kb * n_cb + cb] = sp.s;
+    } else {
+      if (qr == 0 && col < cols) scales[kb * cols + col] = sp.s;
+    }
+    if (col < cols) {
+      uint4 out[2];
+      uint32_t* o = reinterpret_cast<uint32_t*>(out);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        o[j] = cast2(w[2 * j], sp.inv) | (cast2(w[2 * j + 1], sp.inv) << 16);
+      uint4* dst = reinterpret_cast<uint4*>(q + col * rows + kb * kTrRows + 32 * qr);
+      dst[0] = out[0];
+      dst[1] = out[1];
+    }
+    // every thread is done with this buffer (and with part / warp_amax)
+    // before the next iteration refills it
     __syncthreads();
-    gm = fmaxf(fmaxf(part[0][c], part[1][c]), fmaxf(part[2][c], part[3][c]));
   }
-  const ScalePair sp = scales_from_amax(gm);
-  const int64_t col = c0 + c;
-  if constexpr (k128x128) {
-    if (t == 0) scales[kb * ((cols + kTrCols - 1) / kTrCols) + blockIdx.y] = sp.s;
-  } else {
-    if (qr == 0 && col < cols) scales[kb * cols + col] = sp.s;
-  }
-  if (col >= cols) return;
-  uint4 out[2];
-  uint32_t* o = reinterpret_cast<uint32_t*>(out);
-#pragma unroll
-  for (int j = 0; j < 8; ++j) o[j] = cast2(w[2 * j], sp.inv) | (cast2(w[2 * j + 1], sp.inv) << 16);
-  uint4* dst = reinterpret_cast<uint4*>(q + col * rows + kb * kTrRows + 32 * qr);
-  dst[0] = out[0];
-  dst[1] = out[1];
+  cp_async_wait_all();
 }
 
 // ------------------------------------------------------------- tensor
@@ -462,14 +487,27 @@ cudaError_t launch_quantize_transposed(const void* xv, int64_t rows, int64_t col
   if (rows == 0 || cols == 0) return cudaSuccess;
   const uint16_t* x = static_cast<const uint16_t*>(xv);
   uint8_t* q = static_cast<uint8_t*>(qv);
-  const dim3 grid(static_cast<unsigned>(rows / kTrRows),
-                  static_cast<unsigned>((cols + kTrCols - 1) / kTrCols));
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(quant_transposed_kernel<true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kTrSmemBytes));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(quant_transposed_kernel<false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kTrSmemBytes));
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  const int64_t tiles = (rows / kTrRows) * ((cols + kTrCols - 1) / kTrCols);
+  const int64_t max_grid = static_cast<int64_t>(ctx.num_sms) * kTrCtasPerSm;
+  const unsigned grid = static_cast<unsigned>(tiles < max_grid ? tiles : max_grid);
   if (recipe == 3)
-    quant_transposed_kernel<true><<<grid, kTrThreads, 0, ctx.stream>>>(x, rows, cols, ld, q,
-                                                                       scales);
+    quant_transposed_kernel<true><<<grid, kTrThreads, kTrSmemBytes, ctx.stream>>>(
+        x, rows, cols, ld, q, scales);
   else
-    quant_transposed_kernel<false><<<grid, kTrThreads, 0, ctx.stream>>>(x, rows, cols, ld, q,
-                                                                        scales);
+    quant_transposed_kernel<false><<<grid, kTrThreads, kTrSmemBytes, ctx.stream>>>(
+        x, rows, cols, ld, q, scales);
   return cudaGetLastError();
 }
 
