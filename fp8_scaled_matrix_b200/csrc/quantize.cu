@@ -293,14 +293,16 @@ __global__ void __launch_bounds__(k128Threads) quant_128x128_kernel(
 // processed.  Thread t takes column t % 128 and rows 32 (t / 128) .. +31 of
 // the tile: it reads them from shared memory (a warp reads 32 consecutive
 // columns of one row), the four quarter-columns' amax meet in shared memory,
-// and the thread writes its 32 codes as 32 consecutive bytes of the output
-// row (x's column).
+// and the thread stages its 32 codes in shared memory; the tile's 128 output
+// rows (x's columns) then leave as whole 128-byte lines.
 constexpr int kTrRows = 128;
 constexpr int kTrCols = 128;
 constexpr int kTrThreads = 512;
 constexpr int kTrPitch = kTrCols + 8;  // bf16 elements per shared row (16-byte pad)
 constexpr int kTrTileElems = kTrRows * kTrPitch;
-constexpr size_t kTrSmemBytes = 2 * kTrTileElems * sizeof(uint16_t);
+constexpr int kTrOutPitch = kTrRows + 16;  // bytes per staged output row (conflict-free 16-byte stores)
+constexpr size_t kTrSmemBytes =
+    2 * kTrTileElems * sizeof(uint16_t) + static_cast<size_t>(kTrCols) * kTrOutPitch;
 constexpr int kTrCtasPerSm = 2;
 
 template <bool k128x128>
@@ -371,18 +373,31 @@ __global__ void __launch_bounds__(kTrThreads) quant_transposed_kernel(
     } else {
       if (qr == 0 && col < cols) scales[kb * cols + col] = sp.s;
     }
-    if (col < cols) {
+    uint8_t* stage = reinterpret_cast<uint8_t*>(tiles_smem + 2 * kTrTileElems);
+    {
       uint4 out[2];
       uint32_t* o = reinterpret_cast<uint32_t*>(out);
 #pragma unroll
       for (int j = 0; j < 8; ++j)
         o[j] = cast2(w[2 * j], sp.inv) | (cast2(w[2 * j + 1], sp.inv) << 16);
-      uint4* dst = reinterpret_cast<uint4*>(q + col * rows + kb * kTrRows + 32 * qr);
-      dst[0] = out[0];
-      dst[1] = out[1];
+      uint4* sd = reinterpret_cast<uint4*>(stage + c * kTrOutPitch + 32 * qr);
+      sd[0] = out[0];
+      sd[1] = out[1];
     }
-    // every thread is done with this buffer (and with part / warp_amax)
-    // before the next iteration refills it
+    __syncthreads();
+    {
+      // thread t: 32 bytes (chunk t % 4) of output row t / 4 of the tile
+      const int orow = t >> 2, chunk = t & 3;
+      const int64_t ocol = cb * kTrCols + orow;
+      if (ocol < cols) {
+        const uint4* ss = reinterpret_cast<const uint4*>(stage + orow * kTrOutPitch + 32 * chunk);
+        uint4* dst = reinterpret_cast<uint4*>(q + ocol * rows + kb * kTrRows + 32 * chunk);
+        dst[0] = ss[0];
+        dst[1] = ss[1];
+      }
+    }
+    // every thread is done with this buffer, the staging rows and part /
+    // warp_amax before the next iteration refills them
     __syncthreads();
   }
   cp_async_wait_all();
