@@ -84,24 +84,30 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def kernel_sources_hash() -> str:
+# the GEMM kernel's sources: its recorded DRAM traffic stays valid while
+# these are unchanged
+GEMM_SOURCES = ("gemm.cu", "sm100.cuh", "status.cuh")
+
+
+def kernel_sources_hash(files=None) -> str:
+    """Hash of the kernel sources (all of csrc/, or the named files)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "fp8_scaled_matrix_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in sorted(files if files is not None else os.listdir(csrc)):
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(workload: str):
     """DRAM bytes per GEMM launch from the committed ncu summary, if it was
-    taken on the current kernel sources; otherwise None."""
+    taken on the current GEMM kernel sources; otherwise None."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(p):
         return None
     try:
         d = json.load(open(p))
         e = d.get(workload)
-        if e and e.get("sources") == kernel_sources_hash():
+        if e and e.get("sources") == kernel_sources_hash(GEMM_SOURCES):
             return float(e["bytes_per_launch"])
     except Exception:
         return None
