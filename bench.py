@@ -50,6 +50,7 @@ WORKLOADS = {
     "grouped_e16": (4, 0),
     "grad_input_1x128_128x128": (5, 0),
     "grad_weight_1x128_128x1": (6, 0),
+    "grouped_e16_blockwise": (7, 0),
 }
 DEFAULT_WORKLOAD = "rowwise_4096"
 # Page 5's context numbers (TFLOP/s of torch._scaled_mm, hardware not stated)
@@ -60,7 +61,8 @@ PAGE_NUMBERS = {
 OPERAND_GROUPS = {"tensor": ("tensor", "tensor"), "row": ("row", "row"),
                   "1x128_128x128": ("1x128", "128x128"),
                   "1x128_128x1": ("1x128", "1x128"), "grouped": ("row", "row"),
-                  "grad_input": ("1x128", "128x128"), "grad_weight": ("1x128", "1x128")}
+                  "grad_input": ("1x128", "128x128"), "grad_weight": ("1x128", "1x128"),
+                  "grouped_blockwise": ("1x128", "128x128")}
 # GEMM recipe of each workload recipe, and which operands are quantized
 # transposed (the training GEMMs contract along the stored rows)
 GEMM_RECIPE = {"grad_input": "1x128_128x128", "grad_weight": "1x128_128x1"}
@@ -205,7 +207,8 @@ class Step:
         self.qa_recipe = fp8sm.QUANT_RECIPES[ga]
         self.qb_recipe = fp8sm.QUANT_RECIPES[gb]
         self.a = wl.a.to(dev)
-        if wl.recipe == "grouped":
+        self.grouped = wl.recipe in ("grouped", "grouped_blockwise")
+        if self.grouped:
             E, N, K = wl.b.shape
             self.b = wl.b.to(dev).reshape(E * N, K)
             self.offs = wl.offs.to(dev)
@@ -230,6 +233,13 @@ class Step:
         self.ev_join = torch.cuda.Event()
         self.out = torch.empty(wl.M, wl.N, dtype=torch.bfloat16, device=dev)
         self.launches_per_step = 3
+        if wl.recipe == "grouped_blockwise":
+            # each expert's weights are quantized on their own (its 128x128
+            # tiles and scales), into the (E, K/128, N/128) scale layout
+            E, N, K = wl.b.shape
+            self.sb = torch.empty(E * fp8sm.scale_count(N, K, self.qb_recipe),
+                                  dtype=torch.float32, device=dev)
+            self.launches_per_step = 2 + E
 
     def quantize(self):
         """Both operands' quantization; the second runs on a side stream,
@@ -240,7 +250,14 @@ class Step:
         self.ev_fork.record(main)
         self.side.wait_event(self.ev_fork)
         with torch.cuda.stream(self.side):
-            if self.t_b:
+            if self.wl.recipe == "grouped_blockwise":
+                E, N, K = self.wl.b.shape
+                per = self.sb.numel() // E
+                for e in range(E):
+                    f.fp8_quantize(self.b[e * N:(e + 1) * N], self.qb_recipe,
+                                   out=self.qb[e * N:(e + 1) * N],
+                                   scales=self.sb[e * per:(e + 1) * per], stream=self.side)
+            elif self.t_b:
                 f.fp8_quantize_transposed(self.b, self.qb_recipe, out=self.qb, scales=self.sb,
                                           stream=self.side)
             else:
@@ -262,6 +279,10 @@ class Step:
             E, N, K = wl.b.shape
             f.fp8_grouped_scaled_mm(self.qa, self.qb.view(E, N, K), self.sa,
                                     self.sb.view(E, N), self.offs, out=self.out)
+        elif wl.recipe == "grouped_blockwise":
+            E, N, K = wl.b.shape
+            f.fp8_grouped_scaled_mm_blockwise(self.qa, self.qb.view(E, N, K), self.sa,
+                                              self.sb, self.offs, out=self.out)
         else:
             f.fp8_scaled_mm(self.qa, self.qb, self.sa, self.sb,
                             f.MM_RECIPES[GEMM_RECIPE.get(wl.recipe, wl.recipe)],
@@ -355,7 +376,8 @@ def run_e2e(args, wl, dev, world):
     the timed region."""
     from fp8_scaled_matrix_b200 import fp8sm
     ha = wl.a.pin_memory()
-    hb = (wl.b.reshape(-1, wl.K) if wl.recipe == "grouped" else wl.b).contiguous().pin_memory()
+    hb = (wl.b.reshape(-1, wl.K) if wl.recipe in ("grouped", "grouped_blockwise")
+          else wl.b).contiguous().pin_memory()
     hbias = None if wl.bias is None else wl.bias.pin_memory()
     hout = torch.empty(wl.M, wl.N, dtype=torch.bfloat16).pin_memory()
     st = Step(wl, dev)
@@ -414,6 +436,11 @@ def oracle_sample(wl, max_rows: int):
     if wl.recipe == "grouped":
         E, N, K = wl.b.shape
         qb, sb = oracle.quantize(W.bf16_bits(wl.b.reshape(E * N, K)), G[gb])
+    elif wl.recipe == "grouped_blockwise":
+        per_expert = [oracle.quantize(W.bf16_bits(wl.b[e].contiguous()), G[gb])
+                      for e in range(wl.b.shape[0])]
+        qb = np.stack([q for q, _ in per_expert])
+        sb = np.stack([s for _, s in per_expert])
     else:
         qb, sb = oracle.quantize(bits(wl.b, t_b), G[gb])
     tq = time.perf_counter() - t0
@@ -423,6 +450,18 @@ def oracle_sample(wl, max_rows: int):
         E, N, K = wl.b.shape
         oracle.grouped_scaled_mm(qa, qb.reshape(E, N, K), sa, sb.reshape(E, N),
                                  wl.offs.numpy(), rows=rows)
+    elif wl.recipe == "grouped_blockwise":
+        # the dense blockwise GEMM of each group that the sampled rows touch
+        KB = wl.K // 128
+        sa2 = sa.reshape(KB, wl.M)
+        start = 0
+        for e, end in enumerate(wl.offs.numpy()):
+            sel = rows[(rows >= start) & (rows < end)]
+            if sel.size:
+                oracle.scaled_mm(np.ascontiguousarray(qa[start:end]), qb[e],
+                                 np.ascontiguousarray(sa2[:, start:end]).reshape(-1),
+                                 sb[e].reshape(-1), MMR["1x128_128x128"], rows=sel - start)
+            start = int(end)
     else:
         bias = None if wl.bias is None else W.bf16_bits(wl.bias)
         oracle.scaled_mm(qa, qb, sa, sb, MMR[GEMM_RECIPE.get(wl.recipe, wl.recipe)],

@@ -256,33 +256,36 @@ fp8_status fp8_scaled_mm(const void* a, const void* b, int64_t M, int64_t N,
   return finish_launch(e, err, "fp8_scaled_mm");
 }
 
-fp8_status fp8_grouped_scaled_mm(const void* a, const void* b_experts,
-                                 int64_t M_total, int64_t N, int64_t K,
-                                 int32_t E, const float* scale_a,
-                                 const float* scale_b, const int32_t* offs,
-                                 fp8_out_dtype out_dtype, void* out,
-                                 fp8_stream_t stream) {
+namespace {
+
+// Shared by both grouped entry points; recipe 1 (rowwise) or 2 (1x128_128x128).
+fp8_status grouped_common(const char* name, int recipe, const void* a, const void* b_experts,
+                          int64_t M_total, int64_t N, int64_t K, int32_t E,
+                          const float* scale_a, const float* scale_b, const int32_t* offs,
+                          fp8_out_dtype out_dtype, void* out, fp8_stream_t stream) {
+  const std::string n(name);
   if (out_dtype != FP8_OUT_BF16 && out_dtype != FP8_OUT_F32)
-    return fail(FP8_ERR_VALUE, "fp8_grouped_scaled_mm: unknown out_dtype");
-  if (offs == nullptr)
-    return fail(FP8_ERR_VALUE, "fp8_grouped_scaled_mm: offs is required");
+    return fail(FP8_ERR_VALUE, n + ": unknown out_dtype");
+  if (offs == nullptr) return fail(FP8_ERR_VALUE, n + ": offs is required");
   if (M_total < 0 || N < 0 || K < 0 || E < 1 || E > 65535)
-    return fail(FP8_ERR_VALUE, "fp8_grouped_scaled_mm: bad size or expert count");
+    return fail(FP8_ERR_VALUE, n + ": bad size or expert count");
   if (M_total >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
-    return fail(FP8_ERR_VALUE, "fp8_grouped_scaled_mm: size too large");
+    return fail(FP8_ERR_VALUE, n + ": size too large");
   if (K % 16 != 0 || N % 16 != 0)
-    return fail(FP8_ERR_VALUE, "fp8_grouped_scaled_mm: K and N must be multiples of 16");
+    return fail(FP8_ERR_VALUE, n + ": K and N must be multiples of 16");
+  if (recipe == 2 && K % 128 != 0)
+    return fail(FP8_ERR_VALUE, n + ": the blockwise recipe needs K % 128 == 0");
   if (M_total == 0 || N == 0) {
     t_last_error.clear();
     return FP8_OK;
   }
   if (out == nullptr || (K > 0 && (a == nullptr || b_experts == nullptr ||
                                    scale_a == nullptr || scale_b == nullptr)))
-    return fail(FP8_ERR_VALUE, "fp8_grouped_scaled_mm: null pointer");
+    return fail(FP8_ERR_VALUE, n + ": null pointer");
   if (!aligned(out, 16) || (a && !aligned(a, 16)) || (b_experts && !aligned(b_experts, 16)) ||
       (scale_a && !aligned(scale_a, 16)) || (scale_b && !aligned(scale_b, 16)) ||
       !aligned(offs, 4))
-    return fail(FP8_ERR_VALUE, "fp8_grouped_scaled_mm: pointers must be 16-byte aligned");
+    return fail(FP8_ERR_VALUE, n + ": pointers must be 16-byte aligned");
   DeviceInfo* d = nullptr;
   fp8_status s = device_info(&d);
   if (s != FP8_OK) return s;
@@ -290,9 +293,31 @@ fp8_status fp8_grouped_scaled_mm(const void* a, const void* b_experts,
   fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status,
                        d->num_sms, &err};
   cudaError_t e = fp8sm::launch_grouped_scaled_mm(a, b_experts, M_total, N, K, E,
-                                                  scale_a, scale_b, offs,
+                                                  scale_a, scale_b, offs, recipe,
                                                   out_dtype == FP8_OUT_F32, out, ctx);
-  return finish_launch(e, err, "fp8_grouped_scaled_mm");
+  return finish_launch(e, err, name);
+}
+
+}  // namespace
+
+fp8_status fp8_grouped_scaled_mm(const void* a, const void* b_experts,
+                                 int64_t M_total, int64_t N, int64_t K,
+                                 int32_t E, const float* scale_a,
+                                 const float* scale_b, const int32_t* offs,
+                                 fp8_out_dtype out_dtype, void* out,
+                                 fp8_stream_t stream) {
+  return grouped_common("fp8_grouped_scaled_mm", 1, a, b_experts, M_total, N, K, E, scale_a,
+                        scale_b, offs, out_dtype, out, stream);
+}
+
+fp8_status fp8_grouped_scaled_mm_blockwise(const void* a, const void* b_experts,
+                                           int64_t M_total, int64_t N, int64_t K,
+                                           int32_t E, const float* scale_a,
+                                           const float* scale_b, const int32_t* offs,
+                                           fp8_out_dtype out_dtype, void* out,
+                                           fp8_stream_t stream) {
+  return grouped_common("fp8_grouped_scaled_mm_blockwise", 2, a, b_experts, M_total, N, K, E,
+                        scale_a, scale_b, offs, out_dtype, out, stream);
 }
 
 fp8_status fp8_get_device_status(fp8_stream_t stream) {

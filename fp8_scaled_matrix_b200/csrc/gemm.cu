@@ -587,6 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t slot = 0, sphase = 0;
       bool ok = true;
       GroupCursor cur;
+      if constexpr (kGrouped) cur.init(p.offs, kTM);
       for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
         const TileCoord c = tile_coord<kGrouped, kTM>(t, p, cur);
         for (int32_t kb = 0; kb < KB; ++kb) {
@@ -604,9 +605,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if constexpr (kRecipe == kBlock128) {
             if (lane < 2) {
+              // grouped: expert g's scales, layout (E, K/128, ceil(N/128))
+              const int64_t kbg = (kGrouped ? static_cast<int64_t>(c.g) * KB : 0) + kb;
               const bool v = static_cast<int64_t>(c.n0) + 128 * lane < p.N;
               cp_async_4(dst + 128 + lane,
-                         v ? p.sb + static_cast<int64_t>(kb) * NB + c.n0 / 128 + lane : p.sb,
+                         v ? p.sb + kbg * NB + c.n0 / 128 + lane : p.sb,
                          v ? 4u : 0u);
             }
           } else {
@@ -949,6 +952,7 @@ cudaError_t dispatch(int recipe, int out_f32, bool pair, const CUtensorMap& ta,
   }
   if constexpr (kGrouped) {
     FP8SM_CASE(kRow)
+    FP8SM_CASE(kBlock128)
   } else {
     FP8SM_CASE(kTensor)
     FP8SM_CASE(kRow)
@@ -1065,13 +1069,13 @@ cudaError_t launch_grouped_scaled_mm(const void* a, const void* b,
                                      int64_t M_total, int64_t N, int64_t K,
                                      int32_t E, const float* sa,
                                      const float* sb, const int32_t* offs,
-                                     int out_f32, void* out,
+                                     int recipe, int out_f32, void* out,
                                      const LaunchCtx& ctx) {
   if (M_total == 0 || N == 0) return cudaSuccess;
   if (K == 0)
     return launch_scaled_mm(nullptr, nullptr, M_total, N, 0, nullptr, nullptr,
                             1, nullptr, out_f32, out, ctx);
-  const bool pair = use_pair(M_total, kRow);
+  const bool pair = use_pair(M_total, recipe);
   const uint32_t b_rows = pair ? Cfg<true>::kBRows : Cfg<false>::kBRows;
   CUtensorMap ta, tb, to;
   if (!a_map(&ta, a, M_total, K, ctx.err)) return cudaErrorInvalidValue;
@@ -1105,7 +1109,7 @@ cudaError_t launch_grouped_scaled_mm(const void* a, const void* b,
   p.split_start = INT64_MAX;
   p.total_items = 0;
   const unsigned grid = static_cast<unsigned>(pair ? (ctx.num_sms / 2) * 2 : ctx.num_sms);
-  return dispatch<true>(1, out_f32, pair, ta, tb, tb, to, p, grid, ctx.stream);
+  return dispatch<true>(recipe, out_f32, pair, ta, tb, tb, to, p, grid, ctx.stream);
 }
 
 cudaError_t launch_timeout_probe(uint32_t limit_us, const LaunchCtx& ctx) {

@@ -40,12 +40,12 @@ cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
                              const float* sb, int recipe, const void* bias,
                              int out_f32, void* out, const LaunchCtx& ctx);
 
-// Grouped rowwise scaled GEMM (gemm.cu).
+// Grouped scaled GEMM (gemm.cu).  recipe: 1 rowwise, 2 1x128_128x128.
 cudaError_t launch_grouped_scaled_mm(const void* a, const void* b,
                                      int64_t M_total, int64_t N, int64_t K,
                                      int32_t E, const float* sa,
                                      const float* sb, const int32_t* offs,
-                                     int out_f32, void* out,
+                                     int recipe, int out_f32, void* out,
                                      const LaunchCtx& ctx);
 
 // Failure-detection probe (gemm.cu): one CTA waits on a barrier nothing

@@ -33,7 +33,8 @@ MM_RECIPES = {"tensor": FP8_MM_TENSOR_TENSOR, "row": FP8_MM_ROW_ROW,
 EXPORTED = ["fp8_version", "fp8_last_error", "fp8_quantize_workspace_bytes",
             "fp8_quantize", "fp8_scaled_mm", "fp8_grouped_scaled_mm",
             "fp8_get_device_status", "fp8_debug_timeout_probe",
-            "fp8_quantize_noalloc", "fp8_quantize_transposed"]
+            "fp8_quantize_noalloc", "fp8_quantize_transposed",
+            "fp8_grouped_scaled_mm_blockwise"]
 
 
 class Fp8Error(RuntimeError):
@@ -82,6 +83,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fp8_scaled_mm.argtypes = [P, P, I64, I64, I64, P, P, E, P, E, P, P]
     L.fp8_grouped_scaled_mm.restype = E
     L.fp8_grouped_scaled_mm.argtypes = [P, P, I64, I64, I64, I32, P, P, P, E, P, P]
+    L.fp8_grouped_scaled_mm_blockwise.restype = E
+    L.fp8_grouped_scaled_mm_blockwise.argtypes = [P, P, I64, I64, I64, I32, P, P, P, E, P, P]
     L.fp8_get_device_status.restype = E
     L.fp8_get_device_status.argtypes = [P]
     L.fp8_debug_timeout_probe.restype = E
@@ -259,6 +262,29 @@ def fp8_grouped_scaled_mm(a: torch.Tensor, b_experts: torch.Tensor,
     _check(L.fp8_grouped_scaled_mm(_ptr(a), _ptr(b_experts), M, N, K, E, _ptr(scale_a),
                                    _ptr(scale_b), _ptr(offs), od, _ptr(out),
                                    _stream(stream)))
+    return out
+
+
+def fp8_grouped_scaled_mm_blockwise(a: torch.Tensor, b_experts: torch.Tensor,
+                                    scale_a: torch.Tensor, scale_b: torch.Tensor,
+                                    offs: torch.Tensor, out_dtype=torch.bfloat16,
+                                    out: Optional[torch.Tensor] = None,
+                                    stream=None) -> torch.Tensor:
+    """Grouped GEMM with 1x128 (a) / per-expert 128x128 (b_experts) scales."""
+    L = load_library()
+    _need_cuda(a, b_experts, scale_a, scale_b, offs)
+    if offs.dtype != torch.int32:
+        raise ValueError("offs must be int32")
+    M, K = a.shape
+    E, N, K2 = b_experts.shape
+    if K2 != K or offs.numel() != E:
+        raise ValueError("shape mismatch")
+    od = FP8_OUT_F32 if out_dtype == torch.float32 else FP8_OUT_BF16
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=a.device)
+    _check(L.fp8_grouped_scaled_mm_blockwise(_ptr(a), _ptr(b_experts), M, N, K, E,
+                                             _ptr(scale_a), _ptr(scale_b), _ptr(offs), od,
+                                             _ptr(out), _stream(stream)))
     return out
 
 

@@ -30,6 +30,8 @@ descriptions; no public dataset is involved):
   6 grad_weight grad_weight = grad_output_t @ input of the same layer:
                 dY ~ N(0, 1e-3^2) (16640, 5120), X ~ N(0,1) (16640, 8192);
                 GEMM M=5120, N=8192, K=16640
+  7 grouped blockwise  the tensors of workload 4 (same seed), quantized with
+                1x128 activation groups and per-expert 128x128 weight tiles
 """
 from __future__ import annotations
 
@@ -47,6 +49,7 @@ WORKLOAD_NAMES = [
     "grouped_e16",
     "grad_input_1x128_128x128",
     "grad_weight_1x128_128x1",
+    "grouped_e16_blockwise",
 ]
 
 
@@ -99,7 +102,8 @@ def offsets_from_sizes(sizes) -> torch.Tensor:
 @dataclass
 class Workload:
     name: str
-    # tensor | row | 1x128_128x128 | 1x128_128x1 | grouped | grad_input | grad_weight
+    # tensor | row | 1x128_128x128 | 1x128_128x1 | grouped | grouped_blockwise |
+    # grad_input | grad_weight
     recipe: str
     M: int
     N: int
@@ -125,9 +129,13 @@ def make_workload(index: int, shape_index: int = 0, scale_down: int = 1) -> Work
     """Build workload ``index`` (see module doc).  ``scale_down`` > 1 divides M
     (and, for the grouped case, the token count) to make a smaller case with
     the same distributions; sizes stay multiples of 16."""
+    name = WORKLOAD_NAMES[index]
+    if index == 7:  # workload 4's tensors, blockwise-scaled
+        wl = make_workload(4, shape_index, scale_down)
+        wl.name, wl.recipe = name, "grouped_blockwise"
+        return wl
     seed = 1000 + index + 100 * shape_index
     g = generator(seed)
-    name = WORKLOAD_NAMES[index]
     if index == 0:
         M = N = K = 256
         a = randn_bf16((M, K), 1.0, g)

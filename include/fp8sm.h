@@ -236,6 +236,30 @@ FP8SM_API fp8_status fp8_grouped_scaled_mm(const void* a, const void* b_experts,
                                  fp8_stream_t stream);
 
 /*
+ * Grouped (MoE) scaled GEMM with blockwise scales, the 1x128_128x128 recipe
+ * of [P4]/[P5] applied per expert (the blockwise-scaled expert weights that
+ * [P2]'s handler leaves for later):
+ *   for g in 0..E-1, rows m in [offs[g-1], offs[g]):
+ *     out[m, n] = sum_kb scale_a[kb*M_total + m] * scale_b[(g*(K/128) + kb)*ceil(N/128) + n/128]
+ *                        * sum_{k in block kb} a[m,k] * b_experts[g,n,k]
+ *
+ *   a          (M_total, K) e4m3; scale_a (K/128, M_total) fp32 (1x128 groups,
+ *              K-block-major as fp8_quantize writes them).
+ *   b_experts  (E, N, K) e4m3; scale_b (E, K/128, ceil(N/128)) fp32 (each
+ *              expert's 128x128 scales, as fp8_quantize of that expert writes
+ *              them).
+ *   offs, out, out_dtype, alignment and the device-side offs check as for
+ *   fp8_grouped_scaled_mm.
+ * Requirements: K % 128 == 0, N % 16 == 0, 1 <= E <= 65535.
+ */
+FP8SM_API fp8_status fp8_grouped_scaled_mm_blockwise(const void* a, const void* b_experts,
+                                                     int64_t M_total, int64_t N, int64_t K,
+                                                     int32_t E, const float* scale_a,
+                                                     const float* scale_b, const int32_t* offs,
+                                                     fp8_out_dtype out_dtype, void* out,
+                                                     fp8_stream_t stream);
+
+/*
  * Synchronizes `stream`, then returns and clears the current device's status
  * word: FP8_OK, FP8_ERR_VALUE (malformed offs), FP8_ERR_TIMEOUT (a pipeline
  * wait gave up; the kernel released its resources and returned), or
