@@ -37,6 +37,8 @@ def lib():
         L.or_e4m3_encode_bits.argtypes = [P, I64, P]
         L.or_quantize.restype = ctypes.c_int
         L.or_quantize.argtypes = [P, I64, I64, I64, ctypes.c_int, P, P]
+        L.or_quantize_f32.restype = ctypes.c_int
+        L.or_quantize_f32.argtypes = [P, I64, I64, I64, ctypes.c_int, P, P]
         L.or_cast_with_inverse.restype = ctypes.c_int
         L.or_cast_with_inverse.argtypes = [P, I64, I64, I64, ctypes.c_float, P]
         L.or_scaled_mm.restype = ctypes.c_int
@@ -103,6 +105,21 @@ def quantize(x_bits: np.ndarray, group: int):
     rc = lib().or_quantize(_ptr(x_bits), rows, cols, cols, group, _ptr(q), _ptr(s))
     if rc != 0:
         raise ValueError("oracle quantize: bad arguments")
+    return q, s[:scale_count(rows, cols, group)]
+
+
+def quantize_f32(x: np.ndarray, group: int):
+    """The same quantization steps on an fp32 matrix (2-D): for checking a
+    GEMM epilogue that quantizes its fp32 result.
+
+    Returns (q uint8 (rows, cols), scales float32 (scale_count,))."""
+    x = _c(x, np.float32)
+    rows, cols = x.shape
+    q = np.empty((rows, cols), dtype=np.uint8)
+    s = np.empty(max(scale_count(rows, cols, group), 1), dtype=np.float32)
+    rc = lib().or_quantize_f32(_ptr(x), rows, cols, cols, group, _ptr(q), _ptr(s))
+    if rc != 0:
+        raise ValueError("oracle quantize_f32: bad arguments")
     return q, s[:scale_count(rows, cols, group)]
 
 

@@ -144,18 +144,23 @@ float or_bf16_to_float(uint16_t h) {
  *   4. y = x * inv                       (one fp32 multiply)
  *   5. q = e4m3(y), RNE, saturating */
 typedef struct {
-  const uint16_t* x;
+  const uint16_t* x;   /* bf16 input, or */
+  const float* xf;     /* fp32 input (when not NULL) */
   int64_t ld;
   uint8_t* q;
   int64_t ldq;
 } mat_view;
+
+static float mv_get(const mat_view* v, int64_t i) {
+  return v->xf ? v->xf[i] : or_bf16_to_float(v->x[i]);
+}
 
 static float group_scale(const mat_view* v, int64_t r0, int64_t r1, int64_t c0,
                          int64_t c1, float* inv_out) {
   float amax = 0.0f;
   for (int64_t r = r0; r < r1; r++)
     for (int64_t c = c0; c < c1; c++) {
-      float f = fabsf(or_bf16_to_float(v->x[r * v->ld + c]));
+      float f = fabsf(mv_get(v, r * v->ld + c));
       if (f > amax) amax = f;
     }
   float a = amax > OR_EPS ? amax : OR_EPS;
@@ -169,15 +174,14 @@ static void group_cast(const mat_view* v, int64_t r0, int64_t r1, int64_t c0,
                        int64_t c1, float inv) {
   for (int64_t r = r0; r < r1; r++)
     for (int64_t c = c0; c < c1; c++) {
-      volatile float y = or_bf16_to_float(v->x[r * v->ld + c]) * inv;
+      volatile float y = mv_get(v, r * v->ld + c) * inv;
       v->q[r * v->ldq + c] = or_e4m3_encode(y);
     }
 }
 
-int or_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
-                int group, uint8_t* q, float* scales) {
-  if (rows < 0 || cols < 0 || ld < cols || !x || !q || !scales) return -1;
-  mat_view v = {x, ld, q, cols};
+static int quantize_view(const mat_view* vp, int64_t rows, int64_t cols, int group,
+                         float* scales) {
+  const mat_view v = *vp;
   if (group == OR_GROUP_TENSOR) {
     float inv;
     scales[0] = group_scale(&v, 0, rows, 0, cols, &inv);
@@ -225,10 +229,26 @@ int or_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
   return -1;
 }
 
+int or_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                int group, uint8_t* q, float* scales) {
+  if (rows < 0 || cols < 0 || ld < cols || !x || !q || !scales) return -1;
+  mat_view v = {x, NULL, ld, q, cols};
+  return quantize_view(&v, rows, cols, group, scales);
+}
+
+/* The same steps on fp32 input (a GEMM result quantized for the next FP8
+ * operation). */
+int or_quantize_f32(const float* x, int64_t rows, int64_t cols, int64_t ld,
+                    int group, uint8_t* q, float* scales) {
+  if (rows < 0 || cols < 0 || ld < cols || !x || !q || !scales) return -1;
+  mat_view v = {NULL, x, ld, q, cols};
+  return quantize_view(&v, rows, cols, group, scales);
+}
+
 int or_cast_with_inverse(const uint16_t* x, int64_t rows, int64_t cols,
                          int64_t ld, float inv, uint8_t* q) {
   if (rows < 0 || cols < 0 || ld < cols || !x || !q) return -1;
-  mat_view v = {x, ld, q, cols};
+  mat_view v = {x, NULL, ld, q, cols};
   group_cast(&v, 0, rows, 0, cols, inv);
   return 0;
 }

@@ -71,6 +71,11 @@ float or_bf16_to_float(uint16_t h);
 int or_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
                 int group, uint8_t* q, float* scales);
 
+/* or_quantize on fp32 input x (row stride ld): the same steps; used to check
+ * a GEMM whose epilogue quantizes its fp32 result. */
+int or_quantize_f32(const float* x, int64_t rows, int64_t cols, int64_t ld,
+                    int group, uint8_t* q, float* scales);
+
 /* Cast step alone with a caller-supplied inverse scale: q = e4m3(x * inv).
  * Used to pin saturation, which the amax-derived scale never reaches. */
 int or_cast_with_inverse(const uint16_t* x, int64_t rows, int64_t cols,
