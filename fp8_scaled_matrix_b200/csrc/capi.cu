@@ -252,8 +252,48 @@ fp8_status fp8_scaled_mm(const void* a, const void* b, int64_t M, int64_t N,
                        d->num_sms, &err};
   cudaError_t e = fp8sm::launch_scaled_mm(a, b, M, N, K, scale_a, scale_b,
                                           (int)recipe, bias_bf16,
-                                          out_dtype == FP8_OUT_F32, out, ctx);
+                                          out_dtype == FP8_OUT_F32 ? 1 : 0, out, nullptr, ctx);
   return finish_launch(e, err, "fp8_scaled_mm");
+}
+
+fp8_status fp8_scaled_mm_quantized(const void* a, const void* b, int64_t M, int64_t N,
+                                   int64_t K, const float* scale_a, const float* scale_b,
+                                   fp8_mm_recipe recipe, const void* bias_bf16,
+                                   void* out_fp8, float* out_scales, fp8_stream_t stream) {
+  if (recipe < FP8_MM_TENSOR_TENSOR || recipe > FP8_MM_1x128_128x1)
+    return fail(FP8_ERR_VALUE, "fp8_scaled_mm_quantized: unknown recipe");
+  if (M < 0 || N < 0 || K < 0)
+    return fail(FP8_ERR_VALUE, "fp8_scaled_mm_quantized: negative size");
+  if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+    return fail(FP8_ERR_VALUE, "fp8_scaled_mm_quantized: size too large");
+  if (K == 0 || K % 16 != 0)
+    return fail(FP8_ERR_VALUE, "fp8_scaled_mm_quantized: K must be a positive multiple of 16");
+  if (N % 128 != 0)
+    return fail(FP8_ERR_VALUE,
+                "fp8_scaled_mm_quantized: N must be a multiple of 128 (1x128 output groups)");
+  const bool blockwise = recipe == FP8_MM_1x128_128x128 || recipe == FP8_MM_1x128_128x1;
+  if (blockwise && K % 128 != 0)
+    return fail(FP8_ERR_VALUE, "fp8_scaled_mm_quantized: blockwise recipes need K % 128 == 0");
+  if (M == 0 || N == 0) {
+    t_last_error.clear();
+    return FP8_OK;
+  }
+  if (a == nullptr || b == nullptr || scale_a == nullptr || scale_b == nullptr ||
+      out_fp8 == nullptr || out_scales == nullptr)
+    return fail(FP8_ERR_VALUE, "fp8_scaled_mm_quantized: null pointer");
+  if (!aligned(out_fp8, 16) || !aligned(a, 16) || !aligned(b, 16) ||
+      (bias_bf16 && !aligned(bias_bf16, 16)) || !aligned(scale_a, 16) ||
+      !aligned(scale_b, 16) || !aligned(out_scales, 4))
+    return fail(FP8_ERR_VALUE, "fp8_scaled_mm_quantized: misaligned pointer");
+  DeviceInfo* d = nullptr;
+  fp8_status s = device_info(&d);
+  if (s != FP8_OK) return s;
+  std::string err;
+  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status,
+                       d->num_sms, &err};
+  cudaError_t e = fp8sm::launch_scaled_mm(a, b, M, N, K, scale_a, scale_b, (int)recipe,
+                                          bias_bf16, 2, out_fp8, out_scales, ctx);
+  return finish_launch(e, err, "fp8_scaled_mm_quantized");
 }
 
 namespace {

@@ -44,6 +44,7 @@
 
 #include <cstdlib>
 
+#include "fp8cast.cuh"
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -102,6 +103,8 @@ struct Cfg {
 };
 
 enum Recipe : int { kTensor = 0, kRow = 1, kBlock128 = 2, kBlock1 = 3 };
+// Output: bf16, fp32, or e4m3 quantized in 1x128 groups along n (+ scales)
+enum OutKind : int { kOutBf16 = 0, kOutFp32 = 1, kOutE4M3 = 2 };
 
 struct GemmParams {
   int64_t M, N, K;
@@ -109,6 +112,7 @@ struct GemmParams {
   const float* sb;
   const uint16_t* bias;
   void* out;
+  float* out_scales;  // e4m3 output: scale[(n/128) * M + m]
   const int32_t* offs;
   int32_t E;
   int32_t n_tiles;   // tiles along N
@@ -309,7 +313,7 @@ __device__ __forceinline__ void store_cols32(
   }
 }
 
-template <int kRecipe, bool kOutF32, bool kGrouped, bool kPair>
+template <int kRecipe, int kOut, bool kGrouped, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
                     const __grid_constant__ CUtensorMap tm_b,
@@ -317,6 +321,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tm_out,
                     const GemmParams p) {
   constexpr bool kBlockwise = (kRecipe == kBlock128 || kRecipe == kBlock1);
+  constexpr bool kOutF32 = kOut == kOutFp32;
+  constexpr bool kOutQ = kOut == kOutE4M3;
   using C = Cfg<kPair>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -700,20 +706,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         else sa = row_ok ? __ldg(p.sa + row) : 0.0f;
         const float* sbg = p.sb + (kGrouped ? static_cast<int64_t>(c.g) * p.N : 0);
         const uint32_t tcol = tmem_base + lane_base + acc * BN + half * 128;
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
+        // the fp32 results of 32-column chunk cc of this thread's row
+        auto values32 = [&](int cc, float (&v)[32]) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(tcol + cc * 32, r);
           tmem_ld_wait();
-          if (cc == 3) {
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) release_acc(acc);
-          }
           const int64_t n = ncol0 + cc * 32;
           float bias[32];
           load_bias32(p.bias, n, p.N, bias);
-          float v[32];
           if constexpr (kRecipe == kTensor) {
 #pragma unroll
             for (int i = 0; i < 32; ++i)
@@ -725,9 +725,54 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 32; ++i)
               v[i] = fmaf(__uint_as_float(r[i]), sa * sb[i], bias[i]);
           }
-          store_cols32<kOutF32, kGrouped>(ebuf, v, &tm_out,
-                                          static_cast<int32_t>(n), row0,
-                                          c.row_end, p.out, p.N, lane);
+        };
+        auto release_buf = [&]() {
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) release_acc(acc);
+        };
+        if constexpr (!kOutQ) {
+#pragma unroll 1
+          for (int cc = 0; cc < 4; ++cc) {
+            float v[32];
+            values32(cc, v);
+            if (cc == 3) release_buf();
+            store_cols32<kOutF32, kGrouped>(ebuf, v, &tm_out,
+                                            static_cast<int32_t>(ncol0 + cc * 32), row0,
+                                            c.row_end, p.out, p.N, lane);
+          }
+        } else {
+          // e4m3 output in 1x128 groups along n: the group is this thread's
+          // 128 columns of its row.  Pass 1 finds its amax; pass 2 reads the
+          // accumulators again (TMEM reads are cheap next to the MMAs),
+          // recomputes the same fp32 values, casts and stores them.
+          float am = 0.0f;
+#pragma unroll 1
+          for (int cc = 0; cc < 4; ++cc) {
+            float v[32];
+            values32(cc, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(v[i]));
+          }
+          const ScalePair sp = scales_from_amax(am);
+          if (row_ok && ncol0 < p.N) p.out_scales[(ncol0 / 128) * p.M + row] = sp.s;
+#pragma unroll 1
+          for (int bx = 0; bx < 2; ++bx) {
+            uint4 chunk[4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              float v[32];
+              values32(2 * bx + h, v);
+              if (bx == 1 && h == 1) release_buf();
+              uint32_t* w = reinterpret_cast<uint32_t*>(&chunk[2 * h]);
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                w[j] = cast_f32x2(v[4 * j], v[4 * j + 1], sp.inv) |
+                       (cast_f32x2(v[4 * j + 2], v[4 * j + 3], sp.inv) << 16);
+            }
+            store_box64<kGrouped>(ebuf, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
+                                  row0, c.row_end, static_cast<uint8_t*>(p.out), p.N, 1, lane);
+          }
         }
         acc ^= 1u;
         if (acc == 0) acc_phase ^= 1u;
@@ -800,19 +845,52 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (acc == 0) acc_phase ^= 1u;
         }
         if (!ok) break;
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int64_t n = ncol0 + cc * 32;
-          float v[32];
-          load_bias32(p.bias, n, p.N, v);
+        // the tile's fp32 results for chunk cc (bias added)
+        auto result32 = [&](int cc, float (&v)[32]) {
+          load_bias32(p.bias, ncol0 + cc * 32, p.N, v);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             v[2 * i] += accr[cc * 16 + i].x;
             v[2 * i + 1] += accr[cc * 16 + i].y;
           }
-          store_cols32<kOutF32, kGrouped>(ebuf, v, &tm_out,
-                                          static_cast<int32_t>(n), row0,
-                                          c.row_end, p.out, p.N, lane);
+        };
+        if constexpr (!kOutQ) {
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            float v[32];
+            result32(cc, v);
+            store_cols32<kOutF32, kGrouped>(ebuf, v, &tm_out,
+                                            static_cast<int32_t>(ncol0 + cc * 32), row0,
+                                            c.row_end, p.out, p.N, lane);
+          }
+        } else {
+          // e4m3 output in 1x128 groups along n (this thread's 128 columns)
+          float am = 0.0f;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            float v[32];
+            result32(cc, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(v[i]));
+          }
+          const ScalePair sp = scales_from_amax(am);
+          if (row_ok && ncol0 < p.N) p.out_scales[(ncol0 / 128) * p.M + row] = sp.s;
+#pragma unroll
+          for (int bx = 0; bx < 2; ++bx) {
+            uint4 chunk[4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              float v[32];
+              result32(2 * bx + h, v);
+              uint32_t* w = reinterpret_cast<uint32_t*>(&chunk[2 * h]);
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                w[j] = cast_f32x2(v[4 * j], v[4 * j + 1], sp.inv) |
+                       (cast_f32x2(v[4 * j + 2], v[4 * j + 3], sp.inv) << 16);
+            }
+            store_box64<kGrouped>(ebuf, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
+                                  row0, c.row_end, static_cast<uint8_t*>(p.out), p.N, 1, lane);
+          }
         }
       }
     }
@@ -895,17 +973,19 @@ bool make_tmap(CUtensorMap* m, CUtensorMapDataType dt, uint32_t rank,
   return true;
 }
 
-template <int kRecipe, bool kOutF32, bool kGrouped, bool kPair>
+template <int kRecipe, int kOut, bool kGrouped, bool kPair>
 cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb,
                           const CUtensorMap& tbh, const CUtensorMap& to,
                           const GemmParams& p, unsigned grid, cudaStream_t st) {
   constexpr bool kBlockwise = kRecipe == kBlock128 || kRecipe == kBlock1;
   if constexpr (kPair && kBlockwise) {
     return cudaErrorInvalidValue;  // CTA pairs serve the dense recipes only
+  } else if constexpr (kOut == kOutE4M3 && (kPair || kGrouped)) {
+    return cudaErrorInvalidValue;  // quantized output: single-CTA dense GEMM only
   } else {
     using C = Cfg<kPair>;
     static bool configured = false;
-    auto kern = fp8_gemm_kernel<kRecipe, kOutF32, kGrouped, kPair>;
+    auto kern = fp8_gemm_kernel<kRecipe, kOut, kGrouped, kPair>;
     if (!configured) {
       cudaError_t e = cudaFuncSetAttribute(
           kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
@@ -938,17 +1018,19 @@ cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb,
 }
 
 template <bool kGrouped>
-cudaError_t dispatch(int recipe, int out_f32, bool pair, const CUtensorMap& ta,
+cudaError_t dispatch(int recipe, int out_kind, bool pair, const CUtensorMap& ta,
                      const CUtensorMap& tb, const CUtensorMap& tbh,
                      const CUtensorMap& to, const GemmParams& p, unsigned grid,
                      cudaStream_t st) {
 #define FP8SM_CASE(R)                                                                   \
   if (recipe == R) {                                                                    \
+    if (out_kind == kOutE4M3)                                                           \
+      return launch_kernel<R, kOutE4M3, kGrouped, false>(ta, tb, tbh, to, p, grid, st); \
     if (pair)                                                                           \
-      return out_f32 ? launch_kernel<R, true, kGrouped, true>(ta, tb, tbh, to, p, grid, st)   \
-                     : launch_kernel<R, false, kGrouped, true>(ta, tb, tbh, to, p, grid, st); \
-    return out_f32 ? launch_kernel<R, true, kGrouped, false>(ta, tb, tbh, to, p, grid, st)    \
-                   : launch_kernel<R, false, kGrouped, false>(ta, tb, tbh, to, p, grid, st);  \
+      return out_kind ? launch_kernel<R, kOutFp32, kGrouped, true>(ta, tb, tbh, to, p, grid, st) \
+                      : launch_kernel<R, kOutBf16, kGrouped, true>(ta, tb, tbh, to, p, grid, st); \
+    return out_kind ? launch_kernel<R, kOutFp32, kGrouped, false>(ta, tb, tbh, to, p, grid, st)  \
+                    : launch_kernel<R, kOutBf16, kGrouped, false>(ta, tb, tbh, to, p, grid, st); \
   }
   if constexpr (kGrouped) {
     FP8SM_CASE(kRow)
@@ -963,15 +1045,18 @@ cudaError_t dispatch(int recipe, int out_f32, bool pair, const CUtensorMap& ta,
   return cudaErrorInvalidValue;
 }
 
-bool out_map(CUtensorMap* m, void* out, int64_t rows, int64_t N, int out_f32,
+// Output map: 32-row x 64-byte boxes, 64-byte swizzle (the epilogue's
+// staging layout) for bf16, fp32 or e4m3 output.
+bool out_map(CUtensorMap* m, void* out, int64_t rows, int64_t N, int out_kind,
              std::string* err) {
-  const uint64_t eb = out_f32 ? 4 : 2;
+  const uint64_t eb = out_kind == kOutFp32 ? 4 : out_kind == kOutE4M3 ? 1 : 2;
   uint64_t dims[2] = {static_cast<uint64_t>(N), static_cast<uint64_t>(rows)};
   uint64_t strides[1] = {static_cast<uint64_t>(N) * eb};
   uint32_t box[2] = {static_cast<uint32_t>(64 / eb), 32};
-  return make_tmap(m, out_f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
-                              : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                   2, out, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B, err);
+  const CUtensorMapDataType dt = out_kind == kOutFp32   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : out_kind == kOutE4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                                        : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  return make_tmap(m, dt, 2, out, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B, err);
 }
 
 // A operand map: 128-row boxes (one CTA's rows) in both modes.
@@ -1001,8 +1086,11 @@ bool use_pair(int64_t M, int recipe) {
 cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
                              int64_t N, int64_t K, const float* sa,
                              const float* sb, int recipe, const void* bias,
-                             int out_f32, void* out, const LaunchCtx& ctx) {
+                             int out_kind, void* out, float* out_scales,
+                             const LaunchCtx& ctx) {
   if (M == 0 || N == 0) return cudaSuccess;
+  if (K == 0 && out_kind == kOutE4M3) return cudaErrorInvalidValue;
+  const int out_f32 = out_kind == kOutFp32;
   if (K == 0) {
     const int64_t total = M * N;
     int64_t blocks = (total + 255) / 256;
@@ -1031,8 +1119,9 @@ cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
                    CU_TENSOR_MAP_SWIZZLE_128B, ctx.err))
       return cudaErrorInvalidValue;
   }
-  if (!out_map(&to, out, M, N, out_f32, ctx.err)) return cudaErrorInvalidValue;
+  if (!out_map(&to, out, M, N, out_kind, ctx.err)) return cudaErrorInvalidValue;
   GemmParams p{};
+  p.out_scales = out_scales;
   p.M = M;
   p.N = N;
   p.K = K;
@@ -1062,7 +1151,7 @@ cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
   }
   const int64_t units = p.total_items < G ? p.total_items : G;
   const unsigned grid = static_cast<unsigned>(pair ? 2 * units : units);
-  return dispatch<false>(recipe, out_f32, pair, ta, tb, tbh, to, p, grid, ctx.stream);
+  return dispatch<false>(recipe, out_kind, pair, ta, tb, tbh, to, p, grid, ctx.stream);
 }
 
 cudaError_t launch_grouped_scaled_mm(const void* a, const void* b,
@@ -1074,7 +1163,7 @@ cudaError_t launch_grouped_scaled_mm(const void* a, const void* b,
   if (M_total == 0 || N == 0) return cudaSuccess;
   if (K == 0)
     return launch_scaled_mm(nullptr, nullptr, M_total, N, 0, nullptr, nullptr,
-                            1, nullptr, out_f32, out, ctx);
+                            1, nullptr, out_f32 ? kOutFp32 : kOutBf16, out, nullptr, ctx);
   const bool pair = use_pair(M_total, recipe);
   const uint32_t b_rows = pair ? Cfg<true>::kBRows : Cfg<false>::kBRows;
   CUtensorMap ta, tb, to;
@@ -1091,7 +1180,8 @@ cudaError_t launch_grouped_scaled_mm(const void* a, const void* b,
   }
   // The grouped kernel stores with plain masked stores; the map is unused
   // but must be a valid object.
-  if (!out_map(&to, out, M_total, N, out_f32, ctx.err)) return cudaErrorInvalidValue;
+  if (!out_map(&to, out, M_total, N, out_f32 ? kOutFp32 : kOutBf16, ctx.err))
+    return cudaErrorInvalidValue;
   GemmParams p{};
   p.M = M_total;
   p.N = N;

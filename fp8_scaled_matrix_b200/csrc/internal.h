@@ -34,11 +34,13 @@ size_t noalloc_scratch_bytes();
 cudaError_t noalloc_scratch_ptr(int device, void** out);
 
 // Dense scaled GEMM (gemm.cu).  recipe: 0 tensor, 1 row, 2 1x128_128x128,
-// 3 1x128_128x1.  out_f32: 0 -> bf16 output, 1 -> fp32 output.
+// 3 1x128_128x1.  out_kind: 0 bf16, 1 fp32, 2 e4m3 quantized in 1x128
+// groups along n with scales written to out_scales[(n/128) * M + m].
 cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
                              int64_t N, int64_t K, const float* sa,
                              const float* sb, int recipe, const void* bias,
-                             int out_f32, void* out, const LaunchCtx& ctx);
+                             int out_kind, void* out, float* out_scales,
+                             const LaunchCtx& ctx);
 
 // Grouped scaled GEMM (gemm.cu).  recipe: 1 rowwise, 2 1x128_128x128.
 cudaError_t launch_grouped_scaled_mm(const void* a, const void* b,

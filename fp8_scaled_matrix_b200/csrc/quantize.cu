@@ -19,24 +19,12 @@
 
 #include <mutex>
 
+#include "fp8cast.cuh"
 #include "internal.h"
 #include "sm100.cuh"
 
 namespace fp8sm {
 namespace {
-
-constexpr float kE4M3Max = 448.0f;
-constexpr float kEps = 1e-12f;
-
-struct ScalePair {
-  float s;    // dequantization multiplier, stored
-  float inv;  // quantization multiplier
-};
-
-__device__ __forceinline__ ScalePair scales_from_amax(float amax) {
-  const float a = fmaxf(amax, kEps);
-  return {__fdiv_rn(a, kE4M3Max), __fdiv_rn(kE4M3Max, a)};
-}
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) {
   return __uint_as_float(w << 16);
@@ -58,10 +46,7 @@ __device__ __forceinline__ float amax8(const uint4& v, float m) {
 }
 
 __device__ __forceinline__ uint32_t cast2(uint32_t w, float inv) {
-  const float2 y = make_float2(__fmul_rn(bf16_lo(w), inv),
-                               __fmul_rn(bf16_hi(w), inv));
-  return static_cast<uint32_t>(
-      __nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3));
+  return cast_f32x2(bf16_lo(w), bf16_hi(w), inv);
 }
 
 // 8 bf16 -> 8 e4m3 bytes (little-endian order preserved).

@@ -210,6 +210,33 @@ FP8SM_API fp8_status fp8_scaled_mm(const void* a, const void* b, int64_t M, int6
                          fp8_stream_t stream);
 
 /*
+ * Scaled GEMM whose output leaves already quantized for the next layer's
+ * GEMM: the fp32 result of fp8_scaled_mm (same operands, recipes, bias and
+ * K-order of accumulation) is grouped 1x128 along n and each group is cast
+ * to e4m3 with its own scale, exactly as fp8_quantize's 1x128 recipe would
+ * cast those fp32 values:
+ *   y[m, n]       = fp8_scaled_mm(...)[m, n] in fp32
+ *   s[j, m]       = max(amax_{n in group j} |y[m, n]|, 1e-12) / 448
+ *   out[m, n]     = e4m3_satfinite_rn(y[m, n] * (1 / s[n / 128, m]))
+ * This is the chained FP8 linear of [P1] Solution (forward: x_fp8 @ w_fp8^T;
+ * its output is the next layer's x) with the activation quantize of [P3]
+ * and [P5] moved into the producing GEMM's epilogue, so the fp32/bf16 result
+ * never goes to HBM and no separate quantize pass reads it back.
+ *
+ *   a, b, scale_a, scale_b, recipe, bias_bf16: as fp8_scaled_mm.
+ *   out_fp8    (M, N) e4m3 row-major, 16-byte aligned.
+ *   out_scales (N / 128, M) fp32, K-block-major like fp8_quantize's 1x128
+ *              scales (entry [j * M + m]); 4-byte aligned.
+ * Requirements: K > 0, K % 16 == 0 (K % 128 == 0 for the blockwise recipes),
+ * N % 128 == 0.  M is arbitrary; M == 0 or N == 0 is a no-op.
+ */
+FP8SM_API fp8_status fp8_scaled_mm_quantized(const void* a, const void* b, int64_t M,
+                                   int64_t N, int64_t K, const float* scale_a,
+                                   const float* scale_b, fp8_mm_recipe recipe,
+                                   const void* bias_bf16, void* out_fp8,
+                                   float* out_scales, fp8_stream_t stream);
+
+/*
  * Grouped (MoE) scaled GEMM, rowwise recipe only ([P2] Design, RowWise path;
  * other weight granularities return FP8_ERR_UNSUPPORTED as [P2]'s review
  * requires):

@@ -126,6 +126,37 @@ def test_empty_gemm_is_a_noop_without_cuda(lib):
                              None, fp8sm.FP8_OUT_BF16, None, None) == fp8sm.FP8_OK
 
 
+@pytest.mark.parametrize("M,N,K,recipe,frag", [
+    (128, 192, 128, fp8sm.FP8_MM_ROW_ROW, "N must be a multiple of 128"),
+    (128, 128, 0, fp8sm.FP8_MM_ROW_ROW, "K must be a positive multiple of 16"),
+    (128, 128, 100, fp8sm.FP8_MM_TENSOR_TENSOR, "K must be a positive multiple of 16"),
+    (128, 128, 144, fp8sm.FP8_MM_1x128_128x128, "K % 128"),
+    (128, 128, 144, fp8sm.FP8_MM_1x128_128x1, "K % 128"),
+    (128, -128, 128, fp8sm.FP8_MM_ROW_ROW, "negative"),
+    (128, 128, 128, 7, "unknown recipe"),
+])
+def test_scaled_mm_quantized_rejects_bad_arguments(lib, M, N, K, recipe, frag):
+    st = lib.fp8_scaled_mm_quantized(FAKE, FAKE, M, N, K, FAKE, FAKE, recipe, None,
+                                     FAKE, FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE
+    assert frag in lib.fp8_last_error().decode()
+
+
+def test_scaled_mm_quantized_null_alignment_and_empty(lib):
+    st = lib.fp8_scaled_mm_quantized(FAKE, FAKE, 128, 128, 128, FAKE, FAKE,
+                                     fp8sm.FP8_MM_ROW_ROW, None, FAKE, None, None)
+    assert st == fp8sm.FP8_ERR_VALUE and "null" in lib.fp8_last_error().decode()
+    st = lib.fp8_scaled_mm_quantized(FAKE, FAKE, 128, 128, 128, FAKE, FAKE,
+                                     fp8sm.FP8_MM_ROW_ROW, None, P((1 << 20) + 4), FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE and "misaligned" in lib.fp8_last_error().decode()
+    st = lib.fp8_scaled_mm_quantized(FAKE, FAKE, 128, 128, 128, FAKE, FAKE,
+                                     fp8sm.FP8_MM_ROW_ROW, None, FAKE, P((1 << 20) + 2), None)
+    assert st == fp8sm.FP8_ERR_VALUE and "misaligned" in lib.fp8_last_error().decode()
+    assert lib.fp8_scaled_mm_quantized(None, None, 0, 128, 128, None, None,
+                                       fp8sm.FP8_MM_ROW_ROW, None, None, None,
+                                       None) == fp8sm.FP8_OK
+
+
 def test_grouped_requires_offs(lib):
     st = lib.fp8_grouped_scaled_mm(FAKE, FAKE, 64, 128, 128, 4, FAKE, FAKE, None,
                                    fp8sm.FP8_OUT_BF16, FAKE, None)

@@ -1,0 +1,165 @@
+"""The GEMM whose epilogue quantizes its own result (fp8_scaled_mm_quantized).
+
+Two checks per case.  (1) Exactness of the fused quantize: the fp32 result of
+the same GEMM (fp8_scaled_mm with fp32 output, same operands, same kernel
+schedule) quantized by the oracle's fp32 quantizer in 1x128 groups must give
+the same codes and scales bit for bit.  (2) End to end against the oracle's
+fp64 GEMM: the dequantized output (code * scale) is within the GEMM tolerance
+plus half an e4m3 step of the fp64 reference.  The GEMM itself is covered by
+the fp32-output parity tests; (1) pins the epilogue's amax, scale and cast."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp8_scaled_matrix_b200 import fp8sm
+from fp8_scaled_matrix_b200 import workloads as W
+from helpers import MM, OPERAND_GROUPS, QUANT_GROUP, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+MMR = {"tensor": fp8sm.FP8_MM_TENSOR_TENSOR, "row": fp8sm.FP8_MM_ROW_ROW,
+       "1x128_128x128": fp8sm.FP8_MM_1x128_128x128, "1x128_128x1": fp8sm.FP8_MM_1x128_128x1}
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """Value of each e4m3 code (OCP FP8 E4M3: bias 7, no infinities)."""
+    c = codes.astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    v = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * 2.0 ** (e - 7.0))
+    return sign * v
+
+
+def operands(recipe, M, N, K, seed, bias):
+    b_std = 0.02 if recipe != "1x128_128x1" else 1.0
+    a_std = 1.0 if recipe != "1x128_128x1" else 1e-3
+    wl = W.small_case(recipe, M, N, K, seed=seed, a_std=a_std, b_std=b_std, bias=bias)
+    ga, gb = OPERAND_GROUPS[recipe]
+    qa, sa = oracle.quantize(W.bf16_bits(wl.a), QUANT_GROUP[ga])
+    qb, sb = oracle.quantize(W.bf16_bits(wl.b), QUANT_GROUP[gb])
+    return wl, qa, sa, qb, sb
+
+
+def run_both(qa, sa, qb, sb, recipe, bias):
+    a, b = torch.from_numpy(qa).cuda(), torch.from_numpy(qb).cuda()
+    sad, sbd = torch.from_numpy(sa).cuda(), torch.from_numpy(sb).cuda()
+    bd = None if bias is None else bias.cuda()
+    y = fp8sm.fp8_scaled_mm(a, b, sad, sbd, MMR[recipe], bias=bd, out_dtype=torch.float32)
+    q, s = fp8sm.fp8_scaled_mm_quantized(a, b, sad, sbd, MMR[recipe], bias=bd)
+    torch.cuda.synchronize()
+    fp8sm.check_device_status()
+    return y.cpu().numpy(), q.cpu().numpy(), s.cpu().numpy()
+
+
+def check_exact(y, q, s, what):
+    rq, rs = oracle.quantize_f32(y, oracle.GROUP_1x128)
+    rs = rs.reshape(s.shape)
+    bad_s = np.argwhere(rs.view(np.uint32) != s.view(np.uint32))
+    assert bad_s.size == 0, f"{what}: {len(bad_s)} scales differ, first {bad_s[0]}"
+    bad = np.argwhere(rq != q)
+    assert bad.size == 0, (f"{what}: {len(bad)} codes differ, first {bad[0]} "
+                           f"gpu={q[tuple(bad[0])]:#x} oracle={rq[tuple(bad[0])]:#x}")
+
+
+def check_against_fp64(q, s, ref, mag, what):
+    M, N = q.shape
+    scale = s.reshape(N // 128, M).T.repeat(128, axis=1).astype(np.float64)
+    deq = e4m3_decode(q) * scale
+    # the GEMM tolerance for the fp32 value y, then the rounding of y to e4m3:
+    # half a step, 2^-4 |y| for normal codes and 2^-10 scale below them
+    gemm_tol = 1e-2 * np.abs(ref) + 1e-3 * mag
+    tol = gemm_tol + 2.0 ** -4 * (np.abs(ref) + gemm_tol) + scale * 2.0 ** -9
+    err = np.abs(deq - ref)
+    bad = np.argwhere(err > tol)
+    assert bad.size == 0, (f"{what}: {len(bad)} elements out of tolerance, first "
+                           f"{bad[0]} deq={deq[tuple(bad[0])]} ref={ref[tuple(bad[0])]}")
+
+
+CASES = [
+    # recipe, M, N, K, bias
+    ("tensor", 300, 256, 528, True),
+    ("tensor", 1, 128, 16, False),
+    ("row", 129, 512, 4096, True),
+    ("row", 300, 384, 528, False),           # last tile half empty along n
+    ("row", 4096, 4096, 256, True),          # last wave split into 128-wide items
+    ("row", 7, 128, 32, True),
+    ("1x128_128x128", 260, 384, 384, True),
+    ("1x128_128x128", 1100, 2304, 1024, False),
+    ("1x128_128x1", 130, 512, 256, False),
+    ("1x128_128x1", 64, 128, 128, True),
+    ("1x128_128x1", 2304, 4352, 512, False),
+]
+
+
+@pytest.mark.parametrize("recipe,M,N,K,bias", CASES)
+def test_quantized_output_parity(recipe, M, N, K, bias):
+    seed = M * 17 + N * 5 + K + 3
+    wl, qa, sa, qb, sb = operands(recipe, M, N, K, seed, bias)
+    y, q, s = run_both(qa, sa, qb, sb, recipe, wl.bias)
+    what = f"{recipe} {M}x{N}x{K}"
+    check_exact(y, q, s, what)
+    rows = sample_rows(M, n=64, seed=seed)
+    bias_bits = None if wl.bias is None else W.bf16_bits(wl.bias)
+    ref, mag = oracle.scaled_mm(qa, qb, sa, sb, MM[recipe], bias_bits=bias_bits, rows=rows)
+    check_against_fp64(q[rows], s.reshape(N // 128, M)[:, rows].copy(), ref, mag, what)
+
+
+@pytest.mark.parametrize("recipe", ["row", "1x128_128x128"])
+def test_quantized_output_zero_groups(recipe):
+    """Rows of a that are all zero give all-zero groups (no bias): code 0 with
+    the floor scale 1e-12/448; rows that are not zero are unaffected."""
+    M, N, K = 200, 256, 256
+    wl, qa, sa, qb, sb = operands(recipe, M, N, K, 11, False)
+    qa[:3] = 0
+    qa[150] = 0
+    y, q, s = run_both(qa, sa, qb, sb, recipe, None)
+    check_exact(y, q, s, f"{recipe} zero rows")
+    s2 = s.reshape(N // 128, M)
+    floor = np.float32(np.float32(1e-12) / np.float32(448.0))
+    for r in (0, 1, 2, 150):
+        assert (q[r] == 0).all()
+        assert (s2[:, r] == floor).all()
+
+
+def test_quantized_output_constant_group():
+    """A group whose values are all equal maps to code 0x7e (448) exactly."""
+    M, N, K = 64, 128, 128
+    a = torch.zeros(M, K, dtype=torch.uint8, device="cuda")
+    b = torch.zeros(N, K, dtype=torch.uint8, device="cuda")
+    one = torch.ones(1, dtype=torch.float32, device="cuda")
+    bias = torch.full((N,), -3.0, dtype=torch.bfloat16, device="cuda")
+    q, s = fp8sm.fp8_scaled_mm_quantized(a, b, one, one, fp8sm.FP8_MM_TENSOR_TENSOR,
+                                         bias=bias)
+    torch.cuda.synchronize()
+    assert (q.cpu() == 0xFE).all()          # -448
+    assert torch.equal(s.cpu(), torch.full((1, M), float(np.float32(3.0) / np.float32(448.0)),
+                                              dtype=torch.float32))
+
+
+QR = {"row": fp8sm.FP8_SCALE_ROW, "1x128": fp8sm.FP8_SCALE_BLOCK_1x128,
+      "128x128": fp8sm.FP8_SCALE_BLOCK_128x128}
+
+
+@pytest.mark.parametrize("idx,shape_index", [(1, 0), (2, 0), (3, 1)])
+def test_quantized_output_full_size_sampled(idx, shape_index):
+    """Workload shapes (rowwise 4096^3 with bias; blockwise 16640x5120x8192 and
+    16640x8192x5120): the quantized output against the oracle's quantizer on
+    sampled rows of the same kernel schedule's fp32 result."""
+    wl = W.make_workload(idx, shape_index)
+    ga, gb = OPERAND_GROUPS[wl.recipe]
+    a, b = wl.a.cuda(), wl.b.cuda()
+    qa, sa = fp8sm.fp8_quantize(a, QR[ga])
+    qb, sb = fp8sm.fp8_quantize(b, QR[gb])
+    del a, b
+    bd = None if wl.bias is None else wl.bias.cuda()
+    q, s = fp8sm.fp8_scaled_mm_quantized(qa, qb, sa, sb, MMR[wl.recipe], bias=bd)
+    y = fp8sm.fp8_scaled_mm(qa, qb, sa, sb, MMR[wl.recipe], bias=bd, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    fp8sm.check_device_status()
+    rows = torch.from_numpy(sample_rows(wl.M, n=96, seed=idx)).cuda()
+    ys = y.index_select(0, rows).cpu().numpy()
+    qs = q.index_select(0, rows).cpu().numpy()
+    ss = s.index_select(1, rows).cpu().numpy()
+    check_exact(ys, qs, ss, f"{wl.name} full size")
