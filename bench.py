@@ -51,6 +51,7 @@ WORKLOADS = {
     "grad_input_1x128_128x128": (5, 0),
     "grad_weight_1x128_128x1": (6, 0),
     "grouped_e16_blockwise": (7, 0),
+    "linear_chain_1x128_128x128": (8, 0),
 }
 DEFAULT_WORKLOAD = "rowwise_4096"
 # Page 5's context numbers (TFLOP/s of torch._scaled_mm, hardware not stated)
@@ -62,10 +63,11 @@ OPERAND_GROUPS = {"tensor": ("tensor", "tensor"), "row": ("row", "row"),
                   "1x128_128x128": ("1x128", "128x128"),
                   "1x128_128x1": ("1x128", "1x128"), "grouped": ("row", "row"),
                   "grad_input": ("1x128", "128x128"), "grad_weight": ("1x128", "1x128"),
-                  "grouped_blockwise": ("1x128", "128x128")}
+                  "grouped_blockwise": ("1x128", "128x128"), "chain": ("1x128", "128x128")}
 # GEMM recipe of each workload recipe, and which operands are quantized
 # transposed (the training GEMMs contract along the stored rows)
-GEMM_RECIPE = {"grad_input": "1x128_128x128", "grad_weight": "1x128_128x1"}
+GEMM_RECIPE = {"grad_input": "1x128_128x128", "grad_weight": "1x128_128x1",
+               "chain": "1x128_128x128"}
 TRANSPOSED = {"grad_input": (False, True), "grad_weight": (True, True)}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_OVER_BF16 = 2.0   # nominal dense ratio (4.5 / 2.25 PFLOP/s)
@@ -240,6 +242,20 @@ class Step:
             self.sb = torch.empty(E * fp8sm.scale_count(N, K, self.qb_recipe),
                                   dtype=torch.float32, device=dev)
             self.launches_per_step = 2 + E
+        self.chain = wl.recipe == "chain"
+        if self.chain:
+            # second linear: its weight (N2, N) quantized 128x128 like b; the
+            # first GEMM's output leaves as e4m3 codes + 1x128 scales
+            # ((N/128, M), the A-operand scale layout of the second GEMM)
+            self.b2 = wl.extra["b2"].to(dev)
+            n2 = self.b2.shape[0]
+            self.qb2 = torch.empty(n2, wl.N, dtype=torch.uint8, device=dev)
+            self.sb2 = torch.empty(fp8sm.scale_count(n2, wl.N, self.qb_recipe),
+                                   dtype=torch.float32, device=dev)
+            self.y1q = torch.empty(wl.M, wl.N, dtype=torch.uint8, device=dev)
+            self.y1s = torch.empty(wl.N // 128, wl.M, dtype=torch.float32, device=dev)
+            self.out = torch.empty(wl.M, n2, dtype=torch.bfloat16, device=dev)
+            self.launches_per_step = 5
 
     def quantize(self):
         """Both operands' quantization; the second runs on a side stream,
@@ -260,6 +276,11 @@ class Step:
             elif self.t_b:
                 f.fp8_quantize_transposed(self.b, self.qb_recipe, out=self.qb, scales=self.sb,
                                           stream=self.side)
+            elif self.chain:
+                f.fp8_quantize(self.b, self.qb_recipe, out=self.qb, scales=self.sb,
+                               workspace=self.ws_b, stream=self.side)
+                f.fp8_quantize(self.b2, self.qb_recipe, out=self.qb2, scales=self.sb2,
+                               workspace=self.ws_b, stream=self.side)
             else:
                 f.fp8_quantize(self.b, self.qb_recipe, out=self.qb, scales=self.sb,
                                workspace=self.ws_b, stream=self.side)
@@ -283,6 +304,11 @@ class Step:
             E, N, K = wl.b.shape
             f.fp8_grouped_scaled_mm_blockwise(self.qa, self.qb.view(E, N, K), self.sa,
                                               self.sb, self.offs, out=self.out)
+        elif self.chain:
+            r = f.MM_RECIPES["1x128_128x128"]
+            f.fp8_scaled_mm_quantized(self.qa, self.qb, self.sa, self.sb, r,
+                                      out=self.y1q, out_scales=self.y1s)
+            f.fp8_scaled_mm(self.y1q, self.qb2, self.y1s, self.sb2, r, out=self.out)
         else:
             f.fp8_scaled_mm(self.qa, self.qb, self.sa, self.sb,
                             f.MM_RECIPES[GEMM_RECIPE.get(wl.recipe, wl.recipe)],
@@ -292,7 +318,10 @@ class Step:
         """Algorithmic HBM bytes of the two quantize launches: 2 B read +
         1 B written per element, 4 B per scale."""
         n = self.a.numel() + self.b.numel()
-        return 3 * n + 4 * (self.sa.numel() + self.sb.numel())
+        b = 3 * n + 4 * (self.sa.numel() + self.sb.numel())
+        if self.chain:
+            b += 3 * self.b2.numel() + 4 * self.sb2.numel()
+        return b
 
 
 def evict_l2(flush: torch.Tensor):
@@ -379,8 +408,9 @@ def run_e2e(args, wl, dev, world):
     hb = (wl.b.reshape(-1, wl.K) if wl.recipe in ("grouped", "grouped_blockwise")
           else wl.b).contiguous().pin_memory()
     hbias = None if wl.bias is None else wl.bias.pin_memory()
-    hout = torch.empty(wl.M, wl.N, dtype=torch.bfloat16).pin_memory()
+    hb2 = wl.extra["b2"].pin_memory() if "b2" in wl.extra else None
     st = Step(wl, dev)
+    hout = torch.empty(tuple(st.out.shape), dtype=torch.bfloat16).pin_memory()
     da, db = st.a, st.b
     dbias = st.bias
     stream = torch.cuda.current_stream()
@@ -391,6 +421,8 @@ def run_e2e(args, wl, dev, world):
         db.copy_(hb, non_blocking=True)
         if hbias is not None:
             dbias.copy_(hbias, non_blocking=True)
+        if hb2 is not None:
+            st.b2.copy_(hb2, non_blocking=True)
         st.quantize()
         st.gemm()
         hout.copy_(st.out, non_blocking=True)
@@ -408,7 +440,8 @@ def run_e2e(args, wl, dev, world):
     e1.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1) / steps, dev)
-    h2d = ha.numel() * 2 + hb.numel() * 2 + (0 if hbias is None else hbias.numel() * 2)
+    h2d = (ha.numel() * 2 + hb.numel() * 2 + (0 if hbias is None else hbias.numel() * 2)
+           + (0 if hb2 is None else hb2.numel() * 2))
     d2h = hout.numel() * 2
     return {"ms": ms, "h2d": h2d, "d2h": d2h, "steps": steps}
 
@@ -443,6 +476,8 @@ def oracle_sample(wl, max_rows: int):
         sb = np.stack([s for _, s in per_expert])
     else:
         qb, sb = oracle.quantize(bits(wl.b, t_b), G[gb])
+    if wl.recipe == "chain":
+        qb2, sb2 = oracle.quantize(W.bf16_bits(wl.extra["b2"]), G[gb])
     tq = time.perf_counter() - t0
     rows = np.arange(min(max_rows, wl.M), dtype=np.int64)
     t0 = time.perf_counter()
@@ -462,6 +497,12 @@ def oracle_sample(wl, max_rows: int):
                                  np.ascontiguousarray(sa2[:, start:end]).reshape(-1),
                                  sb[e].reshape(-1), MMR["1x128_128x128"], rows=sel - start)
             start = int(end)
+    elif wl.recipe == "chain":
+        # first linear on the sampled rows, its fp32 result quantized 1x128,
+        # then the second linear on those rows
+        y1, _ = oracle.scaled_mm(qa, qb, sa, sb, MMR["1x128_128x128"], rows=rows)
+        y1q, y1s = oracle.quantize_f32(y1.astype(np.float32), oracle.GROUP_1x128)
+        oracle.scaled_mm(y1q, qb2, y1s, sb2, MMR["1x128_128x128"])
     else:
         bias = None if wl.bias is None else W.bf16_bits(wl.bias)
         oracle.scaled_mm(qa, qb, sa, sb, MMR[GEMM_RECIPE.get(wl.recipe, wl.recipe)],
@@ -473,9 +514,12 @@ def oracle_sample(wl, max_rows: int):
 def cpu_baseline(wl, rows: int):
     tg, frac, tq, threads = oracle_sample(wl, rows)
     est_s = tq + tg / frac
+    chain = wl.recipe == "chain"
+    what = "X, W1 and W2" if chain else "both operands"
+    gemm = "both GEMMs (the first one's fp32 output quantized 1x128)" if chain else "GEMM"
     value = wl.flops / est_s / 1e12
     return {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": (f"quantize of both operands in full ({tq:.2f} s) + GEMM on "
+            "sample": (f"quantize of {what} in full ({tq:.2f} s) + {gemm} on "
                        f"{int(round(frac * wl.M))} of {wl.M} output rows ({tg:.2f} s), "
                        f"scaled to all rows"),
             "seconds_est_per_step": est_s}
@@ -585,7 +629,11 @@ def main(argv=None):
             "out_dtype": "bf16",
             "l2": "flushed between steps (256 MB write + read back, outside the step events)",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "step": "quantize A || quantize B (two streams), then scaled GEMM",
+            "step": ("quantize X || quantize W1, W2 (two streams), then GEMM1 with its "
+                     "output quantized 1x128 in the epilogue, then GEMM2"
+                     if wl.recipe == "chain" else
+                     "quantize A || quantize B (two streams), then scaled GEMM"),
+            "N2": (int(wl.extra["b2"].shape[0]) if "b2" in wl.extra else None),
             "launch": ("CUDA graphs of the step's C-ABI launches" if args.graphs
                        else "one C-ABI call per launch"),
         },

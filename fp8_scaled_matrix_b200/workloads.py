@@ -32,6 +32,11 @@ descriptions; no public dataset is involved):
                 GEMM M=5120, N=8192, K=16640
   7 grouped blockwise  the tensors of workload 4 (same seed), quantized with
                 1x128 activation groups and per-expert 128x128 weight tiles
+  8 linear chain  two blockwise (1x128_128x128) linears back to back, the
+                first one's output quantized in its GEMM epilogue and fed to
+                the second as its 1x128 activation: 16640 tokens, 8192 -> 5120
+                -> 8192; X ~ N(0,1) (16640, 8192), W1 ~ N(0, 0.02^2)
+                (5120, 8192), W2 ~ N(0, 0.02^2) (8192, 5120) as stored
 """
 from __future__ import annotations
 
@@ -50,6 +55,7 @@ WORKLOAD_NAMES = [
     "grad_input_1x128_128x128",
     "grad_weight_1x128_128x1",
     "grouped_e16_blockwise",
+    "linear_chain_1x128_128x128",
 ]
 
 
@@ -103,7 +109,7 @@ def offsets_from_sizes(sizes) -> torch.Tensor:
 class Workload:
     name: str
     # tensor | row | 1x128_128x128 | 1x128_128x1 | grouped | grouped_blockwise |
-    # grad_input | grad_weight
+    # grad_input | grad_weight | chain
     recipe: str
     M: int
     N: int
@@ -122,7 +128,11 @@ class Workload:
 
     @property
     def flops(self) -> int:
-        return 2 * self.M * self.N * self.K
+        f = 2 * self.M * self.N * self.K
+        if "b2" in self.extra:   # the chain's second GEMM: (M, N) @ b2^T
+            n2, k2 = self.extra["b2"].shape
+            f += 2 * self.M * n2 * k2
+        return f
 
 
 def make_workload(index: int, shape_index: int = 0, scale_down: int = 1) -> Workload:
@@ -178,6 +188,13 @@ def make_workload(index: int, shape_index: int = 0, scale_down: int = 1) -> Work
         dy = randn_bf16((T, N_out), 1e-3, g)
         x = randn_bf16((T, K_in), 1.0, g)
         return Workload(name, "grad_weight", N_out, K_in, T, dy, x, seed=seed)
+    if index == 8:
+        T, D, F = 16640 // scale_down, 8192, 5120
+        T -= T % 16
+        x = randn_bf16((T, D), 1.0, g)
+        w1 = randn_bf16((F, D), 0.02, g)
+        w2 = randn_bf16((D, F), 0.02, g)
+        return Workload(name, "chain", T, F, D, x, w1, seed=seed, extra={"b2": w2})
     raise ValueError(f"unknown workload {index}")
 
 

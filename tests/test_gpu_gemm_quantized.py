@@ -1,12 +1,18 @@
-"""The GEMM whose epilogue quantizes its own result (fp8_scaled_mm_quantized).
+"""The GEMM whose epilogue quantizes its own result (fp8_scaled_mm_quantized),
+and the chain of two linears it enables.
 
-Two checks per case.  (1) Exactness of the fused quantize: the fp32 result of
-the same GEMM (fp8_scaled_mm with fp32 output, same operands, same kernel
-schedule) quantized by the oracle's fp32 quantizer in 1x128 groups must give
-the same codes and scales bit for bit.  (2) End to end against the oracle's
-fp64 GEMM: the dequantized output (code * scale) is within the GEMM tolerance
-plus half an e4m3 step of the fp64 reference.  The GEMM itself is covered by
-the fp32-output parity tests; (1) pins the epilogue's amax, scale and cast."""
+Two checks per case.  (1) Against the oracle, independently: the oracle
+quantizes the same seeded inputs and computes the fp64 GEMM; the dequantized
+kernel output (code * scale) must be within the GEMM tolerance plus half an
+e4m3 step of it.  (2) A property of the kernel's own output, with no oracle
+involved: its codes and scales are exactly the 1x128 quantization (the scale
+and cast steps of "per-token scaling for fp8 linear", Highlights) of the fp32
+result that the same GEMM writes when asked for fp32 output -- amax of each
+group, scale = amax/448, codes = round-to-nearest-even e4m3 of y * 448/amax,
+saturated -- each step one fp32 operation, restated here with numpy fp32
+arithmetic and torch's float8_e4m3fn cast.  (2) is what makes the fused
+quantize bit-exact; the rounding of the fp32 GEMM itself differs from the
+fp64 reference, so codes cannot be compared with an oracle quantize of it."""
 import numpy as np
 import pytest
 import torch
@@ -54,13 +60,22 @@ def run_both(qa, sa, qb, sb, recipe, bias):
 
 
 def check_exact(y, q, s, what):
-    rq, rs = oracle.quantize_f32(y, oracle.GROUP_1x128)
-    rs = rs.reshape(s.shape)
-    bad_s = np.argwhere(rs.view(np.uint32) != s.view(np.uint32))
+    """q, s (scales (N/128, M)) are the 1x128 quantization of the fp32 y."""
+    M, N = y.shape
+    g = y.astype(np.float32).reshape(M, N // 128, 128)
+    a = np.maximum(np.abs(g).max(axis=2), np.float32(1e-12))      # (M, N/128)
+    s_want = (a / np.float32(448.0)).astype(np.float32)
+    inv = (np.float32(448.0) / a).astype(np.float32)
+    t = np.clip(g * inv[:, :, None], np.float32(-448.0), np.float32(448.0)).reshape(M, N)
+    assert t.dtype == np.float32
+    q_want = torch.from_numpy(np.ascontiguousarray(t)).to(torch.float8_e4m3fn)
+    q_want = q_want.view(torch.uint8).numpy()
+    s = s.reshape(N // 128, M)
+    bad_s = np.argwhere(s_want.T.view(np.uint32) != s.view(np.uint32))
     assert bad_s.size == 0, f"{what}: {len(bad_s)} scales differ, first {bad_s[0]}"
-    bad = np.argwhere(rq != q)
+    bad = np.argwhere(q_want != q)
     assert bad.size == 0, (f"{what}: {len(bad)} codes differ, first {bad[0]} "
-                           f"gpu={q[tuple(bad[0])]:#x} oracle={rq[tuple(bad[0])]:#x}")
+                           f"kernel={q[tuple(bad[0])]:#x} want={q_want[tuple(bad[0])]:#x}")
 
 
 def check_against_fp64(q, s, ref, mag, what):
@@ -163,3 +178,39 @@ def test_quantized_output_full_size_sampled(idx, shape_index):
     qs = q.index_select(0, rows).cpu().numpy()
     ss = s.index_select(1, rows).cpu().numpy()
     check_exact(ys, qs, ss, f"{wl.name} full size")
+
+
+def test_linear_chain_against_oracle():
+    """Two blockwise linears chained through the quantized output (the
+    linear-chain workload at full width, sampled rows): X -> GPU quantize ->
+    GEMM1 quantized -> GEMM2, against the oracle's chain on the same inputs
+    (quantize, fp64 GEMM1 rounded to fp32, 1x128 quantize, fp64 GEMM2); and the
+    chain's SQNR against the unquantized fp64 product (>= 20 dB, the MoE
+    handler's output threshold)."""
+    wl = W.make_workload(8)
+    f = fp8sm
+    x, w1, w2 = wl.a.cuda(), wl.b.cuda(), wl.extra["b2"].cuda()
+    qx, sx = f.fp8_quantize(x, f.FP8_SCALE_BLOCK_1x128)
+    q1, s1 = f.fp8_quantize(w1, f.FP8_SCALE_BLOCK_128x128)
+    q2, s2 = f.fp8_quantize(w2, f.FP8_SCALE_BLOCK_128x128)
+    r = f.FP8_MM_1x128_128x128
+    y1q, y1s = f.fp8_scaled_mm_quantized(qx, q1, sx, s1, r)
+    out = f.fp8_scaled_mm(y1q, q2, y1s, s2, r, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    f.check_device_status()
+    rows = sample_rows(wl.M, 40, seed=8)
+    G = oracle.GROUP_128x128
+    oqx, osx = oracle.quantize(W.bf16_bits(wl.a), oracle.GROUP_1x128)
+    oq1, os1 = oracle.quantize(W.bf16_bits(wl.b), G)
+    oq2, os2 = oracle.quantize(W.bf16_bits(wl.extra["b2"]), G)
+    y1, _ = oracle.scaled_mm(oqx, oq1, osx, os1, oracle.MM_1x128_128x128, rows=rows)
+    oy1q, oy1s = oracle.quantize_f32(y1.astype(np.float32), oracle.GROUP_1x128)
+    ref, mag = oracle.scaled_mm(oy1q, oq2, oy1s, os2, oracle.MM_1x128_128x128)
+    got = out.cpu().numpy().astype(np.float64)[rows]
+    ok = oracle.within_tolerance(got, ref, mag)
+    assert ok.all(), f"chain: {int((~ok).sum())} of {ok.size} out of tolerance"
+    xs = wl.a.double().numpy()[rows]
+    exact = (xs @ wl.b.double().numpy().T) @ wl.extra["b2"].double().numpy().T
+    err = got - exact
+    sqnr = 10 * np.log10((exact ** 2).sum() / (err ** 2).sum())
+    assert sqnr >= 20.0, sqnr
