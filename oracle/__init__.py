@@ -50,6 +50,12 @@ def lib():
         L.or_grouped_scaled_mm.restype = ctypes.c_int
         L.or_grouped_scaled_mm.argtypes = [P, P, I64, I64, I64, ctypes.c_int32,
                                            P, P, P, P, I64, P, P]
+        L.or_mx_quantize.restype = ctypes.c_int
+        L.or_mx_quantize.argtypes = [P, I64, I64, I64, P, P]
+        L.or_mx_scales_to_tiles.restype = ctypes.c_int
+        L.or_mx_scales_to_tiles.argtypes = [P, I64, I64, P]
+        L.or_mx_scaled_mm.restype = ctypes.c_int
+        L.or_mx_scaled_mm.argtypes = [P, P, I64, I64, I64, P, P, P, P, I64, P, P]
         L.or_num_threads.restype = ctypes.c_int
         L.or_num_threads.argtypes = []
         _lib = L
@@ -202,3 +208,54 @@ def within_tolerance(out, ref, mag, rel=1e-2, abs_mag=1e-3):
     Returns a boolean array."""
     out = np.asarray(out, dtype=np.float64)
     return np.abs(out - ref) <= rel * np.abs(ref) + abs_mag * mag
+
+
+# ---------------------------------------------------------------- MXFP8
+
+def mx_quantize(x_bits: np.ndarray):
+    """MXFP8 quantization of a bf16 matrix (uint16 bit patterns, 2-D, cols % 32
+    == 0): returns (q uint8 (rows, cols), e8 uint8 (rows, cols // 32))."""
+    x_bits = _c(x_bits, np.uint16)
+    rows, cols = x_bits.shape
+    q = np.empty((rows, cols), dtype=np.uint8)
+    e8 = np.empty((rows, max(cols // 32, 1)), dtype=np.uint8)
+    rc = lib().or_mx_quantize(_ptr(x_bits), rows, cols, cols, _ptr(q), _ptr(e8))
+    if rc != 0:
+        raise ValueError("oracle mx_quantize: bad arguments")
+    return q, e8[:, :cols // 32]
+
+
+def mx_tile_bytes(rows: int, kblocks: int) -> int:
+    return ((rows + 127) // 128) * ((kblocks + 3) // 4) * 512
+
+
+def mx_scales_to_tiles(e8: np.ndarray) -> np.ndarray:
+    """(rows, kblocks) scale bytes -> the flat scale-factor tile layout."""
+    e8 = _c(e8, np.uint8)
+    rows, kblocks = e8.shape
+    out = np.empty(max(mx_tile_bytes(rows, kblocks), 1), dtype=np.uint8)
+    rc = lib().or_mx_scales_to_tiles(_ptr(e8), rows, kblocks, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle mx_scales_to_tiles: bad arguments")
+    return out[:mx_tile_bytes(rows, kblocks)]
+
+
+def mx_scaled_mm(a, b, ea, eb, bias_bits=None, rows=None):
+    """MXFP8 GEMM reference (ref, mag), fp64: a (M,K), b (N,K) codes; ea
+    (M, K/32), eb (N, K/32) plain scale bytes."""
+    a = _c(a, np.uint8)
+    b = _c(b, np.uint8)
+    ea = _c(ea, np.uint8)
+    eb = _c(eb, np.uint8)
+    M, K = a.shape
+    N = b.shape[0]
+    bias = None if bias_bits is None else _c(bias_bits, np.uint16)
+    r = None if rows is None else _c(rows, np.int64)
+    R = M if r is None else r.size
+    ref = np.empty((R, N), dtype=np.float64)
+    mag = np.empty((R, N), dtype=np.float64)
+    rc = lib().or_mx_scaled_mm(_ptr(a), _ptr(b), M, N, K, _ptr(ea), _ptr(eb), _ptr(bias),
+                               _ptr(r), 0 if r is None else r.size, _ptr(ref), _ptr(mag))
+    if rc != 0:
+        raise ValueError("oracle mx_scaled_mm: bad arguments")
+    return ref, mag

@@ -424,3 +424,118 @@ int or_grouped_scaled_mm(const uint8_t* a, const uint8_t* b_experts,
   }
   return 0;
 }
+
+/* ----------------------------------------------------------------- MXFP8 */
+
+/* "Add _scaled_mm_v2 API" (Blas.cpp review, recipe table) names an "mxfp8"
+ * recipe (MXFP8_MXFP8) without defining it; the name is the OCP Microscaling
+ * (MX) format, whose published definition (OCP MX v1.0) is followed here:
+ * each block of 32 consecutive elements along the contraction dimension has
+ * one E8M0 scale X = 2^e (stored as the byte e + 127), and elements are E4M3.
+ * Converting one block, in the specification's order:
+ *   1. amax = max |v_i| over the block
+ *   2. e = floor(log2(amax)) - 8   (8 = exponent of 256, the largest power of
+ *      two E4M3 represents); an all-zero block takes e = -127; e is clamped
+ *      to the E8M0 range [-127, 127]
+ *   3. q_i = E4M3(v_i / 2^e), round to nearest even, saturating at +-448
+ *      (the specification leaves overflow to the implementation; values of a
+ *      block with amax in [448, 512) * 2^e saturate). */
+static int mx_block_exponent(float amax) {
+  if (amax == 0.0f) return -127;
+  int fe;
+  (void)frexp((double)amax, &fe); /* amax = f * 2^fe, 0.5 <= f < 1 */
+  int e = (fe - 1) - 8;
+  if (e < -127) e = -127;
+  if (e > 127) e = 127;
+  return e;
+}
+
+int or_mx_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                   uint8_t* q, uint8_t* e8) {
+  if (rows < 0 || cols < 0 || cols % 32 != 0 || ld < cols || !x || !q || !e8)
+    return -1;
+  int64_t KB = cols / 32;
+  int64_t r;
+#pragma omp parallel for schedule(static)
+  for (r = 0; r < rows; r++)
+    for (int64_t kb = 0; kb < KB; kb++) {
+      const uint16_t* v = x + r * ld + kb * 32;
+      float amax = 0.0f;
+      for (int i = 0; i < 32; i++) {
+        float f = fabsf(or_bf16_to_float(v[i]));
+        if (f > amax) amax = f;
+      }
+      int e = mx_block_exponent(amax);
+      e8[r * KB + kb] = (uint8_t)(e + 127);
+      for (int i = 0; i < 32; i++) {
+        /* v / 2^e is exact in fp64; below 2^-126 it rounds to zero in E4M3
+         * whatever the fp32 rounding, so the float conversion loses nothing */
+        double y = ldexp((double)or_bf16_to_float(v[i]), -e);
+        q[r * cols + kb * 32 + i] = or_e4m3_encode((float)y);
+      }
+    }
+  return 0;
+}
+
+/* Scale bytes rearranged into the tensor core's scale-factor tiles: one
+ * 512-byte tile per 128 rows x 4 blocks (128 elements of K), tiles ordered
+ * row-tile-major, and inside a tile the byte of (row r, block k) at
+ *   (r % 32) * 16 + (r / 32) * 4 + k        (r < 128, k < 4).
+ * Positions past the matrix (rows beyond `rows`, blocks beyond `kblocks`)
+ * are zero. */
+int or_mx_scales_to_tiles(const uint8_t* e8, int64_t rows, int64_t kblocks,
+                          uint8_t* tiles) {
+  if (rows < 0 || kblocks < 0 || !e8 || !tiles) return -1;
+  int64_t RT = ceil_div(rows, 128), KT = ceil_div(kblocks, 4);
+  memset(tiles, 0, (size_t)(RT * KT * 512));
+  for (int64_t r = 0; r < rows; r++)
+    for (int64_t kb = 0; kb < kblocks; kb++) {
+      int64_t tile = (r / 128) * KT + kb / 4;
+      int64_t rr = r % 128, k = kb % 4;
+      tiles[tile * 512 + (rr % 32) * 16 + (rr / 32) * 4 + k] = e8[r * kblocks + kb];
+    }
+  return 0;
+}
+
+/* MXFP8 GEMM: out[m, n] = sum_k (a[m,k] 2^(ea[m,k/32]-127)) (b[n,k]
+ * 2^(eb[n,k/32]-127)) (+ bias[n]).  Exact integer dot product per 32-block,
+ * scaled by the power of two and summed in fp64; mag as in or_scaled_mm.
+ * ea (M, K/32), eb (N, K/32): plain row-major E8M0 bytes. */
+int or_mx_scaled_mm(const uint8_t* a, const uint8_t* b, int64_t M, int64_t N,
+                    int64_t K, const uint8_t* ea, const uint8_t* eb,
+                    const uint16_t* bias, const int64_t* rows, int64_t n_rows,
+                    double* ref, double* mag) {
+  if (M < 0 || N < 0 || K < 0 || K % 32 != 0 || !ref || !mag) return -1;
+  build_lut();
+  int64_t R = rows ? n_rows : M;
+  for (int64_t i = 0; i < R; i++)
+    if (rows && (rows[i] < 0 || rows[i] >= M)) return -1;
+  int64_t KB = K / 32;
+  int64_t i;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (i = 0; i < R; i++) {
+    int64_t m = rows ? rows[i] : i;
+    const uint8_t* arow = a + m * K;
+    for (int64_t n = 0; n < N; n++) {
+      const uint8_t* brow = b + n * K;
+      double acc = 0.0, accm = 0.0;
+      int any_nan = 0;
+      for (int64_t kb = 0; kb < KB; kb++) {
+        int64_t d = 0, dabs = 0;
+        for (int64_t k = kb * 32; k < kb * 32 + 32; k++) {
+          int64_t p = (int64_t)lut_int[arow[k]] * (int64_t)lut_int[brow[k]];
+          d += p;
+          dabs += p < 0 ? -p : p;
+          any_nan |= lut_nan[arow[k]] | lut_nan[brow[k]];
+        }
+        int ex = (int)ea[m * KB + kb] - 127 + (int)eb[n * KB + kb] - 127;
+        any_nan |= ea[m * KB + kb] == 0xFF || eb[n * KB + kb] == 0xFF;
+        acc += ldexp((double)d, ex - 18);
+        accm += ldexp((double)dabs, ex - 18);
+      }
+      ref[i * N + n] = any_nan ? NAN : acc + bias_at(bias, n);
+      mag[i * N + n] = accm;
+    }
+  }
+  return 0;
+}

@@ -14,6 +14,9 @@
  *   - the quantizer: amax over a group -> scale = max(amax, eps)/448 ->
  *     y = x * (448/max(amax, eps)) -> e4m3 code ("per-token scaling for fp8
  *     linear", Highlights: dynamic per-token scale, pre-scaled input, cast).
+ *   - MXFP8 (the "mxfp8" recipe of "Add _scaled_mm_v2 API", defined by the
+ *     OCP Microscaling specification): power-of-two E8M0 scale per 32
+ *     elements, E4M3 elements, and its GEMM.
  *   - the scaled GEMM as the plain definition "dequantize, then matmul"
  *     ("Fix: Handle LowLevelZeroPlugin with use_fp8=True", Solution, forward
  *     pass): products of exactly decoded values, accumulated exactly in int64
@@ -112,6 +115,26 @@ int or_grouped_scaled_mm(const uint8_t* a, const uint8_t* b_experts,
                          const float* sA, const float* sB, const int32_t* offs,
                          const int64_t* rows, int64_t n_rows, double* ref,
                          double* mag);
+
+/* MXFP8 (OCP Microscaling, E4M3 elements, one E8M0 scale per 32 elements
+ * along each row).  x: (rows, cols) bf16 bit patterns, row stride ld,
+ * cols % 32 == 0.  q: (rows, cols) codes; e8: (rows, cols/32) scale bytes
+ * (2^(byte-127)).  Returns 0, or -1 on bad arguments. */
+int or_mx_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                   uint8_t* q, uint8_t* e8);
+
+/* e8 (rows, kblocks) rearranged into 512-byte scale-factor tiles (128 rows x
+ * 4 blocks each, row-tile-major; byte (r%32)*16 + (r/32)*4 + k inside), zero
+ * past the matrix.  tiles holds ceil(rows/128) * ceil(kblocks/4) * 512 bytes. */
+int or_mx_scales_to_tiles(const uint8_t* e8, int64_t rows, int64_t kblocks,
+                          uint8_t* tiles);
+
+/* MXFP8 GEMM reference: a (M,K), b (N,K) codes; ea (M,K/32), eb (N,K/32)
+ * plain scale bytes; bias, rows, ref, mag as in or_scaled_mm. */
+int or_mx_scaled_mm(const uint8_t* a, const uint8_t* b, int64_t M, int64_t N,
+                    int64_t K, const uint8_t* ea, const uint8_t* eb,
+                    const uint16_t* bias, const int64_t* rows, int64_t n_rows,
+                    double* ref, double* mag);
 
 /* Threads the oracle's OpenMP loops use (1 when built without OpenMP). */
 int or_num_threads(void);
