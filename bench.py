@@ -52,6 +52,8 @@ WORKLOADS = {
     "grad_weight_1x128_128x1": (6, 0),
     "grouped_e16_blockwise": (7, 0),
     "linear_chain_1x128_128x128": (8, 0),
+    "mxfp8_16640x5120x8192": (9, 0),
+    "mxfp8_16640x8192x5120": (9, 1),
 }
 DEFAULT_WORKLOAD = "rowwise_4096"
 # Page 5's context numbers (TFLOP/s of torch._scaled_mm, hardware not stated)
@@ -63,7 +65,8 @@ OPERAND_GROUPS = {"tensor": ("tensor", "tensor"), "row": ("row", "row"),
                   "1x128_128x128": ("1x128", "128x128"),
                   "1x128_128x1": ("1x128", "1x128"), "grouped": ("row", "row"),
                   "grad_input": ("1x128", "128x128"), "grad_weight": ("1x128", "1x128"),
-                  "grouped_blockwise": ("1x128", "128x128"), "chain": ("1x128", "128x128")}
+                  "grouped_blockwise": ("1x128", "128x128"), "chain": ("1x128", "128x128"),
+                  "mxfp8": ("mx", "mx")}
 # GEMM recipe of each workload recipe, and which operands are quantized
 # transposed (the training GEMMs contract along the stored rows)
 GEMM_RECIPE = {"grad_input": "1x128_128x128", "grad_weight": "1x128_128x1",
@@ -206,8 +209,9 @@ class Step:
         self.wl = wl
         self.dev = dev
         ga, gb = OPERAND_GROUPS[wl.recipe]
-        self.qa_recipe = fp8sm.QUANT_RECIPES[ga]
-        self.qb_recipe = fp8sm.QUANT_RECIPES[gb]
+        self.mx = wl.recipe == "mxfp8"
+        self.qa_recipe = None if self.mx else fp8sm.QUANT_RECIPES[ga]
+        self.qb_recipe = None if self.mx else fp8sm.QUANT_RECIPES[gb]
         self.a = wl.a.to(dev)
         self.grouped = wl.recipe in ("grouped", "grouped_blockwise")
         if self.grouped:
@@ -224,10 +228,17 @@ class Step:
         cols = wl.K
         self.qa = torch.empty(rows_a, cols, dtype=torch.uint8, device=dev)
         self.qb = torch.empty(rows_b, cols, dtype=torch.uint8, device=dev)
-        self.sa = torch.empty(max(fp8sm.scale_count(rows_a, cols, self.qa_recipe), 1),
-                              dtype=torch.float32, device=dev)
-        self.sb = torch.empty(max(fp8sm.scale_count(rows_b, cols, self.qb_recipe), 1),
-                              dtype=torch.float32, device=dev)
+        if self.mx:
+            # E8M0 scale-factor tiles
+            self.sa = torch.empty(fp8sm.fp8_mx_scale_bytes(rows_a, cols), dtype=torch.uint8,
+                                  device=dev)
+            self.sb = torch.empty(fp8sm.fp8_mx_scale_bytes(rows_b, cols), dtype=torch.uint8,
+                                  device=dev)
+        else:
+            self.sa = torch.empty(max(fp8sm.scale_count(rows_a, cols, self.qa_recipe), 1),
+                                  dtype=torch.float32, device=dev)
+            self.sb = torch.empty(max(fp8sm.scale_count(rows_b, cols, self.qb_recipe), 1),
+                                  dtype=torch.float32, device=dev)
         self.ws = torch.zeros(64, dtype=torch.uint8, device=dev)
         self.ws_b = torch.zeros(64, dtype=torch.uint8, device=dev)
         self.side = torch.cuda.Stream(device=dev)
@@ -276,6 +287,8 @@ class Step:
             elif self.t_b:
                 f.fp8_quantize_transposed(self.b, self.qb_recipe, out=self.qb, scales=self.sb,
                                           stream=self.side)
+            elif self.mx:
+                f.fp8_quantize_mx(self.b, out=self.qb, scales=self.sb, stream=self.side)
             elif self.chain:
                 f.fp8_quantize(self.b, self.qb_recipe, out=self.qb, scales=self.sb,
                                workspace=self.ws_b, stream=self.side)
@@ -284,7 +297,9 @@ class Step:
             else:
                 f.fp8_quantize(self.b, self.qb_recipe, out=self.qb, scales=self.sb,
                                workspace=self.ws_b, stream=self.side)
-        if self.t_a:
+        if self.mx:
+            f.fp8_quantize_mx(self.a, out=self.qa, scales=self.sa, stream=main)
+        elif self.t_a:
             f.fp8_quantize_transposed(self.a, self.qa_recipe, out=self.qa, scales=self.sa,
                                       stream=main)
         else:
@@ -304,6 +319,8 @@ class Step:
             E, N, K = wl.b.shape
             f.fp8_grouped_scaled_mm_blockwise(self.qa, self.qb.view(E, N, K), self.sa,
                                               self.sb, self.offs, out=self.out)
+        elif self.mx:
+            f.fp8_scaled_mm_mx(self.qa, self.qb, self.sa, self.sb, bias=self.bias, out=self.out)
         elif self.chain:
             r = f.MM_RECIPES["1x128_128x128"]
             f.fp8_scaled_mm_quantized(self.qa, self.qb, self.sa, self.sb, r,
@@ -318,7 +335,8 @@ class Step:
         """Algorithmic HBM bytes of the two quantize launches: 2 B read +
         1 B written per element, 4 B per scale."""
         n = self.a.numel() + self.b.numel()
-        b = 3 * n + 4 * (self.sa.numel() + self.sb.numel())
+        b = 3 * n + self.sa.element_size() * self.sa.numel() + \
+            self.sb.element_size() * self.sb.numel()
         if self.chain:
             b += 3 * self.b2.numel() + 4 * self.sb2.numel()
         return b
@@ -465,6 +483,14 @@ def oracle_sample(wl, max_rows: int):
         b = W.bf16_bits(x)
         return np.ascontiguousarray(b.T) if transposed else b
     t0 = time.perf_counter()
+    if wl.recipe == "mxfp8":
+        qa, sa = oracle.mx_quantize(W.bf16_bits(wl.a))
+        qb, sb = oracle.mx_quantize(W.bf16_bits(wl.b))
+        tq = time.perf_counter() - t0
+        rows = np.arange(min(max_rows, wl.M), dtype=np.int64)
+        t0 = time.perf_counter()
+        oracle.mx_scaled_mm(qa, qb, sa, sb, rows=rows)
+        return time.perf_counter() - t0, rows.size / wl.M, tq, oracle.num_threads()
     qa, sa = oracle.quantize(bits(wl.a, t_a), G[ga])
     if wl.recipe == "grouped":
         E, N, K = wl.b.shape

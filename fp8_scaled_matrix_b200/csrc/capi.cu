@@ -296,6 +296,71 @@ fp8_status fp8_scaled_mm_quantized(const void* a, const void* b, int64_t M, int6
   return finish_launch(e, err, "fp8_scaled_mm_quantized");
 }
 
+size_t fp8_mx_scale_bytes(int64_t rows, int64_t cols) {
+  if (rows < 0 || cols < 0) return 0;
+  return fp8sm::mx_scale_tile_bytes(rows, cols);
+}
+
+fp8_status fp8_quantize_mx(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld_x,
+                           void* out_fp8, void* out_scales_e8m0, fp8_stream_t stream) {
+  if (rows < 0 || cols < 0) return fail(FP8_ERR_VALUE, "fp8_quantize_mx: negative size");
+  if (rows >= (int64_t(1) << 31) || cols >= (int64_t(1) << 31))
+    return fail(FP8_ERR_VALUE, "fp8_quantize_mx: size too large");
+  if (cols % 32 != 0) return fail(FP8_ERR_VALUE, "fp8_quantize_mx: cols must be a multiple of 32");
+  if (ld_x < cols || ld_x % 8 != 0)
+    return fail(FP8_ERR_VALUE, "fp8_quantize_mx: ld_x must be >= cols and a multiple of 8");
+  if (rows == 0 || cols == 0) {
+    t_last_error.clear();
+    return FP8_OK;
+  }
+  if (x_bf16 == nullptr || out_fp8 == nullptr || out_scales_e8m0 == nullptr)
+    return fail(FP8_ERR_VALUE, "fp8_quantize_mx: null pointer");
+  if (!aligned(x_bf16, 16) || !aligned(out_fp8, 16) || !aligned(out_scales_e8m0, 16))
+    return fail(FP8_ERR_VALUE, "fp8_quantize_mx: pointers must be 16-byte aligned");
+  DeviceInfo* d = nullptr;
+  fp8_status s = device_info(&d);
+  if (s != FP8_OK) return s;
+  std::string err;
+  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status, d->num_sms, &err};
+  cudaError_t e = fp8sm::launch_quantize_mx(x_bf16, rows, cols, ld_x, out_fp8,
+                                            out_scales_e8m0, ctx);
+  return finish_launch(e, err, "fp8_quantize_mx");
+}
+
+fp8_status fp8_scaled_mm_mx(const void* a, const void* b, int64_t M, int64_t N, int64_t K,
+                            const void* scale_a_e8m0, const void* scale_b_e8m0,
+                            const void* bias_bf16, fp8_out_dtype out_dtype, void* out,
+                            fp8_stream_t stream) {
+  if (out_dtype != FP8_OUT_BF16 && out_dtype != FP8_OUT_F32)
+    return fail(FP8_ERR_VALUE, "fp8_scaled_mm_mx: unknown out_dtype");
+  if (M < 0 || N < 0 || K < 0) return fail(FP8_ERR_VALUE, "fp8_scaled_mm_mx: negative size");
+  if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+    return fail(FP8_ERR_VALUE, "fp8_scaled_mm_mx: size too large");
+  if (K == 0 || K % 32 != 0)
+    return fail(FP8_ERR_VALUE, "fp8_scaled_mm_mx: K must be a positive multiple of 32");
+  if (N % 16 != 0) return fail(FP8_ERR_VALUE, "fp8_scaled_mm_mx: N must be a multiple of 16");
+  if (M == 0 || N == 0) {
+    t_last_error.clear();
+    return FP8_OK;
+  }
+  if (a == nullptr || b == nullptr || scale_a_e8m0 == nullptr || scale_b_e8m0 == nullptr ||
+      out == nullptr)
+    return fail(FP8_ERR_VALUE, "fp8_scaled_mm_mx: null pointer");
+  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(scale_a_e8m0, 16) ||
+      !aligned(scale_b_e8m0, 16) || !aligned(out, 16) || (bias_bf16 && !aligned(bias_bf16, 16)))
+    return fail(FP8_ERR_VALUE, "fp8_scaled_mm_mx: pointers must be 16-byte aligned");
+  DeviceInfo* d = nullptr;
+  fp8_status s = device_info(&d);
+  if (s != FP8_OK) return s;
+  std::string err;
+  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status, d->num_sms, &err};
+  cudaError_t e = fp8sm::launch_scaled_mm(
+      a, b, M, N, K, static_cast<const float*>(scale_a_e8m0),
+      static_cast<const float*>(scale_b_e8m0), 4, bias_bf16,
+      out_dtype == FP8_OUT_F32 ? 1 : 0, out, nullptr, ctx);
+  return finish_launch(e, err, "fp8_scaled_mm_mx");
+}
+
 namespace {
 
 // Shared by both grouped entry points; recipe 1 (rowwise) or 2 (1x128_128x128).

@@ -6,8 +6,11 @@
 // fixes what is computed: the scaled matmul equals dequantize-then-matmul plus
 // bias.  Recipes: tensorwise and rowwise ("Add _scaled_mm_v2 API"),
 // blockwise 1x128_128x128 and 1x128_128x1 ("improve fp8 blockwise gemm
-// perf"), and the grouped rowwise MoE form over (E, N, K) experts with
-// cumulative offs ("Add _grouped_mm dispatch handler to Float8Tensor").
+// perf"), the grouped rowwise MoE form over (E, N, K) experts with
+// cumulative offs ("Add _grouped_mm dispatch handler to Float8Tensor"), and
+// MXFP8 (the "mxfp8" recipe of "Add _scaled_mm_v2 API": one E8M0 scale per
+// 32 elements of K, applied by the tensor core itself through
+// tcgen05.mma.kind::mxf8f6f4.block_scale with the scales staged in TMEM).
 //
 // One persistent kernel, one CTA per SM, 12 warps with fixed roles:
 //   warp 0      TMA producer: A (128 x 128 B) and B (256 x 128 B) tiles into
@@ -75,6 +78,13 @@ constexpr uint32_t kEpiBuf = 32 * 64;  // 32 rows x 64 bytes, 64-byte swizzle
 constexpr int kSclSlots = 8;
 constexpr int kSclSlotFloats = 128 + 256;
 constexpr uint32_t kSclBytes = kSclSlots * kSclSlotFloats * 4;
+// MXFP8: per stage, three 512-byte scale-factor tiles (A's 128 rows, B's two
+// 128-row halves) land next to the operands, in the scale-ring region (which
+// the MXFP8 kernel does not otherwise use); in TMEM each stage has a
+// 16-column slot after the accumulator (A: 4 columns, B: 8).
+constexpr uint32_t kMxSfTile = 512;
+constexpr uint32_t kMxSfStage = 3 * kMxSfTile;
+constexpr uint32_t kMxSfCols = 16;
 
 // Shared-memory layout.  Single-CTA tiles are 128 x 256: each stage holds
 // A (128 rows) and B (256 rows) of a 128-byte K slice.  CTA-pair tiles are
@@ -100,9 +110,11 @@ struct Cfg {
   static constexpr uint32_t kSmemUsed = kOffMisc + 16;
   static constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // + alignment slack
   static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kStages * kMxSfStage <= kSclBytes, "MXFP8 scale tiles fit the ring region");
+  static_assert(BN + kStages * kMxSfCols <= kTmemCols, "MXFP8 TMEM slots");
 };
 
-enum Recipe : int { kTensor = 0, kRow = 1, kBlock128 = 2, kBlock1 = 3 };
+enum Recipe : int { kTensor = 0, kRow = 1, kBlock128 = 2, kBlock1 = 3, kMxfp8 = 4 };
 // Output: bf16, fp32, or e4m3 quantized in 1x128 groups along n (+ scales)
 enum OutKind : int { kOutBf16 = 0, kOutFp32 = 1, kOutE4M3 = 2 };
 
@@ -110,6 +122,8 @@ struct GemmParams {
   int64_t M, N, K;
   const float* sa;
   const float* sb;
+  const uint8_t* sfa;  // MXFP8: scale-factor tiles of A and B (E8M0 bytes)
+  const uint8_t* sfb;
   const uint16_t* bias;
   void* out;
   float* out_scales;  // e4m3 output: scale[(n/128) * M + m]
@@ -321,6 +335,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tm_out,
                     const GemmParams p) {
   constexpr bool kBlockwise = (kRecipe == kBlock128 || kRecipe == kBlock1);
+  constexpr bool kIsMx = kRecipe == kMxfp8;
+  // epilogue threads that hold a whole 128-column row slice in registers
+  constexpr bool kBigEpi = kBlockwise || kIsMx;
   constexpr bool kOutF32 = kOut == kOutFp32;
   constexpr bool kOutQ = kOut == kOutE4M3;
   using C = Cfg<kPair>;
@@ -416,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < kFirstEpiWarp) {
    // warpgroup 0: all four warps execute the same setmaxnreg
-   if constexpr (kBlockwise) warpgroup_reg_dealloc<kRegsLow>();
+   if constexpr (kBigEpi) warpgroup_reg_dealloc<kRegsLow>();
    if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -449,6 +466,24 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_3d_pair(b_dst, &tm_b, lead_full, kb * BK, b_row, c.g);
             else
               tma_load_2d_pair(b_dst, c.half_n ? &tm_b_half : &tm_b, lead_full, kb * BK, b_row);
+          } else if constexpr (kIsMx) {
+            // operands plus their scale-factor tiles (tile (i, kb) of a
+            // matrix's scales is its 128 rows 128 i .. and K elements
+            // 128 kb ..); B's second half-tile exists only below N
+            const int64_t nb0 = c.n0 / 128;
+            const bool two = !c.half_n && nb0 + 1 < (p.N + 127) / 128;
+            mbar_arrive_expect_tx(&full[stage], C::kAStage + b_bytes +
+                                                    (two ? 3u : 2u) * kMxSfTile);
+            tma_load_2d(a_dst, &tm_a, &full[stage], kb * BK, c.m0);
+            tma_load_2d(b_dst, c.half_n ? &tm_b_half : &tm_b, &full[stage], kb * BK, c.n0);
+            uint8_t* sf_dst = smem + C::kOffScl + stage * kMxSfStage;
+            const int64_t ka = (static_cast<int64_t>(c.m0 / 128) * KB + kb) * kMxSfTile;
+            const int64_t kbb = (nb0 * KB + kb) * kMxSfTile;
+            bulk_load_g2s(sf_dst, p.sfa + ka, kMxSfTile, &full[stage]);
+            bulk_load_g2s(sf_dst + kMxSfTile, p.sfb + kbb, kMxSfTile, &full[stage]);
+            if (two)
+              bulk_load_g2s(sf_dst + 2 * kMxSfTile, p.sfb + kbb + static_cast<int64_t>(KB) * kMxSfTile,
+                            kMxSfTile, &full[stage]);
           } else {
             mbar_arrive_expect_tx(&full[stage], C::kAStage + b_bytes);
             tma_load_2d(a_dst, &tm_a, &full[stage], kb * BK, c.m0);
@@ -489,7 +524,59 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the barrier), and the next stage's barrier is peeked while this
       // stage's MMAs go out.
       bool ready = mbar_test_wait<kPair>(&full[stage], phase);
-      if constexpr (!kBlockwise) {
+      if constexpr (kIsMx) {
+        // MXFP8: per stage, the scale-factor tiles go from shared memory to
+        // the stage's TMEM slot (tcgen05.cp: 32 rows x 16 bytes copied to
+        // all four lane quarters; ordered before this thread's later MMAs),
+        // then four block-scaled MMAs, MMA k reading byte k (its 32-wide K
+        // block) of each scale word.  One accumulator buffer: the scale
+        // slots take the other half of TMEM, and the epilogue hands the
+        // buffer back as soon as it has read it into registers.
+        uint32_t idesc_f[4], idesc_h[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          idesc_f[k] = idesc_mx_e4m3(kTM, BN, k, k);
+          idesc_h[k] = idesc_mx_e4m3(kTM, BN / 2, k, k);
+        }
+        for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
+          const bool hn = t >= p.split_start;
+          if (!mbar_wait(&acc_empty[0], acc_phase ^ 1u, abort_flag, p.status,
+                         SITE_MMA_ACC_EMPTY, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          for (int32_t kb = 0; kb < KB; ++kb) {
+            if (!ready && !mbar_wait(&full[stage], phase, abort_flag, p.status, SITE_MMA_FULL,
+                                     kWaitLimitNs)) {
+              ok = false;
+              break;
+            }
+            const uint32_t cur = stage;
+            if (++stage == C::kStages) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            ready = mbar_test_wait(&full[stage], phase);
+            const uint32_t sf_t = tmem_base + BN + cur * kMxSfCols;
+            const uint32_t sf_s = smem_u32(smem + C::kOffScl + cur * kMxSfStage);
+            tmem_cp_32x128b_warpx4(sf_t, smem_desc_rows16(sf_s));
+            tmem_cp_32x128b_warpx4(sf_t + 4, smem_desc_rows16(sf_s + kMxSfTile));
+            if (!hn) tmem_cp_32x128b_warpx4(sf_t + 8, smem_desc_rows16(sf_s + 2 * kMxSfTile));
+            const uint64_t da = smem_desc_k_sw128(smem_u32(smem + C::kOffA + cur * C::kAStage));
+            const uint64_t db = smem_desc_k_sw128(smem_u32(smem + C::kOffB + cur * C::kBStage));
+#pragma unroll
+            for (int k = 0; k < BK / UMMA_K; ++k)
+              mma_mx_e4m3(tmem_base, da + (k * UMMA_K) / 16, db + (k * UMMA_K) / 16,
+                          hn ? idesc_h[k] : idesc_f[k], sf_t, sf_t + 4, (kb > 0) || (k > 0));
+            mma_commit(&empty[cur]);
+          }
+          if (ok) {
+            mma_commit(&acc_full[0]);
+            acc_phase ^= 1u;
+          }
+        }
+      } else if constexpr (!kBlockwise) {
         for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
           const uint32_t idesc = (!kGrouped && t >= p.split_start) ? idesc_half : idesc_full;
           if (!mbar_wait<kPair>(&acc_empty[acc], acc_phase ^ 1u, abort_flag, p.status,
@@ -639,7 +726,7 @@ __global__ void __launch_bounds__(kThreads, 1)
    }
   } else {
     // --------------------------------------------------------- epilogue
-    if constexpr (kBlockwise) warpgroup_reg_alloc<kRegsHigh>();
+    if constexpr (kBigEpi) warpgroup_reg_alloc<kRegsHigh>();
     const uint32_t ew = warp - kFirstEpiWarp;  // 0..7
     const uint32_t q = warp & 3u;          // TMEM lane quarter of this warp
     const uint32_t half = ew >> 2;         // which 128 columns of the tile
@@ -686,6 +773,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t ncol0 = static_cast<int64_t>(c.n0) + half * 128;
       const int32_t row0 = cta_m0 + static_cast<int32_t>(q * 32);
 
+      // next accumulator buffer (MXFP8: the one buffer, next phase)
+      auto next_acc = [&]() {
+        if constexpr (kIsMx) {
+          acc_phase ^= 1u;
+        } else {
+          acc ^= 1u;
+          if (acc == 0) acc_phase ^= 1u;
+        }
+      };
       if constexpr (!kBlockwise) {
         if (!mbar_wait<kPair>(&acc_full[acc], acc_phase, abort_flag, p.status,
                        SITE_EPI_ACC_FULL, kWaitLimitNs)) {
@@ -697,8 +793,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           // 128-wide item: this warp's columns are not part of it
           __syncwarp();
           if (lane == 0) release_acc(acc);
-          acc ^= 1u;
-          if (acc == 0) acc_phase ^= 1u;
+          next_acc();
+          continue;
+        }
+        if constexpr (kIsMx) {
+          // scales were applied by the MMA: read the whole row slice, hand
+          // the buffer back, then add bias and store
+          const uint32_t tcol = tmem_base + lane_base + half * 128;
+          uint32_t r[4][32];
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) tmem_ld_32x32b_x32(tcol + cc * 32, r[cc]);
+          tmem_ld_wait();
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) release_acc(0);
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            const int64_t n = ncol0 + cc * 32;
+            float v[32];
+            load_bias32(p.bias, n, p.N, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __fadd_rn(__uint_as_float(r[cc][i]), v[i]);
+            store_cols32<kOutF32, kGrouped>(ebuf, v, &tm_out, static_cast<int32_t>(n), row0,
+                                            c.row_end, p.out, p.N, lane);
+          }
+          next_acc();
           continue;
         }
         float sa;
@@ -774,8 +893,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                   row0, c.row_end, static_cast<uint8_t*>(p.out), p.N, 1, lane);
           }
         }
-        acc ^= 1u;
-        if (acc == 0) acc_phase ^= 1u;
+        next_acc();
       } else {
         // Blockwise: promote each K block's partial product into registers.
         // Warp (q, half) reads TMEM lanes 32q.. and the 128 columns of its
@@ -978,8 +1096,11 @@ cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb,
                           const CUtensorMap& tbh, const CUtensorMap& to,
                           const GemmParams& p, unsigned grid, cudaStream_t st) {
   constexpr bool kBlockwise = kRecipe == kBlock128 || kRecipe == kBlock1;
+  constexpr bool kBigEpi = kBlockwise || kRecipe == kMxfp8;
   if constexpr (kPair && kBlockwise) {
     return cudaErrorInvalidValue;  // CTA pairs serve the dense recipes only
+  } else if constexpr (kRecipe == kMxfp8 && (kPair || kGrouped || kOut == kOutE4M3)) {
+    return cudaErrorInvalidValue;  // MXFP8: single-CTA dense GEMM, bf16/fp32 out
   } else if constexpr (kOut == kOutE4M3 && (kPair || kGrouped)) {
     return cudaErrorInvalidValue;  // quantized output: single-CTA dense GEMM only
   } else {
@@ -990,7 +1111,7 @@ cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb,
       cudaError_t e = cudaFuncSetAttribute(
           kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
       if (e != cudaSuccess) return e;
-      if (kBlockwise) {
+      if (kBigEpi) {
         // setmaxnreg.inc would wait forever if the launch allocation were
         // smaller than the split assumes: check before the first launch.
         cudaFuncAttributes attr;
@@ -1040,6 +1161,7 @@ cudaError_t dispatch(int recipe, int out_kind, bool pair, const CUtensorMap& ta,
     FP8SM_CASE(kRow)
     FP8SM_CASE(kBlock128)
     FP8SM_CASE(kBlock1)
+    FP8SM_CASE(kMxfp8)
   }
 #undef FP8SM_CASE
   return cudaErrorInvalidValue;
@@ -1078,7 +1200,8 @@ bool a_map(CUtensorMap* m, const void* a, int64_t rows, int64_t K, std::string* 
 // kernels always run on single CTAs.
 bool use_pair(int64_t M, int recipe) {
   const char* e = std::getenv("FP8SM_CTA_PAIRS");
-  return e != nullptr && e[0] == '1' && M > BM && recipe != kBlock128 && recipe != kBlock1;
+  return e != nullptr && e[0] == '1' && M > BM && recipe != kBlock128 && recipe != kBlock1 &&
+         recipe != kMxfp8;
 }
 
 }  // namespace
@@ -1125,8 +1248,14 @@ cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
   p.M = M;
   p.N = N;
   p.K = K;
-  p.sa = sa;
-  p.sb = sb;
+  if (recipe == kMxfp8) {
+    // MXFP8: sa, sb carry the E8M0 scale-factor tiles
+    p.sfa = reinterpret_cast<const uint8_t*>(sa);
+    p.sfb = reinterpret_cast<const uint8_t*>(sb);
+  } else {
+    p.sa = sa;
+    p.sb = sb;
+  }
   p.bias = static_cast<const uint16_t*>(bias);
   p.out = out;
   p.offs = nullptr;

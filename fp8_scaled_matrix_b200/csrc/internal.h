@@ -27,6 +27,13 @@ cudaError_t launch_quantize_transposed(const void* x, int64_t rows, int64_t cols
                                        int64_t ld, int recipe, void* q, float* scales,
                                        const LaunchCtx& ctx);
 
+// MXFP8 quantization (quantize.cu): q (rows, cols) e4m3, scale bytes in the
+// GEMM's scale-factor tiles (mx_scale_tile_bytes(rows, cols) bytes).
+// cols % 32 == 0.
+size_t mx_scale_tile_bytes(int64_t rows, int64_t cols);
+cudaError_t launch_quantize_mx(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                               void* q, void* sf, const LaunchCtx& ctx);
+
 // Library-owned scratch for the no-allocation quantize entry point
 // (quantize.cu): its size, and its device address on `device` (looked up
 // once per device; the device must be current).
@@ -34,7 +41,7 @@ size_t noalloc_scratch_bytes();
 cudaError_t noalloc_scratch_ptr(int device, void** out);
 
 // Dense scaled GEMM (gemm.cu).  recipe: 0 tensor, 1 row, 2 1x128_128x128,
-// 3 1x128_128x1.  out_kind: 0 bf16, 1 fp32, 2 e4m3 quantized in 1x128
+// 3 1x128_128x1, 4 MXFP8 (sa, sb then point to E8M0 scale-factor tiles).  out_kind: 0 bf16, 1 fp32, 2 e4m3 quantized in 1x128
 // groups along n with scales written to out_scales[(n/128) * M + m].
 cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
                              int64_t N, int64_t K, const float* sa,

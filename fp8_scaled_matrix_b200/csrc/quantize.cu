@@ -220,6 +220,76 @@ __global__ void __launch_bounds__(256) quant_1x128_kernel(
   }
 }
 
+// ------------------------------------------------------------ MXFP8
+// OCP Microscaling (the "mxfp8" recipe of "Add _scaled_mm_v2 API"): per block
+// of 32 elements along a row, e = floor(log2(amax)) - 8 clamped to
+// [-127, 127] (an all-zero block: -127), scale byte e + 127 (E8M0), codes
+// e4m3_satfinite(x * 2^-e).  Both the exponent (from the bits of amax) and
+// the scaling (by a power of two) are exact.
+// One warp per 2048-element span of a row: lane l holds 16-byte chunks
+// l + 32 i (i < 8), so each load instruction reads 512 contiguous bytes and
+// four consecutive lanes hold one block (amax over 2 shuffles).  Scale bytes
+// go straight into the GEMM's scale-factor tiles: tile (row / 128, block / 4),
+// byte (row % 32) * 16 + ((row % 128) / 32) * 4 + block % 4.  Warps past the
+// last row (up to the next multiple of 128) and the blocks past the last one
+// of a row (up to the next multiple of 4) write zero scale bytes, so the
+// tiles hold no stale bytes.
+constexpr int kMxChunks = 8;                 // 16-byte chunks per lane
+constexpr int kMxSpan = 32 * kMxChunks * 8;  // elements per warp
+
+__device__ __forceinline__ int64_t mx_tile_byte(int64_t row, int64_t kb, int64_t KT) {
+  const int64_t r = row & 127;
+  return ((row >> 7) * KT + (kb >> 2)) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (kb & 3);
+}
+
+__global__ void __launch_bounds__(256) quant_mx_kernel(
+    const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+    uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+  const int lane = threadIdx.x & 31;
+  const int64_t spans = (cols + kMxSpan - 1) / kMxSpan;
+  const int64_t warp = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int64_t row = warp / spans;
+  const int64_t c0 = (warp % spans) * (kMxSpan / 8);  // first chunk of the span
+  const int64_t C8 = cols >> 3;                       // chunks per row
+  const int64_t KB = cols >> 5;
+  const int64_t KT = (KB + 3) >> 2;
+  const int64_t rows_pad = (rows + 127) & ~int64_t(127);
+  if (row >= rows_pad) return;
+  if (row >= rows) {
+    // padding rows of the last row tile: zero scale bytes
+    for (int64_t kb = (c0 >> 2) + lane; kb < KT * 4 && kb < (c0 >> 2) + kMxSpan / 32; kb += 32)
+      sf[mx_tile_byte(row, kb, KT)] = 0;
+    return;
+  }
+  uint4 v[kMxChunks];
+#pragma unroll
+  for (int i = 0; i < kMxChunks; ++i) {
+    const int64_t c = c0 + lane + 32 * i;
+    if (c < C8) v[i] = ld_stream(reinterpret_cast<const uint4*>(x + row * ld + c * 8));
+  }
+#pragma unroll
+  for (int i = 0; i < kMxChunks; ++i) {
+    const int64_t c = c0 + lane + 32 * i;
+    // C8 is a multiple of 4, so a block's four lanes agree on c < C8
+    float m = c < C8 ? amax8(v[i], 0.0f) : 0.0f;
+    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+    if (c >= C8) continue;
+    // floor(log2(m)) = biased exponent - 127 for normal m; zero and
+    // subnormal m clamp to -127 like every exponent below it
+    const int be = static_cast<int>(__float_as_uint(m) >> 23);
+    const int e = max(be - 127 - 8, -127);               // <= 119 for finite m
+    const float inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e
+    *reinterpret_cast<uint2*>(q + row * cols + c * 8) = cast8(v[i], inv);
+    if ((lane & 3) == 0) {
+      const int64_t kb = c >> 2;
+      sf[mx_tile_byte(row, kb, KT)] = static_cast<uint8_t>(e + 127);
+      if (kb == KB - 1)
+        for (int64_t k = KB; k < KT * 4; ++k) sf[mx_tile_byte(row, k, KT)] = 0;
+    }
+  }
+}
+
 // ------------------------------------------------------------ 128x128
 // One CTA (512 threads) per 128x128 tile: thread t covers the 16-byte chunk
 // t%16 of rows t/16 + 32 i (i < 4), so each warp-wide load reads two whole
@@ -479,6 +549,23 @@ cudaError_t noalloc_scratch_ptr(int device, void** out) {
   }
   *out = g_noalloc_ptr[device];
   return cudaSuccess;
+}
+
+size_t mx_scale_tile_bytes(int64_t rows, int64_t cols) {
+  const int64_t KT = (cols / 32 + 3) / 4;
+  return static_cast<size_t>(((rows + 127) / 128) * KT * 512);
+}
+
+cudaError_t launch_quantize_mx(const void* xv, int64_t rows, int64_t cols, int64_t ld,
+                               void* qv, void* sfv, const LaunchCtx& ctx) {
+  if (rows == 0 || cols == 0) return cudaSuccess;
+  const int64_t spans = (cols + kMxSpan - 1) / kMxSpan;
+  const int64_t warps = ((rows + 127) / 128) * 128 * spans;
+  const unsigned grid = static_cast<unsigned>((warps + 7) / 8);
+  quant_mx_kernel<<<grid, 256, 0, ctx.stream>>>(static_cast<const uint16_t*>(xv), rows, cols,
+                                                ld, static_cast<uint8_t*>(qv),
+                                                static_cast<uint8_t*>(sfv));
+  return cudaGetLastError();
 }
 
 cudaError_t launch_quantize_transposed(const void* xv, int64_t rows, int64_t cols,

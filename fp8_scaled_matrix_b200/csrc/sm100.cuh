@@ -484,6 +484,63 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(uint32_t M, uint32_t N) {
   return (1u << 4) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
+// ------------------------------------------------- block-scaled (MXFP8) MMA
+// Contiguous global -> shared bulk copy completing on `bar` (bytes counted in
+// its transaction count).  dst, src 16-byte aligned, bytes % 16 == 0.  No
+// cluster multicast.
+__device__ __forceinline__ void bulk_load_g2s(void* smem_dst, const void* src,
+                                              uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1], %2, [%3];" ::"r"(smem_u32(smem_dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Shared-memory descriptor of a K-major, unswizzled matrix of 16-byte rows
+// (core matrices of 8 rows x 16 bytes, 128 bytes apart): the source of
+// tcgen05.cp for a 32 x 128-bit scale-factor block.
+__device__ __forceinline__ uint64_t smem_desc_rows16(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(128u >> 4) << 16;   // leading byte offset
+  d |= static_cast<uint64_t>(128u >> 4) << 32;   // stride byte offset (8-row groups)
+  d |= static_cast<uint64_t>(1u) << 46;          // descriptor version
+  return d;                                      // layout type 0: no swizzle
+}
+
+// Copy a 32-row x 128-bit block from shared memory into TMEM columns
+// [taddr, taddr + 4) of all four 32-lane quarters (row i -> lane 32 q + i of
+// every quarter q).  Ordered before later tcgen05.mma of the same thread.
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
+// D (+)= (A * 2^sfa) (B * 2^sfb)^T with one E8M0 scale per 32 elements of K
+// for each row of A and of B, read from TMEM (kind::mxf8f6f4, block32).
+__device__ __forceinline__ void mma_mx_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t sfa_tmem,
+                                            uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.scale_vec::1X "
+      "[%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor for kind::mxf8f6f4 block-scaled, A = B = e4m3,
+// D = fp32, both K-major, E8M0 scales:
+//   [4,6) B scale-factor byte   [7,10) A format (0 = e4m3)  [10,13) B format
+//   [17,23) N >> 3              [23] scale type (1 = E8M0)   [24,29) M >> 4
+//   [29,31) A scale-factor byte
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3(uint32_t M, uint32_t N, uint32_t sf_a,
+                                                     uint32_t sf_b) {
+  return (sf_b << 4) | ((N >> 3) << 17) | (1u << 23) | ((M >> 4) << 24) | (sf_a << 29);
+}
+
 // 16-byte asynchronous global -> shared copy (no registers involved);
 // src_bytes = 0 writes zeros without reading `src` (which must still be a
 // valid address).  Completion is tracked per thread with commit/wait groups.

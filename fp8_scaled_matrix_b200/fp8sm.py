@@ -34,7 +34,8 @@ EXPORTED = ["fp8_version", "fp8_last_error", "fp8_quantize_workspace_bytes",
             "fp8_quantize", "fp8_scaled_mm", "fp8_grouped_scaled_mm",
             "fp8_get_device_status", "fp8_debug_timeout_probe",
             "fp8_quantize_noalloc", "fp8_quantize_transposed",
-            "fp8_grouped_scaled_mm_blockwise", "fp8_scaled_mm_quantized"]
+            "fp8_grouped_scaled_mm_blockwise", "fp8_scaled_mm_quantized",
+            "fp8_mx_scale_bytes", "fp8_quantize_mx", "fp8_scaled_mm_mx"]
 
 
 class Fp8Error(RuntimeError):
@@ -81,6 +82,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fp8_quantize.argtypes = [P, I64, I64, I64, E, P, P, P, SZ, P]
     L.fp8_scaled_mm.restype = E
     L.fp8_scaled_mm.argtypes = [P, P, I64, I64, I64, P, P, E, P, E, P, P]
+    L.fp8_mx_scale_bytes.restype = SZ
+    L.fp8_mx_scale_bytes.argtypes = [I64, I64]
+    L.fp8_quantize_mx.restype = E
+    L.fp8_quantize_mx.argtypes = [P, I64, I64, I64, P, P, P]
+    L.fp8_scaled_mm_mx.restype = E
+    L.fp8_scaled_mm_mx.argtypes = [P, P, I64, I64, I64, P, P, P, E, P, P]
     L.fp8_scaled_mm_quantized.restype = E
     L.fp8_scaled_mm_quantized.argtypes = [P, P, I64, I64, I64, P, P, E, P, P, P, P]
     L.fp8_grouped_scaled_mm.restype = E
@@ -274,6 +281,60 @@ def fp8_scaled_mm_quantized(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Ten
                                      _ptr(scale_b), recipe, _ptr(bias), _ptr(out),
                                      _ptr(out_scales), _stream(stream)))
     return out, out_scales
+
+
+def fp8_mx_scale_bytes(rows: int, cols: int) -> int:
+    return int(load_library().fp8_mx_scale_bytes(rows, cols))
+
+
+def fp8_quantize_mx(x: torch.Tensor, out: Optional[torch.Tensor] = None,
+                    scales: Optional[torch.Tensor] = None,
+                    stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """MXFP8 quantization of a 2-D bf16 CUDA tensor: returns (codes uint8
+    (rows, cols), E8M0 scale bytes uint8 in the scale-factor tile layout)."""
+    L = load_library()
+    _need_cuda(x)
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D bf16 tensor with unit column stride")
+    rows, cols = x.shape
+    if out is None:
+        out = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    nbytes = fp8_mx_scale_bytes(rows, cols)
+    if scales is None:
+        scales = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=x.device)
+    if out.numel() < rows * cols or scales.numel() < nbytes:
+        raise ValueError("out or scales too small")
+    _check(L.fp8_quantize_mx(_ptr(x), rows, cols, x.stride(0), _ptr(out), _ptr(scales),
+                             _stream(stream)))
+    return out, scales[:nbytes] if scales.numel() > nbytes else scales
+
+
+def fp8_scaled_mm_mx(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor,
+                     scale_b: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                     out_dtype=torch.bfloat16, out: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """MXFP8 GEMM: a (M,K), b (N,K) e4m3 codes; scale_a, scale_b E8M0 bytes
+    in the scale-factor tile layout (as fp8_quantize_mx returns them)."""
+    L = load_library()
+    _need_cuda(a, b, scale_a, scale_b, bias)
+    M, K = a.shape
+    N = b.shape[0]
+    if b.shape[1] != K:
+        raise ValueError("a and b must share K")
+    for t in (a, b):
+        if t.dtype not in (torch.uint8, torch.float8_e4m3fn) or not t.is_contiguous():
+            raise ValueError("a and b must be contiguous e4m3 (uint8 codes)")
+    if (scale_a.numel() < fp8_mx_scale_bytes(M, K) or
+            scale_b.numel() < fp8_mx_scale_bytes(N, K)):
+        raise ValueError("scale tiles too small")
+    if bias is not None and (bias.dtype != torch.bfloat16 or not bias.is_contiguous()):
+        raise ValueError("bias must be a contiguous bf16 tensor")
+    od = FP8_OUT_F32 if out_dtype == torch.float32 else FP8_OUT_BF16
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=a.device)
+    _check(L.fp8_scaled_mm_mx(_ptr(a), _ptr(b), M, N, K, _ptr(scale_a), _ptr(scale_b),
+                              _ptr(bias), od, _ptr(out), _stream(stream)))
+    return out
 
 
 def fp8_grouped_scaled_mm(a: torch.Tensor, b_experts: torch.Tensor,

@@ -37,6 +37,8 @@ descriptions; no public dataset is involved):
                 the second as its 1x128 activation: 16640 tokens, 8192 -> 5120
                 -> 8192; X ~ N(0,1) (16640, 8192), W1 ~ N(0, 0.02^2)
                 (5120, 8192), W2 ~ N(0, 0.02^2) (8192, 5120) as stored
+  9 mxfp8       the tensors of workload 2 (same seeds, both (N, K) shapes),
+                quantized MXFP8 (E8M0 scale per 32 elements of K)
 """
 from __future__ import annotations
 
@@ -56,6 +58,7 @@ WORKLOAD_NAMES = [
     "grad_weight_1x128_128x1",
     "grouped_e16_blockwise",
     "linear_chain_1x128_128x128",
+    "mxfp8",
 ]
 
 
@@ -109,7 +112,7 @@ def offsets_from_sizes(sizes) -> torch.Tensor:
 class Workload:
     name: str
     # tensor | row | 1x128_128x128 | 1x128_128x1 | grouped | grouped_blockwise |
-    # grad_input | grad_weight | chain
+    # grad_input | grad_weight | chain | mxfp8
     recipe: str
     M: int
     N: int
@@ -143,6 +146,10 @@ def make_workload(index: int, shape_index: int = 0, scale_down: int = 1) -> Work
     if index == 7:  # workload 4's tensors, blockwise-scaled
         wl = make_workload(4, shape_index, scale_down)
         wl.name, wl.recipe = name, "grouped_blockwise"
+        return wl
+    if index == 9:  # workload 2's tensors, MXFP8
+        wl = make_workload(2, shape_index, scale_down)
+        wl.name, wl.recipe = name, "mxfp8"
         return wl
     seed = 1000 + index + 100 * shape_index
     g = generator(seed)

@@ -237,6 +237,54 @@ FP8SM_API fp8_status fp8_scaled_mm_quantized(const void* a, const void* b, int64
                                    float* out_scales, fp8_stream_t stream);
 
 /*
+ * MXFP8 ("mxfp8" in the recipe table of [P4]; the pages name the recipe but
+ * do not define it, so the OCP Microscaling (MX) specification's definition
+ * is used): one power-of-two E8M0 scale per block of 32 consecutive elements
+ * along K, E4M3 elements.  Per block:
+ *   e     = floor(log2(max |x|)) - 8, clamped to [-127, 127]; -127 for an
+ *           all-zero block (8: 2^8 = 256 is the largest power of two in E4M3)
+ *   byte  = e + 127                       (the block's scale is 2^e)
+ *   q     = e4m3_satfinite_rn(x * 2^-e)   (exact scaling; amax/2^e < 512)
+ *
+ * Scale bytes are stored in the tensor core's scale-factor tiles: for a
+ * (rows, cols) matrix, tiles of 128 rows x 4 blocks (128 elements of K),
+ * 512 bytes each, ordered tile (i, j) at byte offset (i * ceil(cols/128) + j)
+ * * 512; inside a tile the byte of row r (< 128) and block k (< 4) sits at
+ *   (r % 32) * 16 + (r / 32) * 4 + k.
+ * fp8_mx_scale_bytes(rows, cols) = ceil(rows/128) * ceil(cols/128) * 512.
+ * Bytes for rows past `rows` and blocks past cols/32 are padding;
+ * fp8_quantize_mx writes them as zero.
+ */
+FP8SM_API size_t fp8_mx_scale_bytes(int64_t rows, int64_t cols);
+
+/*
+ *   x_bf16          (rows, cols) bf16, row stride ld_x (elements, a multiple
+ *                   of 8), 16-byte aligned; finite values.
+ *   out_fp8         (rows, cols) e4m3 codes, row stride cols, 16-byte aligned.
+ *   out_scales_e8m0 fp8_mx_scale_bytes(rows, cols) bytes, 16-byte aligned.
+ * Requirements: cols % 32 == 0.  rows == 0 or cols == 0 is a no-op.
+ */
+FP8SM_API fp8_status fp8_quantize_mx(const void* x_bf16, int64_t rows, int64_t cols,
+                           int64_t ld_x, void* out_fp8, void* out_scales_e8m0,
+                           fp8_stream_t stream);
+
+/*
+ * MXFP8 GEMM:
+ *   out[m, n] = sum_k (a[m,k] 2^(sa[m, k/32] - 127)) (b[n,k] 2^(sb[n, k/32] - 127))
+ *               (+ bias[n])
+ * with sa, sb the E8M0 scale bytes of a (M, K) and b (N, K) in the
+ * scale-factor tile layout above (fp8_mx_scale_bytes(M, K) and
+ * fp8_mx_scale_bytes(N, K) bytes, 16-byte aligned; padding bytes must not be
+ * 0xFF).  The tensor core applies the scales (tcgen05.mma block_scale); fp32
+ * accumulation.  out (M, N) bf16 or fp32, 16-byte aligned.
+ * Requirements: K > 0, K % 32 == 0, N % 16 == 0.  M == 0 or N == 0 is a no-op.
+ */
+FP8SM_API fp8_status fp8_scaled_mm_mx(const void* a, const void* b, int64_t M, int64_t N,
+                            int64_t K, const void* scale_a_e8m0,
+                            const void* scale_b_e8m0, const void* bias_bf16,
+                            fp8_out_dtype out_dtype, void* out, fp8_stream_t stream);
+
+/*
  * Grouped (MoE) scaled GEMM, rowwise recipe only ([P2] Design, RowWise path;
  * other weight granularities return FP8_ERR_UNSUPPORTED as [P2]'s review
  * requires):

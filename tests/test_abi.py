@@ -180,3 +180,54 @@ def test_missing_library_fails_loudly(tmp_path):
             fp8sm.load_library(str(tmp_path / "nope.so"))
         finally:
             fp8sm._lib = saved
+
+
+def test_mx_scale_bytes(lib):
+    assert lib.fp8_mx_scale_bytes(128, 128) == 512
+    assert lib.fp8_mx_scale_bytes(129, 128) == 1024
+    assert lib.fp8_mx_scale_bytes(1, 32) == 512
+    assert lib.fp8_mx_scale_bytes(16640, 8192) == 130 * 64 * 512
+    assert lib.fp8_mx_scale_bytes(0, 64) == 0
+
+
+@pytest.mark.parametrize("rows,cols,ld,frag", [
+    (128, 48, 48, "multiple of 32"),
+    (128, 64, 60, "ld_x"),
+    (128, 64, 68, "ld_x"),
+    (-1, 64, 64, "negative"),
+])
+def test_quantize_mx_rejects_bad_arguments(lib, rows, cols, ld, frag):
+    st = lib.fp8_quantize_mx(FAKE, rows, cols, ld, FAKE, FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE and frag in lib.fp8_last_error().decode()
+
+
+def test_quantize_mx_null_alignment_and_empty(lib):
+    assert lib.fp8_quantize_mx(FAKE, 4, 64, 64, FAKE, None, None) == fp8sm.FP8_ERR_VALUE
+    st = lib.fp8_quantize_mx(FAKE, 4, 64, 64, FAKE, P((1 << 20) + 8), None)
+    assert st == fp8sm.FP8_ERR_VALUE and "aligned" in lib.fp8_last_error().decode()
+    assert lib.fp8_quantize_mx(None, 0, 64, 64, None, None, None) == fp8sm.FP8_OK
+
+
+@pytest.mark.parametrize("M,N,K,frag", [
+    (128, 128, 0, "positive multiple of 32"),
+    (128, 128, 48, "positive multiple of 32"),
+    (128, 120, 64, "N must be a multiple of 16"),
+    (128, -16, 64, "negative"),
+])
+def test_scaled_mm_mx_rejects_bad_arguments(lib, M, N, K, frag):
+    st = lib.fp8_scaled_mm_mx(FAKE, FAKE, M, N, K, FAKE, FAKE, None, fp8sm.FP8_OUT_BF16,
+                              FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE and frag in lib.fp8_last_error().decode()
+
+
+def test_scaled_mm_mx_null_alignment_dtype_and_empty(lib):
+    st = lib.fp8_scaled_mm_mx(FAKE, FAKE, 64, 64, 64, None, FAKE, None, fp8sm.FP8_OUT_BF16,
+                              FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE and "null" in lib.fp8_last_error().decode()
+    st = lib.fp8_scaled_mm_mx(FAKE, FAKE, 64, 64, 64, FAKE, P((1 << 20) + 4), None,
+                              fp8sm.FP8_OUT_BF16, FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE and "aligned" in lib.fp8_last_error().decode()
+    st = lib.fp8_scaled_mm_mx(FAKE, FAKE, 64, 64, 64, FAKE, FAKE, None, 7, FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE and "out_dtype" in lib.fp8_last_error().decode()
+    assert lib.fp8_scaled_mm_mx(None, None, 0, 64, 64, None, None, None, fp8sm.FP8_OUT_BF16,
+                                None, None) == fp8sm.FP8_OK
