@@ -226,20 +226,27 @@ __global__ void __launch_bounds__(256) quant_1x128_kernel(
 // [-127, 127] (an all-zero block: -127), scale byte e + 127 (E8M0), codes
 // e4m3_satfinite(x * 2^-e).  Both the exponent (from the bits of amax) and
 // the scaling (by a power of two) are exact.
-// One warp per 2048-element span of a row: lane l holds 16-byte chunks
-// l + 32 i (i < 8), so each load instruction reads 512 contiguous bytes and
-// four consecutive lanes hold one block (amax over 2 shuffles).  Scale bytes
-// go straight into the GEMM's scale-factor tiles: tile (row / 128, block / 4),
-// byte (row % 32) * 16 + ((row % 128) / 32) * 4 + block % 4.  Warps past the
-// last row (up to the next multiple of 128) and the blocks past the last one
-// of a row (up to the next multiple of 4) write zero scale bytes, so the
-// tiles hold no stale bytes.
-constexpr int kMxChunks = 8;                 // 16-byte chunks per lane
-constexpr int kMxSpan = 32 * kMxChunks * 8;  // elements per warp
+// One warp per 2048-element span of a row: lane l holds the 32-byte
+// (16-element) pieces l + 32 i (i < 4), so two consecutive lanes hold one
+// block (amax over one shuffle) and each lane writes 16 codes at once.
+// Scale bytes go straight into the GEMM's scale-factor tiles: tile (row / 128,
+// block / 4), byte (row % 32) * 16 + ((row % 128) / 32) * 4 + block % 4.
+// Warps past the last row (up to the next multiple of 128) and the blocks
+// past the last one of a row (up to the next multiple of 4) write zero scale
+// bytes, so the tiles hold no stale bytes.
+constexpr int kMxItems = 4;                  // 16-element pieces per lane
+constexpr int kMxSpan = 32 * kMxItems * 16;  // elements per warp
 
-__device__ __forceinline__ int64_t mx_tile_byte(int64_t row, int64_t kb, int64_t KT) {
-  const int64_t r = row & 127;
-  return ((row >> 7) * KT + (kb >> 2)) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (kb & 3);
+// Block maximum of |x| as bf16 magnitude bits: for finite values the order of
+// |x| is the unsigned order of (bits & 0x7FFF), so two bf16 per word are
+// compared at once; the exponent of the maximum is then bits >> 7.
+__device__ __forceinline__ uint32_t absmax_bits16(const uint4& a, const uint4& b) {
+  const uint32_t m0 = __vmaxu2(__vmaxu2(a.x & 0x7FFF7FFFu, a.y & 0x7FFF7FFFu),
+                               __vmaxu2(a.z & 0x7FFF7FFFu, a.w & 0x7FFF7FFFu));
+  const uint32_t m1 = __vmaxu2(__vmaxu2(b.x & 0x7FFF7FFFu, b.y & 0x7FFF7FFFu),
+                               __vmaxu2(b.z & 0x7FFF7FFFu, b.w & 0x7FFF7FFFu));
+  const uint32_t m = __vmaxu2(m0, m1);
+  return max(m & 0xFFFFu, m >> 16);
 }
 
 __global__ void __launch_bounds__(256) quant_mx_kernel(
@@ -249,43 +256,51 @@ __global__ void __launch_bounds__(256) quant_mx_kernel(
   const int64_t spans = (cols + kMxSpan - 1) / kMxSpan;
   const int64_t warp = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int64_t row = warp / spans;
-  const int64_t c0 = (warp % spans) * (kMxSpan / 8);  // first chunk of the span
-  const int64_t C8 = cols >> 3;                       // chunks per row
+  const int64_t p0 = (warp % spans) * (kMxSpan / 16);  // first 16-element piece of the span
+  const int64_t P = cols >> 4;                          // pieces per row (even)
   const int64_t KB = cols >> 5;
   const int64_t KT = (KB + 3) >> 2;
   const int64_t rows_pad = (rows + 127) & ~int64_t(127);
   if (row >= rows_pad) return;
+  const int64_t r7 = row & 127;
+  // this row's scale bytes: tile row (row / 128), byte (row % 32) * 16 + (row % 128 / 32) * 4
+  uint8_t* sfr = sf + (row >> 7) * KT * 512 + (r7 & 31) * 16 + (r7 >> 5) * 4;
   if (row >= rows) {
     // padding rows of the last row tile: zero scale bytes
-    for (int64_t kb = (c0 >> 2) + lane; kb < KT * 4 && kb < (c0 >> 2) + kMxSpan / 32; kb += 32)
-      sf[mx_tile_byte(row, kb, KT)] = 0;
+    for (int64_t kb = (p0 >> 1) + lane; kb < KT * 4 && kb < (p0 >> 1) + kMxSpan / 32; kb += 32)
+      sfr[(kb >> 2) * 512 + (kb & 3)] = 0;
     return;
   }
-  uint4 v[kMxChunks];
+  // pieces of this span inside the row (even, as P is)
+  const int np = static_cast<int>(P - p0 < kMxSpan / 16 ? P - p0 : kMxSpan / 16);
+  const uint4* xs = reinterpret_cast<const uint4*>(x + row * ld) + 2 * p0;
+  uint4* qs = reinterpret_cast<uint4*>(q + row * cols) + p0;
+  uint4 v[kMxItems][2];
 #pragma unroll
-  for (int i = 0; i < kMxChunks; ++i) {
-    const int64_t c = c0 + lane + 32 * i;
-    if (c < C8) v[i] = ld_stream(reinterpret_cast<const uint4*>(x + row * ld + c * 8));
-  }
+  for (int i = 0; i < kMxItems; ++i)
+    if (lane + 32 * i < np) {
+      v[i][0] = ld_stream(xs + 2 * (lane + 32 * i));
+      v[i][1] = ld_stream(xs + 2 * (lane + 32 * i) + 1);
+    }
 #pragma unroll
-  for (int i = 0; i < kMxChunks; ++i) {
-    const int64_t c = c0 + lane + 32 * i;
-    // C8 is a multiple of 4, so a block's four lanes agree on c < C8
-    float m = c < C8 ? amax8(v[i], 0.0f) : 0.0f;
-    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-    if (c >= C8) continue;
-    // floor(log2(m)) = biased exponent - 127 for normal m; zero and
-    // subnormal m clamp to -127 like every exponent below it
-    const int be = static_cast<int>(__float_as_uint(m) >> 23);
-    const int e = max(be - 127 - 8, -127);               // <= 119 for finite m
+  for (int i = 0; i < kMxItems; ++i) {
+    const int pl = lane + 32 * i;
+    // a block's two lanes agree on pl < np
+    uint32_t m = pl < np ? absmax_bits16(v[i][0], v[i][1]) : 0u;
+    m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+    if (pl >= np) continue;
+    // floor(log2(amax)) = biased exponent - 127 for normal amax; zero and
+    // subnormal amax clamp to -127 like every exponent below it
+    const int e = max(static_cast<int>(m >> 7) - 127 - 8, -127);   // <= 119 for finite amax
     const float inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e
-    *reinterpret_cast<uint2*>(q + row * cols + c * 8) = cast8(v[i], inv);
-    if ((lane & 3) == 0) {
-      const int64_t kb = c >> 2;
-      sf[mx_tile_byte(row, kb, KT)] = static_cast<uint8_t>(e + 127);
+    const uint2 lo = cast8(v[i][0], inv);
+    const uint2 hi = cast8(v[i][1], inv);
+    qs[pl] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+    if ((lane & 1) == 0) {
+      const int64_t kb = (p0 + pl) >> 1;
+      sfr[(kb >> 2) * 512 + (kb & 3)] = static_cast<uint8_t>(e + 127);
       if (kb == KB - 1)
-        for (int64_t k = KB; k < KT * 4; ++k) sf[mx_tile_byte(row, k, KT)] = 0;
+        for (int64_t k = KB; k < KT * 4; ++k) sfr[(k >> 2) * 512 + (k & 3)] = 0;
     }
   }
 }
