@@ -52,6 +52,8 @@ def lib():
                                            P, P, P, P, I64, P, P]
         L.or_mx_quantize.restype = ctypes.c_int
         L.or_mx_quantize.argtypes = [P, I64, I64, I64, P, P]
+        L.or_mx_quantize_f32.restype = ctypes.c_int
+        L.or_mx_quantize_f32.argtypes = [P, I64, I64, I64, P, P]
         L.or_mx_scales_to_tiles.restype = ctypes.c_int
         L.or_mx_scales_to_tiles.argtypes = [P, I64, I64, P]
         L.or_mx_scaled_mm.restype = ctypes.c_int
@@ -222,6 +224,18 @@ def mx_quantize(x_bits: np.ndarray):
     rc = lib().or_mx_quantize(_ptr(x_bits), rows, cols, cols, _ptr(q), _ptr(e8))
     if rc != 0:
         raise ValueError("oracle mx_quantize: bad arguments")
+    return q, e8[:, :cols // 32]
+
+
+def mx_quantize_f32(x: np.ndarray):
+    """The same MXFP8 conversion of an fp32 matrix (2-D, cols % 32 == 0)."""
+    x = _c(x, np.float32)
+    rows, cols = x.shape
+    q = np.empty((rows, cols), dtype=np.uint8)
+    e8 = np.empty((rows, max(cols // 32, 1)), dtype=np.uint8)
+    rc = lib().or_mx_quantize_f32(_ptr(x), rows, cols, cols, _ptr(q), _ptr(e8))
+    if rc != 0:
+        raise ValueError("oracle mx_quantize_f32: bad arguments")
     return q, e8[:, :cols // 32]
 
 

@@ -450,30 +450,47 @@ static int mx_block_exponent(float amax) {
   return e;
 }
 
+/* One row of blocks; x values read through mv_get (bf16 or fp32 input). */
+static void mx_quantize_row(const mat_view* v, int64_t r, int64_t cols, uint8_t* e8) {
+  int64_t KB = cols / 32;
+  for (int64_t kb = 0; kb < KB; kb++) {
+    float amax = 0.0f;
+    for (int i = 0; i < 32; i++) {
+      float f = fabsf(mv_get(v, r * v->ld + kb * 32 + i));
+      if (f > amax) amax = f;
+    }
+    int e = mx_block_exponent(amax);
+    e8[r * KB + kb] = (uint8_t)(e + 127);
+    for (int i = 0; i < 32; i++) {
+      /* v / 2^e is exact in fp64; below 2^-126 it rounds to zero in E4M3
+       * whatever the fp32 rounding, so the float conversion loses nothing */
+      double y = ldexp((double)mv_get(v, r * v->ld + kb * 32 + i), -e);
+      v->q[r * v->ldq + kb * 32 + i] = or_e4m3_encode((float)y);
+    }
+  }
+}
+
 int or_mx_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
                    uint8_t* q, uint8_t* e8) {
   if (rows < 0 || cols < 0 || cols % 32 != 0 || ld < cols || !x || !q || !e8)
     return -1;
-  int64_t KB = cols / 32;
+  mat_view v = {x, NULL, ld, q, cols};
   int64_t r;
 #pragma omp parallel for schedule(static)
-  for (r = 0; r < rows; r++)
-    for (int64_t kb = 0; kb < KB; kb++) {
-      const uint16_t* v = x + r * ld + kb * 32;
-      float amax = 0.0f;
-      for (int i = 0; i < 32; i++) {
-        float f = fabsf(or_bf16_to_float(v[i]));
-        if (f > amax) amax = f;
-      }
-      int e = mx_block_exponent(amax);
-      e8[r * KB + kb] = (uint8_t)(e + 127);
-      for (int i = 0; i < 32; i++) {
-        /* v / 2^e is exact in fp64; below 2^-126 it rounds to zero in E4M3
-         * whatever the fp32 rounding, so the float conversion loses nothing */
-        double y = ldexp((double)or_bf16_to_float(v[i]), -e);
-        q[r * cols + kb * 32 + i] = or_e4m3_encode((float)y);
-      }
-    }
+  for (r = 0; r < rows; r++) mx_quantize_row(&v, r, cols, e8);
+  return 0;
+}
+
+/* The same conversion of an fp32 matrix (a GEMM result quantized for the
+ * next MXFP8 GEMM). */
+int or_mx_quantize_f32(const float* x, int64_t rows, int64_t cols, int64_t ld,
+                       uint8_t* q, uint8_t* e8) {
+  if (rows < 0 || cols < 0 || cols % 32 != 0 || ld < cols || !x || !q || !e8)
+    return -1;
+  mat_view v = {NULL, x, ld, q, cols};
+  int64_t r;
+#pragma omp parallel for schedule(static)
+  for (r = 0; r < rows; r++) mx_quantize_row(&v, r, cols, e8);
   return 0;
 }
 

@@ -123,6 +123,10 @@ int or_grouped_scaled_mm(const uint8_t* a, const uint8_t* b_experts,
 int or_mx_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
                    uint8_t* q, uint8_t* e8);
 
+/* or_mx_quantize on fp32 input x (row stride ld): the same steps. */
+int or_mx_quantize_f32(const float* x, int64_t rows, int64_t cols, int64_t ld,
+                       uint8_t* q, uint8_t* e8);
+
 /* e8 (rows, kblocks) rearranged into 512-byte scale-factor tiles (128 rows x
  * 4 blocks each, row-tile-major; byte (r%32)*16 + (r/32)*4 + k inside), zero
  * past the matrix.  tiles holds ceil(rows/128) * ceil(kblocks/4) * 512 bytes. */

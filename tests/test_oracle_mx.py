@@ -178,3 +178,30 @@ def test_scale_tiles_is_a_bijection():
             assert pos not in seen
             seen.add(pos)
     assert len(seen) == rows * kb == oracle.mx_tile_bytes(rows, kb)
+
+
+def test_quantize_f32_matches_bf16_path_on_bf16_values():
+    xb = _random_blocks(45, 192, 11)
+    q1, e1 = oracle.mx_quantize(W.bf16_bits(xb))
+    q2, e2 = oracle.mx_quantize_f32(xb.float().numpy())
+    assert np.array_equal(q1, q2) and np.array_equal(e1, e2)
+
+
+def test_quantize_f32_against_torch_cast():
+    # fp32 values with full 24-bit significands, spread over 2^-60 .. 2^60
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal((20, 256)) * np.exp2(rng.integers(-60, 61, (20, 8))).repeat(32, axis=1)
+    x = x.astype(np.float32)
+    x[3, 64:96] = 0.0
+    x[4, 5] = np.float32(2.0 ** -140)                 # a subnormal block maximum
+    x[4, 0:5] = 0.0
+    x[4, 6:32] = 0.0
+    q, e8 = oracle.mx_quantize_f32(x)
+    e = e8.astype(np.int64) - 127
+    amax = np.abs(x.astype(np.float64)).reshape(20, 8, 32).max(axis=2)
+    scaled = amax / np.ldexp(1.0, e)
+    assert (((scaled >= 256) & (scaled < 512)) | (e == -127)).all()
+    assert e8[4, 0] == 0 and e8[3, 2] == 0
+    y = np.clip(x.astype(np.float64).reshape(20, 8, 32) / np.ldexp(1.0, e)[:, :, None], -448, 448)
+    want = torch.from_numpy(y.reshape(20, 256).astype(np.float32)).to(torch.float8_e4m3fn)
+    assert np.array_equal(q, want.view(torch.uint8).numpy())
