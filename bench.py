@@ -54,6 +54,7 @@ WORKLOADS = {
     "linear_chain_1x128_128x128": (8, 0),
     "mxfp8_16640x5120x8192": (9, 0),
     "mxfp8_16640x8192x5120": (9, 1),
+    "linear_chain_mxfp8": (10, 0),
 }
 DEFAULT_WORKLOAD = "rowwise_4096"
 # Page 5's context numbers (TFLOP/s of torch._scaled_mm, hardware not stated)
@@ -66,7 +67,7 @@ OPERAND_GROUPS = {"tensor": ("tensor", "tensor"), "row": ("row", "row"),
                   "1x128_128x1": ("1x128", "1x128"), "grouped": ("row", "row"),
                   "grad_input": ("1x128", "128x128"), "grad_weight": ("1x128", "1x128"),
                   "grouped_blockwise": ("1x128", "128x128"), "chain": ("1x128", "128x128"),
-                  "mxfp8": ("mx", "mx")}
+                  "mxfp8": ("mx", "mx"), "chain_mx": ("mx", "mx")}
 # GEMM recipe of each workload recipe, and which operands are quantized
 # transposed (the training GEMMs contract along the stored rows)
 GEMM_RECIPE = {"grad_input": "1x128_128x128", "grad_weight": "1x128_128x1",
@@ -209,7 +210,7 @@ class Step:
         self.wl = wl
         self.dev = dev
         ga, gb = OPERAND_GROUPS[wl.recipe]
-        self.mx = wl.recipe == "mxfp8"
+        self.mx = wl.recipe in ("mxfp8", "chain_mx")
         self.qa_recipe = None if self.mx else fp8sm.QUANT_RECIPES[ga]
         self.qb_recipe = None if self.mx else fp8sm.QUANT_RECIPES[gb]
         self.a = wl.a.to(dev)
@@ -253,7 +254,7 @@ class Step:
             self.sb = torch.empty(E * fp8sm.scale_count(N, K, self.qb_recipe),
                                   dtype=torch.float32, device=dev)
             self.launches_per_step = 2 + E
-        self.chain = wl.recipe == "chain"
+        self.chain = wl.recipe in ("chain", "chain_mx")
         if self.chain:
             # second linear: its weight (N2, N) quantized 128x128 like b; the
             # first GEMM's output leaves as e4m3 codes + 1x128 scales
@@ -261,10 +262,16 @@ class Step:
             self.b2 = wl.extra["b2"].to(dev)
             n2 = self.b2.shape[0]
             self.qb2 = torch.empty(n2, wl.N, dtype=torch.uint8, device=dev)
-            self.sb2 = torch.empty(fp8sm.scale_count(n2, wl.N, self.qb_recipe),
-                                   dtype=torch.float32, device=dev)
             self.y1q = torch.empty(wl.M, wl.N, dtype=torch.uint8, device=dev)
-            self.y1s = torch.empty(wl.N // 128, wl.M, dtype=torch.float32, device=dev)
+            if self.mx:
+                self.sb2 = torch.empty(fp8sm.fp8_mx_scale_bytes(n2, wl.N), dtype=torch.uint8,
+                                       device=dev)
+                self.y1s = torch.empty(fp8sm.fp8_mx_scale_bytes(wl.M, wl.N), dtype=torch.uint8,
+                                       device=dev)
+            else:
+                self.sb2 = torch.empty(fp8sm.scale_count(n2, wl.N, self.qb_recipe),
+                                       dtype=torch.float32, device=dev)
+                self.y1s = torch.empty(wl.N // 128, wl.M, dtype=torch.float32, device=dev)
             self.out = torch.empty(wl.M, n2, dtype=torch.bfloat16, device=dev)
             self.launches_per_step = 5
 
@@ -289,6 +296,8 @@ class Step:
                                           stream=self.side)
             elif self.mx:
                 f.fp8_quantize_mx(self.b, out=self.qb, scales=self.sb, stream=self.side)
+                if self.chain:
+                    f.fp8_quantize_mx(self.b2, out=self.qb2, scales=self.sb2, stream=self.side)
             elif self.chain:
                 f.fp8_quantize(self.b, self.qb_recipe, out=self.qb, scales=self.sb,
                                workspace=self.ws_b, stream=self.side)
@@ -319,6 +328,10 @@ class Step:
             E, N, K = wl.b.shape
             f.fp8_grouped_scaled_mm_blockwise(self.qa, self.qb.view(E, N, K), self.sa,
                                               self.sb, self.offs, out=self.out)
+        elif self.mx and self.chain:
+            f.fp8_scaled_mm_mx_quantized(self.qa, self.qb, self.sa, self.sb,
+                                         out=self.y1q, out_scales=self.y1s)
+            f.fp8_scaled_mm_mx(self.y1q, self.qb2, self.y1s, self.sb2, out=self.out)
         elif self.mx:
             f.fp8_scaled_mm_mx(self.qa, self.qb, self.sa, self.sb, bias=self.bias, out=self.out)
         elif self.chain:
@@ -338,7 +351,7 @@ class Step:
         b = 3 * n + self.sa.element_size() * self.sa.numel() + \
             self.sb.element_size() * self.sb.numel()
         if self.chain:
-            b += 3 * self.b2.numel() + 4 * self.sb2.numel()
+            b += 3 * self.b2.numel() + self.sb2.element_size() * self.sb2.numel()
         return b
 
 
@@ -483,6 +496,17 @@ def oracle_sample(wl, max_rows: int):
         b = W.bf16_bits(x)
         return np.ascontiguousarray(b.T) if transposed else b
     t0 = time.perf_counter()
+    if wl.recipe == "chain_mx":
+        qa, sa = oracle.mx_quantize(W.bf16_bits(wl.a))
+        qb, sb = oracle.mx_quantize(W.bf16_bits(wl.b))
+        qb2, sb2 = oracle.mx_quantize(W.bf16_bits(wl.extra["b2"]))
+        tq = time.perf_counter() - t0
+        rows = np.arange(min(max_rows, wl.M), dtype=np.int64)
+        t0 = time.perf_counter()
+        y1, _ = oracle.mx_scaled_mm(qa, qb, sa, sb, rows=rows)
+        y1q, y1e = oracle.mx_quantize_f32(y1.astype(np.float32))
+        oracle.mx_scaled_mm(y1q, qb2, y1e, sb2)
+        return time.perf_counter() - t0, rows.size / wl.M, tq, oracle.num_threads()
     if wl.recipe == "mxfp8":
         qa, sa = oracle.mx_quantize(W.bf16_bits(wl.a))
         qb, sb = oracle.mx_quantize(W.bf16_bits(wl.b))
@@ -540,9 +564,10 @@ def oracle_sample(wl, max_rows: int):
 def cpu_baseline(wl, rows: int):
     tg, frac, tq, threads = oracle_sample(wl, rows)
     est_s = tq + tg / frac
-    chain = wl.recipe == "chain"
+    chain = wl.recipe in ("chain", "chain_mx")
     what = "X, W1 and W2" if chain else "both operands"
-    gemm = "both GEMMs (the first one's fp32 output quantized 1x128)" if chain else "GEMM"
+    gemm = (("both GEMMs (the first one's fp32 output quantized "
+             + ("MXFP8)" if wl.recipe == "chain_mx" else "1x128)")) if chain else "GEMM")
     value = wl.flops / est_s / 1e12
     return {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
             "sample": (f"quantize of {what} in full ({tq:.2f} s) + {gemm} on "
@@ -658,6 +683,8 @@ def main(argv=None):
             "step": ("quantize X || quantize W1, W2 (two streams), then GEMM1 with its "
                      "output quantized 1x128 in the epilogue, then GEMM2"
                      if wl.recipe == "chain" else
+                     "MXFP8 quantize X || W1, W2 (two streams), then GEMM1 with MXFP8 "
+                     "output, then GEMM2" if wl.recipe == "chain_mx" else
                      "quantize A || quantize B (two streams), then scaled GEMM"),
             "N2": (int(wl.extra["b2"].shape[0]) if "b2" in wl.extra else None),
             "launch": ("CUDA graphs of the step's C-ABI launches" if args.graphs

@@ -361,6 +361,43 @@ fp8_status fp8_scaled_mm_mx(const void* a, const void* b, int64_t M, int64_t N, 
   return finish_launch(e, err, "fp8_scaled_mm_mx");
 }
 
+fp8_status fp8_scaled_mm_mx_quantized(const void* a, const void* b, int64_t M, int64_t N,
+                                      int64_t K, const void* scale_a_e8m0,
+                                      const void* scale_b_e8m0, const void* bias_bf16,
+                                      void* out_fp8, void* out_scales_e8m0,
+                                      fp8_stream_t stream) {
+  if (M < 0 || N < 0 || K < 0)
+    return fail(FP8_ERR_VALUE, "fp8_scaled_mm_mx_quantized: negative size");
+  if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+    return fail(FP8_ERR_VALUE, "fp8_scaled_mm_mx_quantized: size too large");
+  if (K == 0 || K % 32 != 0)
+    return fail(FP8_ERR_VALUE,
+                "fp8_scaled_mm_mx_quantized: K must be a positive multiple of 32");
+  if (N % 128 != 0)
+    return fail(FP8_ERR_VALUE, "fp8_scaled_mm_mx_quantized: N must be a multiple of 128");
+  if (M == 0 || N == 0) {
+    t_last_error.clear();
+    return FP8_OK;
+  }
+  if (a == nullptr || b == nullptr || scale_a_e8m0 == nullptr || scale_b_e8m0 == nullptr ||
+      out_fp8 == nullptr || out_scales_e8m0 == nullptr)
+    return fail(FP8_ERR_VALUE, "fp8_scaled_mm_mx_quantized: null pointer");
+  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(scale_a_e8m0, 16) ||
+      !aligned(scale_b_e8m0, 16) || !aligned(out_fp8, 16) || !aligned(out_scales_e8m0, 16) ||
+      (bias_bf16 && !aligned(bias_bf16, 16)))
+    return fail(FP8_ERR_VALUE, "fp8_scaled_mm_mx_quantized: pointers must be 16-byte aligned");
+  DeviceInfo* d = nullptr;
+  fp8_status s = device_info(&d);
+  if (s != FP8_OK) return s;
+  std::string err;
+  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status, d->num_sms, &err};
+  cudaError_t e = fp8sm::launch_scaled_mm(
+      a, b, M, N, K, static_cast<const float*>(scale_a_e8m0),
+      static_cast<const float*>(scale_b_e8m0), 4, bias_bf16, 3, out_fp8,
+      static_cast<float*>(out_scales_e8m0), ctx);
+  return finish_launch(e, err, "fp8_scaled_mm_mx_quantized");
+}
+
 namespace {
 
 // Shared by both grouped entry points; recipe 1 (rowwise) or 2 (1x128_128x128).

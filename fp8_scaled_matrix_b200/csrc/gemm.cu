@@ -115,8 +115,10 @@ struct Cfg {
 };
 
 enum Recipe : int { kTensor = 0, kRow = 1, kBlock128 = 2, kBlock1 = 3, kMxfp8 = 4 };
-// Output: bf16, fp32, or e4m3 quantized in 1x128 groups along n (+ scales)
-enum OutKind : int { kOutBf16 = 0, kOutFp32 = 1, kOutE4M3 = 2 };
+// Output: bf16, fp32, e4m3 quantized in 1x128 groups along n (+ fp32
+// scales), or MXFP8 (e4m3 + one E8M0 scale per 32 columns, in scale-factor
+// tiles: the A operand of the next MXFP8 GEMM)
+enum OutKind : int { kOutBf16 = 0, kOutFp32 = 1, kOutE4M3 = 2, kOutMx = 3 };
 
 struct GemmParams {
   int64_t M, N, K;
@@ -126,7 +128,7 @@ struct GemmParams {
   const uint8_t* sfb;
   const uint16_t* bias;
   void* out;
-  float* out_scales;  // e4m3 output: scale[(n/128) * M + m]
+  float* out_scales;  // e4m3 output: scale[(n/128) * M + m]; MXFP8 output: tiles
   const int32_t* offs;
   int32_t E;
   int32_t n_tiles;   // tiles along N
@@ -340,6 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr bool kBigEpi = kBlockwise || kIsMx;
   constexpr bool kOutF32 = kOut == kOutFp32;
   constexpr bool kOutQ = kOut == kOutE4M3;
+  constexpr bool kOutMxq = kOut == kOutMx;
   using C = Cfg<kPair>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -807,15 +810,57 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before_sync();
           __syncwarp();
           if (lane == 0) release_acc(0);
+          if constexpr (!kOutMxq) {
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            const int64_t n = ncol0 + cc * 32;
-            float v[32];
-            load_bias32(p.bias, n, p.N, v);
+            for (int cc = 0; cc < 4; ++cc) {
+              const int64_t n = ncol0 + cc * 32;
+              float v[32];
+              load_bias32(p.bias, n, p.N, v);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __fadd_rn(__uint_as_float(r[cc][i]), v[i]);
-            store_cols32<kOutF32, kGrouped>(ebuf, v, &tm_out, static_cast<int32_t>(n), row0,
-                                            c.row_end, p.out, p.N, lane);
+              for (int i = 0; i < 32; ++i) v[i] = __fadd_rn(__uint_as_float(r[cc][i]), v[i]);
+              store_cols32<kOutF32, kGrouped>(ebuf, v, &tm_out, static_cast<int32_t>(n), row0,
+                                              c.row_end, p.out, p.N, lane);
+            }
+          } else {
+            // MXFP8 output: the thread's 128 columns are four 32-wide blocks
+            // of its row.  Per block: e = floor(log2(amax)) - 8 clamped to
+            // [-127, 127] (from the bits of the fp32 amax), codes
+            // e4m3_satfinite(v * 2^-e).  The four scale bytes leave as one
+            // word of the output's scale-factor tiles (rows past M: zero).
+            uint32_t sc = 0;
+#pragma unroll
+            for (int bx = 0; bx < 2; ++bx) {
+              uint4 chunk[4];
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int cc = 2 * bx + h;
+                float v[32];
+                load_bias32(p.bias, ncol0 + cc * 32, p.N, v);
+                float am = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                  v[i] = __fadd_rn(__uint_as_float(r[cc][i]), v[i]);
+                  am = fmaxf(am, fabsf(v[i]));
+                }
+                const int e = max(static_cast<int>(__float_as_uint(am) >> 23) - 127 - 8, -127);
+                const float inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+                sc |= static_cast<uint32_t>(e + 127) << (8 * cc);
+                uint32_t* w = reinterpret_cast<uint32_t*>(&chunk[2 * h]);
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                  w[j] = cast_f32x2(v[4 * j], v[4 * j + 1], inv) |
+                         (cast_f32x2(v[4 * j + 2], v[4 * j + 3], inv) << 16);
+              }
+              store_box64<kGrouped>(ebuf, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
+                                    row0, c.row_end, static_cast<uint8_t*>(p.out), p.N, 1, lane);
+            }
+            if (ncol0 < p.N) {
+              const int64_t r7 = row & 127;
+              uint8_t* tiles = reinterpret_cast<uint8_t*>(p.out_scales);
+              const int64_t off = ((row >> 7) * (p.N / 128) + ncol0 / 128) * kMxSfTile +
+                                  (r7 & 31) * 16 + (r7 >> 5) * 4;
+              *reinterpret_cast<uint32_t*>(tiles + off) = row_ok ? sc : 0u;
+            }
           }
           next_acc();
           continue;
@@ -1100,7 +1145,9 @@ cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb,
   if constexpr (kPair && kBlockwise) {
     return cudaErrorInvalidValue;  // CTA pairs serve the dense recipes only
   } else if constexpr (kRecipe == kMxfp8 && (kPair || kGrouped || kOut == kOutE4M3)) {
-    return cudaErrorInvalidValue;  // MXFP8: single-CTA dense GEMM, bf16/fp32 out
+    return cudaErrorInvalidValue;  // MXFP8: single-CTA dense GEMM, bf16/fp32/MXFP8 out
+  } else if constexpr (kOut == kOutMx && kRecipe != kMxfp8) {
+    return cudaErrorInvalidValue;  // MXFP8 output from the MXFP8 GEMM only
   } else if constexpr (kOut == kOutE4M3 && (kPair || kGrouped)) {
     return cudaErrorInvalidValue;  // quantized output: single-CTA dense GEMM only
   } else {
@@ -1147,6 +1194,8 @@ cudaError_t dispatch(int recipe, int out_kind, bool pair, const CUtensorMap& ta,
   if (recipe == R) {                                                                    \
     if (out_kind == kOutE4M3)                                                           \
       return launch_kernel<R, kOutE4M3, kGrouped, false>(ta, tb, tbh, to, p, grid, st); \
+    if (out_kind == kOutMx)                                                             \
+      return launch_kernel<R, kOutMx, kGrouped, false>(ta, tb, tbh, to, p, grid, st);   \
     if (pair)                                                                           \
       return out_kind ? launch_kernel<R, kOutFp32, kGrouped, true>(ta, tb, tbh, to, p, grid, st) \
                       : launch_kernel<R, kOutBf16, kGrouped, true>(ta, tb, tbh, to, p, grid, st); \
@@ -1171,13 +1220,14 @@ cudaError_t dispatch(int recipe, int out_kind, bool pair, const CUtensorMap& ta,
 // staging layout) for bf16, fp32 or e4m3 output.
 bool out_map(CUtensorMap* m, void* out, int64_t rows, int64_t N, int out_kind,
              std::string* err) {
-  const uint64_t eb = out_kind == kOutFp32 ? 4 : out_kind == kOutE4M3 ? 1 : 2;
+  const bool q8 = out_kind == kOutE4M3 || out_kind == kOutMx;
+  const uint64_t eb = out_kind == kOutFp32 ? 4 : q8 ? 1 : 2;
   uint64_t dims[2] = {static_cast<uint64_t>(N), static_cast<uint64_t>(rows)};
   uint64_t strides[1] = {static_cast<uint64_t>(N) * eb};
   uint32_t box[2] = {static_cast<uint32_t>(64 / eb), 32};
-  const CUtensorMapDataType dt = out_kind == kOutFp32   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
-                                 : out_kind == kOutE4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
-                                                        : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUtensorMapDataType dt = out_kind == kOutFp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : q8                 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                                      : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   return make_tmap(m, dt, 2, out, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B, err);
 }
 
@@ -1212,7 +1262,7 @@ cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
                              int out_kind, void* out, float* out_scales,
                              const LaunchCtx& ctx) {
   if (M == 0 || N == 0) return cudaSuccess;
-  if (K == 0 && out_kind == kOutE4M3) return cudaErrorInvalidValue;
+  if (K == 0 && (out_kind == kOutE4M3 || out_kind == kOutMx)) return cudaErrorInvalidValue;
   const int out_f32 = out_kind == kOutFp32;
   if (K == 0) {
     const int64_t total = M * N;

@@ -41,8 +41,10 @@ size_t noalloc_scratch_bytes();
 cudaError_t noalloc_scratch_ptr(int device, void** out);
 
 // Dense scaled GEMM (gemm.cu).  recipe: 0 tensor, 1 row, 2 1x128_128x128,
-// 3 1x128_128x1, 4 MXFP8 (sa, sb then point to E8M0 scale-factor tiles).  out_kind: 0 bf16, 1 fp32, 2 e4m3 quantized in 1x128
-// groups along n with scales written to out_scales[(n/128) * M + m].
+// 3 1x128_128x1, 4 MXFP8 (sa, sb then point to E8M0 scale-factor tiles).
+// out_kind: 0 bf16, 1 fp32, 2 e4m3 quantized in 1x128 groups along n with
+// fp32 scales written to out_scales[(n/128) * M + m], 3 MXFP8 (recipe 4
+// only; E8M0 scale-factor tiles written to out_scales as bytes).
 cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
                              int64_t N, int64_t K, const float* sa,
                              const float* sb, int recipe, const void* bias,

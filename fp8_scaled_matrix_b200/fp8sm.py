@@ -35,7 +35,8 @@ EXPORTED = ["fp8_version", "fp8_last_error", "fp8_quantize_workspace_bytes",
             "fp8_get_device_status", "fp8_debug_timeout_probe",
             "fp8_quantize_noalloc", "fp8_quantize_transposed",
             "fp8_grouped_scaled_mm_blockwise", "fp8_scaled_mm_quantized",
-            "fp8_mx_scale_bytes", "fp8_quantize_mx", "fp8_scaled_mm_mx"]
+            "fp8_mx_scale_bytes", "fp8_quantize_mx", "fp8_scaled_mm_mx",
+            "fp8_scaled_mm_mx_quantized"]
 
 
 class Fp8Error(RuntimeError):
@@ -88,6 +89,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fp8_quantize_mx.argtypes = [P, I64, I64, I64, P, P, P]
     L.fp8_scaled_mm_mx.restype = E
     L.fp8_scaled_mm_mx.argtypes = [P, P, I64, I64, I64, P, P, P, E, P, P]
+    L.fp8_scaled_mm_mx_quantized.restype = E
+    L.fp8_scaled_mm_mx_quantized.argtypes = [P, P, I64, I64, I64, P, P, P, P, P, P]
     L.fp8_scaled_mm_quantized.restype = E
     L.fp8_scaled_mm_quantized.argtypes = [P, P, I64, I64, I64, P, P, E, P, P, P, P]
     L.fp8_grouped_scaled_mm.restype = E
@@ -335,6 +338,38 @@ def fp8_scaled_mm_mx(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor,
     _check(L.fp8_scaled_mm_mx(_ptr(a), _ptr(b), M, N, K, _ptr(scale_a), _ptr(scale_b),
                               _ptr(bias), od, _ptr(out), _stream(stream)))
     return out
+
+
+def fp8_scaled_mm_mx_quantized(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor,
+                               scale_b: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                               out: Optional[torch.Tensor] = None,
+                               out_scales: Optional[torch.Tensor] = None,
+                               stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """MXFP8 GEMM with MXFP8 output: returns (codes (M, N) uint8, E8M0 scale
+    bytes in the scale-factor tile layout) -- the A operand of a next
+    fp8_scaled_mm_mx."""
+    L = load_library()
+    _need_cuda(a, b, scale_a, scale_b, bias)
+    M, K = a.shape
+    N = b.shape[0]
+    if b.shape[1] != K:
+        raise ValueError("a and b must share K")
+    for t in (a, b):
+        if t.dtype not in (torch.uint8, torch.float8_e4m3fn) or not t.is_contiguous():
+            raise ValueError("a and b must be contiguous e4m3 (uint8 codes)")
+    if bias is not None and (bias.dtype != torch.bfloat16 or not bias.is_contiguous()):
+        raise ValueError("bias must be a contiguous bf16 tensor")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.uint8, device=a.device)
+    nbytes = fp8_mx_scale_bytes(M, N)
+    if out_scales is None:
+        out_scales = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=a.device)
+    if out.numel() < M * N or out_scales.numel() < nbytes:
+        raise ValueError("out or out_scales too small")
+    _check(L.fp8_scaled_mm_mx_quantized(_ptr(a), _ptr(b), M, N, K, _ptr(scale_a),
+                                        _ptr(scale_b), _ptr(bias), _ptr(out),
+                                        _ptr(out_scales), _stream(stream)))
+    return out, out_scales[:nbytes] if out_scales.numel() > nbytes else out_scales
 
 
 def fp8_grouped_scaled_mm(a: torch.Tensor, b_experts: torch.Tensor,

@@ -39,6 +39,8 @@ descriptions; no public dataset is involved):
                 (5120, 8192), W2 ~ N(0, 0.02^2) (8192, 5120) as stored
   9 mxfp8       the tensors of workload 2 (same seeds, both (N, K) shapes),
                 quantized MXFP8 (E8M0 scale per 32 elements of K)
+ 10 linear chain, MXFP8  the tensors of workload 8, every operand MXFP8 and
+                the first GEMM writing MXFP8
 """
 from __future__ import annotations
 
@@ -59,6 +61,7 @@ WORKLOAD_NAMES = [
     "grouped_e16_blockwise",
     "linear_chain_1x128_128x128",
     "mxfp8",
+    "linear_chain_mxfp8",
 ]
 
 
@@ -112,7 +115,7 @@ def offsets_from_sizes(sizes) -> torch.Tensor:
 class Workload:
     name: str
     # tensor | row | 1x128_128x128 | 1x128_128x1 | grouped | grouped_blockwise |
-    # grad_input | grad_weight | chain | mxfp8
+    # grad_input | grad_weight | chain | mxfp8 | chain_mx
     recipe: str
     M: int
     N: int
@@ -146,6 +149,10 @@ def make_workload(index: int, shape_index: int = 0, scale_down: int = 1) -> Work
     if index == 7:  # workload 4's tensors, blockwise-scaled
         wl = make_workload(4, shape_index, scale_down)
         wl.name, wl.recipe = name, "grouped_blockwise"
+        return wl
+    if index == 10:  # workload 8's tensors, MXFP8 throughout
+        wl = make_workload(8, shape_index, scale_down)
+        wl.name, wl.recipe = name, "chain_mx"
         return wl
     if index == 9:  # workload 2's tensors, MXFP8
         wl = make_workload(2, shape_index, scale_down)

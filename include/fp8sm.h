@@ -285,6 +285,25 @@ FP8SM_API fp8_status fp8_scaled_mm_mx(const void* a, const void* b, int64_t M, i
                             fp8_out_dtype out_dtype, void* out, fp8_stream_t stream);
 
 /*
+ * MXFP8 GEMM whose output leaves MXFP8-quantized, ready to be the A operand
+ * of the next MXFP8 GEMM (the chained linear of [P1] Solution, forward pass,
+ * with the next layer's activation quantize moved into this GEMM's
+ * epilogue).  With y the fp32 result of fp8_scaled_mm_mx (same operands, bias
+ * and accumulation order), each block of 32 consecutive columns of a row is
+ * quantized exactly as fp8_quantize_mx quantizes a block (e from the fp32
+ * amax of y, codes e4m3_satfinite_rn(y * 2^-e)).
+ *   out_fp8          (M, N) e4m3 codes, 16-byte aligned.
+ *   out_scales_e8m0  fp8_mx_scale_bytes(M, N) bytes in the scale-factor tile
+ *                    layout, 16-byte aligned; padding rows are written zero.
+ * Requirements: K > 0, K % 32 == 0, N % 128 == 0.
+ */
+FP8SM_API fp8_status fp8_scaled_mm_mx_quantized(const void* a, const void* b, int64_t M,
+                                      int64_t N, int64_t K, const void* scale_a_e8m0,
+                                      const void* scale_b_e8m0, const void* bias_bf16,
+                                      void* out_fp8, void* out_scales_e8m0,
+                                      fp8_stream_t stream);
+
+/*
  * Grouped (MoE) scaled GEMM, rowwise recipe only ([P2] Design, RowWise path;
  * other weight granularities return FP8_ERR_UNSUPPORTED as [P2]'s review
  * requires):

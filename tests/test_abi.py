@@ -231,3 +231,25 @@ def test_scaled_mm_mx_null_alignment_dtype_and_empty(lib):
     assert st == fp8sm.FP8_ERR_VALUE and "out_dtype" in lib.fp8_last_error().decode()
     assert lib.fp8_scaled_mm_mx(None, None, 0, 64, 64, None, None, None, fp8sm.FP8_OUT_BF16,
                                 None, None) == fp8sm.FP8_OK
+
+
+@pytest.mark.parametrize("M,N,K,frag", [
+    (128, 192, 64, "N must be a multiple of 128"),
+    (128, 128, 0, "positive multiple of 32"),
+    (128, 128, 80, "positive multiple of 32"),
+    (-2, 128, 64, "negative"),
+])
+def test_scaled_mm_mx_quantized_rejects_bad_arguments(lib, M, N, K, frag):
+    st = lib.fp8_scaled_mm_mx_quantized(FAKE, FAKE, M, N, K, FAKE, FAKE, None, FAKE, FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE and frag in lib.fp8_last_error().decode()
+
+
+def test_scaled_mm_mx_quantized_null_alignment_and_empty(lib):
+    st = lib.fp8_scaled_mm_mx_quantized(FAKE, FAKE, 64, 128, 64, FAKE, FAKE, None, FAKE, None,
+                                        None)
+    assert st == fp8sm.FP8_ERR_VALUE and "null" in lib.fp8_last_error().decode()
+    st = lib.fp8_scaled_mm_mx_quantized(FAKE, FAKE, 64, 128, 64, FAKE, FAKE, None, FAKE,
+                                        P((1 << 20) + 4), None)
+    assert st == fp8sm.FP8_ERR_VALUE and "aligned" in lib.fp8_last_error().decode()
+    assert lib.fp8_scaled_mm_mx_quantized(None, None, 0, 128, 64, None, None, None, None, None,
+                                          None) == fp8sm.FP8_OK

@@ -145,3 +145,108 @@ def test_mx_end_to_end_full_size_sampled(shape_index):
     exact = wl.a.double().numpy()[rows] @ wl.b.double().numpy().T
     err = got - exact
     assert 10 * np.log10((exact ** 2).sum() / (err ** 2).sum()) >= 20.0
+
+
+# ------------------------------------------------ MXFP8 output (next layer's A)
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.ascontiguousarray(codes)).view(torch.float8_e4m3fn).double().numpy()
+
+
+def tile_words(M: int, N: int) -> np.ndarray:
+    """Byte offsets of (row m, 128-column group j)'s 4 scale bytes in the
+    scale-factor tiles of an (M, N) matrix: tile (m / 128, j), byte
+    (m % 32) * 16 + (m % 128 / 32) * 4 + (block % 4)."""
+    m = np.arange(M)[:, None]
+    j = np.arange(N // 128)[None, :]
+    return ((m // 128) * (N // 128) + j) * 512 + (m % 32) * 16 + (m % 128 // 32) * 4
+
+
+def check_mx_output_property(y, q, tiles, what):
+    """q, tiles are the MXFP8 quantization of the fp32 y, restated here:
+    per 32-column block, e = floor(log2(amax)) - 8 clamped to [-127, 127]
+    (from the fp32 bits of amax), codes = RNE e4m3 of y * 2^-e saturated."""
+    M, N = y.shape
+    g = y.astype(np.float32).reshape(M, N // 32, 32)
+    amax = np.abs(g).max(axis=2)
+    be = (amax.view(np.uint32) >> 23).astype(np.int64)
+    e = np.maximum(be - 127 - 8, -127)
+    t = np.clip(g.astype(np.float64) / np.ldexp(1.0, e)[:, :, None], -448, 448)
+    q_want = torch.from_numpy(t.reshape(M, N).astype(np.float32)).to(torch.float8_e4m3fn)
+    q_want = q_want.view(torch.uint8).numpy()
+    bad = np.argwhere(q_want != q)
+    assert bad.size == 0, f"{what}: {len(bad)} codes differ, first {bad[0]}"
+    off = tile_words(M, N)
+    got_e = np.stack([tiles[off + k] for k in range(4)], axis=2).reshape(M, N // 32)
+    bad = np.argwhere(got_e.astype(np.int64) != e + 127)
+    assert bad.size == 0, f"{what}: {len(bad)} scale bytes differ, first {bad[0]}"
+    return e
+
+
+@pytest.mark.parametrize("M,N,K,bias", [(128, 256, 128, False), (130, 384, 96, True),
+                                        (300, 512, 4096, True), (2048, 4096, 256, False),
+                                        (4096, 4096, 256, True)])
+def test_mx_output_parity(M, N, K, bias):
+    seed = M + N * 3 + K * 7
+    qa, ea, qb, eb = mx_operands(M, N, K, seed)
+    g = W.generator(seed + 2)
+    bb = (torch.randn(N, generator=g) * 0.5).to(torch.bfloat16) if bias else None
+    args = (torch.from_numpy(qa).cuda(), torch.from_numpy(qb).cuda(),
+            torch.from_numpy(oracle.mx_scales_to_tiles(ea)).cuda(),
+            torch.from_numpy(oracle.mx_scales_to_tiles(eb)).cuda())
+    bd = None if bb is None else bb.cuda()
+    y = fp8sm.fp8_scaled_mm_mx(*args, bias=bd, out_dtype=torch.float32)
+    q, tiles = fp8sm.fp8_scaled_mm_mx_quantized(*args, bias=bd)
+    torch.cuda.synchronize()
+    fp8sm.check_device_status()
+    y, q, tiles = y.cpu().numpy(), q.cpu().numpy(), tiles.cpu().numpy()
+    e = check_mx_output_property(y, q, tiles, f"mx out {M}x{N}x{K}")
+    # rows past M in the last tile are written as zero
+    if M % 128:
+        pad = tile_words(((M + 127) // 128) * 128, N)[M:]
+        assert not np.stack([tiles[pad + k] for k in range(4)]).any()
+    # against the oracle's fp64 GEMM: GEMM tolerance, plus half an e4m3 step,
+    # plus the saturation of the format (a block maximum lands in
+    # [256, 512) * 2^e, and values past 448 * 2^e are clamped to it)
+    rows = sample_rows(M, 48, seed=seed) if M > 256 else np.arange(M)
+    ref, mag = oracle.mx_scaled_mm(qa, qb, ea, eb,
+                                   bias_bits=None if bb is None else W.bf16_bits(bb), rows=rows)
+    scale = np.ldexp(1.0, e[rows]).repeat(32, axis=1)
+    deq = e4m3_decode(q[rows]) * scale
+    gemm_tol = 1e-2 * np.abs(ref) + 1e-3 * mag
+    clamp = np.maximum(np.abs(ref) + gemm_tol - 448.0 * scale, 0.0)
+    tol = gemm_tol + 2.0 ** -4 * (np.abs(ref) + gemm_tol) + scale * 2.0 ** -10 + clamp
+    bad = np.argwhere(np.abs(deq - ref) > tol)
+    assert bad.size == 0, f"{len(bad)} out of tolerance, first {bad[0]}"
+
+
+def test_mx_linear_chain_against_oracle():
+    """X -> MXFP8 quantize -> GEMM1 with MXFP8 output -> GEMM2 (MXFP8), the
+    16640-token layer pair 8192 -> 5120 -> 8192 (the linear-chain workload's
+    tensors), sampled rows against the oracle's chain (MX quantize, fp64
+    GEMM1 rounded to fp32, MX quantize of it, fp64 GEMM2) and SQNR >= 20 dB
+    against the unquantized product."""
+    wl = W.make_workload(8)
+    f = fp8sm
+    x, w1, w2 = wl.a.cuda(), wl.b.cuda(), wl.extra["b2"].cuda()
+    qx, sx = f.fp8_quantize_mx(x)
+    q1, s1 = f.fp8_quantize_mx(w1)
+    q2, s2 = f.fp8_quantize_mx(w2)
+    y1q, y1s = f.fp8_scaled_mm_mx_quantized(qx, q1, sx, s1)
+    out = f.fp8_scaled_mm_mx(y1q, q2, y1s, s2, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    f.check_device_status()
+    rows = sample_rows(wl.M, 40, seed=8)
+    oqx, oex = oracle.mx_quantize(W.bf16_bits(wl.a))
+    oq1, oe1 = oracle.mx_quantize(W.bf16_bits(wl.b))
+    oq2, oe2 = oracle.mx_quantize(W.bf16_bits(wl.extra["b2"]))
+    y1, _ = oracle.mx_scaled_mm(oqx, oq1, oex, oe1, rows=rows)
+    oy1q, oy1e = oracle.mx_quantize_f32(y1.astype(np.float32))
+    ref, mag = oracle.mx_scaled_mm(oy1q, oq2, oy1e, oe2)
+    got = out.cpu().numpy().astype(np.float64)[rows]
+    ok = oracle.within_tolerance(got, ref, mag)
+    assert ok.all(), f"chain: {int((~ok).sum())} of {ok.size} out of tolerance"
+    exact = (wl.a.double().numpy()[rows] @ wl.b.double().numpy().T) @ \
+        wl.extra["b2"].double().numpy().T
+    err = got - exact
+    assert 10 * np.log10((exact ** 2).sum() / (err ** 2).sum()) >= 20.0
