@@ -55,6 +55,7 @@ WORKLOADS = {
     "mxfp8_16640x5120x8192": (9, 0),
     "mxfp8_16640x8192x5120": (9, 1),
     "linear_chain_mxfp8": (10, 0),
+    "grouped_e16_mxfp8": (11, 0),
 }
 DEFAULT_WORKLOAD = "rowwise_4096"
 # Page 5's context numbers (TFLOP/s of torch._scaled_mm, hardware not stated)
@@ -67,7 +68,7 @@ OPERAND_GROUPS = {"tensor": ("tensor", "tensor"), "row": ("row", "row"),
                   "1x128_128x1": ("1x128", "1x128"), "grouped": ("row", "row"),
                   "grad_input": ("1x128", "128x128"), "grad_weight": ("1x128", "1x128"),
                   "grouped_blockwise": ("1x128", "128x128"), "chain": ("1x128", "128x128"),
-                  "mxfp8": ("mx", "mx"), "chain_mx": ("mx", "mx")}
+                  "mxfp8": ("mx", "mx"), "chain_mx": ("mx", "mx"), "grouped_mx": ("mx", "mx")}
 # GEMM recipe of each workload recipe, and which operands are quantized
 # transposed (the training GEMMs contract along the stored rows)
 GEMM_RECIPE = {"grad_input": "1x128_128x128", "grad_weight": "1x128_128x1",
@@ -210,11 +211,11 @@ class Step:
         self.wl = wl
         self.dev = dev
         ga, gb = OPERAND_GROUPS[wl.recipe]
-        self.mx = wl.recipe in ("mxfp8", "chain_mx")
+        self.mx = wl.recipe in ("mxfp8", "chain_mx", "grouped_mx")
         self.qa_recipe = None if self.mx else fp8sm.QUANT_RECIPES[ga]
         self.qb_recipe = None if self.mx else fp8sm.QUANT_RECIPES[gb]
         self.a = wl.a.to(dev)
-        self.grouped = wl.recipe in ("grouped", "grouped_blockwise")
+        self.grouped = wl.recipe in ("grouped", "grouped_blockwise", "grouped_mx")
         if self.grouped:
             E, N, K = wl.b.shape
             self.b = wl.b.to(dev).reshape(E * N, K)
@@ -328,6 +329,10 @@ class Step:
             E, N, K = wl.b.shape
             f.fp8_grouped_scaled_mm_blockwise(self.qa, self.qb.view(E, N, K), self.sa,
                                               self.sb, self.offs, out=self.out)
+        elif wl.recipe == "grouped_mx":
+            E, N, K = wl.b.shape
+            f.fp8_grouped_scaled_mm_mx(self.qa, self.qb.view(E, N, K), self.sa, self.sb,
+                                       self.offs, out=self.out)
         elif self.mx and self.chain:
             f.fp8_scaled_mm_mx_quantized(self.qa, self.qb, self.sa, self.sb,
                                          out=self.y1q, out_scales=self.y1s)
@@ -440,7 +445,7 @@ def run_e2e(args, wl, dev, world):
     copy of every step is still made and timed."""
     from fp8_scaled_matrix_b200 import fp8sm  # noqa: F401
     ha = wl.a.pin_memory()
-    hb = (wl.b.reshape(-1, wl.K) if wl.recipe in ("grouped", "grouped_blockwise")
+    hb = (wl.b.reshape(-1, wl.K) if wl.recipe in ("grouped", "grouped_blockwise", "grouped_mx")
           else wl.b).contiguous().pin_memory()
     hbias = None if wl.bias is None else wl.bias.pin_memory()
     hb2 = wl.extra["b2"].pin_memory() if "b2" in wl.extra else None
@@ -536,6 +541,22 @@ def oracle_sample(wl, max_rows: int):
         rows = np.arange(min(max_rows, wl.M), dtype=np.int64)
         t0 = time.perf_counter()
         oracle.mx_scaled_mm(qa, qb, sa, sb, rows=rows)
+        return time.perf_counter() - t0, rows.size / wl.M, tq, oracle.num_threads()
+    if wl.recipe == "grouped_mx":
+        E, N, K = wl.b.shape
+        qa, sa = oracle.mx_quantize(W.bf16_bits(wl.a))
+        qb, sb = oracle.mx_quantize(W.bf16_bits(wl.b.reshape(E * N, K)))
+        tq = time.perf_counter() - t0
+        rows = np.arange(min(max_rows, wl.M), dtype=np.int64)
+        t0 = time.perf_counter()
+        start = 0
+        for e, end in enumerate(wl.offs.numpy()):
+            sel = rows[(rows >= start) & (rows < end)]
+            if sel.size:
+                oracle.mx_scaled_mm(np.ascontiguousarray(qa[start:end]), qb[e * N:(e + 1) * N],
+                                    np.ascontiguousarray(sa[start:end]), sb[e * N:(e + 1) * N],
+                                    rows=sel - start)
+            start = int(end)
         return time.perf_counter() - t0, rows.size / wl.M, tq, oracle.num_threads()
     qa, sa = oracle.quantize(bits(wl.a, t_a), G[ga])
     if wl.recipe == "grouped":

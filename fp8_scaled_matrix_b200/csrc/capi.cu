@@ -417,6 +417,8 @@ fp8_status grouped_common(const char* name, int recipe, const void* a, const voi
     return fail(FP8_ERR_VALUE, n + ": K and N must be multiples of 16");
   if (recipe == 2 && K % 128 != 0)
     return fail(FP8_ERR_VALUE, n + ": the blockwise recipe needs K % 128 == 0");
+  if (recipe == 4 && (K == 0 || K % 32 != 0))
+    return fail(FP8_ERR_VALUE, n + ": MXFP8 needs K to be a positive multiple of 32");
   if (M_total == 0 || N == 0) {
     t_last_error.clear();
     return FP8_OK;
@@ -460,6 +462,16 @@ fp8_status fp8_grouped_scaled_mm_blockwise(const void* a, const void* b_experts,
                                            fp8_stream_t stream) {
   return grouped_common("fp8_grouped_scaled_mm_blockwise", 2, a, b_experts, M_total, N, K, E,
                         scale_a, scale_b, offs, out_dtype, out, stream);
+}
+
+fp8_status fp8_grouped_scaled_mm_mx(const void* a, const void* b_experts, int64_t M_total,
+                                    int64_t N, int64_t K, int32_t E,
+                                    const void* scale_a_e8m0, const void* scale_b_e8m0,
+                                    const int32_t* offs, fp8_out_dtype out_dtype, void* out,
+                                    fp8_stream_t stream) {
+  return grouped_common("fp8_grouped_scaled_mm_mx", 4, a, b_experts, M_total, N, K, E,
+                        static_cast<const float*>(scale_a_e8m0),
+                        static_cast<const float*>(scale_b_e8m0), offs, out_dtype, out, stream);
 }
 
 fp8_status fp8_get_device_status(fp8_stream_t stream) {

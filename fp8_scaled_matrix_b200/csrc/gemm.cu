@@ -338,6 +338,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const GemmParams p) {
   constexpr bool kBlockwise = (kRecipe == kBlock128 || kRecipe == kBlock1);
   constexpr bool kIsMx = kRecipe == kMxfp8;
+  // grouped MXFP8: a group's 128-row tile rarely starts on a 128-row
+  // boundary, so warp 2 gathers A's scale words into each stage
+  constexpr bool kMxGather = kIsMx && kGrouped;
   // epilogue threads that hold a whole 128-column row slice in registers
   constexpr bool kBigEpi = kBlockwise || kIsMx;
   constexpr bool kOutF32 = kOut == kOutFp32;
@@ -366,7 +369,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], 1);
+      // grouped MXFP8: each lane of warp 2 also arrives once its copies of
+      // the stage's A scale words have landed
+      mbar_init(&full[s], kMxGather ? 1 + 32 : 1);
       mbar_init(&empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) mbar_init(&acc_full[i], 1);
@@ -473,16 +478,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             // operands plus their scale-factor tiles (tile (i, kb) of a
             // matrix's scales is its 128 rows 128 i .. and K elements
             // 128 kb ..); B's second half-tile exists only below N
+            // (grouped: expert g's tile set follows the g earlier ones; A's
+            // scale tile is gathered by warp 2)
+            const int64_t NB = (p.N + 127) / 128;
             const int64_t nb0 = c.n0 / 128;
-            const bool two = !c.half_n && nb0 + 1 < (p.N + 127) / 128;
+            const bool two = !c.half_n && nb0 + 1 < NB;
             mbar_arrive_expect_tx(&full[stage], C::kAStage + b_bytes +
-                                                    (two ? 3u : 2u) * kMxSfTile);
+                                                    ((two ? 2u : 1u) + (kGrouped ? 0u : 1u)) *
+                                                        kMxSfTile);
             tma_load_2d(a_dst, &tm_a, &full[stage], kb * BK, c.m0);
-            tma_load_2d(b_dst, c.half_n ? &tm_b_half : &tm_b, &full[stage], kb * BK, c.n0);
+            if constexpr (kGrouped)
+              tma_load_3d(b_dst, &tm_b, &full[stage], kb * BK, c.n0, c.g);
+            else
+              tma_load_2d(b_dst, c.half_n ? &tm_b_half : &tm_b, &full[stage], kb * BK, c.n0);
             uint8_t* sf_dst = smem + C::kOffScl + stage * kMxSfStage;
-            const int64_t ka = (static_cast<int64_t>(c.m0 / 128) * KB + kb) * kMxSfTile;
-            const int64_t kbb = (nb0 * KB + kb) * kMxSfTile;
-            bulk_load_g2s(sf_dst, p.sfa + ka, kMxSfTile, &full[stage]);
+            const int64_t kbb =
+                ((kGrouped ? static_cast<int64_t>(c.g) * NB * KB : 0) + nb0 * KB + kb) * kMxSfTile;
+            if constexpr (!kGrouped) {
+              const int64_t ka = (static_cast<int64_t>(c.m0 / 128) * KB + kb) * kMxSfTile;
+              bulk_load_g2s(sf_dst, p.sfa + ka, kMxSfTile, &full[stage]);
+            }
             bulk_load_g2s(sf_dst + kMxSfTile, p.sfb + kbb, kMxSfTile, &full[stage]);
             if (two)
               bulk_load_g2s(sf_dst + 2 * kMxSfTile, p.sfb + kbb + static_cast<int64_t>(KB) * kMxSfTile,
@@ -563,6 +578,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             ready = mbar_test_wait(&full[stage], phase);
             const uint32_t sf_t = tmem_base + BN + cur * kMxSfCols;
             const uint32_t sf_s = smem_u32(smem + C::kOffScl + cur * kMxSfStage);
+            // grouped: warp 2's cp.async wrote A's scale words (generic
+            // proxy); order them before tcgen05.cp reads them (async proxy)
+            if constexpr (kMxGather) fence_proxy_async_smem();
             tmem_cp_32x128b_warpx4(sf_t, smem_desc_rows16(sf_s));
             tmem_cp_32x128b_warpx4(sf_t + 4, smem_desc_rows16(sf_s + kMxSfTile));
             if (!hn) tmem_cp_32x128b_warpx4(sf_t + 8, smem_desc_rows16(sf_s + 2 * kMxSfTile));
@@ -721,6 +739,47 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (++slot == kSclSlots) {
             slot = 0;
             sphase ^= 1u;
+          }
+        }
+      }
+      cp_async_wait_all();  // nothing lands in shared memory after the CTA exits
+    } else if constexpr (kMxGather) {
+      // ------------------------------------- grouped MXFP8: A scale gather
+      // For each stage, in the producer's order: the tile's 128 rows' four
+      // scale bytes of this K tile (one word per row, read from A's
+      // scale-factor tiles at the row's own position) are copied into the
+      // stage's A slot at row r's position ((r % 32) * 16 + (r / 32) * 4) by
+      // 4-byte cp.async (zero fill past the matrix); each lane's copies then
+      // arrive on the stage's full barrier when they land
+      // (cp.async.mbarrier.arrive.noinc), so the warp never waits for them.
+      // The MMA thread fences them into the async proxy before tcgen05.cp.
+      GroupCursor cur;
+      cur.init(p.offs, kTM);
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
+        const TileCoord c = tile_coord<kGrouped, kTM>(t, p, cur);
+        for (int32_t kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, SITE_SCALE_EMPTY,
+                         kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          uint8_t* slot = smem + C::kOffScl + stage * kMxSfStage;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t r = lane + 32u * j;
+            const int64_t row = static_cast<int64_t>(c.m0) + r;
+            const int64_t r7 = row & 127;
+            const uint8_t* src =
+                row < p.M ? p.sfa + ((row >> 7) * KB + kb) * kMxSfTile + (r7 & 31) * 16 + (r7 >> 5) * 4
+                          : p.sfa;
+            cp_async_4(slot + (r & 31u) * 16 + (r >> 5) * 4, src, row < p.M ? 4u : 0u);
+          }
+          cp_async_mbar_arrive_noinc(&full[stage]);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
           }
         }
       }
@@ -1144,8 +1203,9 @@ cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb,
   constexpr bool kBigEpi = kBlockwise || kRecipe == kMxfp8;
   if constexpr (kPair && kBlockwise) {
     return cudaErrorInvalidValue;  // CTA pairs serve the dense recipes only
-  } else if constexpr (kRecipe == kMxfp8 && (kPair || kGrouped || kOut == kOutE4M3)) {
-    return cudaErrorInvalidValue;  // MXFP8: single-CTA dense GEMM, bf16/fp32/MXFP8 out
+  } else if constexpr (kRecipe == kMxfp8 &&
+                       (kPair || kOut == kOutE4M3 || (kGrouped && kOut == kOutMx))) {
+    return cudaErrorInvalidValue;  // MXFP8: single CTAs; bf16/fp32 out (dense: also MXFP8)
   } else if constexpr (kOut == kOutMx && kRecipe != kMxfp8) {
     return cudaErrorInvalidValue;  // MXFP8 output from the MXFP8 GEMM only
   } else if constexpr (kOut == kOutE4M3 && (kPair || kGrouped)) {
@@ -1205,6 +1265,7 @@ cudaError_t dispatch(int recipe, int out_kind, bool pair, const CUtensorMap& ta,
   if constexpr (kGrouped) {
     FP8SM_CASE(kRow)
     FP8SM_CASE(kBlock128)
+    FP8SM_CASE(kMxfp8)
   } else {
     FP8SM_CASE(kTensor)
     FP8SM_CASE(kRow)
@@ -1365,8 +1426,13 @@ cudaError_t launch_grouped_scaled_mm(const void* a, const void* b,
   p.M = M_total;
   p.N = N;
   p.K = K;
-  p.sa = sa;
-  p.sb = sb;
+  if (recipe == kMxfp8) {
+    p.sfa = reinterpret_cast<const uint8_t*>(sa);
+    p.sfb = reinterpret_cast<const uint8_t*>(sb);
+  } else {
+    p.sa = sa;
+    p.sb = sb;
+  }
   p.bias = nullptr;
   p.out = out;
   p.offs = offs;

@@ -36,7 +36,7 @@ EXPORTED = ["fp8_version", "fp8_last_error", "fp8_quantize_workspace_bytes",
             "fp8_quantize_noalloc", "fp8_quantize_transposed",
             "fp8_grouped_scaled_mm_blockwise", "fp8_scaled_mm_quantized",
             "fp8_mx_scale_bytes", "fp8_quantize_mx", "fp8_scaled_mm_mx",
-            "fp8_scaled_mm_mx_quantized"]
+            "fp8_scaled_mm_mx_quantized", "fp8_grouped_scaled_mm_mx"]
 
 
 class Fp8Error(RuntimeError):
@@ -95,6 +95,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fp8_scaled_mm_quantized.argtypes = [P, P, I64, I64, I64, P, P, E, P, P, P, P]
     L.fp8_grouped_scaled_mm.restype = E
     L.fp8_grouped_scaled_mm.argtypes = [P, P, I64, I64, I64, I32, P, P, P, E, P, P]
+    L.fp8_grouped_scaled_mm_mx.restype = E
+    L.fp8_grouped_scaled_mm_mx.argtypes = [P, P, I64, I64, I64, I32, P, P, P, E, P, P]
     L.fp8_grouped_scaled_mm_blockwise.restype = E
     L.fp8_grouped_scaled_mm_blockwise.argtypes = [P, P, I64, I64, I64, I32, P, P, P, E, P, P]
     L.fp8_get_device_status.restype = E
@@ -430,3 +432,29 @@ def check_device_status(stream=None):
 
 def fp8_debug_timeout_probe(limit_us: int, stream=None):
     _check(load_library().fp8_debug_timeout_probe(limit_us, _stream(stream)))
+
+
+def fp8_grouped_scaled_mm_mx(a: torch.Tensor, b_experts: torch.Tensor,
+                             scale_a: torch.Tensor, scale_b: torch.Tensor,
+                             offs: torch.Tensor, out_dtype=torch.bfloat16,
+                             out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Grouped MXFP8 GEMM: rows [offs[g-1], offs[g]) of a times expert g;
+    scale_a A's scale-factor tiles, scale_b the experts' tile sets in order."""
+    L = load_library()
+    _need_cuda(a, b_experts, scale_a, scale_b, offs)
+    if offs.dtype != torch.int32:
+        raise ValueError("offs must be int32")
+    M, K = a.shape
+    E, N, K2 = b_experts.shape
+    if K2 != K or offs.numel() != E:
+        raise ValueError("shape mismatch")
+    if (scale_a.numel() < fp8_mx_scale_bytes(M, K) or
+            scale_b.numel() < E * fp8_mx_scale_bytes(N, K)):
+        raise ValueError("scale tiles too small")
+    od = FP8_OUT_F32 if out_dtype == torch.float32 else FP8_OUT_BF16
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=a.device)
+    _check(L.fp8_grouped_scaled_mm_mx(_ptr(a), _ptr(b_experts), M, N, K, E, _ptr(scale_a),
+                                      _ptr(scale_b), _ptr(offs), od, _ptr(out),
+                                      _stream(stream)))
+    return out

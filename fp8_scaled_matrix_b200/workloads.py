@@ -41,6 +41,7 @@ descriptions; no public dataset is involved):
                 quantized MXFP8 (E8M0 scale per 32 elements of K)
  10 linear chain, MXFP8  the tensors of workload 8, every operand MXFP8 and
                 the first GEMM writing MXFP8
+ 11 grouped MXFP8  the tensors of workload 4 (same seed), MXFP8 throughout
 """
 from __future__ import annotations
 
@@ -62,6 +63,7 @@ WORKLOAD_NAMES = [
     "linear_chain_1x128_128x128",
     "mxfp8",
     "linear_chain_mxfp8",
+    "grouped_e16_mxfp8",
 ]
 
 
@@ -115,7 +117,7 @@ def offsets_from_sizes(sizes) -> torch.Tensor:
 class Workload:
     name: str
     # tensor | row | 1x128_128x128 | 1x128_128x1 | grouped | grouped_blockwise |
-    # grad_input | grad_weight | chain | mxfp8 | chain_mx
+    # grad_input | grad_weight | chain | mxfp8 | chain_mx | grouped_mx
     recipe: str
     M: int
     N: int
@@ -149,6 +151,10 @@ def make_workload(index: int, shape_index: int = 0, scale_down: int = 1) -> Work
     if index == 7:  # workload 4's tensors, blockwise-scaled
         wl = make_workload(4, shape_index, scale_down)
         wl.name, wl.recipe = name, "grouped_blockwise"
+        return wl
+    if index == 11:  # workload 4's tensors, MXFP8
+        wl = make_workload(4, shape_index, scale_down)
+        wl.name, wl.recipe = name, "grouped_mx"
         return wl
     if index == 10:  # workload 8's tensors, MXFP8 throughout
         wl = make_workload(8, shape_index, scale_down)

@@ -354,6 +354,25 @@ FP8SM_API fp8_status fp8_grouped_scaled_mm_blockwise(const void* a, const void* 
                                                      fp8_stream_t stream);
 
 /*
+ * Grouped (MoE) MXFP8 GEMM: for g in 0..E-1, rows m in [offs[g-1], offs[g]):
+ *   out[m, n] = sum_k (a[m,k] 2^(sa[m, k/32] - 127)) (b_experts[g,n,k] 2^(sb_g[n, k/32] - 127))
+ * (the MoE form of [P2] with the MXFP8 recipe of fp8_scaled_mm_mx).
+ *   scale_a_e8m0  A's scale-factor tiles, fp8_mx_scale_bytes(M_total, K)
+ *                 bytes (fp8_quantize_mx of a); groups may start anywhere.
+ *   scale_b_e8m0  E consecutive per-expert tile sets of fp8_mx_scale_bytes(N, K)
+ *                 bytes each (fp8_quantize_mx of each expert's (N, K) weight;
+ *                 when N % 128 == 0, also one fp8_quantize_mx of the (E*N, K)
+ *                 view).
+ *   offs, out, out_dtype as fp8_grouped_scaled_mm.
+ * Requirements: K > 0, K % 32 == 0, N % 16 == 0, 1 <= E <= 65535.
+ */
+FP8SM_API fp8_status fp8_grouped_scaled_mm_mx(const void* a, const void* b_experts,
+                                    int64_t M_total, int64_t N, int64_t K, int32_t E,
+                                    const void* scale_a_e8m0, const void* scale_b_e8m0,
+                                    const int32_t* offs, fp8_out_dtype out_dtype, void* out,
+                                    fp8_stream_t stream);
+
+/*
  * Synchronizes `stream`, then returns and clears the current device's status
  * word: FP8_OK, FP8_ERR_VALUE (malformed offs), FP8_ERR_TIMEOUT (a pipeline
  * wait gave up; the kernel released its resources and returned), or

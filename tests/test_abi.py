@@ -253,3 +253,15 @@ def test_scaled_mm_mx_quantized_null_alignment_and_empty(lib):
     assert st == fp8sm.FP8_ERR_VALUE and "aligned" in lib.fp8_last_error().decode()
     assert lib.fp8_scaled_mm_mx_quantized(None, None, 0, 128, 64, None, None, None, None, None,
                                           None) == fp8sm.FP8_OK
+
+
+@pytest.mark.parametrize("M,N,K,E,frag", [
+    (64, 128, 48, 2, "MXFP8 needs K"),
+    (64, 128, 0, 2, "MXFP8 needs K"),
+    (64, 120, 64, 2, "multiples of 16"),
+    (64, 128, 64, 0, "expert count"),
+])
+def test_grouped_mx_rejects_bad_arguments(lib, M, N, K, E, frag):
+    st = lib.fp8_grouped_scaled_mm_mx(FAKE, FAKE, M, N, K, E, FAKE, FAKE, FAKE,
+                                      fp8sm.FP8_OUT_BF16, FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE and frag in lib.fp8_last_error().decode()
