@@ -56,6 +56,7 @@ WORKLOADS = {
     "mxfp8_16640x8192x5120": (9, 1),
     "linear_chain_mxfp8": (10, 0),
     "grouped_e16_mxfp8": (11, 0),
+    "grouped_e16_grad_input": (12, 0),
 }
 DEFAULT_WORKLOAD = "rowwise_4096"
 # Page 5's context numbers (TFLOP/s of torch._scaled_mm, hardware not stated)
@@ -68,7 +69,8 @@ OPERAND_GROUPS = {"tensor": ("tensor", "tensor"), "row": ("row", "row"),
                   "1x128_128x1": ("1x128", "1x128"), "grouped": ("row", "row"),
                   "grad_input": ("1x128", "128x128"), "grad_weight": ("1x128", "1x128"),
                   "grouped_blockwise": ("1x128", "128x128"), "chain": ("1x128", "128x128"),
-                  "mxfp8": ("mx", "mx"), "chain_mx": ("mx", "mx"), "grouped_mx": ("mx", "mx")}
+                  "mxfp8": ("mx", "mx"), "chain_mx": ("mx", "mx"), "grouped_mx": ("mx", "mx"),
+                  "grouped_grad_input": ("1x128", "128x128")}
 # GEMM recipe of each workload recipe, and which operands are quantized
 # transposed (the training GEMMs contract along the stored rows)
 GEMM_RECIPE = {"grad_input": "1x128_128x128", "grad_weight": "1x128_128x1",
@@ -215,8 +217,14 @@ class Step:
         self.qa_recipe = None if self.mx else fp8sm.QUANT_RECIPES[ga]
         self.qb_recipe = None if self.mx else fp8sm.QUANT_RECIPES[gb]
         self.a = wl.a.to(dev)
-        self.grouped = wl.recipe in ("grouped", "grouped_blockwise", "grouped_mx")
-        if self.grouped:
+        self.grouped = wl.recipe in ("grouped", "grouped_blockwise", "grouped_mx",
+                                     "grouped_grad_input")
+        self.gin = wl.recipe == "grouped_grad_input"
+        if self.gin:
+            # the experts as stored (E, out, in); each is quantized transposed
+            self.b = wl.b.to(dev)
+            self.offs = wl.offs.to(dev)
+        elif self.grouped:
             E, N, K = wl.b.shape
             self.b = wl.b.to(dev).reshape(E * N, K)
             self.offs = wl.offs.to(dev)
@@ -227,6 +235,8 @@ class Step:
         self.t_a, self.t_b = TRANSPOSED.get(wl.recipe, (False, False))
         # quantized operands: A (M, K), B (N, K) (grouped: (E N, K))
         rows_a, rows_b = wl.M, self.b.shape[1] if self.t_b else self.b.shape[0]
+        if self.gin:
+            rows_b = wl.b.shape[0] * wl.N    # (E * in, out) codes
         cols = wl.K
         self.qa = torch.empty(rows_a, cols, dtype=torch.uint8, device=dev)
         self.qb = torch.empty(rows_b, cols, dtype=torch.uint8, device=dev)
@@ -253,6 +263,12 @@ class Step:
             # tiles and scales), into the (E, K/128, N/128) scale layout
             E, N, K = wl.b.shape
             self.sb = torch.empty(E * fp8sm.scale_count(N, K, self.qb_recipe),
+                                  dtype=torch.float32, device=dev)
+            self.launches_per_step = 2 + E
+        if self.gin:
+            # per expert W_g^T quantized 128x128: (out/128, in/128) scales each
+            E = wl.b.shape[0]
+            self.sb = torch.empty(E * fp8sm.scale_count(wl.N, wl.K, self.qb_recipe),
                                   dtype=torch.float32, device=dev)
             self.launches_per_step = 2 + E
         self.chain = wl.recipe in ("chain", "chain_mx")
@@ -285,7 +301,15 @@ class Step:
         self.ev_fork.record(main)
         self.side.wait_event(self.ev_fork)
         with torch.cuda.stream(self.side):
-            if self.wl.recipe == "grouped_blockwise":
+            if self.gin:
+                E, Kin = self.wl.b.shape[0], self.wl.N
+                per = self.sb.numel() // E
+                for e in range(E):
+                    f.fp8_quantize_transposed(self.b[e], self.qb_recipe,
+                                              out=self.qb[e * Kin:(e + 1) * Kin],
+                                              scales=self.sb[e * per:(e + 1) * per],
+                                              stream=self.side)
+            elif self.wl.recipe == "grouped_blockwise":
                 E, N, K = self.wl.b.shape
                 per = self.sb.numel() // E
                 for e in range(E):
@@ -328,6 +352,10 @@ class Step:
         elif wl.recipe == "grouped_blockwise":
             E, N, K = wl.b.shape
             f.fp8_grouped_scaled_mm_blockwise(self.qa, self.qb.view(E, N, K), self.sa,
+                                              self.sb, self.offs, out=self.out)
+        elif self.gin:
+            E = wl.b.shape[0]
+            f.fp8_grouped_scaled_mm_blockwise(self.qa, self.qb.view(E, wl.N, wl.K), self.sa,
                                               self.sb, self.offs, out=self.out)
         elif wl.recipe == "grouped_mx":
             E, N, K = wl.b.shape
@@ -446,7 +474,7 @@ def run_e2e(args, wl, dev, world):
     from fp8_scaled_matrix_b200 import fp8sm  # noqa: F401
     ha = wl.a.pin_memory()
     hb = (wl.b.reshape(-1, wl.K) if wl.recipe in ("grouped", "grouped_blockwise", "grouped_mx")
-          else wl.b).contiguous().pin_memory()
+          else wl.b).contiguous().pin_memory()     # grouped_grad_input: (E, out, in) as stored
     hbias = None if wl.bias is None else wl.bias.pin_memory()
     hb2 = wl.extra["b2"].pin_memory() if "b2" in wl.extra else None
     sets = [Step(wl, dev), Step(wl, dev)]
@@ -541,6 +569,23 @@ def oracle_sample(wl, max_rows: int):
         rows = np.arange(min(max_rows, wl.M), dtype=np.int64)
         t0 = time.perf_counter()
         oracle.mx_scaled_mm(qa, qb, sa, sb, rows=rows)
+        return time.perf_counter() - t0, rows.size / wl.M, tq, oracle.num_threads()
+    if wl.recipe == "grouped_grad_input":
+        qa, sa = oracle.quantize(W.bf16_bits(wl.a), G["1x128"])
+        per_expert = [oracle.quantize(np.ascontiguousarray(W.bf16_bits(wl.b[e]).T), G["128x128"])
+                      for e in range(wl.b.shape[0])]
+        tq = time.perf_counter() - t0
+        rows = np.arange(min(max_rows, wl.M), dtype=np.int64)
+        t0 = time.perf_counter()
+        sa2 = sa.reshape(wl.K // 128, wl.M)
+        start = 0
+        for e, end in enumerate(wl.offs.numpy()):
+            sel = rows[(rows >= start) & (rows < end)]
+            if sel.size:
+                oracle.scaled_mm(np.ascontiguousarray(qa[start:end]), per_expert[e][0],
+                                 np.ascontiguousarray(sa2[:, start:end]).reshape(-1),
+                                 per_expert[e][1], MMR["1x128_128x128"], rows=sel - start)
+            start = int(end)
         return time.perf_counter() - t0, rows.size / wl.M, tq, oracle.num_threads()
     if wl.recipe == "grouped_mx":
         E, N, K = wl.b.shape

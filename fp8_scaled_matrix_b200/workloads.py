@@ -42,6 +42,11 @@ descriptions; no public dataset is involved):
  10 linear chain, MXFP8  the tensors of workload 8, every operand MXFP8 and
                 the first GEMM writing MXFP8
  11 grouped MXFP8  the tensors of workload 4 (same seed), MXFP8 throughout
+ 12 grouped grad_input  the MoE layer's backward dX_g = dY_g @ W_g with the
+                1x128_128x128 recipe: dY ~ N(0,1) (32768, 4096) (drawn as
+                workload 4's activations, same seed and group split), W =
+                workload 4's experts (16, 4096 out, 4096 in); GEMM M=32768,
+                N=4096 (in), K=4096 (out)
 """
 from __future__ import annotations
 
@@ -64,6 +69,7 @@ WORKLOAD_NAMES = [
     "mxfp8",
     "linear_chain_mxfp8",
     "grouped_e16_mxfp8",
+    "grouped_e16_grad_input",
 ]
 
 
@@ -117,7 +123,8 @@ def offsets_from_sizes(sizes) -> torch.Tensor:
 class Workload:
     name: str
     # tensor | row | 1x128_128x128 | 1x128_128x1 | grouped | grouped_blockwise |
-    # grad_input | grad_weight | chain | mxfp8 | chain_mx | grouped_mx
+    # grad_input | grad_weight | chain | mxfp8 | chain_mx | grouped_mx |
+    # grouped_grad_input
     recipe: str
     M: int
     N: int
@@ -125,7 +132,8 @@ class Workload:
     # GEMM sizes M, N, K; the bf16 operands as a caller holds them (CPU):
     #   a  (M, K); grad_weight: (K, M) (grad_output, tokens x out)
     #   b  (N, K) or (E, N, K); grad_input: (K, N) (the weight as stored);
-    #      grad_weight: (K, N) (the layer input, tokens x in)
+    #      grad_weight: (K, N) (the layer input, tokens x in);
+    #      grouped_grad_input: (E, K, N) (the experts as stored, out x in)
     a: torch.Tensor
     b: torch.Tensor
     bias: Optional[torch.Tensor] = None   # bf16 (N,) CPU
@@ -151,6 +159,12 @@ def make_workload(index: int, shape_index: int = 0, scale_down: int = 1) -> Work
     if index == 7:  # workload 4's tensors, blockwise-scaled
         wl = make_workload(4, shape_index, scale_down)
         wl.name, wl.recipe = name, "grouped_blockwise"
+        return wl
+    if index == 12:  # workload 4's tensors as (dY, W) of the backward
+        wl = make_workload(4, shape_index, scale_down)
+        E, Nout, Kin = wl.b.shape
+        wl.name, wl.recipe = name, "grouped_grad_input"
+        wl.N, wl.K = Kin, Nout
         return wl
     if index == 11:  # workload 4's tensors, MXFP8
         wl = make_workload(4, shape_index, scale_down)
