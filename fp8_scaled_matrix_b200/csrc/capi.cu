@@ -474,6 +474,79 @@ fp8_status fp8_grouped_scaled_mm_mx(const void* a, const void* b_experts, int64_
                         static_cast<const float*>(scale_b_e8m0), offs, out_dtype, out, stream);
 }
 
+int64_t fp8_grouped_padded_tokens(int64_t tokens, int32_t E) {
+  if (tokens < 0 || E < 1) return 0;
+  return fp8sm::grouped_padded_tokens(tokens, E);
+}
+
+fp8_status fp8_quantize_transposed_grouped(const void* x_bf16, int64_t tokens, int64_t cols,
+                                           int64_t ld_x, const int32_t* offs, int32_t E,
+                                           void* out_fp8, float* out_scales,
+                                           fp8_stream_t stream) {
+  const char* n = "fp8_quantize_transposed_grouped";
+  if (tokens < 0 || cols < 0) return fail(FP8_ERR_VALUE, std::string(n) + ": negative size");
+  if (tokens >= (int64_t(1) << 31) || cols >= (int64_t(1) << 31))
+    return fail(FP8_ERR_VALUE, std::string(n) + ": size too large");
+  if (E < 1 || E > 2048)
+    return fail(FP8_ERR_VALUE, std::string(n) + ": expert count must be in [1, 2048]");
+  if (cols % 8 != 0 || ld_x % 8 != 0 || ld_x < cols)
+    return fail(FP8_ERR_VALUE,
+                std::string(n) + ": cols and ld_x must be multiples of 8, ld_x >= cols");
+  if (offs == nullptr) return fail(FP8_ERR_VALUE, std::string(n) + ": offs is required");
+  if (tokens == 0 || cols == 0) {
+    t_last_error.clear();
+    return FP8_OK;
+  }
+  if (x_bf16 == nullptr || out_fp8 == nullptr || out_scales == nullptr)
+    return fail(FP8_ERR_VALUE, std::string(n) + ": null pointer");
+  if (!aligned(x_bf16, 16) || !aligned(out_fp8, 16) || !aligned(out_scales, 4) ||
+      !aligned(offs, 4))
+    return fail(FP8_ERR_VALUE, std::string(n) + ": misaligned pointer");
+  DeviceInfo* d = nullptr;
+  fp8_status s = device_info(&d);
+  if (s != FP8_OK) return s;
+  std::string err;
+  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status, d->num_sms, &err};
+  cudaError_t e = fp8sm::launch_quantize_transposed_grouped(x_bf16, tokens, cols, ld_x, offs, E,
+                                                            out_fp8, out_scales, ctx);
+  return finish_launch(e, err, n);
+}
+
+fp8_status fp8_grouped_scaled_mm_wgrad(const void* a_t, const void* b_t, int64_t M, int64_t N,
+                                       int64_t tokens, int32_t E, const float* scale_a,
+                                       const float* scale_b, const int32_t* offs,
+                                       fp8_out_dtype out_dtype, void* out, fp8_stream_t stream) {
+  const std::string n("fp8_grouped_scaled_mm_wgrad");
+  if (out_dtype != FP8_OUT_BF16 && out_dtype != FP8_OUT_F32)
+    return fail(FP8_ERR_VALUE, n + ": unknown out_dtype");
+  if (offs == nullptr) return fail(FP8_ERR_VALUE, n + ": offs is required");
+  if (M < 0 || N < 0 || tokens < 0 || E < 1 || E > 65535)
+    return fail(FP8_ERR_VALUE, n + ": bad size or expert count");
+  if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || tokens >= (int64_t(1) << 31))
+    return fail(FP8_ERR_VALUE, n + ": size too large");
+  if (M % 128 != 0) return fail(FP8_ERR_VALUE, n + ": M must be a multiple of 128");
+  if (N % 16 != 0) return fail(FP8_ERR_VALUE, n + ": N must be a multiple of 16");
+  if (M == 0 || N == 0) {
+    t_last_error.clear();
+    return FP8_OK;
+  }
+  if (a_t == nullptr || b_t == nullptr || scale_a == nullptr || scale_b == nullptr ||
+      out == nullptr)
+    return fail(FP8_ERR_VALUE, n + ": null pointer");
+  if (!aligned(a_t, 16) || !aligned(b_t, 16) || !aligned(scale_a, 16) || !aligned(scale_b, 16) ||
+      !aligned(out, 16) || !aligned(offs, 4))
+    return fail(FP8_ERR_VALUE, n + ": pointers must be 16-byte aligned");
+  DeviceInfo* d = nullptr;
+  fp8_status s = device_info(&d);
+  if (s != FP8_OK) return s;
+  std::string err;
+  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status, d->num_sms, &err};
+  const int64_t P = fp8sm::grouped_padded_tokens(tokens, E);
+  cudaError_t e = fp8sm::launch_grouped_wgrad(a_t, b_t, M, N, P, tokens, E, scale_a, scale_b,
+                                              offs, out_dtype == FP8_OUT_F32, out, ctx);
+  return finish_launch(e, err, n.c_str());
+}
+
 fp8_status fp8_get_device_status(fp8_stream_t stream) {
   DeviceInfo* d = nullptr;
   fp8_status s = device_info(&d);

@@ -131,6 +131,7 @@ struct GemmParams {
   float* out_scales;  // e4m3 output: scale[(n/128) * M + m]; MXFP8 output: tiles
   const int32_t* offs;
   int32_t E;
+  int64_t tokens;    // K-grouped (weight gradient): offs[E-1] must equal this
   int32_t n_tiles;   // tiles along N
   int32_t m_tiles;   // tiles along M (dense)
   int32_t k_blocks;
@@ -172,6 +173,33 @@ struct TileCoord {
   int32_t m0, n0, g;
   int64_t row_end;
   bool half_n;  // 128-wide item (columns n0 .. n0+127 only)
+  int32_t out_m0;  // first output row (differs from m0 for the K-grouped GEMM)
+  int64_t kb0;     // K-grouped: first (padded) K block of the item's group
+  int32_t nkb;     // K-grouped: K blocks of the group
+};
+
+// K-grouped GEMM (per-expert weight gradient): walks the groups' padded K
+// block ranges in increasing group order.
+struct KGroupCursor {
+  int32_t g;
+  int64_t kb0;  // padded 128-blocks of groups < g
+  int32_t nkb;  // padded 128-blocks of group g
+  __device__ static int32_t blocks(const int32_t* offs, int32_t g) {
+    const int32_t prev = g ? offs[g - 1] : 0;
+    return (offs[g] - prev + BK - 1) / BK;
+  }
+  __device__ void init(const int32_t* offs) {
+    g = 0;
+    kb0 = 0;
+    nkb = blocks(offs, 0);
+  }
+  __device__ void seek(int32_t target, const int32_t* offs) {
+    while (g < target) {
+      kb0 += nkb;
+      ++g;
+      nkb = blocks(offs, g);
+    }
+  }
 };
 
 // Work item t -> output tile (rows m0 .. m0 + kTM - 1).
@@ -189,6 +217,8 @@ __device__ __forceinline__ TileCoord tile_coord(int64_t t, const GemmParams& p,
       c.half_n = true;
     }
   }
+  c.kb0 = 0;
+  c.nkb = 0;
   const int64_t mt = t / p.n_tiles;
   c.n0 = static_cast<int32_t>((t % p.n_tiles) * BN) + sub * (BN / 2);
   if constexpr (kGrouped) {
@@ -201,6 +231,27 @@ __device__ __forceinline__ TileCoord tile_coord(int64_t t, const GemmParams& p,
     c.m0 = static_cast<int32_t>(mt * kTM);
     c.row_end = p.M;
   }
+  c.out_m0 = c.m0;
+  return c;
+}
+
+// K-grouped work item t -> (group g, A rows m0.., B rows n0..) with the
+// group's K blocks; output rows g * M + m0 ...
+__device__ __forceinline__ TileCoord kgroup_coord(int64_t t, const GemmParams& p,
+                                                  KGroupCursor& kc) {
+  TileCoord c;
+  c.half_n = false;
+  const int64_t per_group = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
+  const int32_t g = static_cast<int32_t>(t / per_group);
+  const int64_t r = t % per_group;
+  kc.seek(g, p.offs);
+  c.g = g;
+  c.m0 = static_cast<int32_t>((r / p.n_tiles) * BM);
+  c.n0 = static_cast<int32_t>((r % p.n_tiles) * BN);
+  c.out_m0 = static_cast<int32_t>(static_cast<int64_t>(g) * p.M + c.m0);
+  c.row_end = static_cast<int64_t>(g + 1) * p.M;
+  c.kb0 = kc.kb0;
+  c.nkb = kc.nkb;
   return c;
 }
 
@@ -341,6 +392,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // grouped MXFP8: a group's 128-row tile rarely starts on a 128-row
   // boundary, so warp 2 gathers A's scale words into each stage
   constexpr bool kMxGather = kIsMx && kGrouped;
+  // grouped 1x128_128x1 = the per-expert weight gradient: groups split K
+  // (tokens), every group has its own (M, N) output
+  constexpr bool kKGroups = kGrouped && kRecipe == kBlock1;
   // epilogue threads that hold a whole 128-column row slice in registers
   constexpr bool kBigEpi = kBlockwise || kIsMx;
   constexpr bool kOutF32 = kOut == kOutFp32;
@@ -413,12 +467,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (e < prev || prev < 0) bad = true;
         else mt += (static_cast<int64_t>(e) - prev + C::kTileM - 1) / C::kTileM;
       }
-      if (lane == 0 && static_cast<int64_t>(p.offs[p.E - 1]) != p.M) bad = true;
+      if (lane == 0 && static_cast<int64_t>(p.offs[p.E - 1]) != (kKGroups ? p.tokens : p.M))
+        bad = true;
+      int64_t kblocks = 0;  // K-grouped: the groups' padded K blocks must fit in K
+      if constexpr (kKGroups) {
+        for (int32_t i = static_cast<int32_t>(lane); i < p.E; i += 32) {
+          const int32_t prev = i ? p.offs[i - 1] : 0;
+          kblocks += (static_cast<int64_t>(p.offs[i]) - prev + BK - 1) / BK;
+        }
+      }
       bad = __any_sync(0xFFFFFFFFu, bad);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1)
+      for (int o = 16; o > 0; o >>= 1) {
         mt += __shfl_xor_sync(0xFFFFFFFFu, mt, o);
-      total = bad ? 0 : mt * p.n_tiles;
+        kblocks += __shfl_xor_sync(0xFFFFFFFFu, kblocks, o);
+      }
+      if constexpr (kKGroups) {
+        if (kblocks > p.k_blocks) bad = true;
+        total = bad ? 0 : static_cast<int64_t>(p.E) * p.m_tiles * p.n_tiles;
+      } else {
+        total = bad ? 0 : mt * p.n_tiles;
+      }
       if (bad && lane == 0 && blockIdx.x == 0)
         record_status(p.status, FP8_DEV_VALUE, SITE_OFFS);
     } else {
@@ -446,13 +515,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
       GroupCursor cur;
-      if constexpr (kGrouped) cur.init(p.offs, kTM);
+      KGroupCursor kc;
+      if constexpr (kKGroups) kc.init(p.offs);
+      else if constexpr (kGrouped) cur.init(p.offs, kTM);
       uint32_t stage = 0, phase = 0;
       uint64_t issued = 0;
       bool ok = true;
       for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
-        const TileCoord c = tile_coord<kGrouped, kTM>(t, p, cur);
-        for (int32_t kb = 0; kb < KB; ++kb) {
+        const TileCoord c =
+            kKGroups ? kgroup_coord(t, p, kc) : tile_coord<kGrouped, kTM>(t, p, cur);
+        const int32_t nkb = kKGroups ? c.nkb : KB;
+        for (int32_t kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait<kPair>(&empty[stage], phase ^ 1u, abort_flag, p.status,
                          SITE_PRODUCER_EMPTY, kWaitLimitNs)) {
             ok = false;
@@ -502,6 +575,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (two)
               bulk_load_g2s(sf_dst + 2 * kMxSfTile, p.sfb + kbb + static_cast<int64_t>(KB) * kMxSfTile,
                             kMxSfTile, &full[stage]);
+          } else if constexpr (kKGroups) {
+            // the group's padded K range; A and B are (rows, padded tokens)
+            const int32_t kx = static_cast<int32_t>((c.kb0 + kb) * BK);
+            mbar_arrive_expect_tx(&full[stage], C::kAStage + b_bytes);
+            tma_load_2d(a_dst, &tm_a, &full[stage], kx, c.m0);
+            tma_load_2d(b_dst, &tm_b, &full[stage], kx, c.n0);
           } else {
             mbar_arrive_expect_tx(&full[stage], C::kAStage + b_bytes);
             tma_load_2d(a_dst, &tm_a, &full[stage], kb * BK, c.m0);
@@ -648,8 +727,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // into two N = 128 halves with their own hand-back costs twice the
         // MMA instructions and commits, and the single issuing thread, not
         // the tensor core, then sets the pace.)
+        KGroupCursor kc;
+        if constexpr (kKGroups) kc.init(p.offs);
         for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
-          for (int32_t kb = 0; kb < KB; ++kb) {
+          const int32_t nkb = kKGroups ? kgroup_coord(t, p, kc).nkb : KB;
+          for (int32_t kb = 0; kb < nkb; ++kb) {
             if (!mbar_wait<kPair>(&acc_empty[acc], acc_phase ^ 1u, abort_flag, p.status,
                                   SITE_MMA_ACC_EMPTY, kWaitLimitNs)) {
               ok = false;
@@ -701,17 +783,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t slot = 0, sphase = 0;
       bool ok = true;
       GroupCursor cur;
-      if constexpr (kGrouped) cur.init(p.offs, kTM);
+      KGroupCursor kc;
+      if constexpr (kKGroups) kc.init(p.offs);
+      else if constexpr (kGrouped) cur.init(p.offs, kTM);
       for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
-        const TileCoord c = tile_coord<kGrouped, kTM>(t, p, cur);
-        for (int32_t kb = 0; kb < KB; ++kb) {
+        const TileCoord c =
+            kKGroups ? kgroup_coord(t, p, kc) : tile_coord<kGrouped, kTM>(t, p, cur);
+        const int32_t nkb = kKGroups ? c.nkb : KB;
+        for (int32_t kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&sempty[slot], sphase ^ 1u, abort_flag, p.status, SITE_SCALE_EMPTY,
                          kWaitLimitNs)) {
             ok = false;
             break;
           }
           float* dst = scl + slot * kSclSlotFloats;
-          const float* sa_k = p.sa + static_cast<int64_t>(kb) * p.M;
+          // K-grouped: the group's padded K blocks index the scale rows
+          const int64_t kbs = kKGroups ? c.kb0 + kb : kb;
+          const float* sa_k = p.sa + kbs * p.M;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int64_t r = static_cast<int64_t>(c.m0) + lane + 32 * i;
@@ -731,7 +819,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 2; ++i) {
               const int64_t n = static_cast<int64_t>(c.n0) + 8 * lane + 4 * i;
               cp_async_16(dst + 128 + 8 * lane + 4 * i,
-                          n < p.N ? p.sb + static_cast<int64_t>(kb) * p.N + n : p.sb,
+                          n < p.N ? p.sb + kbs * p.N + n : p.sb,
                           n < p.N ? 16u : 0u);
             }
           }
@@ -795,7 +883,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* ebuf = smem + C::kOffEpi + ew * kEpiBuf;
     const uint32_t lane_base = (q * 32u) << 16;
     GroupCursor cur;
-    if constexpr (kGrouped) cur.init(p.offs, kTM);
+    KGroupCursor kc;
+    if constexpr (kKGroups) kc.init(p.offs);
+    else if constexpr (kGrouped) cur.init(p.offs, kTM);
     uint32_t acc = 0, acc_phase = 0;
     uint32_t ep_stage = 0, ep_phase = 0;  // blockwise: mirrors the MMA's stage sequence
     uint32_t sslot = 0, sphase = 0;       // blockwise: scale ring position
@@ -828,12 +918,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       else mbar_arrive(&acc_empty[a]);
     };
     for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
-      const TileCoord c = tile_coord<kGrouped, kTM>(t, p, cur);
-      const int32_t cta_m0 = c.m0 + static_cast<int32_t>(rank) * BM;  // this CTA's rows
+      const TileCoord c =
+          kKGroups ? kgroup_coord(t, p, kc) : tile_coord<kGrouped, kTM>(t, p, cur);
+      // this CTA's output rows (K-grouped: group g's block of the output)
+      const int32_t cta_m0 = c.out_m0 + static_cast<int32_t>(rank) * BM;
       const int64_t row = static_cast<int64_t>(cta_m0) + q * 32 + lane;
       const bool row_ok = row < c.row_end;
       const int64_t ncol0 = static_cast<int64_t>(c.n0) + half * 128;
       const int32_t row0 = cta_m0 + static_cast<int32_t>(q * 32);
+      const int32_t nkb = kKGroups ? c.nkb : KB;
 
       // next accumulator buffer (MXFP8: the one buffer, next phase)
       auto next_acc = [&]() {
@@ -1014,7 +1107,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float2 accr[64];  // accr[16 c + i]: columns 32c + 2i, 32c + 2i + 1 of the warp's 128
 #pragma unroll
         for (int i = 0; i < 64; ++i) accr[i] = make_float2(0.0f, 0.0f);
-        for (int32_t kb = 0; kb < KB && ok; ++kb) {
+        for (int32_t kb = 0; kb < nkb && ok; ++kb) {
           const float* sl = wait_scales();
           if (sl == nullptr) {
             ok = false;
@@ -1265,6 +1358,7 @@ cudaError_t dispatch(int recipe, int out_kind, bool pair, const CUtensorMap& ta,
   if constexpr (kGrouped) {
     FP8SM_CASE(kRow)
     FP8SM_CASE(kBlock128)
+    FP8SM_CASE(kBlock1)  // K-grouped: the per-expert weight gradient
     FP8SM_CASE(kMxfp8)
   } else {
     FP8SM_CASE(kTensor)
@@ -1445,6 +1539,46 @@ cudaError_t launch_grouped_scaled_mm(const void* a, const void* b,
   p.total_items = 0;
   const unsigned grid = static_cast<unsigned>(pair ? (ctx.num_sms / 2) * 2 : ctx.num_sms);
   return dispatch<true>(recipe, out_f32, pair, ta, tb, tb, to, p, grid, ctx.stream);
+}
+
+cudaError_t launch_grouped_wgrad(const void* a_t, const void* b_t, int64_t M, int64_t N,
+                                 int64_t P, int64_t tokens, int32_t E, const float* sa,
+                                 const float* sb, const int32_t* offs, int out_f32, void* out,
+                                 const LaunchCtx& ctx) {
+  if (M == 0 || N == 0) return cudaSuccess;
+  CUtensorMap ta, tb, to;
+  if (!a_map(&ta, a_t, M, P, ctx.err)) return cudaErrorInvalidValue;
+  {
+    uint64_t dims[2] = {static_cast<uint64_t>(P), static_cast<uint64_t>(N)};
+    uint64_t strides[1] = {static_cast<uint64_t>(P)};
+    uint32_t box[2] = {BK, Cfg<false>::kBRows};
+    if (!make_tmap(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, b_t, dims, strides, box,
+                   CU_TENSOR_MAP_SWIZZLE_128B, ctx.err))
+      return cudaErrorInvalidValue;
+  }
+  // the kernel stores with plain masked stores; the map must be a valid object
+  if (!out_map(&to, out, static_cast<int64_t>(E) * M, N, out_f32 ? kOutFp32 : kOutBf16, ctx.err))
+    return cudaErrorInvalidValue;
+  GemmParams p{};
+  p.M = M;
+  p.N = N;
+  p.K = P;
+  p.sa = sa;
+  p.sb = sb;
+  p.bias = nullptr;
+  p.out = out;
+  p.offs = offs;
+  p.E = E;
+  p.tokens = tokens;
+  p.n_tiles = static_cast<int32_t>((N + BN - 1) / BN);
+  p.m_tiles = static_cast<int32_t>(M / BM);
+  p.k_blocks = static_cast<int32_t>(P / BK);
+  p.status = ctx.status;
+  p.split_start = INT64_MAX;
+  p.total_items = 0;
+  const int64_t items = static_cast<int64_t>(E) * p.m_tiles * p.n_tiles;
+  const unsigned grid = static_cast<unsigned>(items < ctx.num_sms ? items : ctx.num_sms);
+  return dispatch<true>(kBlock1, out_f32, false, ta, tb, tb, to, p, grid, ctx.stream);
 }
 
 cudaError_t launch_timeout_probe(uint32_t limit_us, const LaunchCtx& ctx) {

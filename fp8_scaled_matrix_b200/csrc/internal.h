@@ -34,6 +34,16 @@ size_t mx_scale_tile_bytes(int64_t rows, int64_t cols);
 cudaError_t launch_quantize_mx(const void* x, int64_t rows, int64_t cols, int64_t ld,
                                void* q, void* sf, const LaunchCtx& ctx);
 
+// Per-expert transposed 1x128 quantization (quantize.cu): x (rows = tokens,
+// cols) with groups of tokens by cumulative offs (device, E entries); the
+// output (cols, P) codes with P = grouped_padded_tokens(rows, E) hold each
+// group's tokens padded to a multiple of 128 (zero codes in the padding);
+// scales (P/128, cols).  E <= 2048.
+int64_t grouped_padded_tokens(int64_t tokens, int32_t E);
+cudaError_t launch_quantize_transposed_grouped(const void* x, int64_t rows, int64_t cols,
+                                               int64_t ld, const int32_t* offs, int32_t E,
+                                               void* q, float* scales, const LaunchCtx& ctx);
+
 // Library-owned scratch for the no-allocation quantize entry point
 // (quantize.cu): its size, and its device address on `device` (looked up
 // once per device; the device must be current).
@@ -58,6 +68,16 @@ cudaError_t launch_grouped_scaled_mm(const void* a, const void* b,
                                      const float* sb, const int32_t* offs,
                                      int recipe, int out_f32, void* out,
                                      const LaunchCtx& ctx);
+
+// Per-expert weight gradient (gemm.cu): for g < E, out[g] (M, N) =
+// sum over group g's padded K blocks of (a_t * sa)(b_t * sb)^T with the
+// 1x128_128x1 recipe.  a_t (M, P), b_t (N, P): per-expert padded transposed
+// codes (launch_quantize_transposed_grouped); sa (P/128, M), sb (P/128, N);
+// offs (device, E) token offsets ending at `tokens`.  M % 128 == 0.
+cudaError_t launch_grouped_wgrad(const void* a_t, const void* b_t, int64_t M, int64_t N,
+                                 int64_t P, int64_t tokens, int32_t E, const float* sa,
+                                 const float* sb, const int32_t* offs, int out_f32, void* out,
+                                 const LaunchCtx& ctx);
 
 // Failure-detection probe (gemm.cu): one CTA waits on a barrier nothing
 // completes, with the given limit.

@@ -375,29 +375,102 @@ constexpr size_t kTrSmemBytes =
     2 * kTrTileElems * sizeof(uint16_t) + static_cast<size_t>(kTrCols) * kTrOutPitch;
 constexpr int kTrCtasPerSm = 2;
 
-template <bool k128x128>
+// Grouped (per-expert) variant, 1x128 only: rows are tokens split into
+// groups by cumulative offsets; each group's tokens are laid out in the
+// output padded to a multiple of 128 (group g starts at output column
+// 128 * pb0[g], pb0 = exclusive prefix of ceil(size / 128)), so no 128-token
+// block mixes two groups; the padding is zero.  ldq = the output row stride.
+constexpr int kTrMaxGroups = 2048;
+
+template <bool k128x128, bool kGroupedT>
 __global__ void __launch_bounds__(kTrThreads) quant_transposed_kernel(
     const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
-    uint8_t* __restrict__ q, float* __restrict__ scales) {
+    uint8_t* __restrict__ q, float* __restrict__ scales, const int32_t* __restrict__ offs,
+    int32_t E, int64_t ldq, int64_t n_kb, uint32_t* status) {
   extern __shared__ __align__(16) uint16_t tiles_smem[];
   __shared__ float part[4][kTrCols];
   __shared__ float warp_amax[kTrThreads / 32];
-  const int64_t n_kb = rows / kTrRows;
   const int64_t n_cb = (cols + kTrCols - 1) / kTrCols;
   const int64_t n_tiles = n_kb * n_cb;
   const int t = threadIdx.x;
+  int32_t* pb0 = nullptr;  // grouped: pb0[g] = padded blocks before group g; pb0[E] = total
+  if constexpr (kGroupedT) {
+    __shared__ int32_t table[kTrMaxGroups + 1];
+    __shared__ int32_t bad;
+    pb0 = table;
+    if (t < 32) {
+      // lane l: groups [l * per, (l + 1) * per); block counts, then a scan
+      const int32_t per = (E + 31) / 32;
+      const int32_t g0 = t * per, g1 = min(E, g0 + per);
+      int32_t sum = 0, bad_l = 0;
+      for (int32_t g = g0; g < g1; ++g) {
+        const int32_t prev = g ? offs[g - 1] : 0;
+        const int32_t e = offs[g];
+        if (e < prev || prev < 0) bad_l = 1;
+        sum += (max(e - prev, 0) + kTrRows - 1) / kTrRows;
+      }
+      int32_t incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (t >= o) incl += v;
+      }
+      int32_t run = incl - sum;
+      for (int32_t g = g0; g < g1; ++g) {
+        table[g] = run;
+        const int32_t prev = g ? offs[g - 1] : 0;
+        run += (max(offs[g] - prev, 0) + kTrRows - 1) / kTrRows;
+      }
+      if (t == 31) table[E] = incl;
+      bad_l = __any_sync(0xFFFFFFFFu, bad_l);
+      if (t == 0) bad = bad_l || offs[E - 1] != rows;
+    }
+    __syncthreads();
+    if (bad || pb0[E] > n_kb) {
+      if (t == 0 && blockIdx.x == 0) record_status(status, FP8_DEV_VALUE, SITE_OFFS);
+      return;
+    }
+  }
+  // padded block kb -> first input row and the rows it holds (grouped: the
+  // block's group by binary search over pb0)
+  auto block_rows = [&](int64_t kb, int64_t& row0, int32_t& nrows) {
+    if constexpr (kGroupedT) {
+      int32_t lo = 0, hi = E - 1;
+      while (lo < hi) {  // last g with pb0[g] <= kb
+        const int32_t mid = (lo + hi + 1) >> 1;
+        if (pb0[mid] <= kb) lo = mid;
+        else hi = mid - 1;
+      }
+      const int64_t start = lo ? offs[lo - 1] : 0;
+      row0 = start + (kb - pb0[lo]) * kTrRows;
+      const int64_t left = static_cast<int64_t>(offs[lo]) - row0;
+      nrows = static_cast<int32_t>(left < kTrRows ? left : kTrRows);
+    } else {
+      row0 = kb * kTrRows;
+      nrows = kTrRows;
+    }
+  };
+  const int64_t n_kb_used = kGroupedT ? pb0[E] : n_kb;
   // copy tile `tile` into buffer `buf`: chunk t % 16 (8 columns) of rows
-  // t / 16 + 32 i; columns past the end are zero-filled (no effect on the max)
+  // t / 16 + 32 i; columns past the end (and grouped: rows past the group)
+  // are zero-filled (no effect on the max, zero codes)
   auto issue = [&](int64_t tile, int buf) {
     const int64_t kb = tile % n_kb, cb = tile / n_kb;
+    if (kb >= n_kb_used) {
+      cp_async_commit();
+      return;
+    }
+    int64_t row0;
+    int32_t nrows;
+    block_rows(kb, row0, nrows);
     const int ch = t & 15;
     const int64_t col = cb * kTrCols + ch * 8;
     uint16_t* dst = tiles_smem + buf * kTrTileElems;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int r = (t >> 4) + 32 * i;
-      const bool in = col < cols;
-      cp_async_16(dst + r * kTrPitch + ch * 8, in ? x + (kb * kTrRows + r) * ld + col : x,
+      const bool in = col < cols && r < nrows;
+      cp_async_16(dst + r * kTrPitch + ch * 8, in ? x + (row0 + r) * ld + col : x,
                   in ? 16u : 0u);
     }
     cp_async_commit();
@@ -414,6 +487,7 @@ __global__ void __launch_bounds__(kTrThreads) quant_transposed_kernel(
     __syncthreads();
     const uint16_t* tl = tiles_smem + buf * kTrTileElems;
     const int64_t kb = tile % n_kb, cb = tile / n_kb;
+    if (kb >= n_kb_used) continue;   // grouped: past the last group's blocks (uniform)
     uint32_t w[16];                  // the 32 values, packed bf16 pairs
     float m = 0.0f;
 #pragma unroll
@@ -461,7 +535,7 @@ __global__ void __launch_bounds__(kTrThreads) quant_transposed_kernel(
       const int64_t ocol = cb * kTrCols + orow;
       if (ocol < cols) {
         const uint4* ss = reinterpret_cast<const uint4*>(stage + orow * kTrOutPitch + 32 * chunk);
-        uint4* dst = reinterpret_cast<uint4*>(q + ocol * rows + kb * kTrRows + 32 * chunk);
+        uint4* dst = reinterpret_cast<uint4*>(q + ocol * ldq + kb * kTrRows + 32 * chunk);
         dst[0] = ss[0];
         dst[1] = ss[1];
       }
@@ -583,33 +657,60 @@ cudaError_t launch_quantize_mx(const void* xv, int64_t rows, int64_t cols, int64
   return cudaGetLastError();
 }
 
+static cudaError_t configure_transposed() {
+  static bool configured = false;
+  if (configured) return cudaSuccess;
+  const void* fns[] = {(const void*)quant_transposed_kernel<true, false>,
+                       (const void*)quant_transposed_kernel<false, false>,
+                       (const void*)quant_transposed_kernel<false, true>};
+  for (const void* f : fns) {
+    cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kTrSmemBytes));
+    if (e != cudaSuccess) return e;
+  }
+  configured = true;
+  return cudaSuccess;
+}
+
 cudaError_t launch_quantize_transposed(const void* xv, int64_t rows, int64_t cols,
                                        int64_t ld, int recipe, void* qv, float* scales,
                                        const LaunchCtx& ctx) {
   if (rows == 0 || cols == 0) return cudaSuccess;
   const uint16_t* x = static_cast<const uint16_t*>(xv);
   uint8_t* q = static_cast<uint8_t*>(qv);
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(quant_transposed_kernel<true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kTrSmemBytes));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(quant_transposed_kernel<false>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kTrSmemBytes));
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
-  const int64_t tiles = (rows / kTrRows) * ((cols + kTrCols - 1) / kTrCols);
+  cudaError_t e = configure_transposed();
+  if (e != cudaSuccess) return e;
+  const int64_t n_kb = rows / kTrRows;
+  const int64_t tiles = n_kb * ((cols + kTrCols - 1) / kTrCols);
   const int64_t max_grid = static_cast<int64_t>(ctx.num_sms) * kTrCtasPerSm;
   const unsigned grid = static_cast<unsigned>(tiles < max_grid ? tiles : max_grid);
   if (recipe == 3)
-    quant_transposed_kernel<true><<<grid, kTrThreads, kTrSmemBytes, ctx.stream>>>(
-        x, rows, cols, ld, q, scales);
+    quant_transposed_kernel<true, false><<<grid, kTrThreads, kTrSmemBytes, ctx.stream>>>(
+        x, rows, cols, ld, q, scales, nullptr, 0, rows, n_kb, ctx.status);
   else
-    quant_transposed_kernel<false><<<grid, kTrThreads, kTrSmemBytes, ctx.stream>>>(
-        x, rows, cols, ld, q, scales);
+    quant_transposed_kernel<false, false><<<grid, kTrThreads, kTrSmemBytes, ctx.stream>>>(
+        x, rows, cols, ld, q, scales, nullptr, 0, rows, n_kb, ctx.status);
+  return cudaGetLastError();
+}
+
+int64_t grouped_padded_tokens(int64_t tokens, int32_t E) {
+  return ((tokens + kTrRows - 1) / kTrRows + E) * kTrRows;
+}
+
+cudaError_t launch_quantize_transposed_grouped(const void* xv, int64_t rows, int64_t cols,
+                                               int64_t ld, const int32_t* offs, int32_t E,
+                                               void* qv, float* scales, const LaunchCtx& ctx) {
+  if (cols == 0) return cudaSuccess;
+  cudaError_t e = configure_transposed();
+  if (e != cudaSuccess) return e;
+  const int64_t P = grouped_padded_tokens(rows, E);
+  const int64_t n_kb = P / kTrRows;
+  const int64_t tiles = n_kb * ((cols + kTrCols - 1) / kTrCols);
+  const int64_t max_grid = static_cast<int64_t>(ctx.num_sms) * kTrCtasPerSm;
+  const unsigned grid = static_cast<unsigned>(tiles < max_grid ? tiles : max_grid);
+  quant_transposed_kernel<false, true><<<grid, kTrThreads, kTrSmemBytes, ctx.stream>>>(
+      static_cast<const uint16_t*>(xv), rows, cols, ld, static_cast<uint8_t*>(qv), scales,
+      offs, E, P, n_kb, ctx.status);
   return cudaGetLastError();
 }
 

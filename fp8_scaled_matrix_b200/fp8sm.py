@@ -36,7 +36,9 @@ EXPORTED = ["fp8_version", "fp8_last_error", "fp8_quantize_workspace_bytes",
             "fp8_quantize_noalloc", "fp8_quantize_transposed",
             "fp8_grouped_scaled_mm_blockwise", "fp8_scaled_mm_quantized",
             "fp8_mx_scale_bytes", "fp8_quantize_mx", "fp8_scaled_mm_mx",
-            "fp8_scaled_mm_mx_quantized", "fp8_grouped_scaled_mm_mx"]
+            "fp8_scaled_mm_mx_quantized", "fp8_grouped_scaled_mm_mx",
+            "fp8_grouped_padded_tokens", "fp8_quantize_transposed_grouped",
+            "fp8_grouped_scaled_mm_wgrad"]
 
 
 class Fp8Error(RuntimeError):
@@ -95,6 +97,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fp8_scaled_mm_quantized.argtypes = [P, P, I64, I64, I64, P, P, E, P, P, P, P]
     L.fp8_grouped_scaled_mm.restype = E
     L.fp8_grouped_scaled_mm.argtypes = [P, P, I64, I64, I64, I32, P, P, P, E, P, P]
+    L.fp8_grouped_padded_tokens.restype = I64
+    L.fp8_grouped_padded_tokens.argtypes = [I64, I32]
+    L.fp8_quantize_transposed_grouped.restype = E
+    L.fp8_quantize_transposed_grouped.argtypes = [P, I64, I64, I64, P, I32, P, P, P]
+    L.fp8_grouped_scaled_mm_wgrad.restype = E
+    L.fp8_grouped_scaled_mm_wgrad.argtypes = [P, P, I64, I64, I64, I32, P, P, P, E, P, P]
     L.fp8_grouped_scaled_mm_mx.restype = E
     L.fp8_grouped_scaled_mm_mx.argtypes = [P, P, I64, I64, I64, I32, P, P, P, E, P, P]
     L.fp8_grouped_scaled_mm_blockwise.restype = E
@@ -457,4 +465,59 @@ def fp8_grouped_scaled_mm_mx(a: torch.Tensor, b_experts: torch.Tensor,
     _check(L.fp8_grouped_scaled_mm_mx(_ptr(a), _ptr(b_experts), M, N, K, E, _ptr(scale_a),
                                       _ptr(scale_b), _ptr(offs), od, _ptr(out),
                                       _stream(stream)))
+    return out
+
+
+def fp8_grouped_padded_tokens(tokens: int, E: int) -> int:
+    return int(load_library().fp8_grouped_padded_tokens(tokens, E))
+
+
+def fp8_quantize_transposed_grouped(x: torch.Tensor, offs: torch.Tensor,
+                                    out: Optional[torch.Tensor] = None,
+                                    scales: Optional[torch.Tensor] = None,
+                                    stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Per-expert 1x128 quantization of x^T (x: tokens x cols bf16), each
+    group of tokens padded to a multiple of 128: returns (codes (cols, P),
+    scales (P/128, cols)), P = fp8_grouped_padded_tokens(tokens, E)."""
+    L = load_library()
+    _need_cuda(x, offs)
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D bf16 tensor with unit column stride")
+    if offs.dtype != torch.int32:
+        raise ValueError("offs must be int32")
+    T, cols = x.shape
+    E = offs.numel()
+    P = fp8_grouped_padded_tokens(T, E)
+    if out is None:
+        out = torch.empty((cols, P), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((P // 128, cols), dtype=torch.float32, device=x.device)
+    if out.numel() < cols * P or scales.numel() < (P // 128) * cols:
+        raise ValueError("out or scales too small")
+    _check(L.fp8_quantize_transposed_grouped(_ptr(x), T, cols, x.stride(0), _ptr(offs), E,
+                                             _ptr(out), _ptr(scales), _stream(stream)))
+    return out, scales
+
+
+def fp8_grouped_scaled_mm_wgrad(a_t: torch.Tensor, b_t: torch.Tensor, scale_a: torch.Tensor,
+                                scale_b: torch.Tensor, offs: torch.Tensor, tokens: int,
+                                out_dtype=torch.bfloat16, out: Optional[torch.Tensor] = None,
+                                stream=None) -> torch.Tensor:
+    """Per-expert weight gradient: out[g] = dY_g^T @ X_g from the padded
+    transposed codes of fp8_quantize_transposed_grouped; returns (E, M, N)."""
+    L = load_library()
+    _need_cuda(a_t, b_t, scale_a, scale_b, offs)
+    if offs.dtype != torch.int32:
+        raise ValueError("offs must be int32")
+    E = offs.numel()
+    M, P = a_t.shape
+    N = b_t.shape[0]
+    if b_t.shape[1] != P or P != fp8_grouped_padded_tokens(tokens, E):
+        raise ValueError("operands must have the padded width of fp8_quantize_transposed_grouped")
+    od = FP8_OUT_F32 if out_dtype == torch.float32 else FP8_OUT_BF16
+    if out is None:
+        out = torch.empty((E, M, N), dtype=out_dtype, device=a_t.device)
+    _check(L.fp8_grouped_scaled_mm_wgrad(_ptr(a_t), _ptr(b_t), M, N, tokens, E, _ptr(scale_a),
+                                         _ptr(scale_b), _ptr(offs), od, _ptr(out),
+                                         _stream(stream)))
     return out

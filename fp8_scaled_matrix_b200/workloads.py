@@ -47,6 +47,11 @@ descriptions; no public dataset is involved):
                 workload 4's activations, same seed and group split), W =
                 workload 4's experts (16, 4096 out, 4096 in); GEMM M=32768,
                 N=4096 (in), K=4096 (out)
+ 13 grouped grad_weight  the MoE layer's per-expert weight gradient
+                dW_g = dY_g^T @ X_g with the 1x128_128x1 recipe over each
+                group's tokens: dY ~ N(0, 1e-3^2) (32768, 4096 out), X ~ N(0,1)
+                (32768, 4096 in), workload 4's group split; GEMM M=4096 (out),
+                N=4096 (in), K=32768 tokens in 16 groups
 """
 from __future__ import annotations
 
@@ -70,6 +75,7 @@ WORKLOAD_NAMES = [
     "linear_chain_mxfp8",
     "grouped_e16_mxfp8",
     "grouped_e16_grad_input",
+    "grouped_e16_grad_weight",
 ]
 
 
@@ -124,7 +130,7 @@ class Workload:
     name: str
     # tensor | row | 1x128_128x128 | 1x128_128x1 | grouped | grouped_blockwise |
     # grad_input | grad_weight | chain | mxfp8 | chain_mx | grouped_mx |
-    # grouped_grad_input
+    # grouped_grad_input | grouped_grad_weight
     recipe: str
     M: int
     N: int
@@ -133,7 +139,9 @@ class Workload:
     #   a  (M, K); grad_weight: (K, M) (grad_output, tokens x out)
     #   b  (N, K) or (E, N, K); grad_input: (K, N) (the weight as stored);
     #      grad_weight: (K, N) (the layer input, tokens x in);
-    #      grouped_grad_input: (E, K, N) (the experts as stored, out x in)
+    #      grouped_grad_input: (E, K, N) (the experts as stored, out x in);
+    #   grouped_grad_weight: a (K, M) = dY (tokens x out), b (K, N) = X
+    #      (tokens x in), K = tokens split by offs
     a: torch.Tensor
     b: torch.Tensor
     bias: Optional[torch.Tensor] = None   # bf16 (N,) CPU
@@ -160,6 +168,16 @@ def make_workload(index: int, shape_index: int = 0, scale_down: int = 1) -> Work
         wl = make_workload(4, shape_index, scale_down)
         wl.name, wl.recipe = name, "grouped_blockwise"
         return wl
+    if index == 13:
+        ref = make_workload(4, shape_index, scale_down)
+        T, D = ref.a.shape
+        E = ref.E
+        seed = 1000 + index + 100 * shape_index
+        g = generator(seed)
+        dy = randn_bf16((T, D), 1e-3, g)
+        x = randn_bf16((T, D), 1.0, g)
+        return Workload(name, "grouped_grad_weight", D, D, T, dy, x, offs=ref.offs, E=E,
+                        seed=seed)
     if index == 12:  # workload 4's tensors as (dY, W) of the backward
         wl = make_workload(4, shape_index, scale_down)
         E, Nout, Kin = wl.b.shape

@@ -373,6 +373,48 @@ FP8SM_API fp8_status fp8_grouped_scaled_mm_mx(const void* a, const void* b_exper
                                     fp8_stream_t stream);
 
 /*
+ * MoE weight gradient ([P2]'s grouped layer, backward; the grad_weight GEMM
+ * of [P5] with the 1x128_128x1 recipe): for every expert g,
+ *   out[g] (M, N) = dY_g^T @ X_g = sum over the tokens t of group g of
+ *                   (a_t[m, t] * sa) (b_t[n, t] * sb)
+ * where group g's tokens are [offs[g-1], offs[g]).  The contraction runs
+ * over each group's own tokens, so 128-token quantization blocks must not
+ * mix groups: the operands are quantized per group with
+ * fp8_quantize_transposed_grouped, which lays every group's tokens out
+ * padded to a multiple of 128 (zero codes in the padding).
+ *
+ * fp8_grouped_padded_tokens(T, E) = (ceil(T/128) + E) * 128 = P, the padded
+ * width (an upper bound of sum_g ceil(size_g/128) * 128, known on the host).
+ *
+ * fp8_quantize_transposed_grouped: x_bf16 (T, cols) bf16 (row stride ld_x,
+ *   a multiple of 8; cols % 8 == 0), offs DEVICE (E) int32 cumulative token
+ *   ends (non-decreasing, offs[E-1] == T), 1 <= E <= 2048.  Writes
+ *   out_fp8 (cols, P) e4m3 (row stride P; group g's tokens at columns
+ *   128 * pb0[g] .., pb0[g] = sum_{h<g} ceil(size_h/128)) and out_scales
+ *   (P/128, cols) fp32 (scale[(pb) * cols + c] for padded block pb), each
+ *   block's scale from its own group's tokens only.  Columns of the padded
+ *   width past the last group are not written.  A malformed offs writes
+ *   nothing and sets the device status to FP8_ERR_VALUE.
+ * fp8_grouped_scaled_mm_wgrad: a_t (M, P), b_t (N, P) from the quantizer
+ *   above (a_t = dY^T with M = the layer's outputs, b_t = X^T with N = its
+ *   inputs), scale_a (P/128, M), scale_b (P/128, N), offs as above with
+ *   tokens = T; out (E, M, N) bf16 or fp32 (an empty group's gradient is
+ *   zero).  Requirements: M % 128 == 0, N % 16 == 0, 1 <= E <= 65535.
+ */
+FP8SM_API int64_t fp8_grouped_padded_tokens(int64_t tokens, int32_t E);
+
+FP8SM_API fp8_status fp8_quantize_transposed_grouped(const void* x_bf16, int64_t tokens,
+                                           int64_t cols, int64_t ld_x, const int32_t* offs,
+                                           int32_t E, void* out_fp8, float* out_scales,
+                                           fp8_stream_t stream);
+
+FP8SM_API fp8_status fp8_grouped_scaled_mm_wgrad(const void* a_t, const void* b_t, int64_t M,
+                                       int64_t N, int64_t tokens, int32_t E,
+                                       const float* scale_a, const float* scale_b,
+                                       const int32_t* offs, fp8_out_dtype out_dtype,
+                                       void* out, fp8_stream_t stream);
+
+/*
  * Synchronizes `stream`, then returns and clears the current device's status
  * word: FP8_OK, FP8_ERR_VALUE (malformed offs), FP8_ERR_TIMEOUT (a pipeline
  * wait gave up; the kernel released its resources and returned), or

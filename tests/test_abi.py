@@ -265,3 +265,33 @@ def test_grouped_mx_rejects_bad_arguments(lib, M, N, K, E, frag):
     st = lib.fp8_grouped_scaled_mm_mx(FAKE, FAKE, M, N, K, E, FAKE, FAKE, FAKE,
                                       fp8sm.FP8_OUT_BF16, FAKE, None)
     assert st == fp8sm.FP8_ERR_VALUE and frag in lib.fp8_last_error().decode()
+
+
+def test_grouped_padded_tokens(lib):
+    assert lib.fp8_grouped_padded_tokens(0, 4) == 512
+    assert lib.fp8_grouped_padded_tokens(300, 2) == (3 + 2) * 128
+    assert lib.fp8_grouped_padded_tokens(32768, 16) == (256 + 16) * 128
+
+
+@pytest.mark.parametrize("args,frag", [
+    ((FAKE, 64, 100, 100, FAKE, 2), "multiples of 8"),
+    ((FAKE, 64, 128, 128, None, 2), "offs is required"),
+    ((FAKE, 64, 128, 128, FAKE, 0), "expert count"),
+    ((FAKE, 64, 128, 128, FAKE, 4096), "expert count"),
+    ((FAKE, -1, 128, 128, FAKE, 2), "negative"),
+])
+def test_quantize_transposed_grouped_rejects_bad_arguments(lib, args, frag):
+    x, T, cols, ld, offs, E = args
+    st = lib.fp8_quantize_transposed_grouped(x, T, cols, ld, offs, E, FAKE, FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE and frag in lib.fp8_last_error().decode()
+
+
+@pytest.mark.parametrize("M,N,T,E,frag", [
+    (100, 128, 64, 2, "M must be a multiple of 128"),
+    (128, 100, 64, 2, "N must be a multiple of 16"),
+    (128, 128, 64, 0, "expert count"),
+])
+def test_grouped_wgrad_rejects_bad_arguments(lib, M, N, T, E, frag):
+    st = lib.fp8_grouped_scaled_mm_wgrad(FAKE, FAKE, M, N, T, E, FAKE, FAKE, FAKE,
+                                         fp8sm.FP8_OUT_BF16, FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE and frag in lib.fp8_last_error().decode()

@@ -85,3 +85,102 @@ def test_grouped_grad_input_full_size_sampled():
     rows = np.array(sorted(r for r in rows if 0 <= r < wl.M))
     ref, mag = oracle_grad_input(wl.a, wl.b, ends, rows=rows)
     check_gemm(out_f64(out)[rows], ref, mag, "grouped grad_input full size")
+
+
+# -------------------------------------------------- weight gradient per expert
+
+def padded_t_bits(x: torch.Tensor, start: int, end: int) -> np.ndarray:
+    """Group [start, end) of x (tokens x cols), transposed and padded with zero
+    tokens to a multiple of 128: the definition of the per-expert layout."""
+    n = end - start
+    pad = -(-n // 128) * 128
+    out = np.zeros((x.shape[1], pad), np.uint16)
+    out[:, :n] = W.bf16_bits(x[start:end]).T
+    return out
+
+
+def oracle_wgrad_group(dy, x, start, end, rows=None):
+    qa, sa = oracle.quantize(padded_t_bits(dy, start, end), oracle.GROUP_1x128)
+    qb, sb = oracle.quantize(padded_t_bits(x, start, end), oracle.GROUP_1x128)
+    return (qa, sa, qb, sb), oracle.scaled_mm(qa, qb, sa, sb, MM["1x128_128x1"], rows=rows)
+
+
+def gpu_wgrad(dy, x, offs_np, out_dtype=torch.float32):
+    offs = torch.as_tensor(offs_np, dtype=torch.int32).cuda()
+    qa, sa = fp8sm.fp8_quantize_transposed_grouped(dy.cuda(), offs)
+    qb, sb = fp8sm.fp8_quantize_transposed_grouped(x.cuda(), offs)
+    out = fp8sm.fp8_grouped_scaled_mm_wgrad(qa, qb, sa, sb, offs, dy.shape[0],
+                                            out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    fp8sm.check_device_status()
+    return qa, sa, qb, sb, out
+
+
+@pytest.mark.parametrize("sizes,M,N", [
+    ([5, 0, 17, 130], 256, 272),
+    ([0, 0, 64, 0], 128, 256),
+    ([300], 128, 512),
+    ([1, 255, 129, 0, 2, 384], 384, 160),
+])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_grouped_wgrad_parity(sizes, M, N, out_dtype):
+    E = len(sizes)
+    T = sum(sizes)
+    g = W.generator(T * 7 + M + N)
+    dy = W.randn_bf16((T, M), 1e-3, g)
+    x = W.randn_bf16((T, N), 1.0, g)
+    ends = np.cumsum(sizes).astype(np.int32)
+    qa, sa, qb, sb, out = gpu_wgrad(dy, x, ends, out_dtype)
+    qa, sa, qb, sb = (t.cpu().numpy() for t in (qa, sa, qb, sb))
+    start, pb = 0, 0
+    for e, end in enumerate(ends):
+        n = int(end) - start
+        nblk = -(-n // 128)
+        if n == 0:
+            assert (out[e] == 0).all(), f"empty group {e} must give a zero gradient"
+            continue
+        (oqa, osa, oqb, osb), (ref, mag) = oracle_wgrad_group(dy, x, start, int(end))
+        # the quantized per-group blocks are the oracle's bit for bit
+        cols = slice(128 * pb, 128 * (pb + nblk))
+        assert np.array_equal(qa[:, cols], oqa) and np.array_equal(qb[:, cols], oqb)
+        assert np.array_equal(sa[pb:pb + nblk].reshape(-1).view(np.uint32), osa.view(np.uint32))
+        assert np.array_equal(sb[pb:pb + nblk].reshape(-1).view(np.uint32), osb.view(np.uint32))
+        check_gemm(out_f64(out[e]), ref, mag, f"wgrad group {e} of {sizes}")
+        start, pb = int(end), pb + nblk
+
+
+def test_grouped_wgrad_full_size_sampled():
+    """The MoE layer's weight gradient on the MoE workload's split (16 experts,
+    32768 tokens, 4096 outputs x 4096 inputs): three experts checked on
+    sampled rows (the largest, a small one and the last)."""
+    wl = W.make_workload(13, 0)
+    dy, x = wl.a, wl.b
+    ends = wl.offs.numpy()
+    _, _, _, _, out = gpu_wgrad(dy, x, ends)
+    sizes = np.diff(np.concatenate([[0], ends]))
+    pick = {int(np.argmax(sizes)), len(ends) - 1}
+    nz = [e for e in range(len(ends)) if sizes[e] > 0]
+    pick.add(int(min(nz, key=lambda e: sizes[e])))
+    for e in sorted(pick):
+        start = int(ends[e - 1]) if e else 0
+        rows = sample_rows(wl.M, 24, seed=e)
+        _, (ref, mag) = oracle_wgrad_group(dy, x, start, int(ends[e]), rows=rows)
+        check_gemm(out_f64(out[e])[rows], ref, mag, f"wgrad expert {e} full size")
+
+
+def test_grouped_wgrad_malformed_offs_reports_value_error():
+    T, M, N, E = 64, 128, 64, 3
+    offs = torch.tensor([40, 20, 64], dtype=torch.int32, device="cuda")
+    dy = torch.zeros(T, M, dtype=torch.bfloat16, device="cuda")
+    fp8sm.fp8_quantize_transposed_grouped(dy, offs)
+    torch.cuda.synchronize()
+    assert fp8sm.fp8_get_device_status() == fp8sm.FP8_ERR_VALUE
+    P = fp8sm.fp8_grouped_padded_tokens(T, E)
+    sentinel = torch.full((E, M, N), 7.0, device="cuda")
+    fp8sm.fp8_grouped_scaled_mm_wgrad(
+        torch.zeros(M, P, dtype=torch.uint8, device="cuda"),
+        torch.zeros(N, P, dtype=torch.uint8, device="cuda"),
+        torch.ones(P // 128, M, device="cuda"), torch.ones(P // 128, N, device="cuda"),
+        offs, T, out_dtype=torch.float32, out=sentinel)
+    assert fp8sm.fp8_get_device_status() == fp8sm.FP8_ERR_VALUE
+    assert (sentinel.cpu() == 7.0).all()
