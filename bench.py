@@ -57,6 +57,7 @@ WORKLOADS = {
     "linear_chain_mxfp8": (10, 0),
     "grouped_e16_mxfp8": (11, 0),
     "grouped_e16_grad_input": (12, 0),
+    "grouped_e16_grad_weight": (13, 0),
 }
 DEFAULT_WORKLOAD = "rowwise_4096"
 # Page 5's context numbers (TFLOP/s of torch._scaled_mm, hardware not stated)
@@ -70,7 +71,8 @@ OPERAND_GROUPS = {"tensor": ("tensor", "tensor"), "row": ("row", "row"),
                   "grad_input": ("1x128", "128x128"), "grad_weight": ("1x128", "1x128"),
                   "grouped_blockwise": ("1x128", "128x128"), "chain": ("1x128", "128x128"),
                   "mxfp8": ("mx", "mx"), "chain_mx": ("mx", "mx"), "grouped_mx": ("mx", "mx"),
-                  "grouped_grad_input": ("1x128", "128x128")}
+                  "grouped_grad_input": ("1x128", "128x128"),
+                  "grouped_grad_weight": ("1x128", "1x128")}
 # GEMM recipe of each workload recipe, and which operands are quantized
 # transposed (the training GEMMs contract along the stored rows)
 GEMM_RECIPE = {"grad_input": "1x128_128x128", "grad_weight": "1x128_128x1",
@@ -220,7 +222,13 @@ class Step:
         self.grouped = wl.recipe in ("grouped", "grouped_blockwise", "grouped_mx",
                                      "grouped_grad_input")
         self.gin = wl.recipe == "grouped_grad_input"
-        if self.gin:
+        self.wg = wl.recipe == "grouped_grad_weight"
+        if self.wg:
+            # (tokens x out) and (tokens x in), quantized per expert, transposed
+            self.grouped = False
+            self.b = wl.b.to(dev)
+            self.offs = wl.offs.to(dev)
+        elif self.gin:
             # the experts as stored (E, out, in); each is quantized transposed
             self.b = wl.b.to(dev)
             self.offs = wl.offs.to(dev)
@@ -238,9 +246,16 @@ class Step:
         if self.gin:
             rows_b = wl.b.shape[0] * wl.N    # (E * in, out) codes
         cols = wl.K
+        if self.wg:
+            # per-expert padded transposed operands: (out, P), (in, P)
+            rows_a, rows_b = wl.M, wl.N
+            cols = fp8sm.fp8_grouped_padded_tokens(wl.K, wl.E)
         self.qa = torch.empty(rows_a, cols, dtype=torch.uint8, device=dev)
         self.qb = torch.empty(rows_b, cols, dtype=torch.uint8, device=dev)
-        if self.mx:
+        if self.wg:
+            self.sa = torch.empty(cols // 128, rows_a, dtype=torch.float32, device=dev)
+            self.sb = torch.empty(cols // 128, rows_b, dtype=torch.float32, device=dev)
+        elif self.mx:
             # E8M0 scale-factor tiles
             self.sa = torch.empty(fp8sm.fp8_mx_scale_bytes(rows_a, cols), dtype=torch.uint8,
                                   device=dev)
@@ -256,7 +271,8 @@ class Step:
         self.side = torch.cuda.Stream(device=dev)
         self.ev_fork = torch.cuda.Event()
         self.ev_join = torch.cuda.Event()
-        self.out = torch.empty(wl.M, wl.N, dtype=torch.bfloat16, device=dev)
+        self.out = torch.empty(((wl.E,) if self.wg else ()) + (wl.M, wl.N),
+                               dtype=torch.bfloat16, device=dev)
         self.launches_per_step = 3
         if wl.recipe == "grouped_blockwise":
             # each expert's weights are quantized on their own (its 128x128
@@ -301,7 +317,10 @@ class Step:
         self.ev_fork.record(main)
         self.side.wait_event(self.ev_fork)
         with torch.cuda.stream(self.side):
-            if self.gin:
+            if self.wg:
+                f.fp8_quantize_transposed_grouped(self.b, self.offs, out=self.qb, scales=self.sb,
+                                                  stream=self.side)
+            elif self.gin:
                 E, Kin = self.wl.b.shape[0], self.wl.N
                 per = self.sb.numel() // E
                 for e in range(E):
@@ -331,7 +350,10 @@ class Step:
             else:
                 f.fp8_quantize(self.b, self.qb_recipe, out=self.qb, scales=self.sb,
                                workspace=self.ws_b, stream=self.side)
-        if self.mx:
+        if self.wg:
+            f.fp8_quantize_transposed_grouped(self.a, self.offs, out=self.qa, scales=self.sa,
+                                              stream=main)
+        elif self.mx:
             f.fp8_quantize_mx(self.a, out=self.qa, scales=self.sa, stream=main)
         elif self.t_a:
             f.fp8_quantize_transposed(self.a, self.qa_recipe, out=self.qa, scales=self.sa,
@@ -353,6 +375,9 @@ class Step:
             E, N, K = wl.b.shape
             f.fp8_grouped_scaled_mm_blockwise(self.qa, self.qb.view(E, N, K), self.sa,
                                               self.sb, self.offs, out=self.out)
+        elif self.wg:
+            f.fp8_grouped_scaled_mm_wgrad(self.qa, self.qb, self.sa, self.sb, self.offs, wl.K,
+                                          out=self.out)
         elif self.gin:
             E = wl.b.shape[0]
             f.fp8_grouped_scaled_mm_blockwise(self.qa, self.qb.view(E, wl.N, wl.K), self.sa,
@@ -569,6 +594,28 @@ def oracle_sample(wl, max_rows: int):
         rows = np.arange(min(max_rows, wl.M), dtype=np.int64)
         t0 = time.perf_counter()
         oracle.mx_scaled_mm(qa, qb, sa, sb, rows=rows)
+        return time.perf_counter() - t0, rows.size / wl.M, tq, oracle.num_threads()
+    if wl.recipe == "grouped_grad_weight":
+        # each expert's zero-padded transposed slices, quantized 1x128; the
+        # GEMM on the first max_rows output rows of every expert
+        ends = wl.offs.numpy()
+        ops = []
+        start = 0
+        for end in ends:
+            n = int(end) - start
+            if n:
+                pad = -(-n // 128) * 128
+                ta = np.zeros((wl.M, pad), np.uint16)
+                tb = np.zeros((wl.N, pad), np.uint16)
+                ta[:, :n] = W.bf16_bits(wl.a[start:int(end)]).T
+                tb[:, :n] = W.bf16_bits(wl.b[start:int(end)]).T
+                ops.append(oracle.quantize(ta, G["1x128"]) + oracle.quantize(tb, G["1x128"]))
+            start = int(end)
+        tq = time.perf_counter() - t0
+        rows = np.arange(min(max_rows, wl.M), dtype=np.int64)
+        t0 = time.perf_counter()
+        for qa, sa, qb, sb in ops:
+            oracle.scaled_mm(qa, qb, sa, sb, MMR["1x128_128x1"], rows=rows)
         return time.perf_counter() - t0, rows.size / wl.M, tq, oracle.num_threads()
     if wl.recipe == "grouped_grad_input":
         qa, sa = oracle.quantize(W.bf16_bits(wl.a), G["1x128"])

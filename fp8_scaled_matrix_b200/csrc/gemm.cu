@@ -395,6 +395,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // grouped 1x128_128x1 = the per-expert weight gradient: groups split K
   // (tokens), every group has its own (M, N) output
   constexpr bool kKGroups = kGrouped && kRecipe == kBlock1;
+  // stores: masked plain stores where a tile's rows may end inside a group
+  // (the row-grouped kernels); TMA stores otherwise (the K-grouped output's
+  // tiles are whole: M % 128 == 0)
+  constexpr bool kMasked = kGrouped && !kKGroups;
   // epilogue threads that hold a whole 128-column row slice in registers
   constexpr bool kBigEpi = kBlockwise || kIsMx;
   constexpr bool kOutF32 = kOut == kOutFp32;
@@ -441,10 +445,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
     prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_b);
-    if constexpr (!kGrouped) {
-      prefetch_tmap(&tm_b_half);
-      prefetch_tmap(&tm_out);
-    }
+    if constexpr (!kGrouped) prefetch_tmap(&tm_b_half);
+    if constexpr (!kMasked) prefetch_tmap(&tm_out);
   }
   if (warp == 1) {
     if constexpr (kPair) {
@@ -970,7 +972,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               load_bias32(p.bias, n, p.N, v);
 #pragma unroll
               for (int i = 0; i < 32; ++i) v[i] = __fadd_rn(__uint_as_float(r[cc][i]), v[i]);
-              store_cols32<kOutF32, kGrouped>(ebuf, v, &tm_out, static_cast<int32_t>(n), row0,
+              store_cols32<kOutF32, kMasked>(ebuf, v, &tm_out, static_cast<int32_t>(n), row0,
                                               c.row_end, p.out, p.N, lane);
             }
           } else {
@@ -1003,7 +1005,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   w[j] = cast_f32x2(v[4 * j], v[4 * j + 1], inv) |
                          (cast_f32x2(v[4 * j + 2], v[4 * j + 3], inv) << 16);
               }
-              store_box64<kGrouped>(ebuf, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
+              store_box64<kMasked>(ebuf, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
                                     row0, c.row_end, static_cast<uint8_t*>(p.out), p.N, 1, lane);
             }
             if (ncol0 < p.N) {
@@ -1053,7 +1055,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float v[32];
             values32(cc, v);
             if (cc == 3) release_buf();
-            store_cols32<kOutF32, kGrouped>(ebuf, v, &tm_out,
+            store_cols32<kOutF32, kMasked>(ebuf, v, &tm_out,
                                             static_cast<int32_t>(ncol0 + cc * 32), row0,
                                             c.row_end, p.out, p.N, lane);
           }
@@ -1086,7 +1088,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 w[j] = cast_f32x2(v[4 * j], v[4 * j + 1], sp.inv) |
                        (cast_f32x2(v[4 * j + 2], v[4 * j + 3], sp.inv) << 16);
             }
-            store_box64<kGrouped>(ebuf, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
+            store_box64<kMasked>(ebuf, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
                                   row0, c.row_end, static_cast<uint8_t*>(p.out), p.N, 1, lane);
           }
         }
@@ -1174,7 +1176,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int cc = 0; cc < 4; ++cc) {
             float v[32];
             result32(cc, v);
-            store_cols32<kOutF32, kGrouped>(ebuf, v, &tm_out,
+            store_cols32<kOutF32, kMasked>(ebuf, v, &tm_out,
                                             static_cast<int32_t>(ncol0 + cc * 32), row0,
                                             c.row_end, p.out, p.N, lane);
           }
@@ -1203,7 +1205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 w[j] = cast_f32x2(v[4 * j], v[4 * j + 1], sp.inv) |
                        (cast_f32x2(v[4 * j + 2], v[4 * j + 3], sp.inv) << 16);
             }
-            store_box64<kGrouped>(ebuf, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
+            store_box64<kMasked>(ebuf, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
                                   row0, c.row_end, static_cast<uint8_t*>(p.out), p.N, 1, lane);
           }
         }
