@@ -126,6 +126,7 @@ struct GemmParams {
   const float* sb;
   const uint8_t* sfa;  // MXFP8: scale-factor tiles of A and B (E8M0 bytes)
   const uint8_t* sfb;
+  int64_t sfa_bytes, sfb_bytes;  // their sizes: every copy is checked against them
   const uint16_t* bias;
   void* out;
   float* out_scales;  // e4m3 output: scale[(n/128) * M + m]; MXFP8 output: tiles
@@ -399,8 +400,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // (the row-grouped kernels); TMA stores otherwise (the K-grouped output's
   // tiles are whole: M % 128 == 0)
   constexpr bool kMasked = kGrouped && !kKGroups;
-  // epilogue threads that hold a whole 128-column row slice in registers
-  constexpr bool kBigEpi = kBlockwise || kIsMx;
+  // epilogue threads that hold a whole 128-column row slice across K blocks
+  // (blockwise promotion) get registers moved from warpgroup 0.  The MXFP8
+  // epilogue reads its accumulators once per tile and runs without the split
+  // (with it, a dense MXFP8 build faulted on the GPU; see the design notes).
+  constexpr bool kBigEpi = kBlockwise;
   constexpr bool kOutF32 = kOut == kOutFp32;
   constexpr bool kOutQ = kOut == kOutE4M3;
   constexpr bool kOutMxq = kOut == kOutMx;
@@ -555,8 +559,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             // 128 kb ..); B's second half-tile exists only below N
             // (grouped: expert g's tile set follows the g earlier ones; A's
             // scale tile is gathered by warp 2)
+            // (the second half of a split last-wave tile can start at or past
+            // N; its columns are never stored, so it takes B's last tile)
             const int64_t NB = (p.N + 127) / 128;
-            const int64_t nb0 = c.n0 / 128;
+            const int64_t nb0 = c.n0 / 128 < NB ? c.n0 / 128 : NB - 1;
             const bool two = !c.half_n && nb0 + 1 < NB;
             mbar_arrive_expect_tx(&full[stage], C::kAStage + b_bytes +
                                                     ((two ? 2u : 1u) + (kGrouped ? 0u : 1u)) *
@@ -569,14 +575,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint8_t* sf_dst = smem + C::kOffScl + stage * kMxSfStage;
             const int64_t kbb =
                 ((kGrouped ? static_cast<int64_t>(c.g) * NB * KB : 0) + nb0 * KB + kb) * kMxSfTile;
-            if constexpr (!kGrouped) {
-              const int64_t ka = (static_cast<int64_t>(c.m0 / 128) * KB + kb) * kMxSfTile;
-              bulk_load_g2s(sf_dst, p.sfa + ka, kMxSfTile, &full[stage]);
+            const int64_t ka = (static_cast<int64_t>(c.m0 / 128) * KB + kb) * kMxSfTile;
+            const int64_t kb2 = kbb + static_cast<int64_t>(KB) * kMxSfTile;
+            if ((!kGrouped && (ka < 0 || ka + kMxSfTile > p.sfa_bytes)) || kbb < 0 ||
+                kbb + kMxSfTile > p.sfb_bytes || (two && kb2 + kMxSfTile > p.sfb_bytes)) {
+              // a scale-tile copy outside the buffers: stop instead of faulting
+              // (the stage's expected bytes never arrive; every waiter gives up)
+              record_status(p.status, FP8_DEV_VALUE, SITE_BOUNDS);
+              *abort_flag = 1u;
+              ok = false;
+              break;
             }
+            if constexpr (!kGrouped) bulk_load_g2s(sf_dst, p.sfa + ka, kMxSfTile, &full[stage]);
             bulk_load_g2s(sf_dst + kMxSfTile, p.sfb + kbb, kMxSfTile, &full[stage]);
-            if (two)
-              bulk_load_g2s(sf_dst + 2 * kMxSfTile, p.sfb + kbb + static_cast<int64_t>(KB) * kMxSfTile,
-                            kMxSfTile, &full[stage]);
+            if (two) bulk_load_g2s(sf_dst + 2 * kMxSfTile, p.sfb + kb2, kMxSfTile, &full[stage]);
           } else if constexpr (kKGroups) {
             // the group's padded K range; A and B are (rows, padded tokens)
             const int32_t kx = static_cast<int32_t>((c.kb0 + kb) * BK);
@@ -861,10 +873,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t r = lane + 32u * j;
             const int64_t row = static_cast<int64_t>(c.m0) + r;
             const int64_t r7 = row & 127;
-            const uint8_t* src =
-                row < p.M ? p.sfa + ((row >> 7) * KB + kb) * kMxSfTile + (r7 & 31) * 16 + (r7 >> 5) * 4
-                          : p.sfa;
-            cp_async_4(slot + (r & 31u) * 16 + (r >> 5) * 4, src, row < p.M ? 4u : 0u);
+            const int64_t off = ((row >> 7) * KB + kb) * kMxSfTile + (r7 & 31) * 16 + (r7 >> 5) * 4;
+            const bool in = row < p.M && off >= 0 && off + 4 <= p.sfa_bytes;
+            cp_async_4(slot + (r & 31u) * 16 + (r >> 5) * 4, in ? p.sfa + off : p.sfa, in ? 4u : 0u);
           }
           cp_async_mbar_arrive_noinc(&full[stage]);
           if (++stage == C::kStages) {
@@ -1459,6 +1470,8 @@ cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
     // MXFP8: sa, sb carry the E8M0 scale-factor tiles
     p.sfa = reinterpret_cast<const uint8_t*>(sa);
     p.sfb = reinterpret_cast<const uint8_t*>(sb);
+    p.sfa_bytes = static_cast<int64_t>(mx_scale_tile_bytes(M, K));
+    p.sfb_bytes = static_cast<int64_t>(mx_scale_tile_bytes(N, K));
   } else {
     p.sa = sa;
     p.sb = sb;
@@ -1525,6 +1538,8 @@ cudaError_t launch_grouped_scaled_mm(const void* a, const void* b,
   if (recipe == kMxfp8) {
     p.sfa = reinterpret_cast<const uint8_t*>(sa);
     p.sfb = reinterpret_cast<const uint8_t*>(sb);
+    p.sfa_bytes = static_cast<int64_t>(mx_scale_tile_bytes(M_total, K));
+    p.sfb_bytes = static_cast<int64_t>(E) * static_cast<int64_t>(mx_scale_tile_bytes(N, K));
   } else {
     p.sa = sa;
     p.sb = sb;

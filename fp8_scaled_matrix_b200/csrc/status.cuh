@@ -27,6 +27,7 @@ enum : uint32_t {
   SITE_PROBE = 8,
   SITE_SCALE_EMPTY = 9,
   SITE_EPI_SCALE_FULL = 10,
+  SITE_BOUNDS = 11,  // a copy index outside its buffer (checked before the copy)
 };
 
 // Wait limit for every pipeline wait inside the GEMM / quantize kernels.
