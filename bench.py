@@ -280,13 +280,11 @@ class Step:
             E, N, K = wl.b.shape
             self.sb = torch.empty(E * fp8sm.scale_count(N, K, self.qb_recipe),
                                   dtype=torch.float32, device=dev)
-            self.launches_per_step = 2 + E
         if self.gin:
             # per expert W_g^T quantized 128x128: (out/128, in/128) scales each
             E = wl.b.shape[0]
             self.sb = torch.empty(E * fp8sm.scale_count(wl.N, wl.K, self.qb_recipe),
                                   dtype=torch.float32, device=dev)
-            self.launches_per_step = 2 + E
         self.chain = wl.recipe in ("chain", "chain_mx")
         if self.chain:
             # second linear: its weight (N2, N) quantized 128x128 like b; the
@@ -321,20 +319,14 @@ class Step:
                 f.fp8_quantize_transposed_grouped(self.b, self.offs, out=self.qb, scales=self.sb,
                                                   stream=self.side)
             elif self.gin:
-                E, Kin = self.wl.b.shape[0], self.wl.N
-                per = self.sb.numel() // E
-                for e in range(E):
-                    f.fp8_quantize_transposed(self.b[e], self.qb_recipe,
-                                              out=self.qb[e * Kin:(e + 1) * Kin],
-                                              scales=self.sb[e * per:(e + 1) * per],
-                                              stream=self.side)
+                # every expert's W_g^T, one launch
+                f.fp8_quantize_transposed_batched(self.b, self.qb_recipe, out=self.qb,
+                                                  scales=self.sb, stream=self.side)
             elif self.wl.recipe == "grouped_blockwise":
+                # every expert's 128x128 tiles and scales, one launch
                 E, N, K = self.wl.b.shape
-                per = self.sb.numel() // E
-                for e in range(E):
-                    f.fp8_quantize(self.b[e * N:(e + 1) * N], self.qb_recipe,
-                                   out=self.qb[e * N:(e + 1) * N],
-                                   scales=self.sb[e * per:(e + 1) * per], stream=self.side)
+                f.fp8_quantize_batched(self.b.view(E, N, K), self.qb_recipe, out=self.qb,
+                                       scales=self.sb, stream=self.side)
             elif self.t_b:
                 f.fp8_quantize_transposed(self.b, self.qb_recipe, out=self.qb, scales=self.sb,
                                           stream=self.side)

@@ -188,6 +188,74 @@ fp8_status fp8_quantize_transposed(const void* x_bf16, int64_t rows, int64_t col
   return finish_launch(e, err, "fp8_quantize_transposed");
 }
 
+fp8_status fp8_quantize_batched(const void* x_bf16, int32_t batch, int64_t rows, int64_t cols,
+                                int64_t ld_x, fp8_quant_recipe recipe, void* out_fp8,
+                                float* out_scales, fp8_stream_t stream) {
+  const std::string n("fp8_quantize_batched");
+  if (recipe < FP8_SCALE_TENSOR || recipe > FP8_SCALE_BLOCK_128x128)
+    return fail(FP8_ERR_VALUE, n + ": unknown recipe");
+  if (recipe != FP8_SCALE_BLOCK_128x128)
+    return fail(FP8_ERR_UNSUPPORTED, n + ": only the 128x128 recipe is implemented");
+  if (batch < 0 || batch > 65535 || rows < 0 || cols < 0)
+    return fail(FP8_ERR_VALUE, n + ": bad batch or size");
+  if (rows >= (int64_t(1) << 31) || cols >= (int64_t(1) << 31))
+    return fail(FP8_ERR_VALUE, n + ": size too large");
+  if (ld_x < cols) return fail(FP8_ERR_VALUE, n + ": ld_x < cols");
+  if (cols % 128 != 0 || ld_x % 8 != 0)
+    return fail(FP8_ERR_VALUE, n + ": cols % 128 == 0 and ld_x % 8 == 0 are required");
+  if (batch == 0 || rows == 0 || cols == 0) {
+    t_last_error.clear();
+    return FP8_OK;
+  }
+  if (x_bf16 == nullptr || out_fp8 == nullptr || out_scales == nullptr)
+    return fail(FP8_ERR_VALUE, n + ": null pointer");
+  if (!aligned(x_bf16, 16) || !aligned(out_fp8, 16) || !aligned(out_scales, 4))
+    return fail(FP8_ERR_VALUE, n + ": x and out_fp8 must be 16-byte aligned, out_scales 4");
+  DeviceInfo* d = nullptr;
+  fp8_status s = device_info(&d);
+  if (s != FP8_OK) return s;
+  std::string err;
+  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status, d->num_sms, &err};
+  cudaError_t e = fp8sm::launch_quantize_128x128_batched(x_bf16, batch, rows, cols, ld_x,
+                                                         out_fp8, out_scales, ctx);
+  return finish_launch(e, err, n.c_str());
+}
+
+fp8_status fp8_quantize_transposed_batched(const void* x_bf16, int32_t batch, int64_t rows,
+                                           int64_t cols, int64_t ld_x, fp8_quant_recipe recipe,
+                                           void* out_fp8, float* out_scales,
+                                           fp8_stream_t stream) {
+  const std::string n("fp8_quantize_transposed_batched");
+  if (recipe < FP8_SCALE_TENSOR || recipe > FP8_SCALE_BLOCK_128x128)
+    return fail(FP8_ERR_VALUE, n + ": unknown recipe");
+  if (recipe != FP8_SCALE_BLOCK_1x128 && recipe != FP8_SCALE_BLOCK_128x128)
+    return fail(FP8_ERR_UNSUPPORTED, n + ": only the 1x128 and 128x128 recipes are implemented");
+  if (batch < 0 || batch > 65535 || rows < 0 || cols < 0)
+    return fail(FP8_ERR_VALUE, n + ": bad batch or size");
+  if (rows >= (int64_t(1) << 31) || cols >= (int64_t(1) << 31))
+    return fail(FP8_ERR_VALUE, n + ": size too large");
+  if (ld_x < cols) return fail(FP8_ERR_VALUE, n + ": ld_x < cols");
+  if (cols % 8 != 0 || ld_x % 8 != 0)
+    return fail(FP8_ERR_VALUE, n + ": cols and ld_x must be multiples of 8");
+  if (rows % 128 != 0) return fail(FP8_ERR_VALUE, n + ": rows must be a multiple of 128");
+  if (batch == 0 || rows == 0 || cols == 0) {
+    t_last_error.clear();
+    return FP8_OK;
+  }
+  if (x_bf16 == nullptr || out_fp8 == nullptr || out_scales == nullptr)
+    return fail(FP8_ERR_VALUE, n + ": null pointer");
+  if (!aligned(x_bf16, 16) || !aligned(out_fp8, 16) || !aligned(out_scales, 4))
+    return fail(FP8_ERR_VALUE, n + ": x and out_fp8 must be 16-byte aligned, out_scales 4");
+  DeviceInfo* d = nullptr;
+  fp8_status s = device_info(&d);
+  if (s != FP8_OK) return s;
+  std::string err;
+  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status, d->num_sms, &err};
+  cudaError_t e = fp8sm::launch_quantize_transposed_batched(x_bf16, batch, rows, cols, ld_x,
+                                                            (int)recipe, out_fp8, out_scales, ctx);
+  return finish_launch(e, err, n.c_str());
+}
+
 fp8_status fp8_quantize_noalloc(const void* x_bf16, int64_t rows, int64_t cols,
                                 int64_t ld_x, fp8_quant_recipe recipe,
                                 void* out_fp8, float* out_scales,

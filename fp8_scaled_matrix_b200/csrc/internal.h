@@ -34,6 +34,19 @@ size_t mx_scale_tile_bytes(int64_t rows, int64_t cols);
 cudaError_t launch_quantize_mx(const void* x, int64_t rows, int64_t cols, int64_t ld,
                                void* q, void* sf, const LaunchCtx& ctx);
 
+// Batched quantization of `batch` equal (rows, cols) matrices stored one after
+// the other (row stride ld; matrix e at x + e * rows * ld), each quantized on
+// its own: 128x128 (codes (batch, rows, cols), scales (batch, cols/128,
+// ceil(rows/128))), and transposed 1x128 / 128x128 (recipe 2 / 3; codes
+// (batch, cols, rows), scales per matrix in the transposed layout; rows %
+// 128 == 0) (quantize.cu).
+cudaError_t launch_quantize_128x128_batched(const void* x, int32_t batch, int64_t rows,
+                                            int64_t cols, int64_t ld, void* q, float* scales,
+                                            const LaunchCtx& ctx);
+cudaError_t launch_quantize_transposed_batched(const void* x, int32_t batch, int64_t rows,
+                                               int64_t cols, int64_t ld, int recipe, void* q,
+                                               float* scales, const LaunchCtx& ctx);
+
 // Per-expert transposed 1x128 quantization (quantize.cu): x (rows = tokens,
 // cols) with groups of tokens by cumulative offs (device, E entries); the
 // output (cols, P) codes with P = grouped_padded_tokens(rows, E) hold each

@@ -312,6 +312,9 @@ __global__ void __launch_bounds__(256) quant_mx_kernel(
 // Ragged last row block: rows past the end take no part in the amax and are
 // not written.
 constexpr int k128Threads = 512;
+// Batched (blockIdx.y = matrix e of a stack of equal matrices, e.g. the
+// experts' weights): matrix e at x + e * rows * ld, its codes at
+// q + e * rows * cols, its scales at scales + e * (cols / 128) * ceil(rows / 128).
 __global__ void __launch_bounds__(k128Threads) quant_128x128_kernel(
     const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
     uint8_t* __restrict__ q, float* __restrict__ scales) {
@@ -320,6 +323,12 @@ __global__ void __launch_bounds__(k128Threads) quant_128x128_kernel(
   constexpr int kRounds = 128 / kRowStep;
   __shared__ float warp_amax[kWarps];
   const int64_t RB = (rows + 127) >> 7;
+  {
+    const int64_t e = blockIdx.y;
+    x += e * rows * ld;
+    q += e * rows * cols;
+    scales += e * (cols >> 7) * RB;
+  }
   const int64_t rb = blockIdx.x % RB;
   const int64_t kb = blockIdx.x / RB;
   const int t = threadIdx.x;
@@ -382,16 +391,21 @@ constexpr int kTrCtasPerSm = 2;
 // block mixes two groups; the padding is zero.  ldq = the output row stride.
 constexpr int kTrMaxGroups = 2048;
 
+// Batched (`batch` equal matrices, not grouped): matrix e at x + e * rows *
+// ld, its transposed codes at q + e * cols * ldq, its scales after the e
+// earlier matrices' scales; tiles are numbered matrix-major.
 template <bool k128x128, bool kGroupedT>
 __global__ void __launch_bounds__(kTrThreads) quant_transposed_kernel(
     const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
     uint8_t* __restrict__ q, float* __restrict__ scales, const int32_t* __restrict__ offs,
-    int32_t E, int64_t ldq, int64_t n_kb, uint32_t* status) {
+    int32_t E, int64_t ldq, int64_t n_kb, uint32_t* status, int32_t batch) {
   extern __shared__ __align__(16) uint16_t tiles_smem[];
   __shared__ float part[4][kTrCols];
   __shared__ float warp_amax[kTrThreads / 32];
   const int64_t n_cb = (cols + kTrCols - 1) / kTrCols;
-  const int64_t n_tiles = n_kb * n_cb;
+  const int64_t per_matrix = n_kb * n_cb;
+  const int64_t n_tiles = per_matrix * batch;
+  const int64_t scales_per_matrix = k128x128 ? n_kb * n_cb : n_kb * cols;
   const int t = threadIdx.x;
   int32_t* pb0 = nullptr;  // grouped: pb0[g] = padded blocks before group g; pb0[E] = total
   if constexpr (kGroupedT) {
@@ -455,6 +469,8 @@ __global__ void __launch_bounds__(kTrThreads) quant_transposed_kernel(
   // t / 16 + 32 i; columns past the end (and grouped: rows past the group)
   // are zero-filled (no effect on the max, zero codes)
   auto issue = [&](int64_t tile, int buf) {
+    const int64_t e = tile / per_matrix;
+    tile -= e * per_matrix;
     const int64_t kb = tile % n_kb, cb = tile / n_kb;
     if (kb >= n_kb_used) {
       cp_async_commit();
@@ -470,7 +486,7 @@ __global__ void __launch_bounds__(kTrThreads) quant_transposed_kernel(
     for (int i = 0; i < 4; ++i) {
       const int r = (t >> 4) + 32 * i;
       const bool in = col < cols && r < nrows;
-      cp_async_16(dst + r * kTrPitch + ch * 8, in ? x + (row0 + r) * ld + col : x,
+      cp_async_16(dst + r * kTrPitch + ch * 8, in ? x + e * rows * ld + (row0 + r) * ld + col : x,
                   in ? 16u : 0u);
     }
     cp_async_commit();
@@ -486,7 +502,10 @@ __global__ void __launch_bounds__(kTrThreads) quant_transposed_kernel(
     cp_async_wait<1>();              // this tile's copies have landed
     __syncthreads();
     const uint16_t* tl = tiles_smem + buf * kTrTileElems;
-    const int64_t kb = tile % n_kb, cb = tile / n_kb;
+    const int64_t e = tile / per_matrix;
+    const int64_t kb = (tile - e * per_matrix) % n_kb, cb = (tile - e * per_matrix) / n_kb;
+    float* const sc = scales + e * scales_per_matrix;
+    uint8_t* const qm = q + e * cols * ldq;
     if (kb >= n_kb_used) continue;   // grouped: past the last group's blocks (uniform)
     uint32_t w[16];                  // the 32 values, packed bf16 pairs
     float m = 0.0f;
@@ -513,9 +532,9 @@ __global__ void __launch_bounds__(kTrThreads) quant_transposed_kernel(
     const ScalePair sp = scales_from_amax(gm);
     const int64_t col = cb * kTrCols + c;
     if constexpr (k128x128) {
-      if (t == 0) scales[kb * n_cb + cb] = sp.s;
+      if (t == 0) sc[kb * n_cb + cb] = sp.s;
     } else {
-      if (qr == 0 && col < cols) scales[kb * cols + col] = sp.s;
+      if (qr == 0 && col < cols) sc[kb * cols + col] = sp.s;
     }
     uint8_t* stage = reinterpret_cast<uint8_t*>(tiles_smem + 2 * kTrTileElems);
     {
@@ -535,7 +554,7 @@ __global__ void __launch_bounds__(kTrThreads) quant_transposed_kernel(
       const int64_t ocol = cb * kTrCols + orow;
       if (ocol < cols) {
         const uint4* ss = reinterpret_cast<const uint4*>(stage + orow * kTrOutPitch + 32 * chunk);
-        uint4* dst = reinterpret_cast<uint4*>(q + ocol * ldq + kb * kTrRows + 32 * chunk);
+        uint4* dst = reinterpret_cast<uint4*>(qm + ocol * ldq + kb * kTrRows + 32 * chunk);
         dst[0] = ss[0];
         dst[1] = ss[1];
       }
@@ -686,10 +705,43 @@ cudaError_t launch_quantize_transposed(const void* xv, int64_t rows, int64_t col
   const unsigned grid = static_cast<unsigned>(tiles < max_grid ? tiles : max_grid);
   if (recipe == 3)
     quant_transposed_kernel<true, false><<<grid, kTrThreads, kTrSmemBytes, ctx.stream>>>(
-        x, rows, cols, ld, q, scales, nullptr, 0, rows, n_kb, ctx.status);
+        x, rows, cols, ld, q, scales, nullptr, 0, rows, n_kb, ctx.status, 1);
   else
     quant_transposed_kernel<false, false><<<grid, kTrThreads, kTrSmemBytes, ctx.stream>>>(
-        x, rows, cols, ld, q, scales, nullptr, 0, rows, n_kb, ctx.status);
+        x, rows, cols, ld, q, scales, nullptr, 0, rows, n_kb, ctx.status, 1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_transposed_batched(const void* xv, int32_t batch, int64_t rows,
+                                               int64_t cols, int64_t ld, int recipe, void* qv,
+                                               float* scales, const LaunchCtx& ctx) {
+  if (batch == 0 || rows == 0 || cols == 0) return cudaSuccess;
+  cudaError_t e = configure_transposed();
+  if (e != cudaSuccess) return e;
+  const int64_t n_kb = rows / kTrRows;
+  const int64_t tiles = n_kb * ((cols + kTrCols - 1) / kTrCols) * batch;
+  const int64_t max_grid = static_cast<int64_t>(ctx.num_sms) * kTrCtasPerSm;
+  const unsigned grid = static_cast<unsigned>(tiles < max_grid ? tiles : max_grid);
+  const uint16_t* x = static_cast<const uint16_t*>(xv);
+  uint8_t* q = static_cast<uint8_t*>(qv);
+  if (recipe == 3)
+    quant_transposed_kernel<true, false><<<grid, kTrThreads, kTrSmemBytes, ctx.stream>>>(
+        x, rows, cols, ld, q, scales, nullptr, 0, rows, n_kb, ctx.status, batch);
+  else
+    quant_transposed_kernel<false, false><<<grid, kTrThreads, kTrSmemBytes, ctx.stream>>>(
+        x, rows, cols, ld, q, scales, nullptr, 0, rows, n_kb, ctx.status, batch);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_128x128_batched(const void* xv, int32_t batch, int64_t rows,
+                                            int64_t cols, int64_t ld, void* qv, float* scales,
+                                            const LaunchCtx& ctx) {
+  if (batch == 0 || rows == 0 || cols == 0) return cudaSuccess;
+  const int64_t tiles = ((rows + 127) / 128) * (cols / 128);
+  quant_128x128_kernel<<<dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(batch)),
+                         k128Threads, 0, ctx.stream>>>(static_cast<const uint16_t*>(xv), rows,
+                                                       cols, ld, static_cast<uint8_t*>(qv),
+                                                       scales);
   return cudaGetLastError();
 }
 
@@ -710,7 +762,7 @@ cudaError_t launch_quantize_transposed_grouped(const void* xv, int64_t rows, int
   const unsigned grid = static_cast<unsigned>(tiles < max_grid ? tiles : max_grid);
   quant_transposed_kernel<false, true><<<grid, kTrThreads, kTrSmemBytes, ctx.stream>>>(
       static_cast<const uint16_t*>(xv), rows, cols, ld, static_cast<uint8_t*>(qv), scales,
-      offs, E, P, n_kb, ctx.status);
+      offs, E, P, n_kb, ctx.status, 1);
   return cudaGetLastError();
 }
 

@@ -38,7 +38,8 @@ EXPORTED = ["fp8_version", "fp8_last_error", "fp8_quantize_workspace_bytes",
             "fp8_mx_scale_bytes", "fp8_quantize_mx", "fp8_scaled_mm_mx",
             "fp8_scaled_mm_mx_quantized", "fp8_grouped_scaled_mm_mx",
             "fp8_grouped_padded_tokens", "fp8_quantize_transposed_grouped",
-            "fp8_grouped_scaled_mm_wgrad"]
+            "fp8_grouped_scaled_mm_wgrad", "fp8_quantize_batched",
+            "fp8_quantize_transposed_batched"]
 
 
 class Fp8Error(RuntimeError):
@@ -97,6 +98,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fp8_scaled_mm_quantized.argtypes = [P, P, I64, I64, I64, P, P, E, P, P, P, P]
     L.fp8_grouped_scaled_mm.restype = E
     L.fp8_grouped_scaled_mm.argtypes = [P, P, I64, I64, I64, I32, P, P, P, E, P, P]
+    L.fp8_quantize_batched.restype = E
+    L.fp8_quantize_batched.argtypes = [P, I32, I64, I64, I64, E, P, P, P]
+    L.fp8_quantize_transposed_batched.restype = E
+    L.fp8_quantize_transposed_batched.argtypes = [P, I32, I64, I64, I64, E, P, P, P]
     L.fp8_grouped_padded_tokens.restype = I64
     L.fp8_grouped_padded_tokens.argtypes = [I64, I32]
     L.fp8_quantize_transposed_grouped.restype = E
@@ -521,3 +526,46 @@ def fp8_grouped_scaled_mm_wgrad(a_t: torch.Tensor, b_t: torch.Tensor, scale_a: t
                                          _ptr(scale_b), _ptr(offs), od, _ptr(out),
                                          _stream(stream)))
     return out
+
+
+def fp8_quantize_batched(x: torch.Tensor, recipe: int, out: Optional[torch.Tensor] = None,
+                         scales: Optional[torch.Tensor] = None,
+                         stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """128x128 quantization of each matrix of a contiguous (B, rows, cols)
+    bf16 stack in one launch: returns (codes (B, rows, cols), scales
+    (B, cols/128, ceil(rows/128)))."""
+    L = load_library()
+    _need_cuda(x)
+    if x.dtype != torch.bfloat16 or x.dim() != 3 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous (B, rows, cols) bf16 tensor")
+    B, rows, cols = x.shape
+    if out is None:
+        out = torch.empty((B, rows, cols), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((B, cols // 128, (rows + 127) // 128), dtype=torch.float32,
+                             device=x.device)
+    _check(L.fp8_quantize_batched(_ptr(x), B, rows, cols, cols, recipe, _ptr(out), _ptr(scales),
+                                  _stream(stream)))
+    return out, scales
+
+
+def fp8_quantize_transposed_batched(x: torch.Tensor, recipe: int,
+                                    out: Optional[torch.Tensor] = None,
+                                    scales: Optional[torch.Tensor] = None,
+                                    stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """1x128 / 128x128 quantization of each matrix's transpose for a
+    contiguous (B, rows, cols) bf16 stack: returns (codes (B, cols, rows),
+    scales, each matrix's fp8_quantize_transposed layout in order)."""
+    L = load_library()
+    _need_cuda(x)
+    if x.dtype != torch.bfloat16 or x.dim() != 3 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous (B, rows, cols) bf16 tensor")
+    B, rows, cols = x.shape
+    per = scale_count(cols, rows, recipe)
+    if out is None:
+        out = torch.empty((B, cols, rows), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((B, per), dtype=torch.float32, device=x.device)
+    _check(L.fp8_quantize_transposed_batched(_ptr(x), B, rows, cols, cols, recipe, _ptr(out),
+                                             _ptr(scales), _stream(stream)))
+    return out, scales

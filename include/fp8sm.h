@@ -187,6 +187,31 @@ FP8SM_API fp8_status fp8_quantize_transposed(const void* x_bf16, int64_t rows,
                                              float* out_scales, fp8_stream_t stream);
 
 /*
+ * Batched quantization of `batch` equal matrices stored one after the other
+ * (matrix e = rows x cols at x_bf16 + e * rows * ld_x, e.g. the (E, N, K)
+ * expert weights of [P2]), each quantized on its own, in one launch: the
+ * same codes and scales as `batch` separate calls.
+ *
+ * fp8_quantize_batched: 128x128 only.  out_fp8 (batch, rows, cols);
+ *   out_scales (batch, cols/128, ceil(rows/128)) -- each matrix's fp8_quantize
+ *   layout, matrices in order (the per-expert layout
+ *   fp8_grouped_scaled_mm_blockwise reads).  cols % 128 == 0.
+ * fp8_quantize_transposed_batched: 1x128 or 128x128 of each matrix's
+ *   transpose.  out_fp8 (batch, cols, rows); out_scales: each matrix's
+ *   fp8_quantize_transposed layout, matrices in order.  rows % 128 == 0.
+ * 1 <= batch <= 65535 (batch == 0 is a no-op); other requirements and
+ * errors as the single-matrix calls.
+ */
+FP8SM_API fp8_status fp8_quantize_batched(const void* x_bf16, int32_t batch, int64_t rows,
+                                int64_t cols, int64_t ld_x, fp8_quant_recipe recipe,
+                                void* out_fp8, float* out_scales, fp8_stream_t stream);
+
+FP8SM_API fp8_status fp8_quantize_transposed_batched(const void* x_bf16, int32_t batch,
+                                           int64_t rows, int64_t cols, int64_t ld_x,
+                                           fp8_quant_recipe recipe, void* out_fp8,
+                                           float* out_scales, fp8_stream_t stream);
+
+/*
  * Scaled GEMM ([P1] forward; [P4] recipes; [P5] blockwise recipes):
  *   out[m, n] = sum_k (a[m,k] * sA) * (b[n,k] * sB)  (+ bias[n])
  * with the scales picked per recipe (see fp8_mm_recipe).  Products are

@@ -295,3 +295,27 @@ def test_grouped_wgrad_rejects_bad_arguments(lib, M, N, T, E, frag):
     st = lib.fp8_grouped_scaled_mm_wgrad(FAKE, FAKE, M, N, T, E, FAKE, FAKE, FAKE,
                                          fp8sm.FP8_OUT_BF16, FAKE, None)
     assert st == fp8sm.FP8_ERR_VALUE and frag in lib.fp8_last_error().decode()
+
+
+@pytest.mark.parametrize("fn,args,status,frag", [
+    ("fp8_quantize_batched", (FAKE, 2, 128, 100, 100, fp8sm.FP8_SCALE_BLOCK_128x128),
+     fp8sm.FP8_ERR_VALUE, "cols % 128"),
+    ("fp8_quantize_batched", (FAKE, 2, 128, 128, 128, fp8sm.FP8_SCALE_BLOCK_1x128),
+     fp8sm.FP8_ERR_UNSUPPORTED, "only the 128x128"),
+    ("fp8_quantize_batched", (FAKE, -1, 128, 128, 128, fp8sm.FP8_SCALE_BLOCK_128x128),
+     fp8sm.FP8_ERR_VALUE, "bad batch"),
+    ("fp8_quantize_transposed_batched", (FAKE, 2, 100, 128, 128, fp8sm.FP8_SCALE_BLOCK_1x128),
+     fp8sm.FP8_ERR_VALUE, "rows must be a multiple of 128"),
+    ("fp8_quantize_transposed_batched", (FAKE, 2, 128, 128, 128, fp8sm.FP8_SCALE_ROW),
+     fp8sm.FP8_ERR_UNSUPPORTED, "only the 1x128 and 128x128"),
+])
+def test_batched_quantize_rejects_bad_arguments(lib, fn, args, status, frag):
+    st = getattr(lib, fn)(*args, FAKE, FAKE, None)
+    assert st == status and frag in lib.fp8_last_error().decode()
+
+
+def test_batched_quantize_empty_is_a_noop(lib):
+    assert lib.fp8_quantize_batched(None, 0, 128, 128, 128, fp8sm.FP8_SCALE_BLOCK_128x128,
+                                    None, None, None) == fp8sm.FP8_OK
+    assert lib.fp8_quantize_transposed_batched(None, 3, 0, 128, 128, fp8sm.FP8_SCALE_BLOCK_1x128,
+                                               None, None, None) == fp8sm.FP8_OK
