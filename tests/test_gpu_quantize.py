@@ -37,6 +37,8 @@ def run_both(x_cpu: torch.Tensor, recipe: str, ld_pad: int = 0):
     ("row", 64, 1000), ("1x128", 301, 384), ("1x128", 7, 1152), ("1x128", 4, 128),
     ("128x128", 300, 640), ("128x128", 128, 128), ("128x128", 1, 256),
     ("tensor", 256, 256), ("tensor", 3000, 1000), ("tensor", 1, 8), ("tensor", 700, 4096),
+    # the single-CTA tensorwise path holds up to 8192 8-element vectors
+    ("tensor", 64, 1024), ("tensor", 257, 256), ("tensor", 1, 65536),
 ])
 def test_quantize_parity_random(recipe, rows, cols):
     g = W.generator(rows * 7 + cols)
