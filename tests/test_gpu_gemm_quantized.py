@@ -214,3 +214,40 @@ def test_linear_chain_against_oracle():
     err = got - exact
     sqnr = 10 * np.log10((exact ** 2).sum() / (err ** 2).sum())
     assert sqnr >= 20.0, sqnr
+
+
+def test_linear_chain_backward_grad_input_against_oracle():
+    """The chain's backward through the grad_input GEMMs ("improve fp8 blockwise
+    gemm perf": grad_input = grad_output @ weight, 1x128_128x128): dY2 ->
+    dY1 = dY2 @ W2 with dY1 quantized 1x128 in that GEMM's epilogue -> dX =
+    dY1 @ W1, each weight quantized transposed (128x128); sampled rows against
+    the oracle's chain (1x128 quantize, fp64 GEMM rounded to fp32, 1x128
+    quantize, fp64 GEMM) and SQNR >= 20 dB against the unquantized product."""
+    wl = W.make_workload(8)          # X (T, 8192), W1 (5120, 8192), W2 (8192, 5120)
+    f = fp8sm
+    g = W.generator(88)
+    T = wl.M
+    dy2 = W.randn_bf16((T, 8192), 1.0, g)
+    w1, w2 = wl.b, wl.extra["b2"]
+    r = f.FP8_MM_1x128_128x128
+    qd, sd = f.fp8_quantize(dy2.cuda(), f.FP8_SCALE_BLOCK_1x128)
+    q2t, s2t = f.fp8_quantize_transposed(w2.cuda(), f.FP8_SCALE_BLOCK_128x128)   # W2^T (5120, 8192)
+    q1t, s1t = f.fp8_quantize_transposed(w1.cuda(), f.FP8_SCALE_BLOCK_128x128)   # W1^T (8192, 5120)
+    dy1q, dy1s = f.fp8_scaled_mm_quantized(qd, q2t, sd, s2t, r)                  # (T, 5120)
+    dx = f.fp8_scaled_mm(dy1q, q1t, dy1s, s1t, r, out_dtype=torch.float32)       # (T, 8192)
+    torch.cuda.synchronize()
+    f.check_device_status()
+    rows = sample_rows(T, 32, seed=18)
+    G = oracle.GROUP_128x128
+    oqd, osd = oracle.quantize(W.bf16_bits(dy2), oracle.GROUP_1x128)
+    oq2t, os2t = oracle.quantize(np.ascontiguousarray(W.bf16_bits(w2).T), G)
+    oq1t, os1t = oracle.quantize(np.ascontiguousarray(W.bf16_bits(w1).T), G)
+    y1, _ = oracle.scaled_mm(oqd, oq2t, osd, os2t, oracle.MM_1x128_128x128, rows=rows)
+    oy1q, oy1s = oracle.quantize_f32(y1.astype(np.float32), oracle.GROUP_1x128)
+    ref, mag = oracle.scaled_mm(oy1q, oq1t, oy1s, os1t, oracle.MM_1x128_128x128)
+    got = dx.cpu().numpy().astype(np.float64)[rows]
+    ok = oracle.within_tolerance(got, ref, mag)
+    assert ok.all(), f"backward chain: {int((~ok).sum())} of {ok.size} out of tolerance"
+    exact = (dy2.double().numpy()[rows] @ w2.double().numpy()) @ w1.double().numpy()
+    err = got - exact
+    assert 10 * np.log10((exact ** 2).sum() / (err ** 2).sum()) >= 20.0
