@@ -429,6 +429,45 @@ fp8_status fp8_scaled_mm_mx(const void* a, const void* b, int64_t M, int64_t N, 
   return finish_launch(e, err, "fp8_scaled_mm_mx");
 }
 
+fp8_status fp8_scaled_mm_quantized_dual(const void* a, const void* b, int64_t M, int64_t N,
+                                        int64_t K, const float* scale_a, const float* scale_b,
+                                        fp8_mm_recipe recipe, const void* bias_bf16,
+                                        void* out_fp8, float* out_scales, void* out_t_fp8,
+                                        float* out_t_scales, fp8_stream_t stream) {
+  const std::string n("fp8_scaled_mm_quantized_dual");
+  if (recipe < FP8_MM_TENSOR_TENSOR || recipe > FP8_MM_1x128_128x1)
+    return fail(FP8_ERR_VALUE, n + ": unknown recipe");
+  if (recipe != FP8_MM_1x128_128x128)
+    return fail(FP8_ERR_UNSUPPORTED, n + ": only the 1x128_128x128 recipe is implemented");
+  if (M < 0 || N < 0 || K < 0) return fail(FP8_ERR_VALUE, n + ": negative size");
+  if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+    return fail(FP8_ERR_VALUE, n + ": size too large");
+  if (K == 0 || K % 128 != 0)
+    return fail(FP8_ERR_VALUE, n + ": K must be a positive multiple of 128");
+  if (M % 128 != 0 || N % 128 != 0)
+    return fail(FP8_ERR_VALUE, n + ": M and N must be multiples of 128");
+  if (M == 0 || N == 0) {
+    t_last_error.clear();
+    return FP8_OK;
+  }
+  if (a == nullptr || b == nullptr || scale_a == nullptr || scale_b == nullptr ||
+      out_fp8 == nullptr || out_scales == nullptr || out_t_fp8 == nullptr ||
+      out_t_scales == nullptr)
+    return fail(FP8_ERR_VALUE, n + ": null pointer");
+  if (!aligned(out_fp8, 16) || !aligned(out_t_fp8, 16) || !aligned(a, 16) || !aligned(b, 16) ||
+      (bias_bf16 && !aligned(bias_bf16, 16)) || !aligned(scale_a, 16) || !aligned(scale_b, 16) ||
+      !aligned(out_scales, 4) || !aligned(out_t_scales, 4))
+    return fail(FP8_ERR_VALUE, n + ": misaligned pointer");
+  DeviceInfo* d = nullptr;
+  fp8_status s = device_info(&d);
+  if (s != FP8_OK) return s;
+  std::string err;
+  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status, d->num_sms, &err};
+  cudaError_t e = fp8sm::launch_scaled_mm(a, b, M, N, K, scale_a, scale_b, (int)recipe, bias_bf16,
+                                          4, out_fp8, out_scales, ctx, out_t_fp8, out_t_scales);
+  return finish_launch(e, err, n.c_str());
+}
+
 fp8_status fp8_scaled_mm_mx_quantized(const void* a, const void* b, int64_t M, int64_t N,
                                       int64_t K, const void* scale_a_e8m0,
                                       const void* scale_b_e8m0, const void* bias_bf16,

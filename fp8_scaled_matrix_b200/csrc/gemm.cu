@@ -104,8 +104,8 @@ struct Cfg {
   static constexpr uint32_t kOffScl = kOffEpi + kEpiWarps * kEpiBuf;
   static constexpr uint32_t kOffBar = kOffScl + kSclBytes;
   // barriers: full[kStages], empty[kStages], acc_full[2], acc_empty[2], drain,
-  // scale ring sfull[kSclSlots], sempty[kSclSlots]
-  static constexpr uint32_t kNumBars = 2 * kStages + 5 + 2 * kSclSlots;
+  // scale ring sfull[kSclSlots], sempty[kSclSlots], epilogue half sync hsync[2]
+  static constexpr uint32_t kNumBars = 2 * kStages + 5 + 2 * kSclSlots + 2;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
   static constexpr uint32_t kSmemUsed = kOffMisc + 16;
   static constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // + alignment slack
@@ -117,8 +117,10 @@ struct Cfg {
 enum Recipe : int { kTensor = 0, kRow = 1, kBlock128 = 2, kBlock1 = 3, kMxfp8 = 4 };
 // Output: bf16, fp32, e4m3 quantized in 1x128 groups along n (+ fp32
 // scales), or MXFP8 (e4m3 + one E8M0 scale per 32 columns, in scale-factor
-// tiles: the A operand of the next MXFP8 GEMM)
-enum OutKind : int { kOutBf16 = 0, kOutFp32 = 1, kOutE4M3 = 2, kOutMx = 3 };
+// tiles: the A operand of the next MXFP8 GEMM), or both e4m3 forms of the
+// result (1x128 along n, and transposed with 1x128 groups along m: the two
+// operands the next layer's backward GEMMs read)
+enum OutKind : int { kOutBf16 = 0, kOutFp32 = 1, kOutE4M3 = 2, kOutMx = 3, kOutE4M3Dual = 4 };
 
 struct GemmParams {
   int64_t M, N, K;
@@ -130,6 +132,8 @@ struct GemmParams {
   const uint16_t* bias;
   void* out;
   float* out_scales;  // e4m3 output: scale[(n/128) * M + m]; MXFP8 output: tiles
+  uint8_t* out_t;      // dual e4m3 output: the result transposed, (N, M) codes
+  float* out_t_scales; //   and its scales, 1x128 along m: scale[(m/128) * N + n]
   const int32_t* offs;
   int32_t E;
   int64_t tokens;    // K-grouped (weight gradient): offs[E-1] must equal this
@@ -406,7 +410,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // (with it, a dense MXFP8 build faulted on the GPU; see the design notes).
   constexpr bool kBigEpi = kBlockwise;
   constexpr bool kOutF32 = kOut == kOutFp32;
-  constexpr bool kOutQ = kOut == kOutE4M3;
+  constexpr bool kOutQT = kOut == kOutE4M3Dual;
+  constexpr bool kOutQ = kOut == kOutE4M3 || kOutQT;
   constexpr bool kOutMxq = kOut == kOutMx;
   using C = Cfg<kPair>;
   extern __shared__ uint8_t smem_raw[];
@@ -420,6 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = bars + 2 * C::kStages + 4;
   uint64_t* sfull = bars + 2 * C::kStages + 5;
   uint64_t* sempty = sfull + kSclSlots;
+  uint64_t* hsync = sempty + kSclSlots;  // the four epilogue warps of each half
   float* scl = reinterpret_cast<float*>(smem + C::kOffScl);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   uint32_t* tmem_slot = misc + 0;
@@ -445,6 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sfull[i], 32);            // one cp.async arrival per lane of warp 2
       mbar_init(&sempty[i], kEpiWarps);
     }
+    for (int i = 0; i < 2; ++i) mbar_init(&hsync[i], kEpiWarps / 2);
     *abort_flag = 0u;
     fence_barrier_init();
     prefetch_tmap(&tm_a);
@@ -926,6 +933,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         kPair ? mapa_shared(smem_u32(&acc_empty[1]), 0) : smem_u32(&acc_empty[1]);
     // Single CTA: a CTA-scope arrive.  Pair: the leader's barrier, at cluster
     // scope (a cluster-scope release costs a fence, so it is used only there).
+    // the four warps of this warp's half meet (bounded; dual e4m3 output)
+    uint32_t hphase = 0;
+    auto half_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&hsync[half]);
+      const bool done = mbar_wait(&hsync[half], hphase, abort_flag, p.status, SITE_EPI_ACC_FULL,
+                                  kWaitLimitNs);
+      hphase ^= 1u;
+      return done;
+    };
     auto release_acc = [&](uint32_t a) {
       if constexpr (kPair) mbar_arrive_cluster(a ? acc_empty_addr1 : acc_empty_addr0);
       else mbar_arrive(&acc_empty[a]);
@@ -1219,6 +1236,104 @@ __global__ void __launch_bounds__(kThreads, 1)
             store_box64<kMasked>(ebuf, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
                                   row0, c.row_end, static_cast<uint8_t*>(p.out), p.N, 1, lane);
           }
+          if constexpr (kOutQT) {
+            // The transposed e4m3 form: for each of this half's 128 columns,
+            // the tile's 128 rows are one 1x128 group along m.  (1) Column
+            // amax over the warp's 32 rows by a butterfly over the lanes
+            // (lane L ends with column 32 cc + L); (2) the four warps of the
+            // half meet through their staging buffers (a bounded mbarrier
+            // per half); (3) codes staged column-major, 64 columns at a time, in
+            // the half's 8 KB of staging buffers and written out as rows of
+            // the transposed matrix.
+            uint8_t* const half_stage = smem + C::kOffEpi + half * 4 * kEpiBuf;
+            float cmax[4];
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              float v[32];
+              result32(cc, v);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] = fabsf(v[i]);
+#pragma unroll
+              for (int sh = 16; sh >= 1; sh >>= 1) {
+                const bool upper = (lane & sh) != 0;
+#pragma unroll
+                for (int k = 0; k < sh; ++k) {
+                  const float send = upper ? v[k] : v[k + sh];
+                  const float keep = upper ? v[k + sh] : v[k];
+                  v[k] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, sh));
+                }
+              }
+              cmax[cc] = v[0];
+            }
+            // this warp's staging buffer is free once its TMA stores have read it
+            if (lane == 0) bulk_wait_group_read0();
+            __syncwarp();
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc)
+              reinterpret_cast<float*>(ebuf)[cc * 32 + lane] = cmax[cc];
+            if (!half_sync()) {
+              ok = false;
+              break;
+            }
+            float inv[4];
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              float am = 0.0f;
+#pragma unroll
+              for (int w = 0; w < 4; ++w)
+                am = fmaxf(am, reinterpret_cast<const float*>(half_stage + w * kEpiBuf)[cc * 32 + lane]);
+              const ScalePair sp = scales_from_amax(am);
+              inv[cc] = sp.inv;
+              const int64_t n = ncol0 + 32 * cc + lane;
+              if (q == 0 && n < p.N) p.out_t_scales[(cta_m0 / 128) * p.N + n] = sp.s;
+            }
+            if (!half_sync()) {  // every warp has read the maxima
+              ok = false;
+              break;
+            }
+            const uint32_t r = q * 32 + lane;   // this thread's row within the tile
+#pragma unroll
+            for (int pass = 0; pass < 2 && ok; ++pass) {
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int cc = 2 * pass + h;
+                float v[32];
+                result32(cc, v);
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                  const float i0 = __shfl_sync(0xFFFFFFFFu, inv[cc], i);
+                  const float i1 = __shfl_sync(0xFFFFFFFFu, inv[cc], i + 1);
+                  const uint32_t two = static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(
+                      make_float2(__fmul_rn(v[i], i0), __fmul_rn(v[i + 1], i1)), __NV_SATFINITE,
+                      __NV_E4M3));
+                  const int j = h * 32 + i;  // column within the pass
+                  half_stage[j * 128 + r] = static_cast<uint8_t>(two & 0xFFu);
+                  half_stage[(j + 1) * 128 + r] = static_cast<uint8_t>(two >> 8);
+                }
+              }
+              if (!half_sync()) {
+                ok = false;
+                break;
+              }
+              {
+                // 128 threads: row j = tid / 2 of the pass, 64 bytes each
+                const uint32_t tid = q * 32 + lane;
+                const int j = static_cast<int>(tid >> 1);
+                const int64_t n = ncol0 + 64 * pass + j;
+                if (n < p.N) {
+                  const uint4* src = reinterpret_cast<const uint4*>(half_stage + j * 128 + 64 * (tid & 1));
+                  uint4* dst = reinterpret_cast<uint4*>(p.out_t + n * p.M + cta_m0 + 64 * (tid & 1));
+#pragma unroll
+                  for (int u = 0; u < 4; ++u) dst[u] = src[u];
+                }
+              }
+              if (!half_sync()) {  // the staging is read before it is refilled
+                ok = false;
+                break;
+              }
+            }
+            if (!ok) break;
+          }
         }
       }
     }
@@ -1314,6 +1429,8 @@ cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb,
     return cudaErrorInvalidValue;  // MXFP8: single CTAs; bf16/fp32 out (dense: also MXFP8)
   } else if constexpr (kOut == kOutMx && kRecipe != kMxfp8) {
     return cudaErrorInvalidValue;  // MXFP8 output from the MXFP8 GEMM only
+  } else if constexpr (kOut == kOutE4M3Dual && (kRecipe != kBlock128 || kGrouped || kPair)) {
+    return cudaErrorInvalidValue;  // dual e4m3 output: dense 1x128_128x128 only
   } else if constexpr (kOut == kOutE4M3 && (kPair || kGrouped)) {
     return cudaErrorInvalidValue;  // quantized output: single-CTA dense GEMM only
   } else {
@@ -1362,6 +1479,8 @@ cudaError_t dispatch(int recipe, int out_kind, bool pair, const CUtensorMap& ta,
       return launch_kernel<R, kOutE4M3, kGrouped, false>(ta, tb, tbh, to, p, grid, st); \
     if (out_kind == kOutMx)                                                             \
       return launch_kernel<R, kOutMx, kGrouped, false>(ta, tb, tbh, to, p, grid, st);   \
+    if (out_kind == kOutE4M3Dual)                                                       \
+      return launch_kernel<R, kOutE4M3Dual, kGrouped, false>(ta, tb, tbh, to, p, grid, st); \
     if (pair)                                                                           \
       return out_kind ? launch_kernel<R, kOutFp32, kGrouped, true>(ta, tb, tbh, to, p, grid, st) \
                       : launch_kernel<R, kOutBf16, kGrouped, true>(ta, tb, tbh, to, p, grid, st); \
@@ -1388,7 +1507,7 @@ cudaError_t dispatch(int recipe, int out_kind, bool pair, const CUtensorMap& ta,
 // staging layout) for bf16, fp32 or e4m3 output.
 bool out_map(CUtensorMap* m, void* out, int64_t rows, int64_t N, int out_kind,
              std::string* err) {
-  const bool q8 = out_kind == kOutE4M3 || out_kind == kOutMx;
+  const bool q8 = out_kind == kOutE4M3 || out_kind == kOutMx || out_kind == kOutE4M3Dual;
   const uint64_t eb = out_kind == kOutFp32 ? 4 : q8 ? 1 : 2;
   uint64_t dims[2] = {static_cast<uint64_t>(N), static_cast<uint64_t>(rows)};
   uint64_t strides[1] = {static_cast<uint64_t>(N) * eb};
@@ -1428,9 +1547,10 @@ cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
                              int64_t N, int64_t K, const float* sa,
                              const float* sb, int recipe, const void* bias,
                              int out_kind, void* out, float* out_scales,
-                             const LaunchCtx& ctx) {
+                             const LaunchCtx& ctx, void* out_t, float* out_t_scales) {
   if (M == 0 || N == 0) return cudaSuccess;
-  if (K == 0 && (out_kind == kOutE4M3 || out_kind == kOutMx)) return cudaErrorInvalidValue;
+  if (K == 0 && (out_kind == kOutE4M3 || out_kind == kOutMx || out_kind == kOutE4M3Dual))
+    return cudaErrorInvalidValue;
   const int out_f32 = out_kind == kOutFp32;
   if (K == 0) {
     const int64_t total = M * N;
@@ -1463,6 +1583,8 @@ cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
   if (!out_map(&to, out, M, N, out_kind, ctx.err)) return cudaErrorInvalidValue;
   GemmParams p{};
   p.out_scales = out_scales;
+  p.out_t = static_cast<uint8_t*>(out_t);
+  p.out_t_scales = out_t_scales;
   p.M = M;
   p.N = N;
   p.K = K;

@@ -67,12 +67,16 @@ cudaError_t noalloc_scratch_ptr(int device, void** out);
 // 3 1x128_128x1, 4 MXFP8 (sa, sb then point to E8M0 scale-factor tiles).
 // out_kind: 0 bf16, 1 fp32, 2 e4m3 quantized in 1x128 groups along n with
 // fp32 scales written to out_scales[(n/128) * M + m], 3 MXFP8 (recipe 4
-// only; E8M0 scale-factor tiles written to out_scales as bytes).
+// only; E8M0 scale-factor tiles written to out_scales as bytes), 4 both
+// e4m3 forms (recipe 2 only, M % 128 == 0): out / out_scales as for 2, and
+// the result transposed in out_t (N, M) with 1x128-along-m scales
+// out_t_scales[(m/128) * N + n].
 cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
                              int64_t N, int64_t K, const float* sa,
                              const float* sb, int recipe, const void* bias,
                              int out_kind, void* out, float* out_scales,
-                             const LaunchCtx& ctx);
+                             const LaunchCtx& ctx, void* out_t = nullptr,
+                             float* out_t_scales = nullptr);
 
 // Grouped scaled GEMM (gemm.cu).  recipe: 1 rowwise, 2 1x128_128x128.
 cudaError_t launch_grouped_scaled_mm(const void* a, const void* b,

@@ -39,7 +39,7 @@ EXPORTED = ["fp8_version", "fp8_last_error", "fp8_quantize_workspace_bytes",
             "fp8_scaled_mm_mx_quantized", "fp8_grouped_scaled_mm_mx",
             "fp8_grouped_padded_tokens", "fp8_quantize_transposed_grouped",
             "fp8_grouped_scaled_mm_wgrad", "fp8_quantize_batched",
-            "fp8_quantize_transposed_batched"]
+            "fp8_quantize_transposed_batched", "fp8_scaled_mm_quantized_dual"]
 
 
 class Fp8Error(RuntimeError):
@@ -98,6 +98,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fp8_scaled_mm_quantized.argtypes = [P, P, I64, I64, I64, P, P, E, P, P, P, P]
     L.fp8_grouped_scaled_mm.restype = E
     L.fp8_grouped_scaled_mm.argtypes = [P, P, I64, I64, I64, I32, P, P, P, E, P, P]
+    L.fp8_scaled_mm_quantized_dual.restype = E
+    L.fp8_scaled_mm_quantized_dual.argtypes = [P, P, I64, I64, I64, P, P, E, P, P, P, P, P, P]
     L.fp8_quantize_batched.restype = E
     L.fp8_quantize_batched.argtypes = [P, I32, I64, I64, I64, E, P, P, P]
     L.fp8_quantize_transposed_batched.restype = E
@@ -569,3 +571,25 @@ def fp8_quantize_transposed_batched(x: torch.Tensor, recipe: int,
     _check(L.fp8_quantize_transposed_batched(_ptr(x), B, rows, cols, cols, recipe, _ptr(out),
                                              _ptr(scales), _stream(stream)))
     return out, scales
+
+
+def fp8_scaled_mm_quantized_dual(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor,
+                                 scale_b: torch.Tensor, recipe: int,
+                                 bias: Optional[torch.Tensor] = None, stream=None):
+    """GEMM writing both e4m3 forms of its result: returns (codes (M, N),
+    scales (N/128, M), transposed codes (N, M), transposed scales (M/128, N))."""
+    L = load_library()
+    _need_cuda(a, b, scale_a, scale_b, bias)
+    M, K = a.shape
+    N = b.shape[0]
+    if b.shape[1] != K:
+        raise ValueError("a and b must share K")
+    dev = a.device
+    out = torch.empty((M, N), dtype=torch.uint8, device=dev)
+    sc = torch.empty((N // 128, M), dtype=torch.float32, device=dev)
+    out_t = torch.empty((N, M), dtype=torch.uint8, device=dev)
+    sc_t = torch.empty((M // 128, N), dtype=torch.float32, device=dev)
+    _check(L.fp8_scaled_mm_quantized_dual(_ptr(a), _ptr(b), M, N, K, _ptr(scale_a),
+                                          _ptr(scale_b), recipe, _ptr(bias), _ptr(out), _ptr(sc),
+                                          _ptr(out_t), _ptr(sc_t), _stream(stream)))
+    return out, sc, out_t, sc_t

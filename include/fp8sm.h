@@ -262,6 +262,29 @@ FP8SM_API fp8_status fp8_scaled_mm_quantized(const void* a, const void* b, int64
                                    float* out_scales, fp8_stream_t stream);
 
 /*
+ * Scaled GEMM that writes both e4m3 forms of its result, for the backward of
+ * a chain of FP8 linears ([P1] Solution, backward pass; [P5]: grad_input
+ * with 1x128_128x128, grad_weight with 1x128_128x1): with y the fp32 result
+ * of fp8_scaled_mm (bias added),
+ *   out_fp8, out_scales     = fp8_scaled_mm_quantized's output: y in 1x128
+ *                             groups along n (the next grad_input's operand)
+ *   out_t_fp8 (N, M), out_t_scales (M/128, N)
+ *                           = y^T quantized with 1x128 groups along m, i.e.
+ *                             fp8_quantize_transposed(y, 1x128) of the fp32
+ *                             values (the next grad_weight's operand):
+ *                             scale[(m/128) * N + n], codes row n = tokens.
+ * Recipe FP8_MM_1x128_128x128 only (others: FP8_ERR_UNSUPPORTED).
+ * Requirements: M % 128 == 0, N % 128 == 0, K > 0, K % 128 == 0; code
+ * buffers 16-byte aligned, scales 4-byte aligned.
+ */
+FP8SM_API fp8_status fp8_scaled_mm_quantized_dual(const void* a, const void* b, int64_t M,
+                                        int64_t N, int64_t K, const float* scale_a,
+                                        const float* scale_b, fp8_mm_recipe recipe,
+                                        const void* bias_bf16, void* out_fp8,
+                                        float* out_scales, void* out_t_fp8,
+                                        float* out_t_scales, fp8_stream_t stream);
+
+/*
  * MXFP8 ("mxfp8" in the recipe table of [P4]; the pages name the recipe but
  * do not define it, so the OCP Microscaling (MX) specification's definition
  * is used): one power-of-two E8M0 scale per block of 32 consecutive elements

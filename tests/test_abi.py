@@ -157,6 +157,37 @@ def test_scaled_mm_quantized_null_alignment_and_empty(lib):
                                        None) == fp8sm.FP8_OK
 
 
+@pytest.mark.parametrize("M,N,K,recipe,status,frag", [
+    (128, 128, 128, fp8sm.FP8_MM_ROW_ROW, fp8sm.FP8_ERR_UNSUPPORTED, "1x128_128x128"),
+    (128, 128, 128, 9, fp8sm.FP8_ERR_VALUE, "unknown recipe"),
+    (100, 128, 128, fp8sm.FP8_MM_1x128_128x128, fp8sm.FP8_ERR_VALUE, "multiples of 128"),
+    (128, 192, 128, fp8sm.FP8_MM_1x128_128x128, fp8sm.FP8_ERR_VALUE, "multiples of 128"),
+    (128, 128, 144, fp8sm.FP8_MM_1x128_128x128, fp8sm.FP8_ERR_VALUE, "K must be"),
+    (128, 128, 0, fp8sm.FP8_MM_1x128_128x128, fp8sm.FP8_ERR_VALUE, "K must be"),
+    (-128, 128, 128, fp8sm.FP8_MM_1x128_128x128, fp8sm.FP8_ERR_VALUE, "negative"),
+])
+def test_scaled_mm_quantized_dual_rejects_bad_arguments(lib, M, N, K, recipe, status, frag):
+    st = lib.fp8_scaled_mm_quantized_dual(FAKE, FAKE, M, N, K, FAKE, FAKE, recipe, None,
+                                          FAKE, FAKE, FAKE, FAKE, None)
+    assert st == status
+    assert frag in lib.fp8_last_error().decode()
+
+
+def test_scaled_mm_quantized_dual_null_alignment_and_empty(lib):
+    r = fp8sm.FP8_MM_1x128_128x128
+    st = lib.fp8_scaled_mm_quantized_dual(FAKE, FAKE, 128, 128, 128, FAKE, FAKE, r, None,
+                                          FAKE, FAKE, None, FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE and "null" in lib.fp8_last_error().decode()
+    st = lib.fp8_scaled_mm_quantized_dual(FAKE, FAKE, 128, 128, 128, FAKE, FAKE, r, None,
+                                          FAKE, FAKE, P((1 << 20) + 8), FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE and "misaligned" in lib.fp8_last_error().decode()
+    st = lib.fp8_scaled_mm_quantized_dual(FAKE, FAKE, 128, 128, 128, FAKE, FAKE, r, None,
+                                          FAKE, FAKE, FAKE, P((1 << 20) + 2), None)
+    assert st == fp8sm.FP8_ERR_VALUE and "misaligned" in lib.fp8_last_error().decode()
+    assert lib.fp8_scaled_mm_quantized_dual(None, None, 0, 128, 128, None, None, r, None,
+                                            None, None, None, None, None) == fp8sm.FP8_OK
+
+
 def test_grouped_requires_offs(lib):
     st = lib.fp8_grouped_scaled_mm(FAKE, FAKE, 64, 128, 128, 4, FAKE, FAKE, None,
                                    fp8sm.FP8_OUT_BF16, FAKE, None)

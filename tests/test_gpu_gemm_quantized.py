@@ -251,3 +251,128 @@ def test_linear_chain_backward_grad_input_against_oracle():
     exact = (dy2.double().numpy()[rows] @ w2.double().numpy()) @ w1.double().numpy()
     err = got - exact
     assert 10 * np.log10((exact ** 2).sum() / (err ** 2).sum()) >= 20.0
+
+
+# ------------------------------------------- both e4m3 forms from one GEMM
+# fp8_scaled_mm_quantized_dual writes the 1x128-along-n form (for the next
+# grad_input GEMM) and the transposed 1x128-along-m form (for the grad_weight
+# GEMM, 1x128_128x1 with the tokens as K) of the same fp32 result.
+
+def run_dual(qa, sa, qb, sb, bias):
+    a, b = torch.from_numpy(qa).cuda(), torch.from_numpy(qb).cuda()
+    sad, sbd = torch.from_numpy(sa).cuda(), torch.from_numpy(sb).cuda()
+    bd = None if bias is None else bias.cuda()
+    r = fp8sm.FP8_MM_1x128_128x128
+    y = fp8sm.fp8_scaled_mm(a, b, sad, sbd, r, bias=bd, out_dtype=torch.float32)
+    q, s, qt, st = fp8sm.fp8_scaled_mm_quantized_dual(a, b, sad, sbd, r, bias=bd)
+    torch.cuda.synchronize()
+    fp8sm.check_device_status()
+    return tuple(t.cpu().numpy() for t in (y, q, s, qt, st))
+
+
+DUAL_CASES = [
+    # M, N, K, bias  (M, N, K multiples of 128)
+    (128, 128, 128, False),
+    (256, 384, 384, True),           # last tile half empty along n
+    (1024, 2304, 1024, False),
+    (384, 640, 256, True),
+    (2304, 4352, 512, False),        # last wave split into 128-wide items
+]
+
+
+@pytest.mark.parametrize("M,N,K,bias", DUAL_CASES)
+def test_dual_output_parity(M, N, K, bias):
+    seed = M * 13 + N * 7 + K
+    wl, qa, sa, qb, sb = operands("1x128_128x128", M, N, K, seed, bias)
+    y, q, s, qt, st = run_dual(qa, sa, qb, sb, wl.bias)
+    what = f"dual {M}x{N}x{K}"
+    check_exact(y, q, s, what + " rows")
+    check_exact(np.ascontiguousarray(y.T), qt, st, what + " transposed")
+    bias_bits = None if wl.bias is None else W.bf16_bits(wl.bias)
+    ref, mag = oracle.scaled_mm(qa, qb, sa, sb, MM["1x128_128x128"], bias_bits=bias_bits)
+    check_against_fp64(q, s, ref, mag, what + " rows")
+    check_against_fp64(qt, st, np.ascontiguousarray(ref.T), np.ascontiguousarray(mag.T),
+                       what + " transposed")
+
+
+def test_dual_output_rejects_other_recipes_and_shapes():
+    z = torch.zeros(128, 128, dtype=torch.uint8, device="cuda")
+    one = torch.ones(1, 128, device="cuda")
+    with pytest.raises(fp8sm.Fp8Unsupported):
+        fp8sm.fp8_scaled_mm_quantized_dual(z, z, one, one, fp8sm.FP8_MM_ROW_ROW)
+    a = torch.zeros(100, 128, dtype=torch.uint8, device="cuda")
+    with pytest.raises(fp8sm.Fp8ValueError):
+        fp8sm.fp8_scaled_mm_quantized_dual(a, z, torch.ones(1, 100, device="cuda"),
+                                           torch.ones(1, 1, device="cuda"),
+                                           fp8sm.FP8_MM_1x128_128x128)
+
+
+def test_dual_output_full_size_sampled():
+    """The blockwise workload (16640 x 5120 x 8192): both forms against the
+    same kernel schedule's fp32 result, on sampled rows and sampled columns."""
+    wl = W.make_workload(2, 0)
+    a, b = wl.a.cuda(), wl.b.cuda()
+    qa, sa = fp8sm.fp8_quantize(a, fp8sm.FP8_SCALE_BLOCK_1x128)
+    qb, sb = fp8sm.fp8_quantize(b, fp8sm.FP8_SCALE_BLOCK_128x128)
+    del a, b
+    r = fp8sm.FP8_MM_1x128_128x128
+    q, s, qt, st = fp8sm.fp8_scaled_mm_quantized_dual(qa, qb, sa, sb, r)
+    y = fp8sm.fp8_scaled_mm(qa, qb, sa, sb, r, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    fp8sm.check_device_status()
+    rows = torch.from_numpy(sample_rows(wl.M, n=64, seed=5)).cuda()
+    check_exact(y.index_select(0, rows).cpu().numpy(), q.index_select(0, rows).cpu().numpy(),
+                s.index_select(1, rows).cpu().numpy(), "dual full size rows")
+    cols = torch.from_numpy(sample_rows(wl.N, n=64, seed=6)).cuda()
+    check_exact(y.index_select(1, cols).t().contiguous().cpu().numpy(),
+                qt.index_select(0, cols).cpu().numpy(),
+                st.index_select(1, cols).cpu().numpy(), "dual full size transposed")
+
+
+def test_linear_chain_backward_with_grad_weight_against_oracle():
+    """A chain of two blockwise linears, X (T, D) -> W1 (F, D) -> W2 (D, F),
+    taken backward: dY1 = dY2 @ W2 (1x128_128x128) writes both e4m3 forms of
+    dY1; dX = dY1 @ W1 from the 1x128-along-F form (1x128_128x128) and
+    dW1 = dY1^T @ X from the 1x128-along-T form (1x128_128x1, K = T), the
+    recipes of "improve fp8 blockwise gemm perf".  Against the oracle's chain
+    (1x128 quantize, fp64 GEMM rounded to fp32, quantize both ways, fp64
+    GEMMs) and SQNR >= 20 dB against the unquantized products."""
+    T, D, F = 2048, 1024, 640
+    g = W.generator(4242)
+    x = W.randn_bf16((T, D), 1.0, g)
+    w1 = W.randn_bf16((F, D), 0.02, g)
+    w2 = W.randn_bf16((D, F), 0.02, g)
+    dy2 = W.randn_bf16((T, D), 1.0, g)
+    f = fp8sm
+    qd, sd = f.fp8_quantize(dy2.cuda(), f.FP8_SCALE_BLOCK_1x128)
+    q2t, s2t = f.fp8_quantize_transposed(w2.cuda(), f.FP8_SCALE_BLOCK_128x128)  # W2^T (F, D)
+    q1t, s1t = f.fp8_quantize_transposed(w1.cuda(), f.FP8_SCALE_BLOCK_128x128)  # W1^T (D, F)
+    qxt, sxt = f.fp8_quantize_transposed(x.cuda(), f.FP8_SCALE_BLOCK_1x128)     # X^T (D, T)
+    dy1q, dy1s, dy1tq, dy1ts = f.fp8_scaled_mm_quantized_dual(
+        qd, q2t, sd, s2t, f.FP8_MM_1x128_128x128)
+    dx = f.fp8_scaled_mm(dy1q, q1t, dy1s, s1t, f.FP8_MM_1x128_128x128, out_dtype=torch.float32)
+    dw1 = f.fp8_scaled_mm(dy1tq, qxt, dy1ts, sxt, f.FP8_MM_1x128_128x1, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    f.check_device_status()
+    G = oracle.GROUP_128x128
+    oqd, osd = oracle.quantize(W.bf16_bits(dy2), oracle.GROUP_1x128)
+    oq2t, os2t = oracle.quantize(np.ascontiguousarray(W.bf16_bits(w2).T), G)
+    oq1t, os1t = oracle.quantize(np.ascontiguousarray(W.bf16_bits(w1).T), G)
+    oqxt, osxt = oracle.quantize(np.ascontiguousarray(W.bf16_bits(x).T), oracle.GROUP_1x128)
+    y1, _ = oracle.scaled_mm(oqd, oq2t, osd, os2t, oracle.MM_1x128_128x128)
+    y1 = y1.astype(np.float32)
+    oy1q, oy1s = oracle.quantize_f32(y1, oracle.GROUP_1x128)
+    oy1tq, oy1ts = oracle.quantize_f32(np.ascontiguousarray(y1.T), oracle.GROUP_1x128)
+    rows = sample_rows(T, 48, seed=42)
+    ref_dx, mag_dx = oracle.scaled_mm(oy1q, oq1t, oy1s, os1t, oracle.MM_1x128_128x128, rows=rows)
+    ref_dw, mag_dw = oracle.scaled_mm(oy1tq, oqxt, oy1ts, osxt, oracle.MM_1x128_128x1)
+    got_dx = dx.cpu().numpy().astype(np.float64)[rows]
+    got_dw = dw1.cpu().numpy().astype(np.float64)
+    for got, ref, mag, what in ((got_dx, ref_dx, mag_dx, "dX"), (got_dw, ref_dw, mag_dw, "dW1")):
+        ok = oracle.within_tolerance(got, ref, mag)
+        assert ok.all(), f"backward {what}: {int((~ok).sum())} of {ok.size} out of tolerance"
+    dy1_exact = dy2.double().numpy() @ w2.double().numpy()
+    for got, exact in ((got_dx, dy1_exact[rows] @ w1.double().numpy()),
+                       (got_dw, dy1_exact.T @ x.double().numpy())):
+        err = got - exact
+        assert 10 * np.log10((exact ** 2).sum() / (err ** 2).sum()) >= 20.0
