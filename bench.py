@@ -58,6 +58,7 @@ WORKLOADS = {
     "grouped_e16_mxfp8": (11, 0),
     "grouped_e16_grad_input": (12, 0),
     "grouped_e16_grad_weight": (13, 0),
+    "linear_chain_train_1x128": (14, 0),
 }
 DEFAULT_WORKLOAD = "rowwise_4096"
 # Page 5's context numbers (TFLOP/s of torch._scaled_mm, hardware not stated)
@@ -72,7 +73,8 @@ OPERAND_GROUPS = {"tensor": ("tensor", "tensor"), "row": ("row", "row"),
                   "grouped_blockwise": ("1x128", "128x128"), "chain": ("1x128", "128x128"),
                   "mxfp8": ("mx", "mx"), "chain_mx": ("mx", "mx"), "grouped_mx": ("mx", "mx"),
                   "grouped_grad_input": ("1x128", "128x128"),
-                  "grouped_grad_weight": ("1x128", "1x128")}
+                  "grouped_grad_weight": ("1x128", "1x128"),
+                  "chain_train": ("1x128", "128x128")}
 # GEMM recipe of each workload recipe, and which operands are quantized
 # transposed (the training GEMMs contract along the stored rows)
 GEMM_RECIPE = {"grad_input": "1x128_128x128", "grad_weight": "1x128_128x1",
@@ -306,6 +308,30 @@ class Step:
             self.out = torch.empty(wl.M, n2, dtype=torch.bfloat16, device=dev)
             self.launches_per_step = 5
 
+    def inputs(self):
+        """The device tensors a step reads, in host_inputs' order."""
+        t = [self.a, self.b]
+        if self.bias is not None:
+            t.append(self.bias)
+        if self.chain:
+            t.append(self.b2)
+        return t
+
+    def host_inputs(self):
+        """The workload's host tensors in the layout of inputs()."""
+        wl = self.wl
+        hb = (wl.b.reshape(-1, wl.K)
+              if wl.recipe in ("grouped", "grouped_blockwise", "grouped_mx") else wl.b)
+        t = [wl.a, hb]
+        if wl.bias is not None:
+            t.append(wl.bias)
+        if self.chain:
+            t.append(wl.extra["b2"])
+        return t
+
+    def outputs(self):
+        return [self.out]
+
     def quantize(self):
         """Both operands' quantization; the second runs on a side stream,
         concurrently with the first (same work, overlapped), and the main
@@ -405,6 +431,107 @@ class Step:
         return b
 
 
+class TrainStep:
+    """Forward and backward of the two-linear chain X -> W1 -> W2, blockwise
+    scaled throughout ("improve fp8 blockwise gemm perf": 1x128_128x128 for
+    the forward and grad_input GEMMs, 1x128_128x1 for grad_weight).
+
+    quantize(): X and dY2 in 1x128 groups along the features and, transposed,
+    along the tokens; W1 and W2 in 128x128 tiles, as stored and transposed.
+    gemm(): Y1 = X W1^T and dY1 = dY2 W2 write both e4m3 forms of their
+    result from the epilogue; Y2 = Y1 W2^T, dX = dY1 W1, dW1 = dY1^T X and
+    dW2 = dY2^T Y1 read them.  All outputs bf16."""
+
+    def __init__(self, wl: W.Workload, dev: torch.device):
+        from fp8_scaled_matrix_b200 import fp8sm
+        self.f = fp8sm
+        self.wl = wl
+        T, F, D = wl.M, wl.N, wl.K
+        self.x, self.w1 = wl.a.to(dev), wl.b.to(dev)
+        self.w2, self.dy2 = wl.extra["b2"].to(dev), wl.extra["dy"].to(dev)
+
+        def u8(r, c):
+            return torch.empty(r, c, dtype=torch.uint8, device=dev)
+
+        def f32(r, c):
+            return torch.empty(r, c, dtype=torch.float32, device=dev)
+
+        def bf(r, c):
+            return torch.empty(r, c, dtype=torch.bfloat16, device=dev)
+        # activations: 1x128 scales (cols/128, rows); weights: 128x128 scales
+        # (cols/128, rows/128)
+        self.qx, self.sx, self.qxt, self.sxt = u8(T, D), f32(D // 128, T), u8(D, T), f32(T // 128, D)
+        self.qd, self.sd, self.qdt, self.sdt = u8(T, D), f32(D // 128, T), u8(D, T), f32(T // 128, D)
+        self.qw1, self.sw1 = u8(F, D), f32(D // 128, F // 128)
+        self.qw1t, self.sw1t = u8(D, F), f32(F // 128, D // 128)
+        self.qw2, self.sw2 = u8(D, F), f32(F // 128, D // 128)
+        self.qw2t, self.sw2t = u8(F, D), f32(D // 128, F // 128)
+        self.y1 = (u8(T, F), f32(F // 128, T), u8(F, T), f32(T // 128, F))
+        self.dy1 = (u8(T, F), f32(F // 128, T), u8(F, T), f32(T // 128, F))
+        self.y2, self.dx, self.dw1, self.dw2 = bf(T, D), bf(T, D), bf(F, D), bf(D, F)
+        self.side = torch.cuda.Stream(device=dev)
+        self.ev_fork = torch.cuda.Event()
+        self.ev_join = torch.cuda.Event()
+        self.launches_per_step = 14
+
+    def inputs(self):
+        return [self.x, self.w1, self.w2, self.dy2]
+
+    def host_inputs(self):
+        wl = self.wl
+        return [wl.a, wl.b, wl.extra["b2"], wl.extra["dy"]]
+
+    def outputs(self):
+        return [self.y2, self.dx, self.dw1, self.dw2]
+
+    def quantize(self):
+        f = self.f
+        B1, B128 = f.FP8_SCALE_BLOCK_1x128, f.FP8_SCALE_BLOCK_128x128
+        main = torch.cuda.current_stream()
+        self.ev_fork.record(main)
+        self.side.wait_event(self.ev_fork)
+        with torch.cuda.stream(self.side):
+            f.fp8_quantize(self.w1, B128, out=self.qw1, scales=self.sw1, stream=self.side)
+            f.fp8_quantize(self.w2, B128, out=self.qw2, scales=self.sw2, stream=self.side)
+            f.fp8_quantize_transposed(self.w1, B128, out=self.qw1t, scales=self.sw1t,
+                                      stream=self.side)
+            f.fp8_quantize_transposed(self.w2, B128, out=self.qw2t, scales=self.sw2t,
+                                      stream=self.side)
+        f.fp8_quantize(self.x, B1, out=self.qx, scales=self.sx, stream=main)
+        f.fp8_quantize_transposed(self.x, B1, out=self.qxt, scales=self.sxt, stream=main)
+        f.fp8_quantize(self.dy2, B1, out=self.qd, scales=self.sd, stream=main)
+        f.fp8_quantize_transposed(self.dy2, B1, out=self.qdt, scales=self.sdt, stream=main)
+        self.ev_join.record(self.side)
+        main.wait_event(self.ev_join)
+
+    def gemm(self):
+        f = self.f
+        R, R1 = f.FP8_MM_1x128_128x128, f.FP8_MM_1x128_128x1
+        y1q, y1s, y1tq, y1ts = self.y1
+        d1q, d1s, d1tq, d1ts = self.dy1
+        f.fp8_scaled_mm_quantized_dual(self.qx, self.qw1, self.sx, self.sw1, R, out=y1q,
+                                       out_scales=y1s, out_t=y1tq, out_t_scales=y1ts)
+        f.fp8_scaled_mm(y1q, self.qw2, y1s, self.sw2, R, out=self.y2)
+        f.fp8_scaled_mm_quantized_dual(self.qd, self.qw2t, self.sd, self.sw2t, R, out=d1q,
+                                       out_scales=d1s, out_t=d1tq, out_t_scales=d1ts)
+        f.fp8_scaled_mm(d1q, self.qw1t, d1s, self.sw1t, R, out=self.dx)
+        f.fp8_scaled_mm(d1tq, self.qxt, d1ts, self.sxt, R1, out=self.dw1)
+        f.fp8_scaled_mm(self.qdt, y1tq, self.sdt, y1ts, R1, out=self.dw2)
+
+    def quant_bytes(self) -> int:
+        """Algorithmic HBM bytes of the eight quantize launches: 2 B read +
+        1 B written per element, 4 B per scale."""
+        act = self.x.numel() + self.dy2.numel()
+        w = self.w1.numel() + self.w2.numel()
+        sc = sum(t.numel() * 4 for t in (self.sx, self.sxt, self.sd, self.sdt, self.sw1,
+                                         self.sw1t, self.sw2, self.sw2t))
+        return 2 * 3 * (act + w) + sc
+
+
+def make_step(wl: W.Workload, dev: torch.device):
+    return TrainStep(wl, dev) if wl.recipe == "chain_train" else Step(wl, dev)
+
+
 def evict_l2(flush: torch.Tensor):
     """Write a buffer twice the size of L2, then read it back: the step's
     inputs leave L2, and the lines left behind are clean, so the next kernel
@@ -423,7 +550,7 @@ def capture(fn, pool=None):
 
 def run_ours(args, wl, dev, rank, world):
     torch.cuda.set_device(dev)
-    st = Step(wl, dev)
+    st = make_step(wl, dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     for _ in range(args.warmup):
         st.quantize()
@@ -483,20 +610,16 @@ def run_ours(args, wl, dev, rank, world):
 def run_e2e(args, wl, dev, world):
     """Same step through the public API from pinned HOST buffers: every step
     copies its bf16 inputs host -> device, quantizes, multiplies, and copies
-    the bf16 result device -> host, all inside the timed region.  Steps are
+    its results device -> host, all inside the timed region.  Steps are
     pipelined the way a serving loop would run them: two sets of device
     buffers and three streams (upload, compute, download), so step i's
     download and step i+1's upload overlap each other and the compute; every
     copy of every step is still made and timed."""
     from fp8_scaled_matrix_b200 import fp8sm  # noqa: F401
-    ha = wl.a.pin_memory()
-    hb = (wl.b.reshape(-1, wl.K) if wl.recipe in ("grouped", "grouped_blockwise", "grouped_mx")
-          else wl.b).contiguous().pin_memory()     # grouped_grad_input: (E, out, in) as stored
-    hbias = None if wl.bias is None else wl.bias.pin_memory()
-    hb2 = wl.extra["b2"].pin_memory() if "b2" in wl.extra else None
-    sets = [Step(wl, dev), Step(wl, dev)]
-    hout = [torch.empty(tuple(sets[0].out.shape), dtype=torch.bfloat16).pin_memory()
-            for _ in range(2)]
+    sets = [make_step(wl, dev), make_step(wl, dev)]
+    hin = [t.contiguous().pin_memory() for t in sets[0].host_inputs()]
+    hout = [[torch.empty(tuple(o.shape), dtype=o.dtype).pin_memory()
+             for o in sets[0].outputs()] for _ in range(2)]
     s_in, s_comp, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_comp = [torch.cuda.Event() for _ in range(2)]
@@ -509,23 +632,20 @@ def run_e2e(args, wl, dev, world):
         with torch.cuda.stream(s_in):
             if i >= 2:
                 s_in.wait_event(ev_comp[k])   # step i-2 has consumed set k's inputs
-            st.a.copy_(ha, non_blocking=True)
-            st.b.copy_(hb, non_blocking=True)
-            if hbias is not None:
-                st.bias.copy_(hbias, non_blocking=True)
-            if hb2 is not None:
-                st.b2.copy_(hb2, non_blocking=True)
+            for d, h in zip(st.inputs(), hin):
+                d.copy_(h, non_blocking=True)
             ev_in[k].record(s_in)
         with torch.cuda.stream(s_comp):
             s_comp.wait_event(ev_in[k])
             if i >= 2:
-                s_comp.wait_event(ev_out[k])  # step i-2's result has left set k
+                s_comp.wait_event(ev_out[k])  # step i-2's results have left set k
             st.quantize()
             st.gemm()
             ev_comp[k].record(s_comp)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_comp[k])
-            hout[k].copy_(st.out, non_blocking=True)
+            for h, d in zip(hout[k], st.outputs()):
+                h.copy_(d, non_blocking=True)
             ev_out[k].record(s_out)
 
     for i in range(2):
@@ -543,9 +663,8 @@ def run_e2e(args, wl, dev, world):
     e1.record(s_out)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1) / steps, dev)
-    h2d = (ha.numel() * 2 + hb.numel() * 2 + (0 if hbias is None else hbias.numel() * 2)
-           + (0 if hb2 is None else hb2.numel() * 2))
-    d2h = hout[0].numel() * 2
+    h2d = sum(t.numel() * t.element_size() for t in hin)
+    d2h = sum(t.numel() * t.element_size() for t in hout[0])
     return {"ms": ms, "h2d": h2d, "d2h": d2h, "steps": steps}
 
 
@@ -568,6 +687,37 @@ def oracle_sample(wl, max_rows: int):
         b = W.bf16_bits(x)
         return np.ascontiguousarray(b.T) if transposed else b
     t0 = time.perf_counter()
+    if wl.recipe == "chain_train":
+        # the whole step on the first tokens (a multiple of 128, the length of
+        # the transposed groups): each of the six GEMMs and the activation
+        # quantizes cost in proportion to the token count; the weights'
+        # quantization (as stored and transposed) is timed in full
+        G1, G128 = oracle.GROUP_1x128, oracle.GROUP_128x128
+        R, R1 = MMR["1x128_128x128"], MMR["1x128_128x1"]
+        w1b, w2b = W.bf16_bits(wl.b), W.bf16_bits(wl.extra["b2"])
+        qw1, sw1 = oracle.quantize(w1b, G128)
+        qw2, sw2 = oracle.quantize(w2b, G128)
+        qw1t, sw1t = oracle.quantize(np.ascontiguousarray(w1b.T), G128)
+        qw2t, sw2t = oracle.quantize(np.ascontiguousarray(w2b.T), G128)
+        tq = time.perf_counter() - t0
+        t = min(wl.M, -(-max(1, max_rows) // 128) * 128)
+        t0 = time.perf_counter()
+        xb, db = W.bf16_bits(wl.a[:t]), W.bf16_bits(wl.extra["dy"][:t])
+        qx, sx = oracle.quantize(xb, G1)
+        qxt, sxt = oracle.quantize(np.ascontiguousarray(xb.T), G1)
+        qd, sd = oracle.quantize(db, G1)
+        qdt, sdt = oracle.quantize(np.ascontiguousarray(db.T), G1)
+        y1 = oracle.scaled_mm(qx, qw1, sx, sw1, R)[0].astype(np.float32)
+        y1q, y1s = oracle.quantize_f32(y1, G1)
+        y1tq, y1ts = oracle.quantize_f32(np.ascontiguousarray(y1.T), G1)
+        oracle.scaled_mm(y1q, qw2, y1s, sw2, R)
+        dy1 = oracle.scaled_mm(qd, qw2t, sd, sw2t, R)[0].astype(np.float32)
+        d1q, d1s = oracle.quantize_f32(dy1, G1)
+        d1tq, d1ts = oracle.quantize_f32(np.ascontiguousarray(dy1.T), G1)
+        oracle.scaled_mm(d1q, qw1t, d1s, sw1t, R)
+        oracle.scaled_mm(d1tq, qxt, d1ts, sxt, R1)
+        oracle.scaled_mm(qdt, y1tq, sdt, y1ts, R1)
+        return time.perf_counter() - t0, t / wl.M, tq, oracle.num_threads()
     if wl.recipe == "chain_mx":
         qa, sa = oracle.mx_quantize(W.bf16_bits(wl.a))
         qb, sb = oracle.mx_quantize(W.bf16_bits(wl.b))
@@ -691,11 +841,19 @@ def oracle_sample(wl, max_rows: int):
 def cpu_baseline(wl, rows: int):
     tg, frac, tq, threads = oracle_sample(wl, rows)
     est_s = tq + tg / frac
+    value = wl.flops / est_s / 1e12
+    if wl.recipe == "chain_train":
+        t = int(round(frac * wl.M))
+        return {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                "sample": (f"quantize of W1 and W2, as stored and transposed, in full "
+                           f"({tq:.2f} s) + the rest of the step (activation quantizes, six "
+                           f"GEMMs, both quantized forms of Y1 and dY1) on the first {t} of "
+                           f"{wl.M} tokens ({tg:.2f} s), scaled to all rows"),
+                "seconds_est_per_step": est_s}
     chain = wl.recipe in ("chain", "chain_mx")
     what = "X, W1 and W2" if chain else "both operands"
     gemm = (("both GEMMs (the first one's fp32 output quantized "
              + ("MXFP8)" if wl.recipe == "chain_mx" else "1x128)")) if chain else "GEMM")
-    value = wl.flops / est_s / 1e12
     return {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
             "sample": (f"quantize of {what} in full ({tq:.2f} s) + {gemm} on "
                        f"{int(round(frac * wl.M))} of {wl.M} output rows ({tg:.2f} s), "
@@ -707,6 +865,8 @@ def baseline_rows(wl, target_s: float = 12.0) -> int:
     """Rows of the GEMM that take about target_s on the oracle (probe with 8)."""
     tg, frac, _, _ = oracle_sample(wl, 8)
     per_row = tg / max(1, int(round(frac * wl.M)))
+    if wl.recipe == "chain_train":   # samples are whole 128-token groups
+        return int(max(128, min(wl.M, 128 * round(target_s / max(per_row * 128, 1e-9)))))
     return int(max(8, min(wl.M, target_s / max(per_row, 1e-9))))
 
 
@@ -812,12 +972,17 @@ def main(argv=None):
                      if wl.recipe == "chain" else
                      "MXFP8 quantize X || W1, W2 (two streams), then GEMM1 with MXFP8 "
                      "output, then GEMM2" if wl.recipe == "chain_mx" else
+                     "quantize X, X^T, dY2, dY2^T || W1, W2, W1^T, W2^T (two streams), then "
+                     "the chain's forward (Y1 = X W1^T writing Y1 and Y1^T in e4m3, Y2 = Y1 "
+                     "W2^T) and backward (dY1 = dY2 W2 writing dY1 and dY1^T in e4m3, dX = "
+                     "dY1 W1, dW1 = dY1^T X, dW2 = dY2^T Y1)"
+                     if wl.recipe == "chain_train" else
                      "quantize A || quantize B (two streams), then scaled GEMM"),
             "N2": (int(wl.extra["b2"].shape[0]) if "b2" in wl.extra else None),
             "launch": ("CUDA graphs of the step's C-ABI launches" if args.graphs
                        else "one C-ABI call per launch"),
-            "e2e": ("pinned host inputs, every step's H2D + quantize + GEMM + D2H of the "
-                    "bf16 result; steps pipelined over two buffer sets and three streams"),
+            "e2e": ("pinned host inputs, every step's H2D + quantize + GEMM + D2H of its "
+                    "bf16 results; steps pipelined over two buffer sets and three streams"),
         },
         "roofline": {
             "bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak,

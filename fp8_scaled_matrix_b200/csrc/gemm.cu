@@ -72,6 +72,9 @@ static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsAtLaunch,
               "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;  // two 256-column fp32 buffers
 constexpr uint32_t kEpiBuf = 32 * 64;  // 32 rows x 64 bytes, 64-byte swizzle
+// dual e4m3 output: per epilogue warp, 16 columns x 32 rows of transposed
+// codes (also the column maxima the half's warps exchange)
+constexpr uint32_t kTposBuf = 512;
 // Blockwise scale ring: one slot per K block, filled ahead by warp 2 with
 // cp.async: [128 row scales sA[kb, m0..] | column scales: sB[kb, nb0],
 // sB[kb, nb0 + 1] (1x128_128x128) or sB[kb, n0 .. n0 + 255] (1x128_128x1)].
@@ -102,7 +105,8 @@ struct Cfg {
   static constexpr uint32_t kOffB = kOffA + kStages * kAStage;
   static constexpr uint32_t kOffEpi = kOffB + kStages * kBStage;
   static constexpr uint32_t kOffScl = kOffEpi + kEpiWarps * kEpiBuf;
-  static constexpr uint32_t kOffBar = kOffScl + kSclBytes;
+  static constexpr uint32_t kOffTpos = kOffScl + kSclBytes;
+  static constexpr uint32_t kOffBar = kOffTpos + kEpiWarps * kTposBuf;
   // barriers: full[kStages], empty[kStages], acc_full[2], acc_empty[2], drain,
   // scale ring sfull[kSclSlots], sempty[kSclSlots], epilogue half sync hsync[2]
   static constexpr uint32_t kNumBars = 2 * kStages + 5 + 2 * kSclSlots + 2;
@@ -934,15 +938,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Single CTA: a CTA-scope arrive.  Pair: the leader's barrier, at cluster
     // scope (a cluster-scope release costs a fence, so it is used only there).
     // the four warps of this warp's half meet (bounded; dual e4m3 output)
-    uint32_t hphase = 0;
-    auto half_sync = [&]() -> bool {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&hsync[half]);
-      const bool done = mbar_wait(&hsync[half], hphase, abort_flag, p.status, SITE_EPI_ACC_FULL,
-                                  kWaitLimitNs);
-      hphase ^= 1u;
-      return done;
-    };
     auto release_acc = [&](uint32_t a) {
       if constexpr (kPair) mbar_arrive_cluster(a ? acc_empty_addr1 : acc_empty_addr0);
       else mbar_arrive(&acc_empty[a]);
@@ -1190,13 +1185,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (acc == 0) acc_phase ^= 1u;
         }
         if (!ok) break;
-        // the tile's fp32 results for chunk cc (bias added)
-        auto result32 = [&](int cc, float (&v)[32]) {
-          load_bias32(p.bias, ncol0 + cc * 32, p.N, v);
+        // the bias joins the accumulators once (one fp32 add per element),
+        // so the output passes below read registers only
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          float bv[32];
+          load_bias32(p.bias, ncol0 + cc * 32, p.N, bv);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            v[2 * i] += accr[cc * 16 + i].x;
-            v[2 * i + 1] += accr[cc * 16 + i].y;
+            accr[cc * 16 + i].x += bv[2 * i];
+            accr[cc * 16 + i].y += bv[2 * i + 1];
+          }
+        }
+        // the tile's fp32 results for chunk cc (bias added)
+        auto result32 = [&](int cc, float (&v)[32]) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            v[2 * i] = accr[cc * 16 + i].x;
+            v[2 * i + 1] = accr[cc * 16 + i].y;
           }
         };
         if constexpr (!kOutQ) {
@@ -1209,130 +1215,113 @@ __global__ void __launch_bounds__(kThreads, 1)
                                             c.row_end, p.out, p.N, lane);
           }
         } else {
-          // e4m3 output in 1x128 groups along n (this thread's 128 columns)
+          // e4m3 output in 1x128 groups along n (this thread's 128 columns).
+          // The dual kind also writes the result transposed, where the
+          // tile's 128 rows of each column form one 1x128 group along m:
+          // the column maxima of the half's four warps meet in shared memory
+          // (two bounded mbarrier meetings per tile), and each warp's codes
+          // for 16 columns x 32 rows pass through its own 512-byte buffer.
           float am = 0.0f;
+          [[maybe_unused]] uint32_t cmax[4];  // lane L: column 32 cc + L, max over the warp's rows
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
             float v[32];
             result32(cc, v);
 #pragma unroll
             for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(v[i]));
+            if constexpr (kOutQT) {
+              // |v| as bits orders like the values
+              uint32_t mine = 0u;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(fabsf(v[i])));
+                mine = lane == static_cast<uint32_t>(i) ? m : mine;
+              }
+              cmax[cc] = mine;
+            }
           }
           const ScalePair sp = scales_from_amax(am);
           if (row_ok && ncol0 < p.N) p.out_scales[(ncol0 / 128) * p.M + row] = sp.s;
-#pragma unroll
-          for (int bx = 0; bx < 2; ++bx) {
-            uint4 chunk[4];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              float v[32];
-              result32(2 * bx + h, v);
-              uint32_t* w = reinterpret_cast<uint32_t*>(&chunk[2 * h]);
-#pragma unroll
-              for (int j = 0; j < 8; ++j)
-                w[j] = cast_f32x2(v[4 * j], v[4 * j + 1], sp.inv) |
-                       (cast_f32x2(v[4 * j + 2], v[4 * j + 3], sp.inv) << 16);
-            }
-            store_box64<kMasked>(ebuf, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
-                                  row0, c.row_end, static_cast<uint8_t*>(p.out), p.N, 1, lane);
-          }
+          [[maybe_unused]] float tinv[4];  // lane L: 1 / scale of column 32 cc + L
+          uint8_t* const tbuf = smem + C::kOffTpos + ew * kTposBuf;
           if constexpr (kOutQT) {
-            // The transposed e4m3 form: for each of this half's 128 columns,
-            // the tile's 128 rows are one 1x128 group along m.  (1) Column
-            // amax over the warp's 32 rows by a butterfly over the lanes
-            // (lane L ends with column 32 cc + L); (2) the four warps of the
-            // half meet through their staging buffers (a bounded mbarrier
-            // per half); (3) codes staged column-major, 64 columns at a time, in
-            // the half's 8 KB of staging buffers and written out as rows of
-            // the transposed matrix.
-            uint8_t* const half_stage = smem + C::kOffEpi + half * 4 * kEpiBuf;
-            float cmax[4];
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-              float v[32];
-              result32(cc, v);
-#pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = fabsf(v[i]);
-#pragma unroll
-              for (int sh = 16; sh >= 1; sh >>= 1) {
-                const bool upper = (lane & sh) != 0;
-#pragma unroll
-                for (int k = 0; k < sh; ++k) {
-                  const float send = upper ? v[k] : v[k + sh];
-                  const float keep = upper ? v[k + sh] : v[k];
-                  v[k] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, sh));
-                }
-              }
-              cmax[cc] = v[0];
-            }
-            // this warp's staging buffer is free once its TMA stores have read it
-            if (lane == 0) bulk_wait_group_read0();
-            __syncwarp();
+            // A tile makes two meetings on hsync[half], so the phase is 0 at
+            // the start of every tile.
+            uint32_t hphase = 0;
+            auto half_sync = [&]() -> bool {
+              __syncwarp();
+              uint64_t* const hb = &hsync[half];
+              if (lane == 0) mbar_arrive(hb);
+              const bool done = mbar_wait(hb, hphase, abort_flag, p.status, SITE_EPI_ACC_FULL,
+                                          kWaitLimitNs);
+              hphase ^= 1u;
+              return done;
+            };
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc)
-              reinterpret_cast<float*>(ebuf)[cc * 32 + lane] = cmax[cc];
+              reinterpret_cast<uint32_t*>(tbuf)[cc * 32 + lane] = cmax[cc];
             if (!half_sync()) {
               ok = false;
               break;
             }
-            float inv[4];
+            const uint8_t* const half_t = smem + C::kOffTpos + half * 4 * kTposBuf;
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
-              float am = 0.0f;
+              uint32_t mx = 0u;
 #pragma unroll
               for (int w = 0; w < 4; ++w)
-                am = fmaxf(am, reinterpret_cast<const float*>(half_stage + w * kEpiBuf)[cc * 32 + lane]);
-              const ScalePair sp = scales_from_amax(am);
-              inv[cc] = sp.inv;
+                mx = max(mx, reinterpret_cast<const uint32_t*>(half_t + w * kTposBuf)[cc * 32 + lane]);
+              const ScalePair tp = scales_from_amax(__uint_as_float(mx));
+              tinv[cc] = tp.inv;
               const int64_t n = ncol0 + 32 * cc + lane;
-              if (q == 0 && n < p.N) p.out_t_scales[(cta_m0 / 128) * p.N + n] = sp.s;
+              if (q == 0 && n < p.N) p.out_t_scales[(cta_m0 / 128) * p.N + n] = tp.s;
             }
             if (!half_sync()) {  // every warp has read the maxima
               ok = false;
               break;
             }
-            const uint32_t r = q * 32 + lane;   // this thread's row within the tile
+          }
 #pragma unroll
-            for (int pass = 0; pass < 2 && ok; ++pass) {
+          for (int bx = 0; bx < 2; ++bx) {
+            uint4 chunk[4];
 #pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const int cc = 2 * pass + h;
-                float v[32];
-                result32(cc, v);
+            for (int h = 0; h < 2; ++h) {
+              const int cc = 2 * bx + h;
+              float v[32];
+              result32(cc, v);
+              uint32_t* w = reinterpret_cast<uint32_t*>(&chunk[2 * h]);
 #pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                  const float i0 = __shfl_sync(0xFFFFFFFFu, inv[cc], i);
-                  const float i1 = __shfl_sync(0xFFFFFFFFu, inv[cc], i + 1);
-                  const uint32_t two = static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(
-                      make_float2(__fmul_rn(v[i], i0), __fmul_rn(v[i + 1], i1)), __NV_SATFINITE,
-                      __NV_E4M3));
-                  const int j = h * 32 + i;  // column within the pass
-                  half_stage[j * 128 + r] = static_cast<uint8_t>(two & 0xFFu);
-                  half_stage[(j + 1) * 128 + r] = static_cast<uint8_t>(two >> 8);
+              for (int j = 0; j < 8; ++j)
+                w[j] = cast_f32x2(v[4 * j], v[4 * j + 1], sp.inv) |
+                       (cast_f32x2(v[4 * j + 2], v[4 * j + 3], sp.inv) << 16);
+              if constexpr (kOutQT) {
+#pragma unroll
+                for (int rd = 0; rd < 2; ++rd) {
+                  // columns 32 cc + 16 rd + i: byte (i, lane) of the buffer
+#pragma unroll
+                  for (int i = 0; i < 16; i += 2) {
+                    const int col = 16 * rd + i;
+                    const float i0 = __shfl_sync(0xFFFFFFFFu, tinv[cc], col);
+                    const float i1 = __shfl_sync(0xFFFFFFFFu, tinv[cc], col + 1);
+                    const uint32_t two = static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(
+                        make_float2(__fmul_rn(v[col], i0), __fmul_rn(v[col + 1], i1)),
+                        __NV_SATFINITE, __NV_E4M3));
+                    tbuf[i * 32 + lane] = static_cast<uint8_t>(two & 0xFFu);
+                    tbuf[(i + 1) * 32 + lane] = static_cast<uint8_t>(two >> 8);
+                  }
+                  __syncwarp();
+                  // lane L: 16 of the 32 rows of column L / 2
+                  const uint4 u =
+                      *reinterpret_cast<const uint4*>(tbuf + (lane >> 1) * 32 + 16 * (lane & 1));
+                  const int64_t n = ncol0 + 32 * cc + 16 * rd + (lane >> 1);
+                  if (n < p.N)
+                    *reinterpret_cast<uint4*>(p.out_t + n * p.M + row0 + 16 * (lane & 1)) = u;
+                  __syncwarp();
                 }
-              }
-              if (!half_sync()) {
-                ok = false;
-                break;
-              }
-              {
-                // 128 threads: row j = tid / 2 of the pass, 64 bytes each
-                const uint32_t tid = q * 32 + lane;
-                const int j = static_cast<int>(tid >> 1);
-                const int64_t n = ncol0 + 64 * pass + j;
-                if (n < p.N) {
-                  const uint4* src = reinterpret_cast<const uint4*>(half_stage + j * 128 + 64 * (tid & 1));
-                  uint4* dst = reinterpret_cast<uint4*>(p.out_t + n * p.M + cta_m0 + 64 * (tid & 1));
-#pragma unroll
-                  for (int u = 0; u < 4; ++u) dst[u] = src[u];
-                }
-              }
-              if (!half_sync()) {  // the staging is read before it is refilled
-                ok = false;
-                break;
               }
             }
-            if (!ok) break;
+            store_box64<kMasked>(ebuf, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
+                                  row0, c.row_end, static_cast<uint8_t*>(p.out), p.N, 1, lane);
           }
         }
       }

@@ -575,21 +575,41 @@ def fp8_quantize_transposed_batched(x: torch.Tensor, recipe: int,
 
 def fp8_scaled_mm_quantized_dual(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor,
                                  scale_b: torch.Tensor, recipe: int,
-                                 bias: Optional[torch.Tensor] = None, stream=None):
-    """GEMM writing both e4m3 forms of its result: returns (codes (M, N),
-    scales (N/128, M), transposed codes (N, M), transposed scales (M/128, N))."""
+                                 bias: Optional[torch.Tensor] = None,
+                                 out: Optional[torch.Tensor] = None,
+                                 out_scales: Optional[torch.Tensor] = None,
+                                 out_t: Optional[torch.Tensor] = None,
+                                 out_t_scales: Optional[torch.Tensor] = None, stream=None):
+    """fp8_scaled_mm writing both e4m3 forms of its result: 1x128 groups along
+    n, and the transpose with 1x128 groups along m.
+
+    Returns (codes (M, N), scales (N/128, M), transposed codes (N, M),
+    transposed scales (M/128, N)); uint8 e4m3 codes, fp32 scales."""
     L = load_library()
     _need_cuda(a, b, scale_a, scale_b, bias)
     M, K = a.shape
     N = b.shape[0]
     if b.shape[1] != K:
         raise ValueError("a and b must share K")
+    for t in (a, b):
+        if t.dtype not in (torch.uint8, torch.float8_e4m3fn) or not t.is_contiguous():
+            raise ValueError("a and b must be contiguous e4m3 (uint8 codes)")
+    if bias is not None and (bias.dtype != torch.bfloat16 or not bias.is_contiguous()):
+        raise ValueError("bias must be a contiguous bf16 tensor")
     dev = a.device
-    out = torch.empty((M, N), dtype=torch.uint8, device=dev)
-    sc = torch.empty((N // 128, M), dtype=torch.float32, device=dev)
-    out_t = torch.empty((N, M), dtype=torch.uint8, device=dev)
-    sc_t = torch.empty((M // 128, N), dtype=torch.float32, device=dev)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.uint8, device=dev)
+    if out_scales is None:
+        out_scales = torch.empty((N // 128, M), dtype=torch.float32, device=dev)
+    if out_t is None:
+        out_t = torch.empty((N, M), dtype=torch.uint8, device=dev)
+    if out_t_scales is None:
+        out_t_scales = torch.empty((M // 128, N), dtype=torch.float32, device=dev)
+    if (out.numel() < M * N or out_t.numel() < M * N or
+            out_scales.numel() < (N // 128) * M or out_t_scales.numel() < (M // 128) * N):
+        raise ValueError("an output buffer is too small")
     _check(L.fp8_scaled_mm_quantized_dual(_ptr(a), _ptr(b), M, N, K, _ptr(scale_a),
-                                          _ptr(scale_b), recipe, _ptr(bias), _ptr(out), _ptr(sc),
-                                          _ptr(out_t), _ptr(sc_t), _stream(stream)))
-    return out, sc, out_t, sc_t
+                                          _ptr(scale_b), recipe, _ptr(bias), _ptr(out),
+                                          _ptr(out_scales), _ptr(out_t), _ptr(out_t_scales),
+                                          _stream(stream)))
+    return out, out_scales, out_t, out_t_scales

@@ -52,6 +52,14 @@ descriptions; no public dataset is involved):
                 group's tokens: dY ~ N(0, 1e-3^2) (32768, 4096 out), X ~ N(0,1)
                 (32768, 4096 in), workload 4's group split; GEMM M=4096 (out),
                 N=4096 (in), K=32768 tokens in 16 groups
+ 14 linear chain training step  workload 8's chain forward and backward
+                with blockwise scaling throughout: X ~ N(0,1) (16640, 8192),
+                W1 ~ N(0, 0.02^2) (5120, 8192), W2 ~ N(0, 0.02^2) (8192, 5120),
+                dY2 ~ N(0, 1e-3^2) (16640, 8192) the gradient arriving at the
+                chain's output; six GEMMs of 16640 x 5120 x 8192 each:
+                Y1 = X W1^T, Y2 = Y1 W2^T, dY1 = dY2 W2, dX = dY1 W1 (all
+                1x128_128x128), dW1 = dY1^T X, dW2 = dY2^T Y1 (1x128_128x1,
+                contracting over the tokens); T must be a multiple of 128
 """
 from __future__ import annotations
 
@@ -76,6 +84,7 @@ WORKLOAD_NAMES = [
     "grouped_e16_mxfp8",
     "grouped_e16_grad_input",
     "grouped_e16_grad_weight",
+    "linear_chain_train_1x128",
 ]
 
 
@@ -130,7 +139,7 @@ class Workload:
     name: str
     # tensor | row | 1x128_128x128 | 1x128_128x1 | grouped | grouped_blockwise |
     # grad_input | grad_weight | chain | mxfp8 | chain_mx | grouped_mx |
-    # grouped_grad_input | grouped_grad_weight
+    # grouped_grad_input | grouped_grad_weight | chain_train
     recipe: str
     M: int
     N: int
@@ -153,6 +162,8 @@ class Workload:
     @property
     def flops(self) -> int:
         f = 2 * self.M * self.N * self.K
+        if self.recipe == "chain_train":   # six GEMMs of the same size
+            return 6 * f
         if "b2" in self.extra:   # the chain's second GEMM: (M, N) @ b2^T
             n2, k2 = self.extra["b2"].shape
             f += 2 * self.M * n2 * k2
@@ -247,6 +258,15 @@ def make_workload(index: int, shape_index: int = 0, scale_down: int = 1) -> Work
         w1 = randn_bf16((F, D), 0.02, g)
         w2 = randn_bf16((D, F), 0.02, g)
         return Workload(name, "chain", T, F, D, x, w1, seed=seed, extra={"b2": w2})
+    if index == 14:
+        T, D, F = 16640 // scale_down, 8192, 5120
+        T = max(128, T - T % 128)
+        x = randn_bf16((T, D), 1.0, g)
+        w1 = randn_bf16((F, D), 0.02, g)
+        w2 = randn_bf16((D, F), 0.02, g)
+        dy2 = randn_bf16((T, D), 1e-3, g)
+        return Workload(name, "chain_train", T, F, D, x, w1, seed=seed,
+                        extra={"b2": w2, "dy": dy2})
     raise ValueError(f"unknown workload {index}")
 
 
