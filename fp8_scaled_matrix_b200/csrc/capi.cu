@@ -256,6 +256,57 @@ fp8_status fp8_quantize_transposed_batched(const void* x_bf16, int32_t batch, in
   return finish_launch(e, err, n.c_str());
 }
 
+// Shape and pointer checks shared by the two steps of the sharded tensorwise
+// quantization.
+static fp8_status check_tensor_shard(const char* name, const void* x, int64_t rows,
+                                     int64_t cols, int64_t ld) {
+  const std::string n(name);
+  if (rows < 0 || cols < 0) return fail(FP8_ERR_VALUE, n + ": negative size");
+  if (rows >= (int64_t(1) << 31) || cols >= (int64_t(1) << 31))
+    return fail(FP8_ERR_VALUE, n + ": size too large");
+  if (ld < cols) return fail(FP8_ERR_VALUE, n + ": ld_x < cols");
+  if (cols % 8 != 0 || ld % 8 != 0)
+    return fail(FP8_ERR_VALUE, n + ": cols and ld_x must be multiples of 8");
+  if (rows > 0 && cols > 0 && (x == nullptr || !aligned(x, 16)))
+    return fail(FP8_ERR_VALUE, n + ": x must be a 16-byte aligned device pointer");
+  return FP8_OK;
+}
+
+fp8_status fp8_tensor_amax(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld_x,
+                           float* amax, fp8_stream_t stream) {
+  fp8_status s = check_tensor_shard("fp8_tensor_amax", x_bf16, rows, cols, ld_x);
+  if (s != FP8_OK) return s;
+  if (amax == nullptr || !aligned(amax, 4))
+    return fail(FP8_ERR_VALUE, "fp8_tensor_amax: amax must be a 4-byte aligned device pointer");
+  DeviceInfo* d = nullptr;
+  s = device_info(&d);
+  if (s != FP8_OK) return s;
+  std::string err;
+  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status, d->num_sms, &err};
+  return finish_launch(fp8sm::launch_tensor_amax(x_bf16, rows, cols, ld_x, amax, ctx), err,
+                       "fp8_tensor_amax");
+}
+
+fp8_status fp8_quantize_tensor_with_amax(const void* x_bf16, int64_t rows, int64_t cols,
+                                         int64_t ld_x, const float* amax, void* out_fp8,
+                                         float* out_scale, fp8_stream_t stream) {
+  const char* n = "fp8_quantize_tensor_with_amax";
+  fp8_status s = check_tensor_shard(n, x_bf16, rows, cols, ld_x);
+  if (s != FP8_OK) return s;
+  if (amax == nullptr || out_scale == nullptr || !aligned(amax, 4) || !aligned(out_scale, 4))
+    return fail(FP8_ERR_VALUE, std::string(n) + ": amax and out_scale must be 4-byte aligned "
+                                                "device pointers");
+  if (rows > 0 && cols > 0 && (out_fp8 == nullptr || !aligned(out_fp8, 16)))
+    return fail(FP8_ERR_VALUE, std::string(n) + ": out_fp8 must be 16-byte aligned");
+  DeviceInfo* d = nullptr;
+  s = device_info(&d);
+  if (s != FP8_OK) return s;
+  std::string err;
+  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status, d->num_sms, &err};
+  return finish_launch(
+      fp8sm::launch_tensor_cast(x_bf16, rows, cols, ld_x, amax, out_fp8, out_scale, ctx), err, n);
+}
+
 fp8_status fp8_quantize_noalloc(const void* x_bf16, int64_t rows, int64_t cols,
                                 int64_t ld_x, fp8_quant_recipe recipe,
                                 void* out_fp8, float* out_scales,

@@ -21,6 +21,15 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t cols,
                             int64_t ld, int recipe, void* q, float* scales,
                             void* workspace, const LaunchCtx& ctx);
 
+// Sharded tensorwise quantization (quantize.cu): max|x| of a shard into
+// amax[0] (device; cleared first), then the cast of a shard with the scale
+// of a given amax (written to scale[0]).  cols % 8 == 0.
+cudaError_t launch_tensor_amax(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                               float* amax, const LaunchCtx& ctx);
+cudaError_t launch_tensor_cast(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                               const float* amax, void* q, float* scale,
+                               const LaunchCtx& ctx);
+
 // Quantization of x^T (quantize.cu), recipe 2 (1x128) or 3 (128x128);
 // rows % 128 == 0.  q is (cols, rows) with row stride rows.
 cudaError_t launch_quantize_transposed(const void* x, int64_t rows, int64_t cols,

@@ -629,6 +629,43 @@ __global__ void __launch_bounds__(256) quant_tensor_kernel(
 
 int g_tensor_blocks_per_sm = -1;
 
+// Sharded tensorwise quantization, step 1: max|x| of this shard folded into
+// amax[0] (fp32 bits, atomic max; amax[0] must be zero on entry).
+__global__ void __launch_bounds__(256) tensor_amax_kernel(
+    const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+    uint32_t* amax) {
+  __shared__ float warp_amax[8];
+  const int64_t nvec = cols >> 3;
+  float m = 0.0f;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + r * ld);
+    for (int64_t c = threadIdx.x; c < nvec; c += blockDim.x) m = amax8(__ldg(xr + c), m);
+  }
+  m = warp_max(m);
+  if ((threadIdx.x & 31) == 0) warp_amax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float bm = warp_amax[0];
+    for (int i = 1; i < (int)(blockDim.x >> 5); ++i) bm = fmaxf(bm, warp_amax[i]);
+    atomicMax(amax, __float_as_uint(bm));
+  }
+}
+
+// Step 2 (after the caller's all-reduce(MAX) of amax over the shards): the
+// tensorwise scale of the whole tensor and the cast of this shard.
+__global__ void __launch_bounds__(256) tensor_cast_kernel(
+    const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+    const float* amax, uint8_t* __restrict__ q, float* __restrict__ scale) {
+  const ScalePair sp = scales_from_amax(*amax);
+  if (blockIdx.x == 0 && threadIdx.x == 0) scale[0] = sp.s;
+  const int64_t nvec = cols >> 3;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + r * ld);
+    uint2* qr = reinterpret_cast<uint2*>(q + r * cols);
+    for (int64_t c = threadIdx.x; c < nvec; c += blockDim.x) qr[c] = cast8(__ldg(xr + c), sp.inv);
+  }
+}
+
 // Scratch for fp8_quantize_noalloc: a fixed array in device memory that the
 // library owns.  Every GPU that loads the library holds one copy until the
 // process exits.  All calls share it; a call leaves its contents behind, so
@@ -832,6 +869,28 @@ cudaError_t launch_quantize(const void* xv, int64_t rows, int64_t cols,
                   (void*)&q, (void*)&scales, (void*)&ws, (void*)&status};
   return cudaLaunchCooperativeKernel((const void*)quant_tensor_kernel, dim3(g),
                                      dim3(256), args, 0, st);
+}
+
+static unsigned tensor_grid(int64_t rows, const LaunchCtx& ctx) {
+  const int64_t g = rows < 8 * static_cast<int64_t>(ctx.num_sms) ? rows : 8 * ctx.num_sms;
+  return static_cast<unsigned>(g < 1 ? 1 : g);
+}
+
+cudaError_t launch_tensor_amax(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                               float* amax, const LaunchCtx& ctx) {
+  cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float), ctx.stream);
+  if (e != cudaSuccess || rows == 0 || cols == 0) return e;
+  tensor_amax_kernel<<<tensor_grid(rows, ctx), 256, 0, ctx.stream>>>(
+      static_cast<const uint16_t*>(x), rows, cols, ld, reinterpret_cast<uint32_t*>(amax));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tensor_cast(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                               const float* amax, void* q, float* scale,
+                               const LaunchCtx& ctx) {
+  tensor_cast_kernel<<<tensor_grid(rows, ctx), 256, 0, ctx.stream>>>(
+      static_cast<const uint16_t*>(x), rows, cols, ld, amax, static_cast<uint8_t*>(q), scale);
+  return cudaGetLastError();
 }
 
 }  // namespace fp8sm

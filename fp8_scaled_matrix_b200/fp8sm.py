@@ -39,7 +39,8 @@ EXPORTED = ["fp8_version", "fp8_last_error", "fp8_quantize_workspace_bytes",
             "fp8_scaled_mm_mx_quantized", "fp8_grouped_scaled_mm_mx",
             "fp8_grouped_padded_tokens", "fp8_quantize_transposed_grouped",
             "fp8_grouped_scaled_mm_wgrad", "fp8_quantize_batched",
-            "fp8_quantize_transposed_batched", "fp8_scaled_mm_quantized_dual"]
+            "fp8_quantize_transposed_batched", "fp8_scaled_mm_quantized_dual",
+            "fp8_tensor_amax", "fp8_quantize_tensor_with_amax"]
 
 
 class Fp8Error(RuntimeError):
@@ -98,6 +99,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fp8_scaled_mm_quantized.argtypes = [P, P, I64, I64, I64, P, P, E, P, P, P, P]
     L.fp8_grouped_scaled_mm.restype = E
     L.fp8_grouped_scaled_mm.argtypes = [P, P, I64, I64, I64, I32, P, P, P, E, P, P]
+    L.fp8_tensor_amax.restype = E
+    L.fp8_tensor_amax.argtypes = [P, I64, I64, I64, P, P]
+    L.fp8_quantize_tensor_with_amax.restype = E
+    L.fp8_quantize_tensor_with_amax.argtypes = [P, I64, I64, I64, P, P, P, P]
     L.fp8_scaled_mm_quantized_dual.restype = E
     L.fp8_scaled_mm_quantized_dual.argtypes = [P, P, I64, I64, I64, P, P, E, P, P, P, P, P, P]
     L.fp8_quantize_batched.restype = E
@@ -613,3 +618,67 @@ def fp8_scaled_mm_quantized_dual(a: torch.Tensor, b: torch.Tensor, scale_a: torc
                                           _ptr(out_scales), _ptr(out_t), _ptr(out_t_scales),
                                           _stream(stream)))
     return out, out_scales, out_t, out_t_scales
+
+
+# ----------------------------------------- tensorwise over row shards (ranks)
+
+def _check_shard(x: torch.Tensor):
+    _need_cuda(x)
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D bf16 tensor with unit column stride")
+    rows, cols = x.shape
+    return rows, cols, (x.stride(0) if (rows > 1 and cols > 0) else cols)
+
+
+def fp8_tensor_amax(x: torch.Tensor, out: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+    """max |x| of a bf16 shard, as a (1,) float32 device tensor."""
+    L = load_library()
+    rows, cols, ld = _check_shard(x)
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=x.device)
+    _check(L.fp8_tensor_amax(_ptr(x), rows, cols, ld, _ptr(out), _stream(stream)))
+    return out
+
+
+def fp8_quantize_tensor_with_amax(x: torch.Tensor, amax: torch.Tensor,
+                                  out: Optional[torch.Tensor] = None,
+                                  scale: Optional[torch.Tensor] = None,
+                                  stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Tensorwise cast of a shard with the scale of a given amax (device
+    float, e.g. all-reduced over the ranks).  Returns (codes, scale (1,))."""
+    L = load_library()
+    rows, cols, ld = _check_shard(x)
+    _need_cuda(amax)
+    if amax.dtype != torch.float32 or amax.numel() < 1:
+        raise ValueError("amax must be a float32 device tensor")
+    if out is None:
+        out = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    if scale is None:
+        scale = torch.empty(1, dtype=torch.float32, device=x.device)
+    _check(L.fp8_quantize_tensor_with_amax(_ptr(x), rows, cols, ld, _ptr(amax), _ptr(out),
+                                           _ptr(scale), _stream(stream)))
+    return out, scale
+
+
+def allreduce_amax(amax: torch.Tensor, group=None) -> torch.Tensor:
+    """The one exchange of the sharded tensorwise quantization: max over the
+    ranks of the process group (in place), when one is initialised."""
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
+        dist.all_reduce(amax, op=dist.ReduceOp.MAX, group=group)
+    return amax
+
+
+def fp8_quantize_tensorwise_sharded(x: torch.Tensor, group=None,
+                                    stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Tensorwise quantization of this rank's row shard of a tensor with the
+    scale of the whole tensor: shard amax, all-reduce(MAX) over the group,
+    cast.  Returns (codes, scale (1,)), the scale equal on every rank."""
+    amax = fp8_tensor_amax(x, stream=stream)
+    if stream is None:
+        allreduce_amax(amax, group)
+    else:
+        with torch.cuda.stream(stream):   # the collective is ordered on that stream
+            allreduce_amax(amax, group)
+    return fp8_quantize_tensor_with_amax(x, amax, stream=stream)

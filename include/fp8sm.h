@@ -161,6 +161,33 @@ FP8SM_API fp8_status fp8_quantize_noalloc(const void* x_bf16, int64_t rows,
                                           fp8_stream_t stream);
 
 /*
+ * Tensorwise quantization of a tensor split by rows across ranks (one process
+ * per GPU, each holding a row shard), with the scale of the WHOLE tensor:
+ * the "tensorwise" recipe of [P4]'s recipe table has one scale per tensor,
+ * i.e. one amax over all of it (then [P3] Highlights' scale and cast steps),
+ * so the ranks exchange their shard maxima once (an all-reduce(MAX) of one
+ * fp32 value, done by the caller, e.g. over NCCL) between the two steps.
+ *   fp8_tensor_amax               amax[0] = max |x| over the shard (0 for an
+ *                                 empty shard); amax is device memory, which
+ *                                 the call clears first.
+ *   fp8_quantize_tensor_with_amax with a = max(amax[0], 1e-12): out_scale[0] =
+ *                                 a / 448 and out_fp8 = e4m3_satfinite(x * (448
+ *                                 / a)), the steps of fp8_quantize's tensorwise
+ *                                 recipe; amax is read on the device.
+ * With one shard the two steps give exactly fp8_quantize(FP8_SCALE_TENSOR).
+ * Layouts as fp8_quantize: x bf16 (rows, cols) row stride ld_x, out_fp8
+ * (rows, cols) row stride cols.  Requirements: cols % 8 == 0, ld_x % 8 == 0,
+ * x and out_fp8 16-byte aligned, amax and out_scale 4-byte aligned.  Errors:
+ * FP8_ERR_VALUE for sizes, null or misaligned pointers.
+ */
+FP8SM_API fp8_status fp8_tensor_amax(const void* x_bf16, int64_t rows, int64_t cols,
+                                     int64_t ld_x, float* amax, fp8_stream_t stream);
+FP8SM_API fp8_status fp8_quantize_tensor_with_amax(const void* x_bf16, int64_t rows,
+                                                   int64_t cols, int64_t ld_x,
+                                                   const float* amax, void* out_fp8,
+                                                   float* out_scale, fp8_stream_t stream);
+
+/*
  * Transposed dynamic quantization, for the training GEMMs of [P5] (the
  * 1x128_128x128 GEMM also serves grad_input = grad_output @ weight, the
  * 1x128_128x1 GEMM serves grad_weight = grad_output_t @ input) and [P1]'s

@@ -188,6 +188,23 @@ def test_scaled_mm_quantized_dual_null_alignment_and_empty(lib):
                                             None, None, None, None, None) == fp8sm.FP8_OK
 
 
+def test_tensor_amax_and_cast_reject_bad_arguments(lib):
+    st = lib.fp8_tensor_amax(FAKE, 4, 12, 12, FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE and "multiples of 8" in lib.fp8_last_error().decode()
+    st = lib.fp8_tensor_amax(FAKE, 4, 16, 8, FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE and "ld_x < cols" in lib.fp8_last_error().decode()
+    st = lib.fp8_tensor_amax(FAKE, 4, 16, 16, None, None)
+    assert st == fp8sm.FP8_ERR_VALUE and "amax" in lib.fp8_last_error().decode()
+    st = lib.fp8_tensor_amax(P((1 << 20) + 8), 4, 16, 16, FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE and "aligned" in lib.fp8_last_error().decode()
+    st = lib.fp8_quantize_tensor_with_amax(FAKE, 4, 16, 16, FAKE, FAKE, None, None)
+    assert st == fp8sm.FP8_ERR_VALUE and "out_scale" in lib.fp8_last_error().decode()
+    st = lib.fp8_quantize_tensor_with_amax(FAKE, 4, 16, 16, FAKE, None, FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE and "out_fp8" in lib.fp8_last_error().decode()
+    st = lib.fp8_quantize_tensor_with_amax(FAKE, -1, 16, 16, FAKE, FAKE, FAKE, None)
+    assert st == fp8sm.FP8_ERR_VALUE and "negative" in lib.fp8_last_error().decode()
+
+
 def test_grouped_requires_offs(lib):
     st = lib.fp8_grouped_scaled_mm(FAKE, FAKE, 64, 128, 128, 4, FAKE, FAKE, None,
                                    fp8sm.FP8_OUT_BF16, FAKE, None)
