@@ -144,6 +144,7 @@ struct GemmParams {
   int32_t n_tiles;   // tiles along N
   int32_t m_tiles;   // tiles along M (dense)
   int32_t k_blocks;
+  int32_t raster_m;  // dense: 0 = M-major tile order, else bands of this many M tiles
   uint32_t* status;
   // Dense kernels: work items [0, split_start) are whole 128 x 256 tiles in
   // M-major order; when the last wave would leave more than half of the SMs
@@ -212,7 +213,7 @@ struct KGroupCursor {
 };
 
 // Work item t -> output tile (rows m0 .. m0 + kTM - 1).
-template <bool kGrouped, int kTM>
+template <bool kGrouped, int kTM, bool kRaster>
 __device__ __forceinline__ TileCoord tile_coord(int64_t t, const GemmParams& p,
                                                 GroupCursor& cur) {
   TileCoord c;
@@ -228,8 +229,22 @@ __device__ __forceinline__ TileCoord tile_coord(int64_t t, const GemmParams& p,
   }
   c.kb0 = 0;
   c.nkb = 0;
-  const int64_t mt = t / p.n_tiles;
-  c.n0 = static_cast<int32_t>((t % p.n_tiles) * BN) + sub * (BN / 2);
+  int64_t mt = t / p.n_tiles;
+  int64_t nt = t % p.n_tiles;
+  if constexpr (!kGrouped && kRaster) {
+    if (p.raster_m > 0) {
+      // grouped raster: bands of raster_m M tiles, N-major inside a band,
+      // so that a wave touches a band of A and a slice of B that fit in L2
+      const int64_t per = static_cast<int64_t>(p.raster_m) * p.n_tiles;
+      const int64_t band = t / per;
+      const int64_t local = t - band * per;
+      const int64_t left = p.m_tiles - band * p.raster_m;
+      const int64_t gm = left < p.raster_m ? left : p.raster_m;
+      mt = band * p.raster_m + local % gm;
+      nt = local / gm;
+    }
+  }
+  c.n0 = static_cast<int32_t>(nt * BN) + sub * (BN / 2);
   if constexpr (kGrouped) {
     cur.seek(mt, p.offs, p.E, kTM);
     c.g = cur.g;
@@ -417,6 +432,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr bool kOutQT = kOut == kOutE4M3Dual;
   constexpr bool kOutQ = kOut == kOutE4M3 || kOutQT;
   constexpr bool kOutMxq = kOut == kOutMx;
+  // the banded tile order (large B operands); the dual-output kernel, whose
+  // epilogue is at the edge of its register budget, keeps the M-major order
+  // (its B is a layer's weight, which fits in L2)
+  constexpr bool kRaster = !kOutQT;
   using C = Cfg<kPair>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -540,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
         const TileCoord c =
-            kKGroups ? kgroup_coord(t, p, kc) : tile_coord<kGrouped, kTM>(t, p, cur);
+            kKGroups ? kgroup_coord(t, p, kc) : tile_coord<kGrouped, kTM, kRaster>(t, p, cur);
         const int32_t nkb = kKGroups ? c.nkb : KB;
         for (int32_t kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait<kPair>(&empty[stage], phase ^ 1u, abort_flag, p.status,
@@ -813,7 +832,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       else if constexpr (kGrouped) cur.init(p.offs, kTM);
       for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
         const TileCoord c =
-            kKGroups ? kgroup_coord(t, p, kc) : tile_coord<kGrouped, kTM>(t, p, cur);
+            kKGroups ? kgroup_coord(t, p, kc) : tile_coord<kGrouped, kTM, kRaster>(t, p, cur);
         const int32_t nkb = kKGroups ? c.nkb : KB;
         for (int32_t kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&sempty[slot], sphase ^ 1u, abort_flag, p.status, SITE_SCALE_EMPTY,
@@ -871,7 +890,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t stage = 0, phase = 0;
       bool ok = true;
       for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
-        const TileCoord c = tile_coord<kGrouped, kTM>(t, p, cur);
+        const TileCoord c = tile_coord<kGrouped, kTM, kRaster>(t, p, cur);
         for (int32_t kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, SITE_SCALE_EMPTY,
                          kWaitLimitNs)) {
@@ -944,7 +963,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
       const TileCoord c =
-          kKGroups ? kgroup_coord(t, p, kc) : tile_coord<kGrouped, kTM>(t, p, cur);
+          kKGroups ? kgroup_coord(t, p, kc) : tile_coord<kGrouped, kTM, kRaster>(t, p, cur);
       // this CTA's output rows (K-grouped: group g's block of the output)
       const int32_t cta_m0 = c.out_m0 + static_cast<int32_t>(rank) * BM;
       const int64_t row = static_cast<int64_t>(cta_m0) + q * 32 + lane;
@@ -1595,6 +1614,12 @@ cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
   p.n_tiles = static_cast<int32_t>((N + BN - 1) / BN);
   p.m_tiles = static_cast<int32_t>((M + tile_m - 1) / tile_m);
   p.k_blocks = static_cast<int32_t>((K + BK - 1) / BK);
+  // Tile order: M-major keeps a band of A and all of B in L2 while B's codes
+  // fit there comfortably; a larger B (the grad_weight shapes, K = tokens)
+  // would be streamed from HBM once per wave, so the tiles go in bands of 16
+  // M tiles instead, N-major inside a band: a wave then reads a band of A
+  // and a slice of B, both L2-resident.
+  p.raster_m = (N * K > (int64_t(64) << 20)) ? 16 : 0;
   p.status = ctx.status;
   const int64_t tiles = static_cast<int64_t>(p.n_tiles) * p.m_tiles;
   const int64_t G = pair ? ctx.num_sms / 2 : ctx.num_sms;  // CTAs or CTA pairs

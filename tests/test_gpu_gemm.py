@@ -144,3 +144,28 @@ def test_gemm_parity_cta_pairs(recipe, M, N, K, bias, monkeypatch):
     selected with FP8SM_CTA_PAIRS=1, against the oracle."""
     monkeypatch.setenv("FP8SM_CTA_PAIRS", "1")
     test_gemm_parity(recipe, M, N, K, bias, torch.float32)
+
+
+@pytest.mark.parametrize("recipe,pairs", [
+    ("row", False), ("row", True), ("tensor", False),
+    ("1x128_128x128", False), ("1x128_128x1", False),
+])
+def test_gemm_banded_tile_order_large_b(recipe, pairs, monkeypatch):
+    """B's codes above 64 MiB (N = 8192, K = 8320): the dense kernels take
+    their tiles in bands of 16 M tiles, N-major inside a band.  M = 2500 gives
+    20 M tiles of 128 rows (a full band and a partial one) or 10 of 256 rows
+    (CTA pairs: one partial band).  Sampled rows of every band, fp32 output,
+    against the oracle."""
+    if pairs:
+        monkeypatch.setenv("FP8SM_CTA_PAIRS", "1")
+    M, N, K = 2500, 8192, 8320
+    b_std = 0.02 if recipe != "1x128_128x1" else 1.0
+    a_std = 1.0 if recipe != "1x128_128x1" else 1e-3
+    wl = W.small_case(recipe, M, N, K, seed=907 + len(recipe), a_std=a_std, b_std=b_std,
+                      bias=recipe == "row")
+    qa, sa, qb, sb = oracle_operands(wl)
+    out = gpu_gemm(qa, sa, qb, sb, recipe, wl.bias, torch.float32)
+    rows = sample_rows(M, 24, seed=7)
+    bias_bits = None if wl.bias is None else W.bf16_bits(wl.bias)
+    ref, mag = oracle.scaled_mm(qa, qb, sa, sb, MM[recipe], bias_bits=bias_bits, rows=rows)
+    check_gemm(out_f64(out)[rows], ref, mag, f"{recipe} banded order")

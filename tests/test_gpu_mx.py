@@ -76,6 +76,7 @@ CASES = [
     (257, 4352, 160, False),       # 17 N tiles, last one half empty
     (2048, 4096, 256, False),      # more tiles than SMs
     (4096, 4096, 256, True),       # last wave split into 128-wide items
+    (2500, 8192, 8320, True),      # B's codes above 64 MiB: banded tile order
 ]
 
 
