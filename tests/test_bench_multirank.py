@@ -34,7 +34,7 @@ def _rank_main(rank, world, port, out):
 def test_max_over_ranks_and_job_throughput_two_gloo_ranks():
     world = 2
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.start_processes(_rank_main, args=(world, port, out), nprocs=world,
                            start_method="spawn", join=True)

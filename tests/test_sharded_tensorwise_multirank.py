@@ -54,7 +54,7 @@ def _rank_main(rank, world, port, out):
 def test_allreduce_amax_gives_the_whole_tensors_amax_on_every_rank():
     world = 2
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.start_processes(_rank_main, args=(world, port, out), nprocs=world,
                            start_method="spawn", join=True)
