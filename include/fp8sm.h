@@ -300,9 +300,14 @@ FP8SM_API fp8_status fp8_scaled_mm_quantized(const void* a, const void* b, int64
  *                             fp8_quantize_transposed(y, 1x128) of the fp32
  *                             values (the next grad_weight's operand):
  *                             scale[(m/128) * N + n], codes row n = tokens.
+ * a (M, K) and b (N, K) e4m3 codes with the recipe's scales as for
+ * fp8_scaled_mm; all buffers are caller-owned device memory; the call is
+ * asynchronous on `stream`.
  * Recipe FP8_MM_1x128_128x128 only (others: FP8_ERR_UNSUPPORTED).
  * Requirements: M % 128 == 0, N % 128 == 0, K > 0, K % 128 == 0; code
- * buffers 16-byte aligned, scales 4-byte aligned.
+ * buffers 16-byte aligned, scales 4-byte aligned.  Errors: FP8_ERR_VALUE
+ * (sizes, null or misaligned pointers; nothing is launched), FP8_ERR_CUDA
+ * (launch); M == 0 or N == 0 returns FP8_OK without a launch.
  */
 FP8SM_API fp8_status fp8_scaled_mm_quantized_dual(const void* a, const void* b, int64_t M,
                                         int64_t N, int64_t K, const float* scale_a,
