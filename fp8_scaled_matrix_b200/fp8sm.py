@@ -663,7 +663,8 @@ def fp8_quantize_tensor_with_amax(x: torch.Tensor, amax: torch.Tensor,
 
 def allreduce_amax(amax: torch.Tensor, group=None) -> torch.Tensor:
     """The one exchange of the sharded tensorwise quantization: max over the
-    ranks of the process group (in place), when one is initialised."""
+    ranks of the process group (in place), when one is initialised.  The
+    group's backend must reduce tensors on amax's device (NCCL for CUDA)."""
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
         dist.all_reduce(amax, op=dist.ReduceOp.MAX, group=group)
