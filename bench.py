@@ -11,14 +11,20 @@ outside the per-step CUDA events (and read back, so that L2 holds clean lines).
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl ours|reference]
 
-Prints ONE JSON line (rank 0).  `value` is GEMM TFLOP/s over the whole step
-(quantize + GEMM) summed over ranks; `roofline` describes the GEMM kernel
-alone against the measured peak; `e2e` is the same metric through the public
-API with host buffers and the copies inside the timed region;
-`cpu_baseline` is the CPU oracle on a bounded sample of the same workload.
+Prints ONE JSON line (rank 0).  The default workload is the blockwise
+1x128_128x128 GEMM at M=16640, N=5120, K=8192.  `value` is GEMM TFLOP/s over
+the whole step (quantize + GEMM) summed over ranks; `roofline` describes the
+GEMM kernel alone against the measured peak (and the nominal one);
+`all_configs` times the quantize step and the GEMM of each of the five
+benchmark configurations (both (N, K) shapes of the blockwise pair) in the
+same process, with the same L2 flush; `e2e` is the same metric through the
+public API with host buffers and the copies inside the timed region;
+`cpu_baseline` is the CPU oracle on a bounded sample of the same workload;
+`clocks` summarises NVML samples taken inside the timed window.
 
 With --impl reference the oracle itself is timed on the host cores (rank 0
-only), as the reference arm.
+only), as the reference arm: every step is the same bounded sample, and the
+line reports the time of the steps it ran.
 """
 from __future__ import annotations
 
@@ -60,7 +66,9 @@ WORKLOADS = {
     "grouped_e16_grad_weight": (13, 0),
     "linear_chain_train_1x128": (14, 0),
 }
-DEFAULT_WORKLOAD = "rowwise_4096"
+# The headline: the blockwise 1x128_128x128 GEMM, M=16640, N=5120, K=8192
+# (the first shape of the "improve fp8 blockwise gemm perf" benchmark table)
+DEFAULT_WORKLOAD = "blockwise_1x128_128x128"
 # Page 5's context numbers (TFLOP/s of torch._scaled_mm, hardware not stated)
 PAGE_NUMBERS = {
     "blockwise_1x128_128x128": 1008.91, "blockwise_1x128_128x128_b": 1002.23,
@@ -82,6 +90,7 @@ GEMM_RECIPE = {"grad_input": "1x128_128x128", "grad_weight": "1x128_128x1",
 TRANSPOSED = {"grad_input": (False, True), "grad_weight": (True, True)}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_OVER_BF16 = 2.0   # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+NOMINAL_FP8_TFLOPS = 4500.0   # B200 dense FP8, nominal
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -150,60 +159,80 @@ def job_tflops(flops_per_rank: float, world: int, ms: float) -> float:
 # ----------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock, power and clock-event reasons of one GPU, read through NVML
+    every few milliseconds on a background thread (nvidia-smi's fields,
+    sampled fast enough that a timed region of a few milliseconds still gets
+    samples).  `window(t0, t1)` summarises the samples taken between two
+    host times (time.perf_counter())."""
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4),
+               ("hw_power_brake_slowdown", 0x80))
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.lines = []
-        self.t = None
+    def __init__(self, dev: torch.device, interval_s: float = 0.004):
+        self.dev = dev
+        self.interval = interval_s
+        self.samples = []      # (t, sm_mhz, power_w, reasons bitmask, gpu util %)
+        self.max_mhz = None
+        self.handle = None
+        self.source = None
+        self._stop = threading.Event()
+        self._t = None
+
+    def _open(self):
+        import pynvml
+        pynvml.nvmlInit()
+        h = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.dev.index or 0)
+        self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+        return pynvml, h
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
+            nv, h = self._open()
         except Exception:
-            self.proc = None
+            self.source = "unavailable"
+            return
+        self.source = "nvml"
+        getr = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons",
+                       getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+        def run():
+            while not self._stop.is_set():
+                try:
+                    t = time.perf_counter()
+                    sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                    pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                    rs = int(getr(h)) if getr else 0
+                    ut = nv.nvmlDeviceGetUtilizationRates(h).gpu
+                    self.samples.append((t, sm, pw, rs, ut))
+                except Exception:
+                    pass
+                self._stop.wait(self.interval)
+        self._t = threading.Thread(target=run, daemon=True)
+        self._t.start()
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        if self.t:
-            self.t.join(timeout=2)
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        self._stop.set()
+        if self._t is not None:
+            self._t.join(timeout=2)
+
+    def window(self, t0: float, t1: float) -> dict:
+        """Samples taken inside [t0, t1]: median SM clock, the reasons seen
+        active, and how many samples fell in the window and under load (GPU
+        utilisation above zero)."""
+        sel = [x for x in self.samples if t0 <= x[0] <= t1]
+        load = [x for x in sel if x[4] > 0]
+        use = load or sel
+        reasons = sorted({n for x in use for n, bit in self.REASONS if x[3] & bit})
+        return {"sm_mhz": float(np.median([x[1] for x in use])) if use else None,
+                "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(sel), "samples_under_load": len(load),
+                "power_w_max": max((x[2] for x in sel), default=None),
+                "window_ms": (t1 - t0) * 1e3, "source": self.source}
 
 
 # ------------------------------------------------------------- our path
@@ -548,7 +577,7 @@ def capture(fn, pool=None):
     return g
 
 
-def run_ours(args, wl, dev, rank, world):
+def run_ours(args, wl, dev, rank, world, sampler):
     torch.cuda.set_device(dev)
     st = make_step(wl, dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -573,12 +602,10 @@ def run_ours(args, wl, dev, rank, world):
 
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-    sampler = ClockSampler(dev.index if dev.index is not None else 0)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    sampler.start()
-    time.sleep(0.25)  # let the sampler start before the timed work
+    t0 = time.perf_counter()
     for i in range(K):
         evict_l2(flush)  # outside the step's events
         ev[i][0].record(stream)
@@ -587,9 +614,9 @@ def run_ours(args, wl, dev, rank, world):
         gemm()
         ev[i][2].record(stream)
     torch.cuda.synchronize()
+    t1 = time.perf_counter()
     if world > 1:
         torch.distributed.barrier()
-    clocks = sampler.stop()
     st.f.check_device_status()
     q_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
     g_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
@@ -600,11 +627,71 @@ def run_ours(args, wl, dev, rank, world):
         "q_ms": float(np.mean(q_ms)), "g_ms": float(np.mean(g_ms)),
         "g_ms_median": float(np.median(g_ms)), "q_ms_median": float(np.median(q_ms)),
         "quant_bytes": st.quant_bytes(), "launches": st.launches_per_step * K,
-        "clocks": clocks,
+        "clocks": sampler.window(t0, t1),
     }
+    del st, flush
+    if args.graphs:
+        del gq, gg
+    torch.cuda.empty_cache()
     if not args.no_e2e:
         res["e2e"] = run_e2e(args, wl, dev, world)
     return res
+
+
+# The five configurations the benchmark is specified on, as workloads: the
+# tensorwise 256^3 GEMM, the rowwise 4096^3 linear, the blockwise
+# 1x128_128x128 and 1x128_128x1 GEMMs at both (N, K) shapes of the
+# "improve fp8 blockwise gemm perf" tables, and the grouped MoE GEMM.
+ALL_CONFIGS = ("tensorwise_256", "rowwise_4096", "blockwise_1x128_128x128",
+               "blockwise_1x128_128x128_b", "blockwise_1x128_128x1", "blockwise_1x128_128x1_b",
+               "grouped_e16")
+
+
+def measure_config(name: str, dev, reps: int, fp8_peak: float, hbm_peak: float) -> dict:
+    """One workload's quantize step and GEMM, each timed on its own with CUDA
+    events (L2 flushed before every timed launch, outside the events; the
+    launches replayed from CUDA graphs); medians over `reps`."""
+    idx, shape_index = WORKLOADS[name]
+    wl = W.make_workload(idx, shape_index)
+    st = make_step(wl, dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    for _ in range(3):
+        st.quantize()
+        st.gemm()
+    torch.cuda.synchronize()
+    st.f.check_device_status()
+    gq = capture(st.quantize)
+    gg = capture(st.gemm, pool=gq.pool())
+    stream = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(reps)]
+    for i in range(reps):
+        evict_l2(flush)
+        ev[i][0].record(stream)
+        gq.replay()
+        ev[i][1].record(stream)
+        evict_l2(flush)
+        ev[i][2].record(stream)
+        gg.replay()
+        ev[i][3].record(stream)
+    torch.cuda.synchronize()
+    st.f.check_device_status()
+    q_us = float(np.median([e[0].elapsed_time(e[1]) for e in ev])) * 1e3
+    g_us = float(np.median([e[2].elapsed_time(e[3]) for e in ev])) * 1e3
+    qbytes = st.quant_bytes()
+    out = {"M": wl.M, "N": wl.N, "K": wl.K, "recipe": wl.recipe, "E": wl.E or None,
+           "gemm_us": g_us, "quantize_us": q_us, "reps": reps}
+    if name == "tensorwise_256":
+        out["note"] = "launch-latency bound (33.6 MFLOP): microseconds only"
+    else:
+        tf = wl.flops / (g_us * 1e-6) / 1e12
+        gbs = qbytes / (q_us * 1e-6) / 1e9
+        out.update({"gemm_tflops": tf, "gemm_frac": tf / fp8_peak,
+                    "gemm_frac_nominal": tf / NOMINAL_FP8_TFLOPS,
+                    "quantize_gbs": gbs, "quantize_frac": gbs / hbm_peak,
+                    "quantize_bytes": qbytes})
+    del gq, gg, st, flush
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_e2e(args, wl, dev, world):
@@ -838,36 +925,94 @@ def oracle_sample(wl, max_rows: int):
     return tg, rows.size / wl.M, tq, oracle.num_threads()
 
 
-def cpu_baseline(wl, rows: int):
+DENSE_RECIPES = ("tensor", "row", "1x128_128x128", "1x128_128x1")
+_B_CODES = {}   # oracle codes of a workload's B operand, made once per process
+
+
+def oracle_dense_sample(wl, rows: int):
+    """A proportional slice of one step of a dense workload on the CPU
+    oracle: quantize rows [0, r) of A and the matching share of B's rows
+    (rounded up to whole 128-row groups), then the GEMM of output rows
+    [0, r) (against B's codes for all N rows, made once, untimed).  Returns
+    (quantize seconds, GEMM seconds, the step's fraction r/M, threads)."""
+    import oracle
+    ga, gb = OPERAND_GROUPS[wl.recipe]
+    G = {"tensor": oracle.GROUP_TENSOR, "row": oracle.GROUP_ROW,
+         "1x128": oracle.GROUP_1x128, "128x128": oracle.GROUP_128x128}
+    MMR = {"tensor": oracle.MM_TENSOR_TENSOR, "row": oracle.MM_ROW_ROW,
+           "1x128_128x128": oracle.MM_1x128_128x128, "1x128_128x1": oracle.MM_1x128_128x1}
+    r = int(max(1, min(wl.M, rows)))
+    key = (id(wl), wl.recipe)
+    if key not in _B_CODES:
+        _B_CODES.clear()
+        _B_CODES[key] = oracle.quantize(W.bf16_bits(wl.b), G[gb])
+    qb, sb = _B_CODES[key]
+    rb = min(wl.N, -(-(r * wl.N // wl.M + 1) // 128) * 128)
+    abits, bbits = W.bf16_bits(wl.a[:r]), W.bf16_bits(wl.b[:rb])
+    t0 = time.perf_counter()
+    qa, sa = oracle.quantize(abits, G[ga])
+    oracle.quantize(bbits, G[gb])
+    tq = time.perf_counter() - t0
+    bias = None if wl.bias is None else W.bf16_bits(wl.bias)
+    t0 = time.perf_counter()
+    oracle.scaled_mm(qa, qb, sa, sb, MMR[wl.recipe], bias_bits=bias)
+    tg = time.perf_counter() - t0
+    return tq, tg, r / wl.M, oracle.num_threads()
+
+
+def sample_rows(wl, flop_budget: float = 6e10) -> int:
+    """Output rows of the oracle's sample: about `flop_budget` of GEMM work
+    (a second or two on a 16-core host), at least 8 rows (a whole 128-token
+    group for the training step), at most all of them.  Fixed by the
+    workload alone, so both benchmark arms time the same sample."""
+    per_row = wl.flops / max(1, wl.M)
+    r = int(round(flop_budget / per_row))
+    if wl.recipe == "chain_train":
+        return int(min(wl.M, max(128, -(-r // 128) * 128)))
+    return int(max(8, min(wl.M, r)))
+
+
+def cpu_baseline(wl, rows: int, repeats: int = 1):
+    """The oracle timed on a bounded sample of one step of the workload.
+    Dense recipes: a proportional slice of the step (quantize and GEMM of
+    r/M of it), value = the slice's GEMM FLOPs / its time.  Other recipes:
+    quantize of the operands in full plus the GEMM on the first rows, the
+    GEMM time scaled to all rows."""
+    if wl.recipe in DENSE_RECIPES:
+        vals, secs = [], []
+        for _ in range(repeats):
+            tq, tg, frac, threads = oracle_dense_sample(wl, rows)
+            secs.append(tq + tg)
+            vals.append(frac * wl.flops / (tq + tg) / 1e12)
+        r = int(round(frac * wl.M))
+        return {"value": float(np.median(vals)), "unit": "TFLOP/s", "cores": threads,
+                "kind": "oracle", "extrapolated": True, "sample_rows": r,
+                "sample": (f"rows 0..{r} of {wl.M}: quantize of those rows of A and of the "
+                           f"matching share of B's rows, then the GEMM of those output rows "
+                           f"({float(np.median(secs)):.2f} s, {r / wl.M:.4f} of the step); "
+                           f"the rate over the slice, scaled to all rows"),
+                "seconds_per_sample": float(np.median(secs)),
+                "seconds_est_per_step": float(np.median(secs)) * wl.M / r}
     tg, frac, tq, threads = oracle_sample(wl, rows)
     est_s = tq + tg / frac
     value = wl.flops / est_s / 1e12
+    r = int(round(frac * wl.M))
+    common = {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+              "extrapolated": True, "sample_rows": r, "seconds_per_sample": tq + tg,
+              "seconds_est_per_step": est_s}
     if wl.recipe == "chain_train":
-        t = int(round(frac * wl.M))
-        return {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                "sample": (f"quantize of W1 and W2, as stored and transposed, in full "
-                           f"({tq:.2f} s) + the rest of the step (activation quantizes, six "
-                           f"GEMMs, both quantized forms of Y1 and dY1) on the first {t} of "
-                           f"{wl.M} tokens ({tg:.2f} s), scaled to all rows"),
-                "seconds_est_per_step": est_s}
+        return dict(common, sample=(
+            f"quantize of W1 and W2, as stored and transposed, in full "
+            f"({tq:.2f} s) + the rest of the step (activation quantizes, six "
+            f"GEMMs, both quantized forms of Y1 and dY1) on the first {r} of "
+            f"{wl.M} tokens ({tg:.2f} s), scaled to all rows"))
     chain = wl.recipe in ("chain", "chain_mx")
     what = "X, W1 and W2" if chain else "both operands"
     gemm = (("both GEMMs (the first one's fp32 output quantized "
              + ("MXFP8)" if wl.recipe == "chain_mx" else "1x128)")) if chain else "GEMM")
-    return {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": (f"quantize of {what} in full ({tq:.2f} s) + {gemm} on "
-                       f"{int(round(frac * wl.M))} of {wl.M} output rows ({tg:.2f} s), "
-                       f"scaled to all rows"),
-            "seconds_est_per_step": est_s}
-
-
-def baseline_rows(wl, target_s: float = 12.0) -> int:
-    """Rows of the GEMM that take about target_s on the oracle (probe with 8)."""
-    tg, frac, _, _ = oracle_sample(wl, 8)
-    per_row = tg / max(1, int(round(frac * wl.M)))
-    if wl.recipe == "chain_train":   # samples are whole 128-token groups
-        return int(max(128, min(wl.M, 128 * round(target_s / max(per_row * 128, 1e-9)))))
-    return int(max(8, min(wl.M, target_s / max(per_row, 1e-9))))
+    return dict(common, sample=(
+        f"quantize of {what} in full ({tq:.2f} s) + {gemm} on {r} of {wl.M} output "
+        f"rows ({tg:.2f} s), scaled to all rows"))
 
 
 # ------------------------------------------------------------------ main
@@ -886,7 +1031,11 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=0,
-                    help="output rows for the CPU oracle sample (0: about 12 s of work)")
+                    help="output rows of the CPU oracle's sample (0: a fixed share of the "
+                         "workload, the same in both arms)")
+    ap.add_argument("--no-all-configs", action="store_true",
+                    help="skip timing the five benchmark configurations after the step")
+    ap.add_argument("--config-reps", type=int, default=20)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -900,24 +1049,31 @@ def main(argv=None):
         if rank != 0:
             return 0
         wl = W.make_workload(idx, shape_index)
-        steps = args.steps or 1
-        rows = args.cpu_rows or baseline_rows(wl, 20.0 / max(1, steps + args.warmup))
-        for _ in range(min(args.warmup, 1)):
-            oracle_sample(wl, max(8, rows // 4))
-        times = []
+        steps = args.steps or 3
+        rows = args.cpu_rows or sample_rows(wl)
+        # every step is the same bounded sample of the workload's step (the
+        # oracle run as it stands); warm-up samples are not timed
+        for _ in range(args.warmup):
+            cpu_baseline(wl, rows)
+        samples = []
+        t_run = time.perf_counter()
         for _ in range(steps):
-            b = cpu_baseline(wl, rows)
-            times.append(b["seconds_est_per_step"])
-        ms = float(np.mean(times)) * 1e3
-        value = wl.flops / (ms * 1e-3) / 1e12
+            samples.append(cpu_baseline(wl, rows))
+        t_run = time.perf_counter() - t_run
+        value = float(np.mean([b["value"] for b in samples]))
+        b = samples[-1]
         line = {
             "impl": "reference", "metric": "fp8_scaled_gemm_tflops", "value": value,
             "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup,
-            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": t_run / steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "fp8e4m3/int64-exact/f64", "data": "synthetic",
             "config": {"workload": args.workload, "M": wl.M, "N": wl.N, "K": wl.K},
+            "extrapolated": True,
+            "sample_rows": b["sample_rows"],
+            "est_full_step_ms": float(np.mean([x["seconds_est_per_step"] for x in samples])) * 1e3,
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": b["cores"],
-                             "kind": "oracle", "sample": b["sample"]},
+                             "kind": "oracle", "sample": b["sample"],
+                             "sample_rows": b["sample_rows"], "extrapolated": True},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0},
         }
@@ -937,16 +1093,28 @@ def main(argv=None):
         # about a second of timed work per workload
         args.steps = {"tensorwise_256": 4000, "rowwise_4096": 3000,
                       "grouped_e16": 1000}.get(args.workload, 600)
-    res = run_ours(args, wl, dev, rank, world)
-
     peaks, peak_src = load_peaks()
     fp8_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])) * FP8_OVER_BF16
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    sampler = ClockSampler(dev)
+    sampler.start()
+    try:
+        res = run_ours(args, wl, dev, rank, world, sampler)
+        configs = None
+        if world == 1 and not args.no_all_configs:
+            t0 = time.perf_counter()
+            configs = {name: measure_config(name, dev, args.config_reps, fp8_peak, hbm_peak)
+                       for name in ALL_CONFIGS}
+            configs["clocks"] = sampler.window(t0, time.perf_counter())
+    finally:
+        sampler.stop()
+
     K = args.steps
     ms_per_step = res["total_ms"] / K
     value = job_tflops(wl.flops, world, ms_per_step)
     gemm_tflops = wl.flops / (res["g_ms"] * 1e-3) / 1e12
     quant_gbs = res["quant_bytes"] / (res["q_ms"] * 1e-3) / 1e9
+    traffic = recorded_traffic(args.workload)
     line = {
         "metric": "fp8_scaled_gemm_tflops",
         "value": value,
@@ -987,9 +1155,15 @@ def main(argv=None):
         "roofline": {
             "bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak,
             "unit": "TFLOP/s", "frac": gemm_tflops / fp8_peak,
-            "traffic": recorded_traffic(args.workload),
+            "traffic": traffic,
+            "traffic_source": ("ncu capture of this GEMM kernel's sources "
+                               "(profiles/dram_traffic.json), not measured in this run"
+                               if traffic is not None else
+                               "none recorded for the current GEMM kernel sources"),
             "kernel": "fp8_gemm_kernel", "peak_source":
                 f"{peak_src} bf16 burst x {FP8_OVER_BF16:g} (nominal fp8/bf16 dense ratio)",
+            "peak_nominal": NOMINAL_FP8_TFLOPS,
+            "frac_nominal": gemm_tflops / NOMINAL_FP8_TFLOPS,
             "ms_per_launch": res["g_ms"],
         },
         "roofline_quantize": {
@@ -1000,15 +1174,18 @@ def main(argv=None):
         "gpu_launches": res["launches"],
         "clocks": res["clocks"],
     }
+    if configs is not None:
+        line["all_configs"] = configs
     if "e2e" in res:
         e = res["e2e"]
         line["e2e"] = {"value": job_tflops(wl.flops, world, e["ms"]), "unit": "TFLOP/s",
                        "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
                        "ms_per_step": e["ms"], "steps": e["steps"]}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rows = args.cpu_rows or baseline_rows(wl)
-        line["cpu_baseline"] = {k: v for k, v in cpu_baseline(wl, rows).items()
-                                if k != "seconds_est_per_step"}
+        rows = args.cpu_rows or sample_rows(wl)
+        cb = cpu_baseline(wl, rows, repeats=2)
+        line["cpu_baseline"] = {k: v for k, v in cb.items()
+                                if k not in ("seconds_est_per_step", "seconds_per_sample")}
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
