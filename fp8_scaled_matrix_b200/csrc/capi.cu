@@ -27,9 +27,10 @@ namespace {
 
 thread_local std::string t_last_error;
 
-constexpr int kMaxDevices = 64;
+using fp8sm::kMaxDevices;
 struct DeviceInfo {
   bool ready = false;
+  int device = 0;
   uint32_t* status = nullptr;
   int num_sms = 0;
 };
@@ -68,12 +69,18 @@ fp8_status device_info(DeviceInfo** out) {
       return fail(FP8_ERR_UNSUPPORTED,
                   "this library is built for sm_100a (B200); device has compute capability " +
                       std::to_string(major) + "." + std::to_string(minor));
+    d.device = dev;
     d.status = static_cast<uint32_t*>(p);
     d.num_sms = sms;
     d.ready = true;
   }
   *out = &d;
   return FP8_OK;
+}
+
+fp8sm::LaunchCtx make_ctx(const DeviceInfo* d, fp8_stream_t stream, std::string* err) {
+  return fp8sm::LaunchCtx{reinterpret_cast<cudaStream_t>(stream), d->status, d->num_sms,
+                          d->device, err};
 }
 
 bool aligned(const void* p, uintptr_t a) {
@@ -143,8 +150,7 @@ fp8_status fp8_quantize(const void* x_bf16, int64_t rows, int64_t cols,
   fp8_status s = device_info(&d);
   if (s != FP8_OK) return s;
   std::string err;
-  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status,
-                       d->num_sms, &err};
+  fp8sm::LaunchCtx ctx = make_ctx(d, stream, &err);
   cudaError_t e = fp8sm::launch_quantize(x_bf16, rows, cols, ld_x, (int)recipe,
                                          out_fp8, out_scales, workspace, ctx);
   return finish_launch(e, err, "fp8_quantize");
@@ -181,8 +187,7 @@ fp8_status fp8_quantize_transposed(const void* x_bf16, int64_t rows, int64_t col
   fp8_status s = device_info(&d);
   if (s != FP8_OK) return s;
   std::string err;
-  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status,
-                       d->num_sms, &err};
+  fp8sm::LaunchCtx ctx = make_ctx(d, stream, &err);
   cudaError_t e = fp8sm::launch_quantize_transposed(x_bf16, rows, cols, ld_x, (int)recipe,
                                                     out_fp8, out_scales, ctx);
   return finish_launch(e, err, "fp8_quantize_transposed");
@@ -215,7 +220,7 @@ fp8_status fp8_quantize_batched(const void* x_bf16, int32_t batch, int64_t rows,
   fp8_status s = device_info(&d);
   if (s != FP8_OK) return s;
   std::string err;
-  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status, d->num_sms, &err};
+  fp8sm::LaunchCtx ctx = make_ctx(d, stream, &err);
   cudaError_t e = fp8sm::launch_quantize_128x128_batched(x_bf16, batch, rows, cols, ld_x,
                                                          out_fp8, out_scales, ctx);
   return finish_launch(e, err, n.c_str());
@@ -250,7 +255,7 @@ fp8_status fp8_quantize_transposed_batched(const void* x_bf16, int32_t batch, in
   fp8_status s = device_info(&d);
   if (s != FP8_OK) return s;
   std::string err;
-  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status, d->num_sms, &err};
+  fp8sm::LaunchCtx ctx = make_ctx(d, stream, &err);
   cudaError_t e = fp8sm::launch_quantize_transposed_batched(x_bf16, batch, rows, cols, ld_x,
                                                             (int)recipe, out_fp8, out_scales, ctx);
   return finish_launch(e, err, n.c_str());
@@ -282,7 +287,7 @@ fp8_status fp8_tensor_amax(const void* x_bf16, int64_t rows, int64_t cols, int64
   s = device_info(&d);
   if (s != FP8_OK) return s;
   std::string err;
-  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status, d->num_sms, &err};
+  fp8sm::LaunchCtx ctx = make_ctx(d, stream, &err);
   return finish_launch(fp8sm::launch_tensor_amax(x_bf16, rows, cols, ld_x, amax, ctx), err,
                        "fp8_tensor_amax");
 }
@@ -302,7 +307,7 @@ fp8_status fp8_quantize_tensor_with_amax(const void* x_bf16, int64_t rows, int64
   s = device_info(&d);
   if (s != FP8_OK) return s;
   std::string err;
-  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status, d->num_sms, &err};
+  fp8sm::LaunchCtx ctx = make_ctx(d, stream, &err);
   return finish_launch(
       fp8sm::launch_tensor_cast(x_bf16, rows, cols, ld_x, amax, out_fp8, out_scale, ctx), err, n);
 }
@@ -367,8 +372,7 @@ fp8_status fp8_scaled_mm(const void* a, const void* b, int64_t M, int64_t N,
   fp8_status s = device_info(&d);
   if (s != FP8_OK) return s;
   std::string err;
-  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status,
-                       d->num_sms, &err};
+  fp8sm::LaunchCtx ctx = make_ctx(d, stream, &err);
   cudaError_t e = fp8sm::launch_scaled_mm(a, b, M, N, K, scale_a, scale_b,
                                           (int)recipe, bias_bf16,
                                           out_dtype == FP8_OUT_F32 ? 1 : 0, out, nullptr, ctx);
@@ -408,8 +412,7 @@ fp8_status fp8_scaled_mm_quantized(const void* a, const void* b, int64_t M, int6
   fp8_status s = device_info(&d);
   if (s != FP8_OK) return s;
   std::string err;
-  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status,
-                       d->num_sms, &err};
+  fp8sm::LaunchCtx ctx = make_ctx(d, stream, &err);
   cudaError_t e = fp8sm::launch_scaled_mm(a, b, M, N, K, scale_a, scale_b, (int)recipe,
                                           bias_bf16, 2, out_fp8, out_scales, ctx);
   return finish_launch(e, err, "fp8_scaled_mm_quantized");
@@ -440,7 +443,7 @@ fp8_status fp8_quantize_mx(const void* x_bf16, int64_t rows, int64_t cols, int64
   fp8_status s = device_info(&d);
   if (s != FP8_OK) return s;
   std::string err;
-  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status, d->num_sms, &err};
+  fp8sm::LaunchCtx ctx = make_ctx(d, stream, &err);
   cudaError_t e = fp8sm::launch_quantize_mx(x_bf16, rows, cols, ld_x, out_fp8,
                                             out_scales_e8m0, ctx);
   return finish_launch(e, err, "fp8_quantize_mx");
@@ -472,7 +475,7 @@ fp8_status fp8_scaled_mm_mx(const void* a, const void* b, int64_t M, int64_t N, 
   fp8_status s = device_info(&d);
   if (s != FP8_OK) return s;
   std::string err;
-  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status, d->num_sms, &err};
+  fp8sm::LaunchCtx ctx = make_ctx(d, stream, &err);
   cudaError_t e = fp8sm::launch_scaled_mm(
       a, b, M, N, K, static_cast<const float*>(scale_a_e8m0),
       static_cast<const float*>(scale_b_e8m0), 4, bias_bf16,
@@ -513,7 +516,7 @@ fp8_status fp8_scaled_mm_quantized_dual(const void* a, const void* b, int64_t M,
   fp8_status s = device_info(&d);
   if (s != FP8_OK) return s;
   std::string err;
-  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status, d->num_sms, &err};
+  fp8sm::LaunchCtx ctx = make_ctx(d, stream, &err);
   cudaError_t e = fp8sm::launch_scaled_mm(a, b, M, N, K, scale_a, scale_b, (int)recipe, bias_bf16,
                                           4, out_fp8, out_scales, ctx, out_t_fp8, out_t_scales);
   return finish_launch(e, err, n.c_str());
@@ -548,7 +551,7 @@ fp8_status fp8_scaled_mm_mx_quantized(const void* a, const void* b, int64_t M, i
   fp8_status s = device_info(&d);
   if (s != FP8_OK) return s;
   std::string err;
-  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status, d->num_sms, &err};
+  fp8sm::LaunchCtx ctx = make_ctx(d, stream, &err);
   cudaError_t e = fp8sm::launch_scaled_mm(
       a, b, M, N, K, static_cast<const float*>(scale_a_e8m0),
       static_cast<const float*>(scale_b_e8m0), 4, bias_bf16, 3, out_fp8,
@@ -592,8 +595,7 @@ fp8_status grouped_common(const char* name, int recipe, const void* a, const voi
   fp8_status s = device_info(&d);
   if (s != FP8_OK) return s;
   std::string err;
-  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status,
-                       d->num_sms, &err};
+  fp8sm::LaunchCtx ctx = make_ctx(d, stream, &err);
   cudaError_t e = fp8sm::launch_grouped_scaled_mm(a, b_experts, M_total, N, K, E,
                                                   scale_a, scale_b, offs, recipe,
                                                   out_dtype == FP8_OUT_F32, out, ctx);
@@ -664,7 +666,7 @@ fp8_status fp8_quantize_transposed_grouped(const void* x_bf16, int64_t tokens, i
   fp8_status s = device_info(&d);
   if (s != FP8_OK) return s;
   std::string err;
-  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status, d->num_sms, &err};
+  fp8sm::LaunchCtx ctx = make_ctx(d, stream, &err);
   cudaError_t e = fp8sm::launch_quantize_transposed_grouped(x_bf16, tokens, cols, ld_x, offs, E,
                                                             out_fp8, out_scales, ctx);
   return finish_launch(e, err, n);
@@ -698,7 +700,7 @@ fp8_status fp8_grouped_scaled_mm_wgrad(const void* a_t, const void* b_t, int64_t
   fp8_status s = device_info(&d);
   if (s != FP8_OK) return s;
   std::string err;
-  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status, d->num_sms, &err};
+  fp8sm::LaunchCtx ctx = make_ctx(d, stream, &err);
   const int64_t P = fp8sm::grouped_padded_tokens(tokens, E);
   cudaError_t e = fp8sm::launch_grouped_wgrad(a_t, b_t, M, N, P, tokens, E, scale_a, scale_b,
                                               offs, out_dtype == FP8_OUT_F32, out, ctx);
@@ -733,8 +735,7 @@ fp8_status fp8_debug_timeout_probe(uint32_t limit_us, fp8_stream_t stream) {
   fp8_status s = device_info(&d);
   if (s != FP8_OK) return s;
   std::string err;
-  fp8sm::LaunchCtx ctx{reinterpret_cast<cudaStream_t>(stream), d->status,
-                       d->num_sms, &err};
+  fp8sm::LaunchCtx ctx = make_ctx(d, stream, &err);
   return finish_launch(fp8sm::launch_timeout_probe(limit_us, ctx), err,
                        "fp8_debug_timeout_probe");
 }

@@ -5,16 +5,39 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
 #include <string>
 
 namespace fp8sm {
+
+// Devices the library keeps per-device state for (indices 0 .. 63).
+constexpr int kMaxDevices = 64;
 
 struct LaunchCtx {
   cudaStream_t stream;
   uint32_t* status;   // device status word of the current device
   int num_sms;
+  int device;         // the current device (set-up below is per device)
   std::string* err;   // filled on failure
 };
+
+// One-time set-up that belongs to a device: kernel attributes (the dynamic
+// shared-memory opt-in) and occupancy queries are per device, so a process
+// that drives several GPUs needs them on each.  `done` holds one flag per
+// device; the first caller on `device` runs `setup` under `mu`, and the
+// flag is set only when it succeeds.  Safe to call from several threads.
+template <class Setup>
+cudaError_t once_per_device(std::atomic<bool> (&done)[kMaxDevices], std::mutex& mu,
+                            int device, Setup&& setup) {
+  if (device < 0 || device >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (done[device].load(std::memory_order_acquire)) return cudaSuccess;
+  std::lock_guard<std::mutex> lk(mu);
+  if (done[device].load(std::memory_order_relaxed)) return cudaSuccess;
+  const cudaError_t e = setup();
+  if (e == cudaSuccess) done[device].store(true, std::memory_order_release);
+  return e;
+}
 
 // Quantizers (quantize.cu).  recipe: 0 tensor, 1 row, 2 1x128, 3 128x128.
 cudaError_t launch_quantize(const void* x, int64_t rows, int64_t cols,

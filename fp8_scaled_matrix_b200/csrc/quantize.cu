@@ -627,7 +627,11 @@ __global__ void __launch_bounds__(256) quant_tensor_kernel(
   }
 }
 
-int g_tensor_blocks_per_sm = -1;
+// Resident quant_tensor_kernel CTAs per SM (the cooperative grid's bound),
+// queried once per device.
+int g_tensor_blocks_per_sm[kMaxDevices];
+std::atomic<bool> g_tensor_occupancy_done[kMaxDevices];
+std::mutex g_tensor_occupancy_mu;
 
 // Sharded tensorwise quantization, step 1: max|x| of this shard folded into
 // amax[0] (fp32 bits, atomic max; amax[0] must be zero on entry).
@@ -713,19 +717,21 @@ cudaError_t launch_quantize_mx(const void* xv, int64_t rows, int64_t cols, int64
   return cudaGetLastError();
 }
 
-static cudaError_t configure_transposed() {
-  static bool configured = false;
-  if (configured) return cudaSuccess;
-  const void* fns[] = {(const void*)quant_transposed_kernel<true, false>,
-                       (const void*)quant_transposed_kernel<false, false>,
-                       (const void*)quant_transposed_kernel<false, true>};
-  for (const void* f : fns) {
-    cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kTrSmemBytes));
-    if (e != cudaSuccess) return e;
-  }
-  configured = true;
-  return cudaSuccess;
+// The transposed kernels' dynamic shared-memory opt-in, once per device.
+static cudaError_t configure_transposed(const LaunchCtx& ctx) {
+  static std::atomic<bool> done[kMaxDevices];
+  static std::mutex mu;
+  return once_per_device(done, mu, ctx.device, [] {
+    const void* fns[] = {(const void*)quant_transposed_kernel<true, false>,
+                         (const void*)quant_transposed_kernel<false, false>,
+                         (const void*)quant_transposed_kernel<false, true>};
+    for (const void* f : fns) {
+      cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(kTrSmemBytes));
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  });
 }
 
 cudaError_t launch_quantize_transposed(const void* xv, int64_t rows, int64_t cols,
@@ -734,7 +740,7 @@ cudaError_t launch_quantize_transposed(const void* xv, int64_t rows, int64_t col
   if (rows == 0 || cols == 0) return cudaSuccess;
   const uint16_t* x = static_cast<const uint16_t*>(xv);
   uint8_t* q = static_cast<uint8_t*>(qv);
-  cudaError_t e = configure_transposed();
+  cudaError_t e = configure_transposed(ctx);
   if (e != cudaSuccess) return e;
   const int64_t n_kb = rows / kTrRows;
   const int64_t tiles = n_kb * ((cols + kTrCols - 1) / kTrCols);
@@ -753,7 +759,7 @@ cudaError_t launch_quantize_transposed_batched(const void* xv, int32_t batch, in
                                                int64_t cols, int64_t ld, int recipe, void* qv,
                                                float* scales, const LaunchCtx& ctx) {
   if (batch == 0 || rows == 0 || cols == 0) return cudaSuccess;
-  cudaError_t e = configure_transposed();
+  cudaError_t e = configure_transposed(ctx);
   if (e != cudaSuccess) return e;
   const int64_t n_kb = rows / kTrRows;
   const int64_t tiles = n_kb * ((cols + kTrCols - 1) / kTrCols) * batch;
@@ -790,7 +796,7 @@ cudaError_t launch_quantize_transposed_grouped(const void* xv, int64_t rows, int
                                                int64_t ld, const int32_t* offs, int32_t E,
                                                void* qv, float* scales, const LaunchCtx& ctx) {
   if (cols == 0) return cudaSuccess;
-  cudaError_t e = configure_transposed();
+  cudaError_t e = configure_transposed(ctx);
   if (e != cudaSuccess) return e;
   const int64_t P = grouped_padded_tokens(rows, E);
   const int64_t n_kb = P / kTrRows;
@@ -852,15 +858,16 @@ cudaError_t launch_quantize(const void* xv, int64_t rows, int64_t cols,
   uint32_t* ws = static_cast<uint32_t*>(workspace);
   cudaError_t e = cudaMemsetAsync(ws, 0, 2 * sizeof(uint32_t), st);
   if (e != cudaSuccess) return e;
-  if (g_tensor_blocks_per_sm < 0) {
+  e = once_per_device(g_tensor_occupancy_done, g_tensor_occupancy_mu, ctx.device, [&] {
     int n = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quant_tensor_kernel,
-                                                      256, 0);
-    if (e != cudaSuccess) return e;
-    g_tensor_blocks_per_sm = n;
-  }
-  int64_t max_grid = static_cast<int64_t>(ctx.num_sms) *
-                     (g_tensor_blocks_per_sm > 0 ? g_tensor_blocks_per_sm : 1);
+    const cudaError_t r =
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quant_tensor_kernel, 256, 0);
+    g_tensor_blocks_per_sm[ctx.device] = n;
+    return r;
+  });
+  if (e != cudaSuccess) return e;
+  const int per_sm = g_tensor_blocks_per_sm[ctx.device];
+  int64_t max_grid = static_cast<int64_t>(ctx.num_sms) * (per_sm > 0 ? per_sm : 1);
   int64_t grid = rows < max_grid ? rows : max_grid;
   if (grid < 1) grid = 1;
   unsigned g = static_cast<unsigned>(grid);

@@ -156,6 +156,23 @@ def _need_cuda(*ts):
             raise ValueError("tensors must live in CUDA device memory")
 
 
+def _check_quant_outputs(x: torch.Tensor, out: torch.Tensor, scales: torch.Tensor,
+                         rows: int, cols: int, recipe: int) -> None:
+    """Caller-passed outputs of a quantization: contiguous, of the right
+    dtype, on x's device and large enough for what the library writes (the
+    codes, rows x cols bytes, and the recipe's scales); the library writes
+    through the raw pointers, so a smaller buffer would be overrun."""
+    if (out.dtype != torch.uint8 or not out.is_contiguous() or out.device != x.device
+            or out.numel() < rows * cols):
+        raise ValueError(f"out must be a contiguous uint8 tensor on {x.device} with at "
+                         f"least {rows * cols} elements")
+    need = max(scale_count(rows, cols, recipe), 1)
+    if (scales.dtype != torch.float32 or not scales.is_contiguous()
+            or scales.device != x.device or scales.numel() < need):
+        raise ValueError(f"scales must be a contiguous float32 tensor on {x.device} with at "
+                         f"least {need} elements")
+
+
 def fp8_version() -> int:
     return load_library().fp8_version()
 
@@ -196,9 +213,13 @@ def fp8_quantize(x: torch.Tensor, recipe: int, out: Optional[torch.Tensor] = Non
     if scales is None:
         scales = torch.empty(max(scale_count(rows, cols, recipe), 1),
                              dtype=torch.float32, device=x.device)
+    _need_cuda(out, scales, workspace)
+    _check_quant_outputs(x, out, scales, rows, cols, recipe)
     ws_bytes = L.fp8_quantize_workspace_bytes(recipe, rows, cols)
     if ws_bytes and workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=x.device)
+    if workspace is not None and (workspace.device != x.device or not workspace.is_contiguous()):
+        raise ValueError(f"workspace must be a contiguous tensor on {x.device}")
     # the row stride only matters when there is more than one non-empty row
     ld = x.stride(0) if (rows > 1 and cols > 0) else cols
     _check(L.fp8_quantize(_ptr(x), rows, cols, ld, recipe, _ptr(out),
@@ -221,6 +242,7 @@ def fp8_quantize_noalloc(x: torch.Tensor, recipe: int, out: torch.Tensor,
     if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
         raise ValueError("x must be a 2-D bf16 tensor with unit column stride")
     rows, cols = x.shape
+    _check_quant_outputs(x, out, scales, rows, cols, recipe)
     ld = x.stride(0) if (rows > 1 and cols > 0) else cols
     _check(L.fp8_quantize_noalloc(_ptr(x), rows, cols, ld, recipe, _ptr(out),
                                   _ptr(scales), _stream(stream)))

@@ -367,3 +367,30 @@ def test_batched_quantize_empty_is_a_noop(lib):
                                     None, None, None) == fp8sm.FP8_OK
     assert lib.fp8_quantize_transposed_batched(None, 3, 0, 128, 128, fp8sm.FP8_SCALE_BLOCK_1x128,
                                                None, None, None) == fp8sm.FP8_OK
+
+
+def test_binding_rejects_caller_outputs_smaller_than_the_library_writes():
+    """fp8_quantize / fp8_quantize_noalloc write through the raw pointers of
+    caller-passed outputs: the binding refuses, before any launch, buffers of
+    the wrong dtype, non-contiguous ones and ones smaller than the codes
+    (rows x cols bytes) or the recipe's scale count."""
+    x = torch.zeros(256, 384, dtype=torch.bfloat16)
+    q = torch.empty(256, 384, dtype=torch.uint8)
+    for recipe in (fp8sm.FP8_SCALE_TENSOR, fp8sm.FP8_SCALE_ROW,
+                   fp8sm.FP8_SCALE_BLOCK_1x128, fp8sm.FP8_SCALE_BLOCK_128x128):
+        n = max(fp8sm.scale_count(256, 384, recipe), 1)
+        s = torch.empty(n, dtype=torch.float32)
+        fp8sm._check_quant_outputs(x, q, s, 256, 384, recipe)      # exact sizes pass
+        with pytest.raises(ValueError):
+            fp8sm._check_quant_outputs(x, q.view(-1)[:-1], s, 256, 384, recipe)
+        if n > 1:
+            with pytest.raises(ValueError):
+                fp8sm._check_quant_outputs(x, q, s[:-1], 256, 384, recipe)
+        with pytest.raises(ValueError):
+            fp8sm._check_quant_outputs(x, q, s.view(torch.int32), 256, 384, recipe)
+        with pytest.raises(ValueError):
+            fp8sm._check_quant_outputs(x, q.to(torch.int8), s, 256, 384, recipe)
+    with pytest.raises(ValueError):   # a column slice is not contiguous
+        fp8sm._check_quant_outputs(x, torch.empty(256, 768, dtype=torch.uint8)[:, :384],
+                                   torch.empty(256, dtype=torch.float32), 256, 384,
+                                   fp8sm.FP8_SCALE_ROW)
