@@ -89,16 +89,12 @@ constexpr uint32_t kMxSfTile = 512;
 constexpr uint32_t kMxSfStage = 3 * kMxSfTile;
 constexpr uint32_t kMxSfCols = 16;
 
-// Shared-memory layout.  Single-CTA tiles are 128 x 256: each stage holds
-// A (128 rows) and B (256 rows) of a 128-byte K slice.  CTA-pair tiles are
-// 256 x 256 (cta_group::2): each CTA holds its own 128 rows of A and its own
-// 128 rows (half of N) of B, so a stage is a third smaller and two more
-// stages fit.
-template <bool kPair>
+// Shared-memory layout.  Tiles are 128 x 256: each stage holds A (128 rows)
+// and B (256 rows) of a 128-byte K slice.
 struct Cfg {
-  static constexpr int kStages = kPair ? 6 : 4;
-  static constexpr int kTileM = kPair ? 2 * BM : BM;   // output rows per work item
-  static constexpr uint32_t kBRows = kPair ? BN / 2 : BN;  // B rows held per CTA
+  static constexpr int kStages = 4;
+  static constexpr int kTileM = BM;   // output rows per work item
+  static constexpr uint32_t kBRows = BN;  // B rows held per stage
   static constexpr uint32_t kAStage = BM * BK;
   static constexpr uint32_t kBStage = kBRows * BK;
   static constexpr uint32_t kOffA = 0;
@@ -404,7 +400,7 @@ __device__ __forceinline__ void store_cols32(
   }
 }
 
-template <int kRecipe, int kOut, bool kGrouped, bool kPair>
+template <int kRecipe, int kOut, bool kGrouped>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
                     const __grid_constant__ CUtensorMap tm_b,
@@ -425,8 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr bool kMasked = kGrouped && !kKGroups;
   // epilogue threads that hold a whole 128-column row slice across K blocks
   // (blockwise promotion) get registers moved from warpgroup 0.  The MXFP8
-  // epilogue reads its accumulators once per tile and runs without the split
-  // (with it, a dense MXFP8 build faulted on the GPU; see the design notes).
+  // epilogue reads its accumulators once per tile and runs without the split.
   constexpr bool kBigEpi = kBlockwise;
   constexpr bool kOutF32 = kOut == kOutFp32;
   constexpr bool kOutQT = kOut == kOutE4M3Dual;
@@ -436,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // epilogue is at the edge of its register budget, keeps the M-major order
   // (its B is a layer's weight, which fits in L2)
   constexpr bool kRaster = !kOutQT;
-  using C = Cfg<kPair>;
+  using C = Cfg;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
@@ -466,9 +461,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) mbar_init(&acc_full[i], 1);
-    // pair: the leader's barrier collects both CTAs' epilogue warps
-    // every epilogue warp hands a buffer back (pair: from both CTAs)
-    for (int i = 0; i < 2; ++i) mbar_init(&acc_empty[i], kPair ? 2 * kEpiWarps : kEpiWarps);
+    // every epilogue warp hands a buffer back
+    for (int i = 0; i < 2; ++i) mbar_init(&acc_empty[i], kEpiWarps);
     mbar_init(drain, 1);
     for (int i = 0; i < kSclSlots; ++i) {
       mbar_init(&sfull[i], 32);            // one cp.async arrival per lane of warp 2
@@ -483,13 +477,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if constexpr (!kMasked) prefetch_tmap(&tm_out);
   }
   if (warp == 1) {
-    if constexpr (kPair) {
-      tmem_alloc_pair(tmem_slot, kTmemCols);
-      tmem_relinquish_pair();
-    } else {
-      tmem_alloc(tmem_slot, kTmemCols);
-      tmem_relinquish();
-    }
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
   }
   if (warp == 2) {
     int64_t total;
@@ -532,16 +521,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) *total_tiles_slot = total;
   }
   __syncthreads();
-  // pair: both CTAs' barriers are initialised before any cross-CTA traffic
-  if constexpr (kPair) cluster_sync();
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
   const int64_t total_tiles = *total_tiles_slot;
   const int32_t KB = p.k_blocks;
-  // work items: one per CTA, or one per CTA pair (cluster of two)
-  const uint32_t rank = kPair ? cluster_ctarank() : 0u;
-  const int64_t item0 = kPair ? (blockIdx.x >> 1) : blockIdx.x;
-  const int64_t item_stride = kPair ? (gridDim.x >> 1) : gridDim.x;
+  const int64_t item0 = blockIdx.x;
+  const int64_t item_stride = gridDim.x;
   constexpr int kTM = C::kTileM;
 
   if (warp < kFirstEpiWarp) {
@@ -562,7 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             kKGroups ? kgroup_coord(t, p, kc) : tile_coord<kGrouped, kTM, kRaster>(t, p, cur);
         const int32_t nkb = kKGroups ? c.nkb : KB;
         for (int32_t kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait<kPair>(&empty[stage], phase ^ 1u, abort_flag, p.status,
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status,
                          SITE_PRODUCER_EMPTY, kWaitLimitNs)) {
             ok = false;
             break;
@@ -570,20 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t b_bytes = c.half_n ? C::kBStage / 2 : C::kBStage;
           uint8_t* a_dst = smem + C::kOffA + stage * C::kAStage;
           uint8_t* b_dst = smem + C::kOffB + stage * C::kBStage;
-          if constexpr (kPair) {
-            // This CTA's 128 rows of A and its half of the item's B rows;
-            // both CTAs' bytes complete on the leader's barrier, which the
-            // leader arms for the pair.
-            const uint32_t lead_full = mapa_shared(smem_u32(&full[stage]), 0);
-            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * (C::kAStage + b_bytes));
-            const int32_t b_row = c.n0 + static_cast<int32_t>(rank) * (c.half_n ? BN / 4 : BN / 2);
-            tma_load_2d_pair(a_dst, &tm_a, lead_full, kb * BK,
-                             c.m0 + static_cast<int32_t>(rank) * BM);
-            if constexpr (kGrouped)
-              tma_load_3d_pair(b_dst, &tm_b, lead_full, kb * BK, b_row, c.g);
-            else
-              tma_load_2d_pair(b_dst, c.half_n ? &tm_b_half : &tm_b, lead_full, kb * BK, b_row);
-          } else if constexpr (kIsMx) {
+          if constexpr (kIsMx) {
             // operands plus their scale-factor tiles (tile (i, kb) of a
             // matrix's scales is its 128 rows 128 i .. and K elements
             // 128 kb ..); B's second half-tile exists only below N
@@ -640,20 +612,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (!ok && rank == 0) {
+      if (!ok) {
         // Let the copies already in flight land before the CTA exits.
         const uint64_t first = issued > C::kStages ? issued - C::kStages : 0;
         for (uint64_t i = first; i < issued; ++i) {
           uint32_t dummy_abort = 0;
-          mbar_wait<kPair>(&full[i % C::kStages], static_cast<uint32_t>((i / C::kStages) & 1u),
+          mbar_wait(&full[i % C::kStages], static_cast<uint32_t>((i / C::kStages) & 1u),
                     &dummy_abort, nullptr, SITE_TEARDOWN, 10000000ull);
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
-    // (pair: the leader CTA issues for both; the peer only drains)
-    if (lane == 0 && rank == 0) {
+    if (lane == 0) {
       const uint32_t idesc_full = idesc_e4m3_f32(kTM, BN);
       const uint32_t idesc_half = idesc_e4m3_f32(kTM, BN / 2);
       uint32_t stage = 0, phase = 0;
@@ -664,7 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // stage wait (TMA writes and MMA reads are both async-proxy, ordered by
       // the barrier), and the next stage's barrier is peeked while this
       // stage's MMAs go out.
-      bool ready = mbar_test_wait<kPair>(&full[stage], phase);
+      bool ready = mbar_test_wait(&full[stage], phase);
       if constexpr (kIsMx) {
         // MXFP8: per stage, the scale-factor tiles go from shared memory to
         // the stage's TMEM slot (tcgen05.cp: 32 rows x 16 bytes copied to
@@ -723,14 +694,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if constexpr (!kBlockwise) {
         for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
           const uint32_t idesc = (!kGrouped && t >= p.split_start) ? idesc_half : idesc_full;
-          if (!mbar_wait<kPair>(&acc_empty[acc], acc_phase ^ 1u, abort_flag, p.status,
+          if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag, p.status,
                                 SITE_MMA_ACC_EMPTY, kWaitLimitNs)) {
             ok = false;
             break;
           }
           tc_fence_after_sync();
           for (int32_t kb = 0; kb < KB; ++kb) {
-            if (!ready && !mbar_wait<kPair>(&full[stage], phase, abort_flag, p.status,
+            if (!ready && !mbar_wait(&full[stage], phase, abort_flag, p.status,
                                             SITE_MMA_FULL, kWaitLimitNs)) {
               ok = false;
               break;
@@ -740,26 +711,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               stage = 0;
               phase ^= 1u;
             }
-            ready = mbar_test_wait<kPair>(&full[stage], phase);  // peek at the next stage
+            ready = mbar_test_wait(&full[stage], phase);  // peek at the next stage
             const uint32_t d = tmem_base + acc * BN;
             const uint64_t da = smem_desc_k_sw128(smem_u32(smem + C::kOffA + cur * C::kAStage));
             const uint64_t db = smem_desc_k_sw128(smem_u32(smem + C::kOffB + cur * C::kBStage));
 #pragma unroll
-            for (int k = 0; k < BK / UMMA_K; ++k) {
-              const uint32_t accumulate = (kb > 0) || (k > 0);
-              if constexpr (kPair)
-                mma_e4m3_pair(d, da + (k * UMMA_K) / 16, db + (k * UMMA_K) / 16, idesc,
-                              accumulate);
-              else
-                mma_e4m3(d, da + (k * UMMA_K) / 16, db + (k * UMMA_K) / 16, idesc,
-                         accumulate);
-            }
-            if constexpr (kPair) mma_commit_pair(&empty[cur], 0x3);
-            else mma_commit(&empty[cur]);
+            for (int k = 0; k < BK / UMMA_K; ++k)
+              mma_e4m3(d, da + (k * UMMA_K) / 16, db + (k * UMMA_K) / 16, idesc,
+                       (kb > 0) || (k > 0));
+            mma_commit(&empty[cur]);
           }
           if (ok) {
-            if constexpr (kPair) mma_commit_pair(&acc_full[acc], 0x3);
-            else mma_commit(&acc_full[acc]);
+            mma_commit(&acc_full[acc]);
             acc ^= 1u;
             if (acc == 0) acc_phase ^= 1u;
           }
@@ -776,13 +739,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
           const int32_t nkb = kKGroups ? kgroup_coord(t, p, kc).nkb : KB;
           for (int32_t kb = 0; kb < nkb; ++kb) {
-            if (!mbar_wait<kPair>(&acc_empty[acc], acc_phase ^ 1u, abort_flag, p.status,
+            if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag, p.status,
                                   SITE_MMA_ACC_EMPTY, kWaitLimitNs)) {
               ok = false;
               break;
             }
             tc_fence_after_sync();
-            if (!ready && !mbar_wait<kPair>(&full[stage], phase, abort_flag, p.status,
+            if (!ready && !mbar_wait(&full[stage], phase, abort_flag, p.status,
                                             SITE_MMA_FULL, kWaitLimitNs)) {
               ok = false;
               break;
@@ -792,7 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               stage = 0;
               phase ^= 1u;
             }
-            ready = mbar_test_wait<kPair>(&full[stage], phase);
+            ready = mbar_test_wait(&full[stage], phase);
             const uint32_t d = tmem_base + acc * BN;
             const uint64_t da = smem_desc_k_sw128(smem_u32(smem + C::kOffA + cur * C::kAStage));
             const uint64_t db = smem_desc_k_sw128(smem_u32(smem + C::kOffB + cur * C::kBStage));
@@ -805,14 +768,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      // All MMAs issued by this thread complete before TMEM is released
-      // (pair: in both CTAs).
-      if constexpr (kPair) mma_commit_pair(drain, 0x3);
-      else mma_commit(drain);
+      // All MMAs issued by this thread complete before TMEM is released.
+      mma_commit(drain);
     }
     if (lane == 0) {
       uint32_t dummy_abort = 0;
-      mbar_wait<kPair>(drain, 0, &dummy_abort, p.status, SITE_TEARDOWN, kWaitLimitNs);
+      mbar_wait(drain, 0, &dummy_abort, p.status, SITE_TEARDOWN, kWaitLimitNs);
     }
    } else if (warp == 2) {
     // ----------------------------------------------- blockwise scale producer
@@ -949,23 +910,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
     bool ok = true;
-    // TMEM buffers are handed back on the leader's barrier (pair: from both CTAs)
-    const uint32_t acc_empty_addr0 =
-        kPair ? mapa_shared(smem_u32(&acc_empty[0]), 0) : smem_u32(&acc_empty[0]);
-    const uint32_t acc_empty_addr1 =
-        kPair ? mapa_shared(smem_u32(&acc_empty[1]), 0) : smem_u32(&acc_empty[1]);
-    // Single CTA: a CTA-scope arrive.  Pair: the leader's barrier, at cluster
-    // scope (a cluster-scope release costs a fence, so it is used only there).
-    // the four warps of this warp's half meet (bounded; dual e4m3 output)
-    auto release_acc = [&](uint32_t a) {
-      if constexpr (kPair) mbar_arrive_cluster(a ? acc_empty_addr1 : acc_empty_addr0);
-      else mbar_arrive(&acc_empty[a]);
-    };
+    auto release_acc = [&](uint32_t a) { mbar_arrive(&acc_empty[a]); };
     for (int64_t t = item0; t < total_tiles && ok; t += item_stride) {
       const TileCoord c =
           kKGroups ? kgroup_coord(t, p, kc) : tile_coord<kGrouped, kTM, kRaster>(t, p, cur);
-      // this CTA's output rows (K-grouped: group g's block of the output)
-      const int32_t cta_m0 = c.out_m0 + static_cast<int32_t>(rank) * BM;
+      // the tile's output rows (K-grouped: group g's block of the output)
+      const int32_t cta_m0 = c.out_m0;
       const int64_t row = static_cast<int64_t>(cta_m0) + q * 32 + lane;
       const bool row_ok = row < c.row_end;
       const int64_t ncol0 = static_cast<int64_t>(c.n0) + half * 128;
@@ -982,7 +932,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
       if constexpr (!kBlockwise) {
-        if (!mbar_wait<kPair>(&acc_full[acc], acc_phase, abort_flag, p.status,
+        if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status,
                        SITE_EPI_ACC_FULL, kWaitLimitNs)) {
           ok = false;
           break;
@@ -1351,13 +1301,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before_sync();
   __syncthreads();
-  // pair: no CTA leaves (or frees TMEM) while the other may still touch its
-  // barriers or shared memory
-  if constexpr (kPair) cluster_sync();
   if (warp == 1) {
     tc_fence_after_sync();
-    if constexpr (kPair) tmem_dealloc_pair(tmem_base, kTmemCols);
-    else tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
@@ -1424,76 +1370,60 @@ bool make_tmap(CUtensorMap* m, CUtensorMapDataType dt, uint32_t rank,
   return true;
 }
 
-template <int kRecipe, int kOut, bool kGrouped, bool kPair>
+template <int kRecipe, int kOut, bool kGrouped>
 cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb,
                           const CUtensorMap& tbh, const CUtensorMap& to,
-                          const GemmParams& p, unsigned grid, cudaStream_t st) {
+                          const GemmParams& p, unsigned grid, const LaunchCtx& ctx) {
   constexpr bool kBlockwise = kRecipe == kBlock128 || kRecipe == kBlock1;
-  constexpr bool kBigEpi = kBlockwise || kRecipe == kMxfp8;
-  if constexpr (kPair && kBlockwise) {
-    return cudaErrorInvalidValue;  // CTA pairs serve the dense recipes only
-  } else if constexpr (kRecipe == kMxfp8 &&
-                       (kPair || kOut == kOutE4M3 || (kGrouped && kOut == kOutMx))) {
-    return cudaErrorInvalidValue;  // MXFP8: single CTAs; bf16/fp32 out (dense: also MXFP8)
+  constexpr bool kBigEpi = kBlockwise;
+  if constexpr (kRecipe == kMxfp8 && (kOut == kOutE4M3 || (kGrouped && kOut == kOutMx))) {
+    return cudaErrorInvalidValue;  // MXFP8: bf16/fp32 out (dense: also MXFP8)
   } else if constexpr (kOut == kOutMx && kRecipe != kMxfp8) {
     return cudaErrorInvalidValue;  // MXFP8 output from the MXFP8 GEMM only
-  } else if constexpr (kOut == kOutE4M3Dual && (kRecipe != kBlock128 || kGrouped || kPair)) {
+  } else if constexpr (kOut == kOutE4M3Dual && (kRecipe != kBlock128 || kGrouped)) {
     return cudaErrorInvalidValue;  // dual e4m3 output: dense 1x128_128x128 only
-  } else if constexpr (kOut == kOutE4M3 && (kPair || kGrouped)) {
-    return cudaErrorInvalidValue;  // quantized output: single-CTA dense GEMM only
+  } else if constexpr (kOut == kOutE4M3 && kGrouped) {
+    return cudaErrorInvalidValue;  // quantized output: dense GEMM only
   } else {
-    using C = Cfg<kPair>;
-    static bool configured = false;
-    auto kern = fp8_gemm_kernel<kRecipe, kOut, kGrouped, kPair>;
-    if (!configured) {
-      cudaError_t e = cudaFuncSetAttribute(
-          kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-      if (e != cudaSuccess) return e;
+    auto kern = fp8_gemm_kernel<kRecipe, kOut, kGrouped>;
+    // the dynamic shared-memory opt-in, once per device
+    static std::atomic<bool> done[kMaxDevices];
+    static std::mutex mu;
+    cudaError_t e = once_per_device(done, mu, ctx.device, [&] {
+      cudaError_t r = cudaFuncSetAttribute(
+          kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
+      if (r != cudaSuccess) return r;
       if (kBigEpi) {
         // setmaxnreg.inc would wait forever if the launch allocation were
         // smaller than the split assumes: check before the first launch.
         cudaFuncAttributes attr;
-        e = cudaFuncGetAttributes(&attr, kern);
-        if (e != cudaSuccess) return e;
+        r = cudaFuncGetAttributes(&attr, kern);
+        if (r != cudaSuccess) return r;
         if (attr.numRegs < static_cast<int>(kRegsAtLaunch)) return cudaErrorInvalidConfiguration;
       }
-      configured = true;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = C::kSmemBytes;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    // single-CTA kernels are launched without a cluster attribute
-    cfg.attrs = attr;
-    cfg.numAttrs = kPair ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kern, ta, tb, tbh, to, p);
+      return cudaSuccess;
+    });
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kThreads, Cfg::kSmemBytes, ctx.stream>>>(ta, tb, tbh, to, p);
+    return cudaGetLastError();
   }
 }
 
 template <bool kGrouped>
-cudaError_t dispatch(int recipe, int out_kind, bool pair, const CUtensorMap& ta,
-                     const CUtensorMap& tb, const CUtensorMap& tbh,
-                     const CUtensorMap& to, const GemmParams& p, unsigned grid,
-                     cudaStream_t st) {
-#define FP8SM_CASE(R)                                                                   \
-  if (recipe == R) {                                                                    \
-    if (out_kind == kOutE4M3)                                                           \
-      return launch_kernel<R, kOutE4M3, kGrouped, false>(ta, tb, tbh, to, p, grid, st); \
-    if (out_kind == kOutMx)                                                             \
-      return launch_kernel<R, kOutMx, kGrouped, false>(ta, tb, tbh, to, p, grid, st);   \
-    if (out_kind == kOutE4M3Dual)                                                       \
-      return launch_kernel<R, kOutE4M3Dual, kGrouped, false>(ta, tb, tbh, to, p, grid, st); \
-    if (pair)                                                                           \
-      return out_kind ? launch_kernel<R, kOutFp32, kGrouped, true>(ta, tb, tbh, to, p, grid, st) \
-                      : launch_kernel<R, kOutBf16, kGrouped, true>(ta, tb, tbh, to, p, grid, st); \
-    return out_kind ? launch_kernel<R, kOutFp32, kGrouped, false>(ta, tb, tbh, to, p, grid, st)  \
-                    : launch_kernel<R, kOutBf16, kGrouped, false>(ta, tb, tbh, to, p, grid, st); \
+cudaError_t dispatch(int recipe, int out_kind, const CUtensorMap& ta, const CUtensorMap& tb,
+                     const CUtensorMap& tbh, const CUtensorMap& to, const GemmParams& p,
+                     unsigned grid, const LaunchCtx& ctx) {
+#define FP8SM_CASE(R)                                                              \
+  if (recipe == R) {                                                               \
+    switch (out_kind) {                                                            \
+      case kOutBf16: return launch_kernel<R, kOutBf16, kGrouped>(ta, tb, tbh, to, p, grid, ctx); \
+      case kOutFp32: return launch_kernel<R, kOutFp32, kGrouped>(ta, tb, tbh, to, p, grid, ctx); \
+      case kOutE4M3: return launch_kernel<R, kOutE4M3, kGrouped>(ta, tb, tbh, to, p, grid, ctx); \
+      case kOutMx: return launch_kernel<R, kOutMx, kGrouped>(ta, tb, tbh, to, p, grid, ctx);     \
+      case kOutE4M3Dual:                                                           \
+        return launch_kernel<R, kOutE4M3Dual, kGrouped>(ta, tb, tbh, to, p, grid, ctx);          \
+      default: return cudaErrorInvalidValue;                                       \
+    }                                                                              \
   }
   if constexpr (kGrouped) {
     FP8SM_CASE(kRow)
@@ -1535,20 +1465,6 @@ bool a_map(CUtensorMap* m, const void* a, int64_t rows, int64_t K, std::string* 
                    CU_TENSOR_MAP_SWIZZLE_128B, err);
 }
 
-// Whether to run a problem on CTA pairs (256-row items, cta_group::2).
-// Measured on B200: the pair kernel halves B traffic per CTA but adds a
-// cross-SM handshake per accumulator hand-off; it is not faster for any
-// recipe here (2x slower for the blockwise recipes, whose hand-off is per
-// K block), so single CTAs are used.  Kept selectable for tuning.
-// FP8SM_CTA_PAIRS=1 selects the pair kernel for the dense recipes (read per
-// call; for tuning and for the tests that keep it covered).  The blockwise
-// kernels always run on single CTAs.
-bool use_pair(int64_t M, int recipe) {
-  const char* e = std::getenv("FP8SM_CTA_PAIRS");
-  return e != nullptr && e[0] == '1' && M > BM && recipe != kBlock128 && recipe != kBlock1 &&
-         recipe != kMxfp8;
-}
-
 }  // namespace
 
 cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
@@ -1572,8 +1488,7 @@ cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
           static_cast<const uint16_t*>(bias), M, N, out);
     return cudaGetLastError();
   }
-  const bool pair = use_pair(M, recipe);
-  const uint32_t b_rows = pair ? Cfg<true>::kBRows : Cfg<false>::kBRows;
+  const uint32_t b_rows = Cfg::kBRows;
   CUtensorMap ta, tb, tbh, to;
   if (!a_map(&ta, a, M, K, ctx.err)) return cudaErrorInvalidValue;
   {
@@ -1610,7 +1525,7 @@ cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
   p.out = out;
   p.offs = nullptr;
   p.E = 0;
-  const int64_t tile_m = pair ? 2 * BM : BM;
+  const int64_t tile_m = BM;
   p.n_tiles = static_cast<int32_t>((N + BN - 1) / BN);
   p.m_tiles = static_cast<int32_t>((M + tile_m - 1) / tile_m);
   p.k_blocks = static_cast<int32_t>((K + BK - 1) / BK);
@@ -1622,7 +1537,7 @@ cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
   p.raster_m = (N * K > (int64_t(64) << 20)) ? 16 : 0;
   p.status = ctx.status;
   const int64_t tiles = static_cast<int64_t>(p.n_tiles) * p.m_tiles;
-  const int64_t G = pair ? ctx.num_sms / 2 : ctx.num_sms;  // CTAs or CTA pairs
+  const int64_t G = ctx.num_sms;  // resident CTAs (one per SM)
   p.split_start = tiles;
   p.total_items = tiles;
   const bool blockwise = recipe == kBlock128 || recipe == kBlock1;
@@ -1635,8 +1550,8 @@ cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
     }
   }
   const int64_t units = p.total_items < G ? p.total_items : G;
-  const unsigned grid = static_cast<unsigned>(pair ? 2 * units : units);
-  return dispatch<false>(recipe, out_kind, pair, ta, tb, tbh, to, p, grid, ctx.stream);
+  const unsigned grid = static_cast<unsigned>(units);
+  return dispatch<false>(recipe, out_kind, ta, tb, tbh, to, p, grid, ctx);
 }
 
 cudaError_t launch_grouped_scaled_mm(const void* a, const void* b,
@@ -1649,8 +1564,7 @@ cudaError_t launch_grouped_scaled_mm(const void* a, const void* b,
   if (K == 0)
     return launch_scaled_mm(nullptr, nullptr, M_total, N, 0, nullptr, nullptr,
                             1, nullptr, out_f32 ? kOutFp32 : kOutBf16, out, nullptr, ctx);
-  const bool pair = use_pair(M_total, recipe);
-  const uint32_t b_rows = pair ? Cfg<true>::kBRows : Cfg<false>::kBRows;
+  const uint32_t b_rows = Cfg::kBRows;
   CUtensorMap ta, tb, to;
   if (!a_map(&ta, a, M_total, K, ctx.err)) return cudaErrorInvalidValue;
   {
@@ -1690,8 +1604,8 @@ cudaError_t launch_grouped_scaled_mm(const void* a, const void* b,
   p.status = ctx.status;
   p.split_start = INT64_MAX;
   p.total_items = 0;
-  const unsigned grid = static_cast<unsigned>(pair ? (ctx.num_sms / 2) * 2 : ctx.num_sms);
-  return dispatch<true>(recipe, out_f32, pair, ta, tb, tb, to, p, grid, ctx.stream);
+  const unsigned grid = static_cast<unsigned>(ctx.num_sms);
+  return dispatch<true>(recipe, out_f32, ta, tb, tb, to, p, grid, ctx);
 }
 
 cudaError_t launch_grouped_wgrad(const void* a_t, const void* b_t, int64_t M, int64_t N,
@@ -1704,7 +1618,7 @@ cudaError_t launch_grouped_wgrad(const void* a_t, const void* b_t, int64_t M, in
   {
     uint64_t dims[2] = {static_cast<uint64_t>(P), static_cast<uint64_t>(N)};
     uint64_t strides[1] = {static_cast<uint64_t>(P)};
-    uint32_t box[2] = {BK, Cfg<false>::kBRows};
+    uint32_t box[2] = {BK, Cfg::kBRows};
     if (!make_tmap(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, b_t, dims, strides, box,
                    CU_TENSOR_MAP_SWIZZLE_128B, ctx.err))
       return cudaErrorInvalidValue;
@@ -1731,7 +1645,7 @@ cudaError_t launch_grouped_wgrad(const void* a_t, const void* b_t, int64_t M, in
   p.total_items = 0;
   const int64_t items = static_cast<int64_t>(E) * p.m_tiles * p.n_tiles;
   const unsigned grid = static_cast<unsigned>(items < ctx.num_sms ? items : ctx.num_sms);
-  return dispatch<true>(kBlock1, out_f32, false, ta, tb, tb, to, p, grid, ctx.stream);
+  return dispatch<true>(kBlock1, out_f32, ta, tb, tb, to, p, grid, ctx);
 }
 
 cudaError_t launch_timeout_probe(uint32_t limit_us, const LaunchCtx& ctx) {

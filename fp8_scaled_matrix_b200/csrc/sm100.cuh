@@ -67,51 +67,28 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar,
       : "memory");
 }
 
-// kCluster: acquire at cluster scope (barriers that the other CTA of a pair
-// arrives on); CTA scope otherwise, which is cheaper.
-template <bool kCluster = false>
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr,
-                                              uint32_t parity) {
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity) {
   uint32_t done;
-  if constexpr (kCluster)
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(bar_addr), "r"(parity)
-        : "memory");
-  else
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(bar_addr), "r"(parity)
-        : "memory");
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar_addr), "r"(parity)
+      : "memory");
   return done != 0;
 }
 
 // Non-blocking check whether the phase with parity `parity` has completed.
-template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   uint32_t done;
-  if constexpr (kCluster)
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-  else
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
   return done != 0;
 }
 
@@ -119,26 +96,16 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 // suspended by the hardware for up to `hint_ns` nanoseconds; it wakes when
 // the phase completes.  Keeps waiting warps from taking issue slots that the
 // warps doing work on the same scheduler need.
-template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar_addr, uint32_t parity,
                                                       uint32_t hint_ns) {
   uint32_t done;
-  if constexpr (kCluster)
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(bar_addr), "r"(parity), "r"(hint_ns)
-        : "memory");
-  else
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(bar_addr), "r"(parity), "r"(hint_ns)
-        : "memory");
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar_addr), "r"(parity), "r"(hint_ns)
+      : "memory");
   return done != 0;
 }
 
@@ -150,17 +117,16 @@ constexpr uint32_t kSuspendHintNs = 200000;
 // Returns false (and records FP8_ERR_TIMEOUT with `site`) when the limit
 // runs out or another role of this CTA has already given up (`abort_flag`).
 // Never traps, never spins forever.
-template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           volatile uint32_t* abort_flag,
                                           uint32_t* status, uint32_t site,
                                           uint64_t limit_ns) {
   const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait<kCluster>(a, parity)) return true;
+  if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
 #pragma unroll 1
   while (true) {
-    if (mbar_try_wait_suspend<kCluster>(a, parity, kSuspendHintNs)) return true;
+    if (mbar_try_wait_suspend(a, parity, kSuspendHintNs)) return true;
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > limit_ns) {
       *abort_flag = 1u;
@@ -237,70 +203,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// ------------------------------------------------------------ clusters
-
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-// Address of the same shared-memory location in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t smem_addr,
-                                                uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
-               : "=r"(r)
-               : "r"(smem_addr), "r"(rank));
-  return r;
-}
-
-// All threads of every CTA in the cluster.
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile(
-      "barrier.cluster.arrive.release.aligned;\n\t"
-      "barrier.cluster.wait.acquire.aligned;" ::
-          : "memory");
-}
-
-// Arrive on an mbarrier given by its shared::cluster address (possibly in
-// the other CTA of the pair).
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile(
-      "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
-          cluster_addr)
-      : "memory");
-}
-
-// 2-D / 3-D tiled loads for a CTA pair: the data lands in this CTA's shared
-// memory, the byte count is signalled on the mbarrier at `bar_cluster_addr`
-// (the pair leader's barrier).  No multicast.
-__device__ __forceinline__ void tma_load_2d_pair(void* smem_dst,
-                                                 const CUtensorMap* map,
-                                                 uint32_t bar_cluster_addr,
-                                                 int32_t c0, int32_t c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::"
-      "complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(c0),
-      "r"(c1)
-      : "memory");
-}
-
-__device__ __forceinline__ void tma_load_3d_pair(void* smem_dst,
-                                                 const CUtensorMap* map,
-                                                 uint32_t bar_cluster_addr,
-                                                 int32_t c0, int32_t c1,
-                                                 int32_t c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::"
-      "complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
-          smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(c0),
-      "r"(c1), "r"(c2)
-      : "memory");
-}
-
 // --------------------------------------------------------------- tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem,
@@ -322,57 +224,6 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
                    taddr),
                "r"(ncols)
                : "memory");
-}
-
-// CTA-pair (cta_group::2) forms: executed by the same warp in both CTAs of
-// the pair; the allocation gives both CTAs the same TMEM address.
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem,
-                                                uint32_t ncols) {
-  asm volatile(
-      "tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-          smem_u32(dst_smem)),
-      "r"(ncols)
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_relinquish_pair() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::
-                   : "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr,
-                                                  uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(
-                   taddr),
-               "r"(ncols)
-               : "memory");
-}
-
-// Pair MMA, issued by one thread of the leader CTA: A rows 0..M/2-1 and
-// B rows 0..N/2-1 come from the leader's shared memory, the other halves from
-// the peer's at the same offsets; D rows are split the same way between the
-// two CTAs' TMEM.
-__device__ __forceinline__ void mma_e4m3_pair(uint32_t d_tmem, uint64_t a_desc,
-                                              uint64_t b_desc, uint32_t idesc,
-                                              uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(
-          d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Arrive once on the mbarrier at this offset in every CTA of `cta_mask` when
-// all pair MMAs issued by this thread so far have completed.
-__device__ __forceinline__ void mma_commit_pair(uint64_t* bar,
-                                                uint16_t cta_mask) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster."
-      "multicast::cluster.b64 [%0], %1;" ::"r"(smem_u32(bar)),
-      "h"(cta_mask)
-      : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before_sync() {

@@ -133,31 +133,12 @@ def test_end_to_end_full_size_sampled(idx, shape_index):
     assert sqnr >= 20.0, sqnr
 
 
-@pytest.mark.parametrize("recipe,M,N,K,bias", [
-    ("row", 300, 272, 528, True),
-    ("row", 4096, 4096, 256, False),
-    ("tensor", 256, 256, 256, False),
-    ("1x128_128x128", 1100, 2304, 1024, False),   # blockwise: stays on single CTAs
-])
-def test_gemm_parity_cta_pairs(recipe, M, N, K, bias, monkeypatch):
-    """The CTA-pair kernel (cta_group::2, 256-row items) of the dense recipes,
-    selected with FP8SM_CTA_PAIRS=1, against the oracle."""
-    monkeypatch.setenv("FP8SM_CTA_PAIRS", "1")
-    test_gemm_parity(recipe, M, N, K, bias, torch.float32)
-
-
-@pytest.mark.parametrize("recipe,pairs", [
-    ("row", False), ("row", True), ("tensor", False),
-    ("1x128_128x128", False), ("1x128_128x1", False),
-])
-def test_gemm_banded_tile_order_large_b(recipe, pairs, monkeypatch):
+@pytest.mark.parametrize("recipe", ["row", "tensor", "1x128_128x128", "1x128_128x1"])
+def test_gemm_banded_tile_order_large_b(recipe):
     """B's codes above 64 MiB (N = 8192, K = 8320): the dense kernels take
     their tiles in bands of 16 M tiles, N-major inside a band.  M = 2500 gives
-    20 M tiles of 128 rows (a full band and a partial one) or 10 of 256 rows
-    (CTA pairs: one partial band).  Sampled rows of every band, fp32 output,
-    against the oracle."""
-    if pairs:
-        monkeypatch.setenv("FP8SM_CTA_PAIRS", "1")
+    20 M tiles of 128 rows (a full band and a partial one).  Sampled rows of
+    every band, fp32 output, against the oracle."""
     M, N, K = 2500, 8192, 8320
     b_std = 0.02 if recipe != "1x128_128x1" else 1.0
     a_std = 1.0 if recipe != "1x128_128x1" else 1e-3

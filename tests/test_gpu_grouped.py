@@ -104,9 +104,3 @@ def test_grouped_full_size_sampled():
     oqa, osa, oqb, osb = oracle_grouped_operands(wl)
     ref, mag = oracle.grouped_scaled_mm(oqa, oqb, osa, osb, wl.offs.numpy(), rows=rows)
     check_gemm(out_f64(out)[rows], ref, mag, "grouped full size")
-
-
-def test_grouped_parity_cta_pairs(monkeypatch):
-    monkeypatch.setenv("FP8SM_CTA_PAIRS", "1")
-    test_grouped_parity([1, 255, 129, 0, 2], 528, 160, torch.bfloat16)
-    test_grouped_parity([5, 0, 17, 130], 272, 256, torch.float32)
