@@ -4,15 +4,14 @@ and the chain of two linears it enables.
 Two checks per case.  (1) Against the oracle, independently: the oracle
 quantizes the same seeded inputs and computes the fp64 GEMM; the dequantized
 kernel output (code * scale) must be within the GEMM tolerance plus half an
-e4m3 step of it.  (2) A property of the kernel's own output, with no oracle
-involved: its codes and scales are exactly the 1x128 quantization (the scale
-and cast steps of "per-token scaling for fp8 linear", Highlights) of the fp32
-result that the same GEMM writes when asked for fp32 output -- amax of each
-group, scale = amax/448, codes = round-to-nearest-even e4m3 of y * 448/amax,
-saturated -- each step one fp32 operation, restated here with numpy fp32
-arithmetic and torch's float8_e4m3fn cast.  (2) is what makes the fused
-quantize bit-exact; the rounding of the fp32 GEMM itself differs from the
-fp64 reference, so codes cannot be compared with an oracle quantize of it."""
+e4m3 step of it.  (2) A property of the kernel's own output: its codes and
+scales are exactly the 1x128 quantization (the scale and cast steps of
+"per-token scaling for fp8 linear", Highlights) of the fp32 result that the
+same GEMM writes when asked for fp32 output -- the oracle's fp32-input
+quantizer applied to that fp32 result must reproduce them bit for bit.  (2) is
+what makes the fused quantize bit-exact; the rounding of the fp32 GEMM itself
+differs from the fp64 reference, so codes cannot be compared with an oracle
+quantize of the fp64 result."""
 import numpy as np
 import pytest
 import torch
@@ -60,18 +59,14 @@ def run_both(qa, sa, qb, sb, recipe, bias):
 
 
 def check_exact(y, q, s, what):
-    """q, s (scales (N/128, M)) are the 1x128 quantization of the fp32 y."""
+    """q, s (scales (N/128, M)) are the 1x128 quantization of the fp32 y: the
+    oracle's fp32-input quantizer is run on the kernel's own fp32 result and
+    must give the same codes and scales bit for bit."""
     M, N = y.shape
-    g = y.astype(np.float32).reshape(M, N // 128, 128)
-    a = np.maximum(np.abs(g).max(axis=2), np.float32(1e-12))      # (M, N/128)
-    s_want = (a / np.float32(448.0)).astype(np.float32)
-    inv = (np.float32(448.0) / a).astype(np.float32)
-    t = np.clip(g * inv[:, :, None], np.float32(-448.0), np.float32(448.0)).reshape(M, N)
-    assert t.dtype == np.float32
-    q_want = torch.from_numpy(np.ascontiguousarray(t)).to(torch.float8_e4m3fn)
-    q_want = q_want.view(torch.uint8).numpy()
-    s = s.reshape(N // 128, M)
-    bad_s = np.argwhere(s_want.T.view(np.uint32) != s.view(np.uint32))
+    q_want, s_want = oracle.quantize_f32(np.ascontiguousarray(y.astype(np.float32)),
+                                         oracle.GROUP_1x128)
+    s = np.ascontiguousarray(s).reshape(-1)[:s_want.size]
+    bad_s = np.argwhere(s_want.view(np.uint32) != s.view(np.uint32))
     assert bad_s.size == 0, f"{what}: {len(bad_s)} scales differ, first {bad_s[0]}"
     bad = np.argwhere(q_want != q)
     assert bad.size == 0, (f"{what}: {len(bad)} codes differ, first {bad[0]} "

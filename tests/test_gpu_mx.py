@@ -164,24 +164,19 @@ def tile_words(M: int, N: int) -> np.ndarray:
 
 
 def check_mx_output_property(y, q, tiles, what):
-    """q, tiles are the MXFP8 quantization of the fp32 y, restated here:
-    per 32-column block, e = floor(log2(amax)) - 8 clamped to [-127, 127]
-    (from the fp32 bits of amax), codes = RNE e4m3 of y * 2^-e saturated."""
+    """q, tiles are the MXFP8 quantization of the fp32 y: the oracle's
+    fp32-input MXFP8 conversion of the kernel's own fp32 result must give the
+    same codes and scale bytes (at each row's place in the scale-factor
+    tiles).  Returns the block exponents e (scale 2^e)."""
     M, N = y.shape
-    g = y.astype(np.float32).reshape(M, N // 32, 32)
-    amax = np.abs(g).max(axis=2)
-    be = (amax.view(np.uint32) >> 23).astype(np.int64)
-    e = np.maximum(be - 127 - 8, -127)
-    t = np.clip(g.astype(np.float64) / np.ldexp(1.0, e)[:, :, None], -448, 448)
-    q_want = torch.from_numpy(t.reshape(M, N).astype(np.float32)).to(torch.float8_e4m3fn)
-    q_want = q_want.view(torch.uint8).numpy()
+    q_want, e8 = oracle.mx_quantize_f32(np.ascontiguousarray(y.astype(np.float32)))
     bad = np.argwhere(q_want != q)
     assert bad.size == 0, f"{what}: {len(bad)} codes differ, first {bad[0]}"
     off = tile_words(M, N)
     got_e = np.stack([tiles[off + k] for k in range(4)], axis=2).reshape(M, N // 32)
-    bad = np.argwhere(got_e.astype(np.int64) != e + 127)
+    bad = np.argwhere(got_e != e8)
     assert bad.size == 0, f"{what}: {len(bad)} scale bytes differ, first {bad[0]}"
-    return e
+    return e8.astype(np.int64) - 127
 
 
 @pytest.mark.parametrize("M,N,K,bias", [(128, 256, 128, False), (130, 384, 96, True),
