@@ -317,6 +317,10 @@ class Step:
             self.sb = torch.empty(E * fp8sm.scale_count(wl.N, wl.K, self.qb_recipe),
                                   dtype=torch.float32, device=dev)
         self.chain = wl.recipe in ("chain", "chain_mx")
+        # both operands on one stream when B takes the 128x128 tile kernel
+        # through fp8_quantize (and A the 1x128 kernel)
+        self.serial_quant = (wl.recipe in ("1x128_128x128", "chain") and not self.t_a
+                             and not self.t_b)
         if self.chain:
             # second linear: its weight (N2, N) quantized 128x128 like b; the
             # first GEMM's output leaves as e4m3 codes + 1x128 scales
@@ -364,9 +368,21 @@ class Step:
     def quantize(self):
         """Both operands' quantization; the second runs on a side stream,
         concurrently with the first (same work, overlapped), and the main
-        stream waits for it before the GEMM."""
+        stream waits for it before the GEMM.  When B is quantized in 128x128
+        tiles (the TMA-fed tile kernel) both run on the main stream, B's
+        first: measured, the tile kernel and the 1x128 kernel run faster one
+        after the other than side by side."""
         f = self.f
         main = torch.cuda.current_stream()
+        if self.serial_quant:
+            f.fp8_quantize(self.b, self.qb_recipe, out=self.qb, scales=self.sb,
+                           workspace=self.ws_b, stream=main)
+            if self.chain:
+                f.fp8_quantize(self.b2, self.qb_recipe, out=self.qb2, scales=self.sb2,
+                               workspace=self.ws_b, stream=main)
+            f.fp8_quantize(self.a, self.qa_recipe, out=self.qa, scales=self.sa,
+                           workspace=self.ws, stream=main)
+            return
         self.ev_fork.record(main)
         self.side.wait_event(self.ev_fork)
         with torch.cuda.stream(self.side):

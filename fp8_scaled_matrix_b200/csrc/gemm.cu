@@ -1337,39 +1337,6 @@ __global__ void timeout_probe_kernel(uint64_t limit_ns, uint32_t* status) {
 
 // ------------------------------------------------------------ host side
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult qres;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr,
-                                cudaEnableDefault, &qres) == cudaSuccess &&
-        qres == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
-bool make_tmap(CUtensorMap* m, CUtensorMapDataType dt, uint32_t rank,
-               const void* base, const uint64_t* dims, const uint64_t* strides,
-               const uint32_t* box, CUtensorMapSwizzle sw, std::string* err) {
-  auto fn = encode_fn();
-  if (!fn) {
-    if (err) *err = "cuTensorMapEncodeTiled is not available from the driver";
-    return false;
-  }
-  uint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, dt, rank, const_cast<void*>(base), dims, strides, box,
-                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) {
-    if (err) *err = "cuTensorMapEncodeTiled failed (code " + std::to_string((int)r) + ")";
-    return false;
-  }
-  return true;
-}
-
 template <int kRecipe, int kOut, bool kGrouped>
 cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb,
                           const CUtensorMap& tbh, const CUtensorMap& to,
@@ -1466,6 +1433,41 @@ bool a_map(CUtensorMap* m, const void* a, int64_t rows, int64_t K, std::string* 
 }
 
 }  // namespace
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr,
+                                cudaEnableDefault, &qres) == cudaSuccess &&
+        qres == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// Tiled tensor map (no interleave, 256-byte L2 promotion, zero fill out of
+// bounds); false with *err set when the driver refuses it.
+bool make_tmap(CUtensorMap* m, CUtensorMapDataType dt, uint32_t rank,
+               const void* base, const uint64_t* dims, const uint64_t* strides,
+               const uint32_t* box, CUtensorMapSwizzle sw, std::string* err) {
+  auto fn = encode_fn();
+  if (!fn) {
+    if (err) *err = "cuTensorMapEncodeTiled is not available from the driver";
+    return false;
+  }
+  uint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, dt, rank, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    if (err) *err = "cuTensorMapEncodeTiled failed (code " + std::to_string((int)r) + ")";
+    return false;
+  }
+  return true;
+}
 
 cudaError_t launch_scaled_mm(const void* a, const void* b, int64_t M,
                              int64_t N, int64_t K, const float* sa,

@@ -2,6 +2,7 @@
 // kernel translation units.  Launchers assume arguments were validated.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -38,6 +39,14 @@ cudaError_t once_per_device(std::atomic<bool> (&done)[kMaxDevices], std::mutex& 
   if (e == cudaSuccess) done[device].store(true, std::memory_order_release);
   return e;
 }
+
+// Tiled TMA tensor map over `base` (gemm.cu): rank 2 or 3, dims/strides in
+// elements/bytes (innermost first, strides of dims 1..rank-1), box in
+// elements; no interleave, 256-byte L2 promotion, zero fill out of bounds.
+// Returns false with *err set when the driver refuses the map.
+bool make_tmap(CUtensorMap* m, CUtensorMapDataType dt, uint32_t rank, const void* base,
+               const uint64_t* dims, const uint64_t* strides, const uint32_t* box,
+               CUtensorMapSwizzle sw, std::string* err);
 
 // Quantizers (quantize.cu).  recipe: 0 tensor, 1 row, 2 1x128, 3 128x128.
 cudaError_t launch_quantize(const void* x, int64_t rows, int64_t cols,

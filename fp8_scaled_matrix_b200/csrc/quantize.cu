@@ -45,8 +45,11 @@ __device__ __forceinline__ float amax8(const uint4& v, float m) {
   return m;
 }
 
+// A packed bf16 pair -> two e4m3 codes: one packed multiply (each lane an
+// IEEE fp32 multiply, bit-identical to two scalar ones), one pair convert.
 __device__ __forceinline__ uint32_t cast2(uint32_t w, float inv) {
-  return cast_f32x2(bf16_lo(w), bf16_hi(w), inv);
+  const float2 y = mul2(make_float2(bf16_lo(w), bf16_hi(w)), make_float2(inv, inv));
+  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3));
 }
 
 // 8 bf16 -> 8 e4m3 bytes (little-endian order preserved).
@@ -306,57 +309,73 @@ __global__ void __launch_bounds__(256) quant_mx_kernel(
 }
 
 // ------------------------------------------------------------ 128x128
-// One CTA (512 threads) per 128x128 tile: thread t covers the 16-byte chunk
-// t%16 of rows t/16 + 32 i (i < 4), so each warp-wide load reads two whole
-// 256-byte row segments (coalesced); the 4 chunks stay in registers.
-// Ragged last row block: rows past the end take no part in the amax and are
-// not written.
-constexpr int k128Threads = 512;
-// Batched (blockIdx.y = matrix e of a stack of equal matrices, e.g. the
-// experts' weights): matrix e at x + e * rows * ld, its codes at
-// q + e * rows * cols, its scales at scales + e * (cols / 128) * ceil(rows / 128).
+// One CTA (256 threads) per 128 x 128 tile, blockIdx.y = the matrix of a
+// stack of equal matrices (the experts' weights).  The tile arrives in
+// shared memory by one TMA load (a 3-D map (cols, rows, matrix): a ragged
+// last row block reads zeros past the matrix's last row, which leave the
+// amax unchanged) and stays there: a first pass reads it for the amax, a
+// second pass reads it again for the cast, so a thread holds one 16-byte
+// chunk at a time.  Few registers and 32 KB of shared memory per CTA let up
+// to seven tiles per SM be in flight, and the short-lived CTAs interleave
+// with those of a concurrent quantization of the other GEMM operand.
+// Thread t takes the chunks t + 256 i (row (t + 256 i) / 16, conflict-free);
+// codes leave as 8-byte stores (16 threads write one row's 128 bytes); rows
+// past the end are not written.  Tile (rb, kb) of matrix e has its scale at
+// scales[e * (cols / 128) * RB + kb * RB + rb].
+constexpr int k128Threads = 256;
+constexpr uint32_t kQTileBytes = 128 * 128 * 2;
+constexpr size_t kQSmemBytes = kQTileBytes + 128;  // + 128-byte alignment slack
+
 __global__ void __launch_bounds__(k128Threads) quant_128x128_kernel(
-    const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
-    uint8_t* __restrict__ q, float* __restrict__ scales) {
-  constexpr int kWarps = k128Threads / 32;
-  constexpr int kRowStep = k128Threads / 16;       // rows covered per load round
-  constexpr int kRounds = 128 / kRowStep;
-  __shared__ float warp_amax[kWarps];
-  const int64_t RB = (rows + 127) >> 7;
-  {
-    const int64_t e = blockIdx.y;
-    x += e * rows * ld;
-    q += e * rows * cols;
-    scales += e * (cols >> 7) * RB;
-  }
-  const int64_t rb = blockIdx.x % RB;
-  const int64_t kb = blockIdx.x / RB;
+    const __grid_constant__ CUtensorMap tm_x, int64_t rows, int64_t cols,
+    uint8_t* __restrict__ q, float* __restrict__ scales, uint32_t* status) {
+  extern __shared__ uint8_t qsmem_raw[];
+  __shared__ uint64_t full;
+  __shared__ float warp_amax[k128Threads / 32];
+  __shared__ uint32_t abort_flag;
+  const uint32_t raw = smem_u32(qsmem_raw);
+  const uint4* tile = reinterpret_cast<const uint4*>(qsmem_raw + (((raw + 127u) & ~127u) - raw));
   const int t = threadIdx.x;
-  const int64_t row0 = rb * 128 + (t >> 4);
-  const int64_t col = kb * 128 + (t & 15) * 8;
-  const uint16_t* xp = x + row0 * ld + col;
-  uint4 v[kRounds];
+  const int64_t RB = (rows + 127) >> 7;
+  const int64_t e = blockIdx.y;
+  const int64_t rb = blockIdx.x % RB, kb = blockIdx.x / RB;
+  if (t == 0) {
+    mbar_init(&full, 1);
+    abort_flag = 0u;
+    fence_barrier_init();
+    mbar_arrive_expect_tx(&full, kQTileBytes);
+    tma_load_3d(const_cast<uint4*>(tile), &tm_x, &full, static_cast<int32_t>(kb * 128),
+                static_cast<int32_t>(rb * 128), static_cast<int32_t>(e));
+  }
+  __syncthreads();
+  const bool got = mbar_wait(&full, 0, &abort_flag, status, SITE_QUANT_TMA, kWaitLimitNs);
+  if (!__syncthreads_and(got)) {
+    // let the load land before the CTA exits
+    if (t == 0) {
+      uint32_t dummy = 0;
+      mbar_wait(&full, 0, &dummy, nullptr, SITE_TEARDOWN, 10000000ull);
+    }
+    return;
+  }
   float m = 0.0f;
 #pragma unroll
-  for (int i = 0; i < kRounds; ++i)
-    v[i] = row0 + kRowStep * i < rows
-               ? ld_stream(reinterpret_cast<const uint4*>(xp + kRowStep * i * ld))
-               : make_uint4(0, 0, 0, 0);  // zero padding does not change the max
-#pragma unroll
-  for (int i = 0; i < kRounds; ++i) m = amax8(v[i], m);
+  for (int k = 0; k < 8; ++k) m = amax8(tile[t + 256 * k], m);
   m = warp_max(m);
   if ((t & 31) == 0) warp_amax[t >> 5] = m;
   __syncthreads();
   float tm = warp_amax[0];
 #pragma unroll
-  for (int i = 1; i < kWarps; ++i) tm = fmaxf(tm, warp_amax[i]);
+  for (int w = 1; w < k128Threads / 32; ++w) tm = fmaxf(tm, warp_amax[w]);
   const ScalePair sp = scales_from_amax(tm);
-  if (t == 0) scales[kb * RB + rb] = sp.s;
-  uint8_t* qp = q + row0 * cols + col;
+  if (t == 0) scales[e * RB * (cols >> 7) + kb * RB + rb] = sp.s;
+  const int64_t nrows = rows - rb * 128 < 128 ? rows - rb * 128 : 128;
+  uint8_t* qt = q + (e * rows + rb * 128) * cols + kb * 128 + (t & 15) * 8;
 #pragma unroll
-  for (int i = 0; i < kRounds; ++i)
-    if (row0 + kRowStep * i < rows)
-      *reinterpret_cast<uint2*>(qp + kRowStep * i * cols) = cast8(v[i], sp.inv);
+  for (int k = 0; k < 8; ++k) {
+    const int row = (t >> 4) + 16 * k;
+    const uint2 c = cast8(tile[t + 256 * k], sp.inv);
+    if (row < nrows) *reinterpret_cast<uint2*>(qt + static_cast<int64_t>(row) * cols) = c;
+  }
 }
 
 // ------------------------------------------------------- transposed
@@ -366,47 +385,63 @@ __global__ void __launch_bounds__(k128Threads) quant_128x128_kernel(
 // x's rows).  The result equals the 1x128 / 128x128 quantization of the
 // transposed matrix: a group is 128 consecutive rows of x within one column
 // (1x128) or a 128 x 128 tile (128x128).
-// Persistent CTAs (512 threads) walk the 128-row x 128-column tiles of x
-// with a two-buffer cp.async pipeline: the next tile's 16-byte chunks
-// (coalesced rows of x) stream into shared memory while this tile is
-// processed.  Thread t takes column t % 128 and rows 32 (t / 128) .. +31 of
-// the tile: it reads them from shared memory (a warp reads 32 consecutive
-// columns of one row), the four quarter-columns' amax meet in shared memory,
-// and the thread stages its 32 codes in shared memory; the tile's 128 output
-// rows (x's columns) then leave as whole 128-byte lines.
+// Persistent CTAs (256 threads, two per SM) walk the 128-row x 128-column
+// tiles of x; each tile arrives in shared memory by TMA (3-D map (cols,
+// rows, matrix); columns past the end read as zero) through a two-buffer
+// ring per CTA.  Thread t reads the 16-byte chunk t % 16 (8 columns) of the
+// 8 consecutive rows 8 (t / 16) .. + 7 (whole 256-byte rows per warp access),
+// so after the cast it holds 8 consecutive codes of each of its 8 columns:
+// one 8-byte word per output row.  The words go to a 16 KB staging area laid
+// out as the tile's 128 output rows of 128 bytes, with the 8-byte slot of a
+// word XOR-swizzled by its column group (conflict-free stores), and leave as
+// 16-byte stores, eight threads per 128-byte output row.  1x128: column
+// maxima over 16 rows per warp (one shuffle), then over the 8 warps through
+// shared memory, where one thread per column forms its scale.
 constexpr int kTrRows = 128;
 constexpr int kTrCols = 128;
-constexpr int kTrThreads = 512;
-constexpr int kTrPitch = kTrCols + 8;  // bf16 elements per shared row (16-byte pad)
-constexpr int kTrTileElems = kTrRows * kTrPitch;
-constexpr int kTrOutPitch = kTrRows + 16;  // bytes per staged output row (conflict-free 16-byte stores)
-constexpr size_t kTrSmemBytes =
-    2 * kTrTileElems * sizeof(uint16_t) + static_cast<size_t>(kTrCols) * kTrOutPitch;
+constexpr int kTrThreads = 256;
+constexpr int kTrStages = 2;
+constexpr uint32_t kTrTileBytes = kTrRows * kTrCols * 2;
+constexpr uint32_t kTrOutBytes = kTrCols * kTrRows;
+constexpr size_t kTrSmemBytes = kTrStages * kTrTileBytes + kTrOutBytes + 1024;  // + alignment
 constexpr int kTrCtasPerSm = 2;
 
 // Grouped (per-expert) variant, 1x128 only: rows are tokens split into
 // groups by cumulative offsets; each group's tokens are laid out in the
 // output padded to a multiple of 128 (group g starts at output column
 // 128 * pb0[g], pb0 = exclusive prefix of ceil(size / 128)), so no 128-token
-// block mixes two groups; the padding is zero.  ldq = the output row stride.
+// block mixes two groups; the padding is zero (rows of the next group that
+// the block's tile load brings in are taken as zero).  ldq = the output row
+// stride.
 constexpr int kTrMaxGroups = 2048;
 
-// Batched (`batch` equal matrices, not grouped): matrix e at x + e * rows *
-// ld, its transposed codes at q + e * cols * ldq, its scales after the e
-// earlier matrices' scales; tiles are numbered matrix-major.
+// Batched (`batch` equal matrices, not grouped): matrix e's transposed codes
+// at q + e * cols * ldq, its scales after the e earlier matrices' scales;
+// tiles are numbered matrix-major.
 template <bool k128x128, bool kGroupedT>
 __global__ void __launch_bounds__(kTrThreads) quant_transposed_kernel(
-    const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+    const __grid_constant__ CUtensorMap tm_x, int64_t rows, int64_t cols,
     uint8_t* __restrict__ q, float* __restrict__ scales, const int32_t* __restrict__ offs,
     int32_t E, int64_t ldq, int64_t n_kb, uint32_t* status, int32_t batch) {
-  extern __shared__ __align__(16) uint16_t tiles_smem[];
-  __shared__ float part[4][kTrCols];
+  extern __shared__ uint8_t tr_smem_raw[];
+  __shared__ uint64_t full[kTrStages];
+  __shared__ __align__(16) float part[kTrThreads / 32][kTrCols];
+  __shared__ __align__(16) float inv_s[kTrCols];  // 1x128: the tile's column inverses
   __shared__ float warp_amax[kTrThreads / 32];
+  __shared__ uint32_t abort_flag;
+  // each buffer's first input row and row count, set by the thread that
+  // issues its load (before its arrive, so the buffer's waiters see them)
+  __shared__ int64_t buf_row0[kTrStages];
+  __shared__ int32_t buf_nrows[kTrStages];
+  const uint32_t raw = smem_u32(tr_smem_raw);
+  uint8_t* const tiles = tr_smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* const stage_out = tiles + kTrStages * kTrTileBytes;
   const int64_t n_cb = (cols + kTrCols - 1) / kTrCols;
   const int64_t per_matrix = n_kb * n_cb;
   const int64_t n_tiles = per_matrix * batch;
   const int64_t scales_per_matrix = k128x128 ? n_kb * n_cb : n_kb * cols;
   const int t = threadIdx.x;
+  const int w = t >> 5;
   int32_t* pb0 = nullptr;  // grouped: pb0[g] = padded blocks before group g; pb0[E] = total
   if constexpr (kGroupedT) {
     __shared__ int32_t table[kTrMaxGroups + 1];
@@ -465,105 +500,178 @@ __global__ void __launch_bounds__(kTrThreads) quant_transposed_kernel(
     }
   };
   const int64_t n_kb_used = kGroupedT ? pb0[E] : n_kb;
-  // copy tile `tile` into buffer `buf`: chunk t % 16 (8 columns) of rows
-  // t / 16 + 32 i; columns past the end (and grouped: rows past the group)
-  // are zero-filled (no effect on the max, zero codes)
-  auto issue = [&](int64_t tile, int buf) {
+  // the load of tile `tile` into buffer s (grouped: blocks past the last
+  // group's complete the buffer's phase without a copy)
+  auto issue = [&](int64_t tile, int s) {
     const int64_t e = tile / per_matrix;
-    tile -= e * per_matrix;
-    const int64_t kb = tile % n_kb, cb = tile / n_kb;
+    const int64_t r = tile - e * per_matrix;
+    const int64_t kb = r % n_kb, cb = r / n_kb;
     if (kb >= n_kb_used) {
-      cp_async_commit();
+      mbar_arrive(&full[s]);
       return;
     }
     int64_t row0;
     int32_t nrows;
     block_rows(kb, row0, nrows);
-    const int ch = t & 15;
-    const int64_t col = cb * kTrCols + ch * 8;
-    uint16_t* dst = tiles_smem + buf * kTrTileElems;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = (t >> 4) + 32 * i;
-      const bool in = col < cols && r < nrows;
-      cp_async_16(dst + r * kTrPitch + ch * 8, in ? x + e * rows * ld + (row0 + r) * ld + col : x,
-                  in ? 16u : 0u);
-    }
-    cp_async_commit();
+    buf_row0[s] = row0;
+    buf_nrows[s] = nrows;
+    mbar_arrive_expect_tx(&full[s], kTrTileBytes);
+    tma_load_3d(tiles + s * kTrTileBytes, &tm_x, &full[s], static_cast<int32_t>(cb * kTrCols),
+                static_cast<int32_t>(row0), static_cast<int32_t>(e));
   };
-  int64_t tile = blockIdx.x;
-  if (tile < n_tiles) issue(tile, 0);
-  const int c = t & (kTrCols - 1);   // column within the tile = output row
-  const int qr = t >> 7;             // rows 32 qr .. 32 qr + 31
-  for (int it = 0; tile < n_tiles; tile += gridDim.x, ++it) {
-    const int buf = it & 1;
-    if (tile + gridDim.x < n_tiles) issue(tile + gridDim.x, buf ^ 1);
-    else cp_async_commit();          // empty group: the wait below counts groups
-    cp_async_wait<1>();              // this tile's copies have landed
-    __syncthreads();
-    const uint16_t* tl = tiles_smem + buf * kTrTileElems;
+  if (t == 0) {
+    for (int s = 0; s < kTrStages; ++s) mbar_init(&full[s], 1);
+    abort_flag = 0u;
+    fence_barrier_init();
+    prefetch_tmap(&tm_x);
+  }
+  __syncthreads();
+  if (t == 0) {
+    int64_t tile = blockIdx.x;
+    for (int s = 0; s < kTrStages && tile < n_tiles; ++s, tile += gridDim.x) issue(tile, s);
+  }
+  int64_t issued_to = blockIdx.x + static_cast<int64_t>(kTrStages) * gridDim.x;
+  const int ch = t & 15;         // 16-byte chunk: columns 8 ch .. 8 ch + 7 of the tile
+  const int rg = t >> 4;         // rows 8 rg .. 8 rg + 7 of the tile
+  int i = 0;
+  for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++i) {
+    const int s = i % kTrStages;
+    const uint32_t parity = static_cast<uint32_t>((i / kTrStages) & 1);
+    const bool got = mbar_wait(&full[s], parity, &abort_flag, status, SITE_QUANT_TMA,
+                               kWaitLimitNs);
+    if (!__syncthreads_and(got)) break;
     const int64_t e = tile / per_matrix;
     const int64_t kb = (tile - e * per_matrix) % n_kb, cb = (tile - e * per_matrix) / n_kb;
-    float* const sc = scales + e * scales_per_matrix;
-    uint8_t* const qm = q + e * cols * ldq;
-    if (kb >= n_kb_used) continue;   // grouped: past the last group's blocks (uniform)
-    uint32_t w[16];                  // the 32 values, packed bf16 pairs
-    float m = 0.0f;
+    if (kb >= n_kb_used) {  // grouped: past the last group's blocks (uniform)
+      if (t == 0 && issued_to < n_tiles) {
+        issue(issued_to, s);
+        issued_to += gridDim.x;
+      }
+      continue;
+    }
+    const int32_t nrows = buf_nrows[s];
+    // this thread's 8 rows x 8 columns (rows past the block's end: zero)
+    const uint8_t* tl = tiles + s * kTrTileBytes;
+    uint4 v[8];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const uint32_t lo = tl[(32 * qr + 2 * j) * kTrPitch + c];
-      const uint32_t hi = tl[(32 * qr + 2 * j + 1) * kTrPitch + c];
-      w[j] = lo | (hi << 16);
-      m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[j])), fabsf(bf16_hi(w[j]))));
+    for (int k = 0; k < 8; ++k) {
+      const int r = 8 * rg + k;
+      v[k] = r < nrows ? *reinterpret_cast<const uint4*>(tl + r * 256 + ch * 16)
+                       : make_uint4(0, 0, 0, 0);
     }
-    float gm;
-    if constexpr (k128x128) {
-      m = warp_max(m);
-      if ((t & 31) == 0) warp_amax[t >> 5] = m;
-      __syncthreads();
-      gm = warp_amax[0];
+    float cm[8];  // column maxima over this thread's 8 rows
 #pragma unroll
-      for (int i = 1; i < kTrThreads / 32; ++i) gm = fmaxf(gm, warp_amax[i]);
-    } else {
-      part[qr][c] = m;
-      __syncthreads();
-      gm = fmaxf(fmaxf(part[0][c], part[1][c]), fmaxf(part[2][c], part[3][c]));
-    }
-    const ScalePair sp = scales_from_amax(gm);
-    const int64_t col = cb * kTrCols + c;
-    if constexpr (k128x128) {
-      if (t == 0) sc[kb * n_cb + cb] = sp.s;
-    } else {
-      if (qr == 0 && col < cols) sc[kb * cols + col] = sp.s;
-    }
-    uint8_t* stage = reinterpret_cast<uint8_t*>(tiles_smem + 2 * kTrTileElems);
-    {
-      uint4 out[2];
-      uint32_t* o = reinterpret_cast<uint32_t*>(out);
+    for (int j = 0; j < 8; ++j) cm[j] = 0.0f;
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        o[j] = cast2(w[2 * j], sp.inv) | (cast2(w[2 * j + 1], sp.inv) << 16);
-      uint4* sd = reinterpret_cast<uint4*>(stage + c * kTrOutPitch + 32 * qr);
-      sd[0] = out[0];
-      sd[1] = out[1];
-    }
-    __syncthreads();
-    {
-      // thread t: 32 bytes (chunk t % 4) of output row t / 4 of the tile
-      const int orow = t >> 2, chunk = t & 3;
-      const int64_t ocol = cb * kTrCols + orow;
-      if (ocol < cols) {
-        const uint4* ss = reinterpret_cast<const uint4*>(stage + orow * kTrOutPitch + 32 * chunk);
-        uint4* dst = reinterpret_cast<uint4*>(qm + ocol * ldq + kb * kTrRows + 32 * chunk);
-        dst[0] = ss[0];
-        dst[1] = ss[1];
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t wd[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        cm[2 * j] = fmaxf(cm[2 * j], fabsf(bf16_lo(wd[j])));
+        cm[2 * j + 1] = fmaxf(cm[2 * j + 1], fabsf(bf16_hi(wd[j])));
       }
     }
-    // every thread is done with this buffer, the staging rows and part /
-    // warp_amax before the next iteration refills them
+    if constexpr (k128x128) {
+      float m = cm[0];
+#pragma unroll
+      for (int j = 1; j < 8; ++j) m = fmaxf(m, cm[j]);
+      m = warp_max(m);
+      if ((t & 31) == 0) warp_amax[w] = m;
+    } else {
+      // lanes l and l + 16 hold rows 16 w .. 16 w + 7 and + 8 .. + 15
+#pragma unroll
+      for (int j = 0; j < 8; ++j) cm[j] = fmaxf(cm[j], __shfl_xor_sync(0xFFFFFFFFu, cm[j], 16));
+      if ((t & 16) == 0) {
+        float4* pw = reinterpret_cast<float4*>(&part[w][8 * ch]);
+        pw[0] = make_float4(cm[0], cm[1], cm[2], cm[3]);
+        pw[1] = make_float4(cm[4], cm[5], cm[6], cm[7]);
+      }
+    }
+    __syncthreads();  // every thread holds its rows: the buffer may be refilled
+    if (t == 0 && issued_to < n_tiles) {
+      fence_proxy_async_smem();
+      issue(issued_to, s);
+      issued_to += gridDim.x;
+    }
+    float* const sc = scales + e * scales_per_matrix;
+    float inv[8];
+    if constexpr (k128x128) {
+      float gm = warp_amax[0];
+#pragma unroll
+      for (int k = 1; k < kTrThreads / 32; ++k) gm = fmaxf(gm, warp_amax[k]);
+      const ScalePair sp = scales_from_amax(gm);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) inv[j] = sp.inv;
+      if (t == 0) sc[kb * n_cb + cb] = sp.s;
+    } else {
+      // thread c < 128: column c's scale from the 8 warps' maxima, once
+      if (t < kTrCols) {
+        float gm = part[0][t];
+#pragma unroll
+        for (int k = 1; k < kTrThreads / 32; ++k) gm = fmaxf(gm, part[k][t]);
+        const ScalePair sp = scales_from_amax(gm);
+        inv_s[t] = sp.inv;
+        const int64_t col = cb * kTrCols + t;
+        if (col < cols) sc[kb * cols + col] = sp.s;
+      }
+      __syncthreads();
+      const float4 a = reinterpret_cast<const float4*>(inv_s)[2 * ch];
+      const float4 b = reinterpret_cast<const float4*>(inv_s)[2 * ch + 1];
+      inv[0] = a.x; inv[1] = a.y; inv[2] = a.z; inv[3] = a.w;
+      inv[4] = b.x; inv[5] = b.y; inv[6] = b.z; inv[7] = b.w;
+    }
+    // the 8 codes of column 8 ch + j (rows 8 rg .. + 7) -> one word of
+    // output row 8 ch + j, at slot rg ^ ch (8-byte slots of a 128-byte row);
+    // two rows per packed multiply (each lane one IEEE fp32 multiply)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float2 inv2 = make_float2(inv[j], inv[j]);
+      uint32_t c16[4];
+#pragma unroll
+      for (int pr = 0; pr < 4; ++pr) {
+        const uint32_t w0 = j < 2 ? v[2 * pr].x : j < 4 ? v[2 * pr].y : j < 6 ? v[2 * pr].z
+                                                                              : v[2 * pr].w;
+        const uint32_t w1 = j < 2 ? v[2 * pr + 1].x : j < 4 ? v[2 * pr + 1].y
+                          : j < 6 ? v[2 * pr + 1].z : v[2 * pr + 1].w;
+        const float2 xy = (j & 1) ? make_float2(bf16_hi(w0), bf16_hi(w1))
+                                  : make_float2(bf16_lo(w0), bf16_lo(w1));
+        c16[pr] = static_cast<uint32_t>(
+            __nv_cvt_float2_to_fp8x2(mul2(xy, inv2), __NV_SATFINITE, __NV_E4M3));
+      }
+      const uint2 codes = make_uint2(c16[0] | (c16[1] << 16), c16[2] | (c16[3] << 16));
+      *reinterpret_cast<uint2*>(stage_out + (8 * ch + j) * 128 + 8 * (rg ^ ch)) = codes;
+    }
+    __syncthreads();
+    {
+      uint8_t* const qm = q + e * cols * ldq;
+      const int seg = t & 7;  // 16-byte segment of an output row
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = (t >> 3) + 32 * u;  // output row within the tile
+        const int64_t ocol = cb * kTrCols + c;
+        const int sw = (c >> 3) & 15;
+        const uint2 lo = *reinterpret_cast<const uint2*>(stage_out + c * 128 + 8 * ((2 * seg) ^ sw));
+        const uint2 hi =
+            *reinterpret_cast<const uint2*>(stage_out + c * 128 + 8 * ((2 * seg + 1) ^ sw));
+        if (ocol < cols)
+          *reinterpret_cast<uint4*>(qm + ocol * ldq + kb * kTrRows + 16 * seg) =
+              make_uint4(lo.x, lo.y, hi.x, hi.y);
+      }
+    }
+    // every thread is done with the staging rows and part / warp_amax
     __syncthreads();
   }
-  cp_async_wait_all();
+  // a CTA that stopped early lets the loads it issued land before it exits
+  if (t == 0) {
+    for (int k = 0; k < kTrStages; ++k) {
+      uint32_t dummy = 0;
+      const int64_t jj = static_cast<int64_t>(i) + k;
+      const int64_t tile_j = blockIdx.x + jj * gridDim.x;
+      if (tile_j < n_tiles && tile_j < issued_to)
+        mbar_wait(&full[jj % kTrStages], static_cast<uint32_t>((jj / kTrStages) & 1), &dummy,
+                  nullptr, SITE_TEARDOWN, 10000000ull);
+    }
+  }
 }
 
 // ------------------------------------------------------------- tensor
@@ -734,58 +842,80 @@ static cudaError_t configure_transposed(const LaunchCtx& ctx) {
   });
 }
 
+// Builds x's tile map ((cols, rows, batch) bf16, 128 x 128 boxes) and
+// launches the persistent transposed kernel on up to kTrCtasPerSm CTAs per SM.
+static cudaError_t launch_transposed(const void* xv, int64_t rows, int64_t cols, int64_t ld,
+                                     bool k128, bool grouped, void* qv, float* scales,
+                                     const int32_t* offs, int32_t E, int64_t ldq, int64_t n_kb,
+                                     int32_t batch, const LaunchCtx& ctx) {
+  cudaError_t e = configure_transposed(ctx);
+  if (e != cudaSuccess) return e;
+  CUtensorMap tm;
+  // (an expert split with no tokens: the map is never read, but must be valid)
+  const uint64_t map_rows = rows > 0 ? static_cast<uint64_t>(rows) : 1;
+  const uint64_t dims[3] = {static_cast<uint64_t>(cols), map_rows, static_cast<uint64_t>(batch)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(ld) * 2, map_rows * ld * 2};
+  const uint32_t box[3] = {kTrCols, kTrRows, 1};
+  if (!make_tmap(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, xv != nullptr ? xv : qv, dims, strides,
+                 box, CU_TENSOR_MAP_SWIZZLE_NONE, ctx.err))
+    return cudaErrorInvalidValue;
+  const int64_t tiles = n_kb * ((cols + kTrCols - 1) / kTrCols) * batch;
+  const int64_t max_grid = static_cast<int64_t>(ctx.num_sms) * kTrCtasPerSm;
+  const unsigned grid = static_cast<unsigned>(tiles < max_grid ? tiles : max_grid);
+  uint8_t* q = static_cast<uint8_t*>(qv);
+  if (grouped)
+    quant_transposed_kernel<false, true><<<grid, kTrThreads, kTrSmemBytes, ctx.stream>>>(
+        tm, rows, cols, q, scales, offs, E, ldq, n_kb, ctx.status, batch);
+  else if (k128)
+    quant_transposed_kernel<true, false><<<grid, kTrThreads, kTrSmemBytes, ctx.stream>>>(
+        tm, rows, cols, q, scales, nullptr, 0, ldq, n_kb, ctx.status, batch);
+  else
+    quant_transposed_kernel<false, false><<<grid, kTrThreads, kTrSmemBytes, ctx.stream>>>(
+        tm, rows, cols, q, scales, nullptr, 0, ldq, n_kb, ctx.status, batch);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quantize_transposed(const void* xv, int64_t rows, int64_t cols,
                                        int64_t ld, int recipe, void* qv, float* scales,
                                        const LaunchCtx& ctx) {
   if (rows == 0 || cols == 0) return cudaSuccess;
-  const uint16_t* x = static_cast<const uint16_t*>(xv);
-  uint8_t* q = static_cast<uint8_t*>(qv);
-  cudaError_t e = configure_transposed(ctx);
-  if (e != cudaSuccess) return e;
-  const int64_t n_kb = rows / kTrRows;
-  const int64_t tiles = n_kb * ((cols + kTrCols - 1) / kTrCols);
-  const int64_t max_grid = static_cast<int64_t>(ctx.num_sms) * kTrCtasPerSm;
-  const unsigned grid = static_cast<unsigned>(tiles < max_grid ? tiles : max_grid);
-  if (recipe == 3)
-    quant_transposed_kernel<true, false><<<grid, kTrThreads, kTrSmemBytes, ctx.stream>>>(
-        x, rows, cols, ld, q, scales, nullptr, 0, rows, n_kb, ctx.status, 1);
-  else
-    quant_transposed_kernel<false, false><<<grid, kTrThreads, kTrSmemBytes, ctx.stream>>>(
-        x, rows, cols, ld, q, scales, nullptr, 0, rows, n_kb, ctx.status, 1);
-  return cudaGetLastError();
+  return launch_transposed(xv, rows, cols, ld, recipe == 3, false, qv, scales, nullptr, 0, rows,
+                           rows / kTrRows, 1, ctx);
 }
 
 cudaError_t launch_quantize_transposed_batched(const void* xv, int32_t batch, int64_t rows,
                                                int64_t cols, int64_t ld, int recipe, void* qv,
                                                float* scales, const LaunchCtx& ctx) {
   if (batch == 0 || rows == 0 || cols == 0) return cudaSuccess;
-  cudaError_t e = configure_transposed(ctx);
-  if (e != cudaSuccess) return e;
-  const int64_t n_kb = rows / kTrRows;
-  const int64_t tiles = n_kb * ((cols + kTrCols - 1) / kTrCols) * batch;
-  const int64_t max_grid = static_cast<int64_t>(ctx.num_sms) * kTrCtasPerSm;
-  const unsigned grid = static_cast<unsigned>(tiles < max_grid ? tiles : max_grid);
-  const uint16_t* x = static_cast<const uint16_t*>(xv);
-  uint8_t* q = static_cast<uint8_t*>(qv);
-  if (recipe == 3)
-    quant_transposed_kernel<true, false><<<grid, kTrThreads, kTrSmemBytes, ctx.stream>>>(
-        x, rows, cols, ld, q, scales, nullptr, 0, rows, n_kb, ctx.status, batch);
-  else
-    quant_transposed_kernel<false, false><<<grid, kTrThreads, kTrSmemBytes, ctx.stream>>>(
-        x, rows, cols, ld, q, scales, nullptr, 0, rows, n_kb, ctx.status, batch);
+  return launch_transposed(xv, rows, cols, ld, recipe == 3, false, qv, scales, nullptr, 0, rows,
+                           rows / kTrRows, batch, ctx);
+}
+
+// The 128x128 quantizer over `batch` equal (rows, cols) matrices stored one
+// after the other (row stride ld, matrix stride rows * ld).
+static cudaError_t launch_128x128(const void* xv, int32_t batch, int64_t rows, int64_t cols,
+                                  int64_t ld, void* qv, float* scales, const LaunchCtx& ctx) {
+  if (batch == 0 || rows == 0 || cols == 0) return cudaSuccess;
+  CUtensorMap tm;
+  const uint64_t dims[3] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows),
+                            static_cast<uint64_t>(batch)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(ld) * 2,
+                               static_cast<uint64_t>(rows) * static_cast<uint64_t>(ld) * 2};
+  const uint32_t box[3] = {128, 128, 1};
+  if (!make_tmap(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, xv, dims, strides, box,
+                 CU_TENSOR_MAP_SWIZZLE_NONE, ctx.err))
+    return cudaErrorInvalidValue;
+  const int64_t tiles = ((rows + 127) / 128) * (cols / 128);
+  quant_128x128_kernel<<<dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(batch)),
+                         k128Threads, kQSmemBytes, ctx.stream>>>(
+      tm, rows, cols, static_cast<uint8_t*>(qv), scales, ctx.status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_quantize_128x128_batched(const void* xv, int32_t batch, int64_t rows,
                                             int64_t cols, int64_t ld, void* qv, float* scales,
                                             const LaunchCtx& ctx) {
-  if (batch == 0 || rows == 0 || cols == 0) return cudaSuccess;
-  const int64_t tiles = ((rows + 127) / 128) * (cols / 128);
-  quant_128x128_kernel<<<dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(batch)),
-                         k128Threads, 0, ctx.stream>>>(static_cast<const uint16_t*>(xv), rows,
-                                                       cols, ld, static_cast<uint8_t*>(qv),
-                                                       scales);
-  return cudaGetLastError();
+  return launch_128x128(xv, batch, rows, cols, ld, qv, scales, ctx);
 }
 
 int64_t grouped_padded_tokens(int64_t tokens, int32_t E) {
@@ -796,17 +926,9 @@ cudaError_t launch_quantize_transposed_grouped(const void* xv, int64_t rows, int
                                                int64_t ld, const int32_t* offs, int32_t E,
                                                void* qv, float* scales, const LaunchCtx& ctx) {
   if (cols == 0) return cudaSuccess;
-  cudaError_t e = configure_transposed(ctx);
-  if (e != cudaSuccess) return e;
   const int64_t P = grouped_padded_tokens(rows, E);
-  const int64_t n_kb = P / kTrRows;
-  const int64_t tiles = n_kb * ((cols + kTrCols - 1) / kTrCols);
-  const int64_t max_grid = static_cast<int64_t>(ctx.num_sms) * kTrCtasPerSm;
-  const unsigned grid = static_cast<unsigned>(tiles < max_grid ? tiles : max_grid);
-  quant_transposed_kernel<false, true><<<grid, kTrThreads, kTrSmemBytes, ctx.stream>>>(
-      static_cast<const uint16_t*>(xv), rows, cols, ld, static_cast<uint8_t*>(qv), scales,
-      offs, E, P, n_kb, ctx.status, 1);
-  return cudaGetLastError();
+  return launch_transposed(xv, rows, cols, ld, false, true, qv, scales, offs, E, P, P / kTrRows,
+                           1, ctx);
 }
 
 cudaError_t launch_quantize(const void* xv, int64_t rows, int64_t cols,
@@ -847,13 +969,8 @@ cudaError_t launch_quantize(const void* xv, int64_t rows, int64_t cols,
     quant_1x128_kernel<<<grid, 256, 0, st>>>(x, rows, cols, ld, q, scales);
     return cudaGetLastError();
   }
-  if (recipe == 3) {  // 128x128
-    if (rows == 0 || cols == 0) return cudaSuccess;
-    const int64_t tiles = ((rows + 127) / 128) * (cols / 128);
-    quant_128x128_kernel<<<static_cast<unsigned>(tiles), k128Threads, 0, st>>>(
-        x, rows, cols, ld, q, scales);
-    return cudaGetLastError();
-  }
+  if (recipe == 3)  // 128x128
+    return launch_128x128(x, 1, rows, cols, ld, q, scales, ctx);
   // tensorwise
   uint32_t* ws = static_cast<uint32_t*>(workspace);
   cudaError_t e = cudaMemsetAsync(ws, 0, 2 * sizeof(uint32_t), st);

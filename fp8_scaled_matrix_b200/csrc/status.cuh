@@ -28,6 +28,7 @@ enum : uint32_t {
   SITE_SCALE_EMPTY = 9,
   SITE_EPI_SCALE_FULL = 10,
   SITE_BOUNDS = 11,  // a copy index outside its buffer (checked before the copy)
+  SITE_QUANT_TMA = 12,  // a quantizer waiting for a tile its TMA load brings
 };
 
 // Wait limit for every pipeline wait inside the GEMM / quantize kernels.
