@@ -171,7 +171,7 @@ class ClockSampler:
     def __init__(self, dev: torch.device, interval_s: float = 0.004):
         self.dev = dev
         self.interval = interval_s
-        self.samples = []      # (t, sm_mhz, power_w, reasons bitmask, gpu util %)
+        self.samples = []      # (t, sm_mhz, power_w, clock-event reasons bitmask, gpu util %)
         self.max_mhz = None
         self.handle = None
         self.source = None
@@ -220,12 +220,14 @@ class ClockSampler:
         if self._t is not None:
             self._t.join(timeout=2)
 
+    GPU_IDLE = 0x1   # NVML clock-event reason: the GPU is idle
+
     def window(self, t0: float, t1: float) -> dict:
         """Samples taken inside [t0, t1]: median SM clock, the reasons seen
-        active, and how many samples fell in the window and under load (GPU
-        utilisation above zero)."""
+        active, and how many samples fell in the window and under load (the
+        driver's GPU-idle clock-event reason not set)."""
         sel = [x for x in self.samples if t0 <= x[0] <= t1]
-        load = [x for x in sel if x[4] > 0]
+        load = [x for x in sel if not (x[3] & self.GPU_IDLE)]
         use = load or sel
         reasons = sorted({n for x in use for n, bit in self.REASONS if x[3] & bit})
         return {"sm_mhz": float(np.median([x[1] for x in use])) if use else None,
@@ -1031,6 +1033,160 @@ def cpu_baseline(wl, rows: int, repeats: int = 1):
         f"rows ({tg:.2f} s), scaled to all rows"))
 
 
+# ------------------------------------------------------------ kernel tables
+
+def _timed_graph(fn, reps: int, flush: torch.Tensor) -> float:
+    """Median device time (µs) of `fn`'s launches replayed from a CUDA graph,
+    L2 flushed before every replay (outside the events)."""
+    from fp8_scaled_matrix_b200 import fp8sm
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        evict_l2(flush)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e3)
+    fp8sm.check_device_status()
+    return float(np.median(ts))
+
+
+def _random_codes(r: int, c: int, dev) -> torch.Tensor:
+    """e4m3 codes of random finite values (no NaN codes)."""
+    x = torch.randint(0, 0x7E, (r, c), dtype=torch.int32, device=dev)
+    s = torch.randint(0, 2, (r, c), dtype=torch.int32, device=dev) << 7
+    return (x | s).to(torch.uint8)
+
+
+def kernel_table(kind: str, only, dev, reps: int = 30) -> dict:
+    """Every quantize kernel (kind "quantize") or GEMM recipe (kind "gemm")
+    timed alone on the benchmark's shapes: one launch per CUDA-graph replay,
+    L2 flushed before each, median of `reps`.  Quantize inputs are N(0,1) bf16
+    (codes and scales do not change the time); GEMM inputs are random e4m3
+    codes with random positive scales."""
+    from fp8_scaled_matrix_b200 import fp8sm
+    torch.manual_seed(0)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    peaks, _ = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    fp8_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])) * FP8_OVER_BF16
+    res = {}
+
+    def want(name):
+        return not only or name in only
+
+    if kind == "quantize":
+        R = {"tensor": fp8sm.FP8_SCALE_TENSOR, "row": fp8sm.FP8_SCALE_ROW,
+             "1x128": fp8sm.FP8_SCALE_BLOCK_1x128, "128x128": fp8sm.FP8_SCALE_BLOCK_128x128}
+
+        def rec(name, nbytes, fn):
+            us = _timed_graph(fn, reps, flush)
+            res[name] = {"us": us, "gbs": nbytes / us / 1e3, "frac": nbytes / us / 1e3 / hbm}
+
+        def bf16(r, c):
+            return torch.randn(r, c, device=dev).to(torch.bfloat16)
+        for rows, cols, rc in [(4096, 4096, "row"), (32768, 4096, "row"), (65536, 4096, "row"),
+                               (16640, 8192, "1x128"), (16640, 5120, "1x128"),
+                               (5120, 8192, "128x128"), (8192, 5120, "128x128"),
+                               (256, 256, "tensor")]:
+            name = f"{rc}_{rows}x{cols}"
+            if not want(name):
+                continue
+            t = bf16(rows, cols)
+            q = torch.empty(rows, cols, dtype=torch.uint8, device=dev)
+            sc = torch.empty(max(fp8sm.scale_count(rows, cols, R[rc]), 1), dtype=torch.float32,
+                             device=dev)
+            ws = torch.zeros(64, dtype=torch.uint8, device=dev)
+            rec(name, 3 * rows * cols + 4 * sc.numel(),
+                lambda: fp8sm.fp8_quantize(t, R[rc], out=q, scales=sc, workspace=ws))
+        for rows, cols, rc in [(16640, 8192, "1x128"), (16640, 5120, "1x128"),
+                               (5120, 8192, "128x128"), (8192, 5120, "128x128")]:
+            name = f"T{rc}_{rows}x{cols}"
+            if not want(name):
+                continue
+            t = bf16(rows, cols)
+            q = torch.empty(cols, rows, dtype=torch.uint8, device=dev)
+            n = ((rows // 128) * cols if rc == "1x128"
+                 else (rows // 128) * ((cols + 127) // 128))
+            sc = torch.empty(n, dtype=torch.float32, device=dev)
+            rec(name, 3 * rows * cols + 4 * n,
+                lambda: fp8sm.fp8_quantize_transposed(t, R[rc], out=q, scales=sc))
+        if want("Tgrouped_32768x4096"):
+            wl = W.make_workload(13, 0)   # the MoE weight gradient's tokens and split
+            t, offs = wl.a.to(dev), wl.offs.to(dev)
+            P = fp8sm.fp8_grouped_padded_tokens(wl.K, wl.E)
+            q = torch.empty(wl.M, P, dtype=torch.uint8, device=dev)
+            sc = torch.empty(P // 128, wl.M, dtype=torch.float32, device=dev)
+            rec("Tgrouped_32768x4096", 3 * t.numel() + 4 * sc.numel(),
+                lambda: fp8sm.fp8_quantize_transposed_grouped(t, offs, out=q, scales=sc))
+        if want("batched128_16x4096x4096") or want("Tbatched128_16x4096x4096"):
+            t = (torch.randn(16 * 4096, 4096, device=dev) * 0.02).to(torch.bfloat16)
+            t = t.view(16, 4096, 4096)
+            q = torch.empty(16 * 4096, 4096, dtype=torch.uint8, device=dev)
+            sc = torch.empty(16 * 32 * 32, dtype=torch.float32, device=dev)
+            nb = 3 * t.numel() + 4 * sc.numel()
+            if want("batched128_16x4096x4096"):
+                rec("batched128_16x4096x4096", nb, lambda: fp8sm.fp8_quantize_batched(
+                    t, fp8sm.FP8_SCALE_BLOCK_128x128, out=q, scales=sc))
+            if want("Tbatched128_16x4096x4096"):
+                rec("Tbatched128_16x4096x4096", nb, lambda: fp8sm.fp8_quantize_transposed_batched(
+                    t, fp8sm.FP8_SCALE_BLOCK_128x128, out=q, scales=sc))
+        if want("mx_16640x8192"):
+            t = bf16(16640, 8192)
+            q = torch.empty(16640, 8192, dtype=torch.uint8, device=dev)
+            sc = torch.empty(fp8sm.fp8_mx_scale_bytes(16640, 8192), dtype=torch.uint8, device=dev)
+            rec("mx_16640x8192", 3 * t.numel() + sc.numel(),
+                lambda: fp8sm.fp8_quantize_mx(t, out=q, scales=sc))
+        return res
+
+    def gemm(name, M, N, K, recipe):
+        if not want(name):
+            return
+        a, b = _random_codes(M, K, dev), _random_codes(N, K, dev)
+        if recipe == "1x128_128x128":
+            na, nb = (K // 128) * M, (K // 128) * ((N + 127) // 128)
+        elif recipe == "1x128_128x1":
+            na, nb = (K // 128) * M, (K // 128) * N
+        else:
+            na, nb = M, N
+        sa = torch.rand(na, device=dev) * 0.01 + 0.001
+        sb = torch.rand(nb, device=dev) * 0.01 + 0.001
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        us = _timed_graph(lambda: fp8sm.fp8_scaled_mm(a, b, sa, sb, fp8sm.MM_RECIPES[recipe],
+                                                      out=out), reps, flush)
+        tf = 2 * M * N * K / us / 1e6
+        res[name] = {"us": us, "tflops": tf, "frac": tf / fp8_peak}
+    gemm("blk128", 16640, 5120, 8192, "1x128_128x128")
+    gemm("blk128_b", 16640, 8192, 5120, "1x128_128x128")
+    gemm("blk1", 16640, 5120, 8192, "1x128_128x1")
+    gemm("blk1_b", 16640, 8192, 5120, "1x128_128x1")
+    gemm("row", 4096, 4096, 4096, "row")
+    gemm("row_16640x5120x8192", 16640, 5120, 8192, "row")
+    if want("mx"):
+        M, N, K = 16640, 5120, 8192
+        a, b = _random_codes(M, K, dev), _random_codes(N, K, dev)
+        sa = torch.randint(120, 130, (fp8sm.fp8_mx_scale_bytes(M, K),), dtype=torch.uint8,
+                           device=dev)
+        sb = torch.randint(120, 130, (fp8sm.fp8_mx_scale_bytes(N, K),), dtype=torch.uint8,
+                           device=dev)
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        us = _timed_graph(lambda: fp8sm.fp8_scaled_mm_mx(a, b, sa, sb, out=out), reps, flush)
+        tf = 2 * M * N * K / us / 1e6
+        res["mx"] = {"us": us, "tflops": tf, "frac": tf / fp8_peak}
+    return res
+
+
 # ------------------------------------------------------------------ main
 
 def main(argv=None):
@@ -1052,6 +1208,11 @@ def main(argv=None):
     ap.add_argument("--no-all-configs", action="store_true",
                     help="skip timing the five benchmark configurations after the step")
     ap.add_argument("--config-reps", type=int, default=20)
+    ap.add_argument("--kernel-table", choices=["quantize", "gemm"], default=None,
+                    help="time every quantize kernel or GEMM recipe alone on the benchmark's "
+                         "shapes and print one JSON line with the table (no step)")
+    ap.add_argument("--only", default="",
+                    help="with --kernel-table: comma-separated entry names to time")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -1094,6 +1255,16 @@ def main(argv=None):
                     "d2h_bytes_per_step": 0},
         }
         print(json.dumps(line), flush=True)
+        return 0
+
+    if args.kernel_table:
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        from fp8_scaled_matrix_b200 import build
+        build.build()
+        only = [x for x in args.only.split(",") if x]
+        print(json.dumps({"kernel_table": args.kernel_table,
+                          "entries": kernel_table(args.kernel_table, only, dev)}), flush=True)
         return 0
 
     if world > 1:

@@ -116,6 +116,33 @@ def gpu_wgrad(dy, x, offs_np, out_dtype=torch.float32):
     return qa, sa, qb, sb, out
 
 
+def test_grouped_transposed_quantize_many_tiles_per_cta():
+    """The per-expert padded transposed quantization on enough tiles that every
+    persistent CTA reuses its tile buffers several times, with empty, ragged
+    and multi-block groups: each group's padded codes and scales bit-exact
+    against the oracle's quantization of that group's zero-padded transpose."""
+    sizes = [0, 3000, 1, 4096, 0, 5000, 128, 3775]
+    T, cols = sum(sizes), 2048
+    g = W.generator(9090)
+    x = W.randn_bf16((T, cols), 1.0, g, outlier_frac=0.001, outlier_mult=50.0)
+    ends = np.cumsum(sizes).astype(np.int32)
+    offs = torch.as_tensor(ends, dtype=torch.int32).cuda()
+    q, s = fp8sm.fp8_quantize_transposed_grouped(x.cuda(), offs)
+    torch.cuda.synchronize()
+    fp8sm.check_device_status()
+    q, s = q.cpu().numpy(), s.cpu().numpy()
+    start, pb = 0, 0
+    for end in ends:
+        n = int(end) - start
+        nblk = -(-n // 128)
+        if n:
+            oq, osc = oracle.quantize(padded_t_bits(x, start, int(end)), oracle.GROUP_1x128)
+            cols_ = slice(128 * pb, 128 * (pb + nblk))
+            assert np.array_equal(q[:, cols_], oq)
+            assert np.array_equal(s[pb:pb + nblk].reshape(-1).view(np.uint32), osc.view(np.uint32))
+        start, pb = int(end), pb + nblk
+
+
 @pytest.mark.parametrize("sizes,M,N", [
     ([5, 0, 17, 130], 256, 272),
     ([0, 0, 64, 0], 128, 256),

@@ -48,6 +48,22 @@ def test_quantize_transposed_parity(group, rows, cols, pad):
     assert np.array_equal(s.cpu().numpy().view(np.uint32), osc.view(np.uint32))
 
 
+@pytest.mark.parametrize("group", ["1x128", "128x128"])
+@pytest.mark.parametrize("rows,cols", [(16384, 2048), (12288, 1544)])
+def test_quantize_transposed_parity_many_tiles_per_cta(group, rows, cols):
+    """Enough 128 x 128 tiles that every persistent CTA walks its two-buffer
+    tile ring several times (buffer reuse, phase flips), with a ragged last
+    column tile in the second case; bit-exact against the oracle."""
+    g = W.generator(rows + 3 * cols)
+    x = W.randn_bf16((rows, cols), 1.0, g, outlier_frac=0.001, outlier_mult=50.0)
+    q, s = fp8sm.fp8_quantize_transposed(x.cuda(), QR[group])
+    torch.cuda.synchronize()
+    fp8sm.check_device_status()
+    oq, osc = oracle_quantize_t(x, group)
+    assert np.array_equal(codes_np(q), oq)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), osc.view(np.uint32))
+
+
 def test_quantize_transposed_matches_forward_quantize_of_transpose():
     """Same codes and scales as fp8_quantize applied to a materialised x^T."""
     g = W.generator(77)
