@@ -324,14 +324,23 @@ __device__ __forceinline__ void load_bias32(const uint16_t* bias, int64_t n,
 
 // Stage 4 x 16-byte chunks of this lane's row in the warp's 32 x 64-byte
 // buffer (64-byte swizzle: chunk j of row r lives at slot j ^ ((r >> 1) & 3)),
-// then write the 32 x 64-byte box to global memory: by TMA store for the
-// dense kernel, by masked 16-byte stores for the grouped kernel.
-template <bool kGrouped>
+// then write the 32 x 64-byte box to global memory.  kStore:
+//   kStoreTma     TMA store (boxes wholly past the last row or column are
+//                 skipped, partial ones clipped at the matrix's edges);
+//   kStoreMixed   (row-grouped kernels, whose tiles may end inside a group)
+//                 TMA store for a box whose 32 rows all lie before row_end,
+//                 masked 16-byte stores for one that crosses row_end;
+//   kStoreMasked  masked 16-byte stores always (the grouped blockwise
+//                 kernel: its epilogue holds 128 accumulators per thread, and
+//                 the second store path's registers cost it more than TMA
+//                 stores save, measured).
+enum StoreMode : int { kStoreTma = 0, kStoreMixed = 1, kStoreMasked = 2 };
+template <int kStore>
 __device__ __forceinline__ void store_box64(
     uint8_t* buf, const uint4 (&chunk)[4], const CUtensorMap* tm_out,
     int32_t col0 /*elements*/, int32_t row0, int64_t row_end, uint8_t* out,
     int64_t N, uint32_t elem_bytes, uint32_t lane) {
-  if constexpr (!kGrouped) {
+  if constexpr (kStore != kStoreMasked) {
     // the previous box's TMA store must have read the buffer
     if (lane == 0) bulk_wait_group_read0();
     __syncwarp();
@@ -341,11 +350,12 @@ __device__ __forceinline__ void store_box64(
     const uint32_t slot = static_cast<uint32_t>(j) ^ ((lane >> 1) & 3u);
     *reinterpret_cast<uint4*>(buf + lane * 64 + slot * 16) = chunk[j];
   }
-  if constexpr (!kGrouped) {
+  // warp-uniform
+  const bool whole = kStore == kStoreTma ||
+                     (kStore == kStoreMixed && static_cast<int64_t>(row0) + 32 <= row_end);
+  if (whole) {
     fence_proxy_async_smem();
     __syncwarp();
-    // Boxes wholly past the last row or column are skipped; partial boxes are
-    // clipped by the TMA unit.
     if (lane == 0 && row0 < row_end && col0 < N) {
       tma_store_2d(tm_out, buf, col0, row0);
       bulk_commit_group();
@@ -370,7 +380,7 @@ __device__ __forceinline__ void store_box64(
 }
 
 // Write 32 fp32 results of this lane's row (columns col0 .. col0+31).
-template <bool kOutF32, bool kGrouped>
+template <bool kOutF32, int kStore>
 __device__ __forceinline__ void store_cols32(
     uint8_t* buf, const float (&v)[32], const CUtensorMap* tm_out, int32_t col0,
     int32_t row0, int64_t row_end, void* out, int64_t N, uint32_t lane) {
@@ -382,8 +392,8 @@ __device__ __forceinline__ void store_cols32(
                         pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
                         pack_bf16x2(v[8 * j + 4], v[8 * j + 5]),
                         pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
-    store_box64<kGrouped>(buf, c, tm_out, col0, row0, row_end,
-                          static_cast<uint8_t*>(out), N, 2, lane);
+    store_box64<kStore>(buf, c, tm_out, col0, row0, row_end,
+                        static_cast<uint8_t*>(out), N, 2, lane);
   } else {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -394,8 +404,8 @@ __device__ __forceinline__ void store_cols32(
                           __float_as_uint(v[16 * h + 4 * j + 1]),
                           __float_as_uint(v[16 * h + 4 * j + 2]),
                           __float_as_uint(v[16 * h + 4 * j + 3]));
-      store_box64<kGrouped>(buf, c, tm_out, col0 + 16 * h, row0, row_end,
-                            static_cast<uint8_t*>(out), N, 4, lane);
+      store_box64<kStore>(buf, c, tm_out, col0 + 16 * h, row0, row_end,
+                          static_cast<uint8_t*>(out), N, 4, lane);
     }
   }
 }
@@ -415,10 +425,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   // grouped 1x128_128x1 = the per-expert weight gradient: groups split K
   // (tokens), every group has its own (M, N) output
   constexpr bool kKGroups = kGrouped && kRecipe == kBlock1;
-  // stores: masked plain stores where a tile's rows may end inside a group
-  // (the row-grouped kernels); TMA stores otherwise (the K-grouped output's
-  // tiles are whole: M % 128 == 0)
+  // stores: TMA stores; the row-grouped kernels' tiles may end inside a
+  // group, so there a 32-row box that crosses the group's end goes out by
+  // masked plain stores instead (the K-grouped output's tiles are whole:
+  // M % 128 == 0)
   constexpr bool kMasked = kGrouped && !kKGroups;
+  constexpr int kStore = !kMasked ? kStoreTma : kBlockwise ? kStoreMasked : kStoreMixed;
   // epilogue threads that hold a whole 128-column row slice across K blocks
   // (blockwise promotion) get registers moved from warpgroup 0.  The MXFP8
   // epilogue reads its accumulators once per tile and runs without the split.
@@ -474,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_b);
     if constexpr (!kGrouped) prefetch_tmap(&tm_b_half);
-    if constexpr (!kMasked) prefetch_tmap(&tm_out);
+    prefetch_tmap(&tm_out);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -964,7 +976,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               load_bias32(p.bias, n, p.N, v);
 #pragma unroll
               for (int i = 0; i < 32; ++i) v[i] = __fadd_rn(__uint_as_float(r[cc][i]), v[i]);
-              store_cols32<kOutF32, kMasked>(ebuf, v, &tm_out, static_cast<int32_t>(n), row0,
+              store_cols32<kOutF32, kStore>(ebuf, v, &tm_out, static_cast<int32_t>(n), row0,
                                               c.row_end, p.out, p.N, lane);
             }
           } else {
@@ -997,7 +1009,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   w[j] = cast_f32x2(v[4 * j], v[4 * j + 1], inv) |
                          (cast_f32x2(v[4 * j + 2], v[4 * j + 3], inv) << 16);
               }
-              store_box64<kMasked>(ebuf, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
+              store_box64<kStore>(ebuf, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
                                     row0, c.row_end, static_cast<uint8_t*>(p.out), p.N, 1, lane);
             }
             if (ncol0 < p.N) {
@@ -1047,7 +1059,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float v[32];
             values32(cc, v);
             if (cc == 3) release_buf();
-            store_cols32<kOutF32, kMasked>(ebuf, v, &tm_out,
+            store_cols32<kOutF32, kStore>(ebuf, v, &tm_out,
                                             static_cast<int32_t>(ncol0 + cc * 32), row0,
                                             c.row_end, p.out, p.N, lane);
           }
@@ -1080,7 +1092,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 w[j] = cast_f32x2(v[4 * j], v[4 * j + 1], sp.inv) |
                        (cast_f32x2(v[4 * j + 2], v[4 * j + 3], sp.inv) << 16);
             }
-            store_box64<kMasked>(ebuf, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
+            store_box64<kStore>(ebuf, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
                                   row0, c.row_end, static_cast<uint8_t*>(p.out), p.N, 1, lane);
           }
         }
@@ -1179,7 +1191,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int cc = 0; cc < 4; ++cc) {
             float v[32];
             result32(cc, v);
-            store_cols32<kOutF32, kMasked>(ebuf, v, &tm_out,
+            store_cols32<kOutF32, kStore>(ebuf, v, &tm_out,
                                             static_cast<int32_t>(ncol0 + cc * 32), row0,
                                             c.row_end, p.out, p.N, lane);
           }
@@ -1289,7 +1301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
               }
             }
-            store_box64<kMasked>(ebuf, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
+            store_box64<kStore>(ebuf, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
                                   row0, c.row_end, static_cast<uint8_t*>(p.out), p.N, 1, lane);
           }
         }
@@ -1579,8 +1591,8 @@ cudaError_t launch_grouped_scaled_mm(const void* a, const void* b,
                    CU_TENSOR_MAP_SWIZZLE_128B, ctx.err))
       return cudaErrorInvalidValue;
   }
-  // The grouped kernel stores with plain masked stores; the map is unused
-  // but must be a valid object.
+  // Output map over all M_total rows: boxes wholly inside a group leave by
+  // TMA store, the box that crosses a group's end by masked stores.
   if (!out_map(&to, out, M_total, N, out_f32 ? kOutFp32 : kOutBf16, ctx.err))
     return cudaErrorInvalidValue;
   GemmParams p{};
@@ -1625,7 +1637,7 @@ cudaError_t launch_grouped_wgrad(const void* a_t, const void* b_t, int64_t M, in
                    CU_TENSOR_MAP_SWIZZLE_128B, ctx.err))
       return cudaErrorInvalidValue;
   }
-  // the kernel stores with plain masked stores; the map must be a valid object
+  // output (E * M, N): every tile is whole and leaves by TMA store
   if (!out_map(&to, out, static_cast<int64_t>(E) * M, N, out_f32 ? kOutFp32 : kOutBf16, ctx.err))
     return cudaErrorInvalidValue;
   GemmParams p{};
