@@ -614,6 +614,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(a_dst, &tm_a, &full[stage], kb * BK, c.m0);
             if constexpr (kGrouped)
               tma_load_3d(b_dst, &tm_b, &full[stage], kb * BK, c.n0, c.g);
+            else if (p.raster_m > 0)
+              // banded order: B is streamed once per band, A's band is reused
+              // by every wave of the band; B's lines go first
+              tma_load_2d_hint(b_dst, c.half_n ? &tm_b_half : &tm_b, &full[stage], kb * BK,
+                               c.n0, l2_policy_evict_first());
             else
               tma_load_2d(b_dst, c.half_n ? &tm_b_half : &tm_b, &full[stage], kb * BK, c.n0);
           }
