@@ -1322,7 +1322,7 @@ def main(argv=None):
             "out_dtype": "bf16",
             "l2": "flushed between steps (256 MB write + read back, outside the step events)",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "step": ("quantize X || quantize W1, W2 (two streams), then GEMM1 with its "
+            "step": ("quantize W1, W2, then X (one stream), then GEMM1 with its "
                      "output quantized 1x128 in the epilogue, then GEMM2"
                      if wl.recipe == "chain" else
                      "MXFP8 quantize X || W1, W2 (two streams), then GEMM1 with MXFP8 "
@@ -1332,6 +1332,8 @@ def main(argv=None):
                      "W2^T) and backward (dY1 = dY2 W2 writing dY1 and dY1^T in e4m3, dX = "
                      "dY1 W1, dW1 = dY1^T X, dW2 = dY2^T Y1)"
                      if wl.recipe == "chain_train" else
+                     "quantize B, then A (one stream), then scaled GEMM"
+                     if wl.recipe == "1x128_128x128" else
                      "quantize A || quantize B (two streams), then scaled GEMM"),
             "N2": (int(wl.extra["b2"].shape[0]) if "b2" in wl.extra else None),
             "launch": ("CUDA graphs of the step's C-ABI launches" if args.graphs
