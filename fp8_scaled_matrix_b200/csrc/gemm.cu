@@ -90,9 +90,12 @@ constexpr uint32_t kMxSfStage = 3 * kMxSfTile;
 constexpr uint32_t kMxSfCols = 16;
 
 // Shared-memory layout.  Tiles are 128 x 256: each stage holds A (128 rows)
-// and B (256 rows) of a 128-byte K slice.
-struct Cfg {
-  static constexpr int kStages = 4;
+// and B (256 rows) of a 128-byte K slice.  kStaged: one stage traded for
+// four output staging buffers per epilogue warp (staged_epilogue below).
+template <bool kStaged>
+struct CfgT {
+  static constexpr int kStages = kStaged ? 3 : 4;
+  static constexpr int kEpiBufs = kStaged ? 4 : 1;  // staging buffers per epilogue warp
   static constexpr int kTileM = BM;   // output rows per work item
   static constexpr uint32_t kBRows = BN;  // B rows held per stage
   static constexpr uint32_t kAStage = BM * BK;
@@ -100,7 +103,7 @@ struct Cfg {
   static constexpr uint32_t kOffA = 0;
   static constexpr uint32_t kOffB = kOffA + kStages * kAStage;
   static constexpr uint32_t kOffEpi = kOffB + kStages * kBStage;
-  static constexpr uint32_t kOffScl = kOffEpi + kEpiWarps * kEpiBuf;
+  static constexpr uint32_t kOffScl = kOffEpi + kEpiWarps * kEpiBufs * kEpiBuf;
   static constexpr uint32_t kOffTpos = kOffScl + kSclBytes;
   static constexpr uint32_t kOffBar = kOffTpos + kEpiWarps * kTposBuf;
   // barriers: full[kStages], empty[kStages], acc_full[2], acc_empty[2], drain,
@@ -113,6 +116,7 @@ struct Cfg {
   static_assert(kStages * kMxSfStage <= kSclBytes, "MXFP8 scale tiles fit the ring region");
   static_assert(BN + kStages * kMxSfCols <= kTmemCols, "MXFP8 TMEM slots");
 };
+using Cfg = CfgT<false>;
 
 enum Recipe : int { kTensor = 0, kRow = 1, kBlock128 = 2, kBlock1 = 3, kMxfp8 = 4 };
 // Output: bf16, fp32, e4m3 quantized in 1x128 groups along n (+ fp32
@@ -121,6 +125,17 @@ enum Recipe : int { kTensor = 0, kRow = 1, kBlock128 = 2, kBlock1 = 3, kMxfp8 = 
 // result (1x128 along n, and transposed with 1x128 groups along m: the two
 // operands the next layer's backward GEMMs read)
 enum OutKind : int { kOutBf16 = 0, kOutFp32 = 1, kOutE4M3 = 2, kOutMx = 3, kOutE4M3Dual = 4 };
+
+// A blockwise epilogue writes its tile only after the last K block, while the
+// MMA can run at most two K blocks ahead; with four staging buffers per warp
+// the tile's boxes leave back to back instead of each waiting for the
+// previous box's TMA store to read the one buffer.  Measured worth the stage
+// it costs for 1x128_128x1 (844 against 867 us on 16640 x 5120 x 8192); the
+// 1x128_128x128 kernels (every output kind) gain nothing from it and keep
+// four stages.
+__host__ __device__ constexpr bool staged_epilogue(int recipe, int /*out_kind*/) {
+  return recipe == kBlock1;
+}
 
 struct GemmParams {
   int64_t M, N, K;
@@ -335,15 +350,22 @@ __device__ __forceinline__ void load_bias32(const uint16_t* bias, int64_t n,
 //                 the second store path's registers cost it more than TMA
 //                 stores save, measured).
 enum StoreMode : int { kStoreTma = 0, kStoreMixed = 1, kStoreMasked = 2 };
-template <int kStore>
+// The warp's kBufs staging buffers (ebase, kEpiBuf bytes each) take the boxes
+// in turn (nbox counts them); before the first buffer is reused, every
+// earlier TMA store of the warp must have read its buffer.
+template <int kStore, int kBufs>
 __device__ __forceinline__ void store_box64(
-    uint8_t* buf, const uint4 (&chunk)[4], const CUtensorMap* tm_out,
+    uint8_t* ebase, uint32_t& nbox, const uint4 (&chunk)[4], const CUtensorMap* tm_out,
     int32_t col0 /*elements*/, int32_t row0, int64_t row_end, uint8_t* out,
     int64_t N, uint32_t elem_bytes, uint32_t lane) {
+  const uint32_t b = kBufs > 1 ? nbox % kBufs : 0u;
+  uint8_t* buf = ebase + b * kEpiBuf;
+  ++nbox;
   if constexpr (kStore != kStoreMasked) {
-    // the previous box's TMA store must have read the buffer
-    if (lane == 0) bulk_wait_group_read0();
-    __syncwarp();
+    if (b == 0) {
+      if (lane == 0) bulk_wait_group_read0();
+      __syncwarp();
+    }
   }
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -380,10 +402,10 @@ __device__ __forceinline__ void store_box64(
 }
 
 // Write 32 fp32 results of this lane's row (columns col0 .. col0+31).
-template <bool kOutF32, int kStore>
+template <bool kOutF32, int kStore, int kBufs>
 __device__ __forceinline__ void store_cols32(
-    uint8_t* buf, const float (&v)[32], const CUtensorMap* tm_out, int32_t col0,
-    int32_t row0, int64_t row_end, void* out, int64_t N, uint32_t lane) {
+    uint8_t* ebase, uint32_t& nbox, const float (&v)[32], const CUtensorMap* tm_out,
+    int32_t col0, int32_t row0, int64_t row_end, void* out, int64_t N, uint32_t lane) {
   if constexpr (!kOutF32) {
     uint4 c[4];
 #pragma unroll
@@ -392,8 +414,8 @@ __device__ __forceinline__ void store_cols32(
                         pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
                         pack_bf16x2(v[8 * j + 4], v[8 * j + 5]),
                         pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
-    store_box64<kStore>(buf, c, tm_out, col0, row0, row_end,
-                        static_cast<uint8_t*>(out), N, 2, lane);
+    store_box64<kStore, kBufs>(ebase, nbox, c, tm_out, col0, row0, row_end,
+                               static_cast<uint8_t*>(out), N, 2, lane);
   } else {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -404,8 +426,8 @@ __device__ __forceinline__ void store_cols32(
                           __float_as_uint(v[16 * h + 4 * j + 1]),
                           __float_as_uint(v[16 * h + 4 * j + 2]),
                           __float_as_uint(v[16 * h + 4 * j + 3]));
-      store_box64<kStore>(buf, c, tm_out, col0 + 16 * h, row0, row_end,
-                          static_cast<uint8_t*>(out), N, 4, lane);
+      store_box64<kStore, kBufs>(ebase, nbox, c, tm_out, col0 + 16 * h, row0, row_end,
+                                 static_cast<uint8_t*>(out), N, 4, lane);
     }
   }
 }
@@ -443,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // epilogue is at the edge of its register budget, keeps the M-major order
   // (its B is a layer's weight, which fits in L2)
   constexpr bool kRaster = !kOutQT;
-  using C = Cfg;
+  using C = CfgT<staged_epilogue(kRecipe, kOut)>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
@@ -901,7 +923,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t ew = warp - kFirstEpiWarp;  // 0..7
     const uint32_t q = warp & 3u;          // TMEM lane quarter of this warp
     const uint32_t half = ew >> 2;         // which 128 columns of the tile
-    uint8_t* ebuf = smem + C::kOffEpi + ew * kEpiBuf;
+    uint8_t* ebuf = smem + C::kOffEpi + ew * C::kEpiBufs * kEpiBuf;
+    uint32_t nbox = 0;  // boxes this warp has staged
     const uint32_t lane_base = (q * 32u) << 16;
     GroupCursor cur;
     KGroupCursor kc;
@@ -981,7 +1004,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               load_bias32(p.bias, n, p.N, v);
 #pragma unroll
               for (int i = 0; i < 32; ++i) v[i] = __fadd_rn(__uint_as_float(r[cc][i]), v[i]);
-              store_cols32<kOutF32, kStore>(ebuf, v, &tm_out, static_cast<int32_t>(n), row0,
+              store_cols32<kOutF32, kStore, C::kEpiBufs>(ebuf, nbox, v, &tm_out, static_cast<int32_t>(n), row0,
                                               c.row_end, p.out, p.N, lane);
             }
           } else {
@@ -1014,7 +1037,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   w[j] = cast_f32x2(v[4 * j], v[4 * j + 1], inv) |
                          (cast_f32x2(v[4 * j + 2], v[4 * j + 3], inv) << 16);
               }
-              store_box64<kStore>(ebuf, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
+              store_box64<kStore, C::kEpiBufs>(ebuf, nbox, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
                                     row0, c.row_end, static_cast<uint8_t*>(p.out), p.N, 1, lane);
             }
             if (ncol0 < p.N) {
@@ -1064,7 +1087,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float v[32];
             values32(cc, v);
             if (cc == 3) release_buf();
-            store_cols32<kOutF32, kStore>(ebuf, v, &tm_out,
+            store_cols32<kOutF32, kStore, C::kEpiBufs>(ebuf, nbox, v, &tm_out,
                                             static_cast<int32_t>(ncol0 + cc * 32), row0,
                                             c.row_end, p.out, p.N, lane);
           }
@@ -1097,7 +1120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 w[j] = cast_f32x2(v[4 * j], v[4 * j + 1], sp.inv) |
                        (cast_f32x2(v[4 * j + 2], v[4 * j + 3], sp.inv) << 16);
             }
-            store_box64<kStore>(ebuf, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
+            store_box64<kStore, C::kEpiBufs>(ebuf, nbox, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
                                   row0, c.row_end, static_cast<uint8_t*>(p.out), p.N, 1, lane);
           }
         }
@@ -1196,7 +1219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int cc = 0; cc < 4; ++cc) {
             float v[32];
             result32(cc, v);
-            store_cols32<kOutF32, kStore>(ebuf, v, &tm_out,
+            store_cols32<kOutF32, kStore, C::kEpiBufs>(ebuf, nbox, v, &tm_out,
                                             static_cast<int32_t>(ncol0 + cc * 32), row0,
                                             c.row_end, p.out, p.N, lane);
           }
@@ -1306,7 +1329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
               }
             }
-            store_box64<kStore>(ebuf, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
+            store_box64<kStore, C::kEpiBufs>(ebuf, nbox, chunk, &tm_out, static_cast<int32_t>(ncol0 + 64 * bx),
                                   row0, c.row_end, static_cast<uint8_t*>(p.out), p.N, 1, lane);
           }
         }
@@ -1370,6 +1393,7 @@ cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb,
     return cudaErrorInvalidValue;  // quantized output: dense GEMM only
   } else {
     auto kern = fp8_gemm_kernel<kRecipe, kOut, kGrouped>;
+    using Cfg = CfgT<staged_epilogue(kRecipe, kOut)>;
     // the dynamic shared-memory opt-in, once per device
     static std::atomic<bool> done[kMaxDevices];
     static std::mutex mu;
