@@ -1276,6 +1276,11 @@ def main(argv=None):
     build.build()
 
     wl = W.make_workload(idx, shape_index)
+    if world > 1:
+        # data parallel over M (weak scaling): rank r works on its own shard of
+        # the global batch, the workload's rows rotated by r * M / world; the
+        # second operand (the weights) is the same on every rank
+        wl.a = torch.roll(wl.a, shifts=rank * (wl.a.shape[0] // world), dims=0)
     if args.steps is None:
         # about a second of timed work per workload
         args.steps = {"tensorwise_256": 4000, "rowwise_4096": 3000,
