@@ -92,6 +92,34 @@ def test_noalloc_on_a_side_stream_after_the_default_stream(recipe):
     _check_oracle(x2, recipe, q2, s2)
 
 
+@pytest.mark.parametrize("recipe", RECIPES)
+def test_noalloc_replayed_from_a_cuda_graph(recipe):
+    """The supported capture pattern: a first call outside any capture (it
+    looks up the library's scratch), then a call captured in a CUDA graph;
+    every replay writes the oracle's codes and scales (the outputs are
+    cleared between replays, so a replay that did nothing would fail)."""
+    g = W.generator(4245 + recipe)
+    x = (W.randn_bf16((384, 512), 1.0, g) * 4).to(torch.bfloat16).cuda()
+    _noalloc(x, recipe)
+    torch.cuda.synchronize()
+    q = torch.empty(384, 512, dtype=torch.uint8, device="cuda")
+    s = torch.empty(max(fp8sm.scale_count(384, 512, recipe), 1), dtype=torch.float32,
+                    device="cuda")
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        fp8sm.fp8_quantize_noalloc(x, recipe, q, s, stream=stream)
+    for _ in range(2):
+        q.zero_()
+        s.zero_()
+        torch.cuda.current_stream().synchronize()
+        graph.replay()
+        torch.cuda.synchronize()
+        fp8sm.check_device_status()
+        _check_oracle(x, recipe, q, s)
+
+
 def test_noalloc_rejects_bad_arguments_like_fp8_quantize():
     x = torch.zeros(4, 100, dtype=torch.bfloat16, device="cuda")
     q = torch.empty(4, 100, dtype=torch.uint8, device="cuda")
