@@ -896,14 +896,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       cp_async_wait_all();  // nothing lands in shared memory after the CTA exits
-      if (!ok) {
-        // the epilogue stopped consuming: let the bulk copies in flight land
-        const uint64_t first = issued > kSclSlots ? issued - kSclSlots : 0;
-        for (uint64_t i = first; i < issued; ++i) {
-          uint32_t dummy_abort = 0;
-          mbar_wait(&sfull[i % kSclSlots], static_cast<uint32_t>((i / kSclSlots) & 1u),
-                    &dummy_abort, nullptr, SITE_TEARDOWN, 10000000ull);
-        }
+      // nor do the bulk copies: wait (bounded) for the last slots' copies,
+      // which the epilogue may not have consumed if it stopped early
+      // (otherwise these phases are complete and the waits return at once)
+      const uint64_t first = issued > kSclSlots ? issued - kSclSlots : 0;
+      for (uint64_t i = first; i < issued; ++i) {
+        uint32_t dummy_abort = 0;
+        mbar_wait(&sfull[i % kSclSlots], static_cast<uint32_t>((i / kSclSlots) & 1u),
+                  &dummy_abort, nullptr, SITE_TEARDOWN, 10000000ull);
       }
     } else if constexpr (kMxGather) {
       // ------------------------------------- grouped MXFP8: A scale gather
