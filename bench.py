@@ -151,6 +151,14 @@ def max_over_ranks(x: float, dev) -> float:
     return float(t.item())
 
 
+def rank_shard_rows(a: torch.Tensor, rank: int, world: int) -> torch.Tensor:
+    """Data parallel over M (weak scaling): rank r works on its own shard of
+    the global batch -- the workload's activation rows rotated by
+    r * M / world, same shape and distribution on every rank -- while the
+    second operand (the weights) is the same everywhere."""
+    return torch.roll(a, shifts=rank * (a.shape[0] // world), dims=0)
+
+
 def job_tflops(flops_per_rank: float, world: int, ms: float) -> float:
     """Whole-job throughput: every rank's work over the slowest rank's time."""
     return flops_per_rank * world / (ms * 1e-3) / 1e12
@@ -1277,10 +1285,7 @@ def main(argv=None):
 
     wl = W.make_workload(idx, shape_index)
     if world > 1:
-        # data parallel over M (weak scaling): rank r works on its own shard of
-        # the global batch, the workload's rows rotated by r * M / world; the
-        # second operand (the weights) is the same on every rank
-        wl.a = torch.roll(wl.a, shifts=rank * (wl.a.shape[0] // world), dims=0)
+        wl.a = rank_shard_rows(wl.a, rank, world)
     if args.steps is None:
         # about a second of timed work per workload
         args.steps = {"tensorwise_256": 4000, "rowwise_4096": 3000,

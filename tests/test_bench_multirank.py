@@ -56,3 +56,18 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     monkeypatch.setenv("WORLD_SIZE", "2")
     assert bench.main(["--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3"]) == 0
     assert capsys.readouterr().out == ""   # rank 1 prints nothing and does no work
+
+
+def test_each_rank_takes_its_own_row_shard():
+    """With N ranks, rank r multiplies the activation rows rotated by r * M / N:
+    every rank sees all rows (same shape and distribution), no two ranks
+    start at the same row, and rank 0 keeps the workload as generated."""
+    a = torch.arange(12 * 3, dtype=torch.float32).view(12, 3)
+    shards = [bench.rank_shard_rows(a, r, 4) for r in range(4)]
+    assert torch.equal(shards[0], a)
+    firsts = {int(s[0, 0]) for s in shards}
+    assert len(firsts) == 4
+    for r, s in enumerate(shards):
+        assert s.shape == a.shape
+        assert torch.equal(torch.sort(s[:, 0]).values, a[:, 0])   # the same rows, reordered
+        assert torch.equal(s[(12 // 4) * r % 12], a[0])
