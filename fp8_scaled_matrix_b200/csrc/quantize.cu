@@ -443,10 +443,13 @@ __global__ void __launch_bounds__(kTrThreads) quant_transposed_kernel(
   const int t = threadIdx.x;
   const int w = t >> 5;
   int32_t* pb0 = nullptr;  // grouped: pb0[g] = padded blocks before group g; pb0[E] = total
+  int32_t* gend = nullptr;  // grouped: gend[g] = offs[g], kept on chip for the tile loads
   if constexpr (kGroupedT) {
     __shared__ int32_t table[kTrMaxGroups + 1];
+    __shared__ int32_t ends[kTrMaxGroups];
     __shared__ int32_t bad;
     pb0 = table;
+    gend = ends;
     if (t < 32) {
       // lane l: groups [l * per, (l + 1) * per); block counts, then a scan
       const int32_t per = (E + 31) / 32;
@@ -468,6 +471,7 @@ __global__ void __launch_bounds__(kTrThreads) quant_transposed_kernel(
       for (int32_t g = g0; g < g1; ++g) {
         table[g] = run;
         const int32_t prev = g ? offs[g - 1] : 0;
+        ends[g] = offs[g];
         run += (max(offs[g] - prev, 0) + kTrRows - 1) / kTrRows;
       }
       if (t == 31) table[E] = incl;
@@ -490,9 +494,9 @@ __global__ void __launch_bounds__(kTrThreads) quant_transposed_kernel(
         if (pb0[mid] <= kb) lo = mid;
         else hi = mid - 1;
       }
-      const int64_t start = lo ? offs[lo - 1] : 0;
+      const int64_t start = lo ? gend[lo - 1] : 0;
       row0 = start + (kb - pb0[lo]) * kTrRows;
-      const int64_t left = static_cast<int64_t>(offs[lo]) - row0;
+      const int64_t left = static_cast<int64_t>(gend[lo]) - row0;
       nrows = static_cast<int32_t>(left < kTrRows ? left : kTrRows);
     } else {
       row0 = kb * kTrRows;
