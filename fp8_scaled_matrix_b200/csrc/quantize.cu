@@ -509,7 +509,10 @@ __global__ void __launch_bounds__(kTrThreads) quant_transposed_kernel(
   auto issue = [&](int64_t tile, int s) {
     const int64_t e = tile / per_matrix;
     const int64_t r = tile - e * per_matrix;
-    const int64_t kb = r % n_kb, cb = r / n_kb;
+    // grouped: column blocks fastest (measured 2 % faster there; the dense
+    // forms keep row blocks fastest, 4 % faster on 16640 x 5120)
+    const int64_t kb = kGroupedT ? r / n_cb : r % n_kb;
+    const int64_t cb = kGroupedT ? r % n_cb : r / n_kb;
     if (kb >= n_kb_used) {
       mbar_arrive(&full[s]);
       return;
@@ -545,7 +548,9 @@ __global__ void __launch_bounds__(kTrThreads) quant_transposed_kernel(
                                kWaitLimitNs);
     if (!__syncthreads_and(got)) break;
     const int64_t e = tile / per_matrix;
-    const int64_t kb = (tile - e * per_matrix) % n_kb, cb = (tile - e * per_matrix) / n_kb;
+    const int64_t rr = tile - e * per_matrix;
+    const int64_t kb = kGroupedT ? rr / n_cb : rr % n_kb;
+    const int64_t cb = kGroupedT ? rr % n_cb : rr / n_kb;
     if (kb >= n_kb_used) {  // grouped: past the last group's blocks (uniform)
       if (t == 0 && issued_to < n_tiles) {
         issue(issued_to, s);
